@@ -1,0 +1,18 @@
+"""Exact softmax attention forward for B200 (sm_100a).
+
+The compute lives in the CUDA C-ABI library ``libattn_b200.so`` (declared in
+``include/attn.h``); this package is its thin ctypes binding plus the seeded
+workload generators.  Importing the package does not load the library; the
+first call does, and raises if the library is missing or no GPU is present.
+"""
+from ._binding import (  # noqa: F401
+    AttnError,
+    attn_decode_paged,
+    attn_decode_workspace_size,
+    attn_fwd,
+    attn_fwd_masked,
+    attn_get_device_error,
+    attn_strerror,
+    library_path,
+    load_library,
+)

@@ -1,0 +1,179 @@
+"""ctypes binding of libattn_b200.so (the C ABI in include/attn.h).
+
+Argument marshalling only: tensors are passed as raw device pointers with
+their sizes, the CUDA stream as its handle.  Every step of the computation
+runs in the library's kernels; there is no fallback of any kind -- if the
+library or a GPU is missing, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_NAME = "libattn_b200.so"
+_lock = threading.Lock()
+_lib = None
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_ALIGNMENT = 3
+ATTN_ERR_WORKSPACE = 4
+ATTN_ERR_CUDA = 5
+ATTN_ERR_DEVICE = 6
+
+DEVERR_WAIT_TIMEOUT = 0x1
+DEVERR_BAD_PAGE = 0x2
+DEVERR_BAD_LENGTH = 0x4
+
+# Every function the header declares, with its ctypes signature.
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+SIGNATURES = {
+    "attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "attn_fwd_masked": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P]),
+    "attn_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P,
+                               _SZ, _P]),
+    "attn_get_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
+    "attn_strerror": (ctypes.c_char_p, [_I]),
+    "attn_split_tokens": (_I, []),
+}
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {attn_strerror(status)} (status {status})" if what
+                         else f"{attn_strerror(status)} (status {status})")
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, LIB_NAME)
+
+
+def load_library():
+    """Load libattn_b200.so from the package directory (raises if it is missing)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = library_path()
+            if not os.path.exists(path):
+                raise RuntimeError(
+                    f"{path} is missing: build it with `python -m exact_softmax_attention_fwd_b200.build`")
+            lib = ctypes.CDLL(path)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def attn_strerror(status: int) -> str:
+    try:
+        return load_library().attn_strerror(int(status)).decode()
+    except Exception:  # library not loadable: still describe the code
+        return {0: "success"}.get(int(status), f"status {status}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status, what):
+    if status != ATTN_OK:
+        raise AttnError(status, what)
+
+
+def _require_cuda(*tensors):
+    for t in tensors:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors (device memory)")
+
+
+def attn_fwd_masked(q, k, v, causal: bool, scale: float, k_lens=None, out=None, lse=None,
+                    return_lse: bool = True, stream=None):
+    """O, LSE = exact attention.  q [B,Hq,Sq,d], k/v [B,Hkv,Sk,d] bf16 CUDA tensors."""
+    import torch
+    _require_cuda(q, k, v, k_lens)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bfloat16")
+    B, Hq, Sq, d = q.shape
+    Bk, Hkv, Sk, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or dk != d:
+        raise ValueError("q/k/v shapes disagree")
+    if k_lens is not None and (k_lens.dtype != torch.int32 or tuple(k_lens.shape) != (B,)):
+        raise ValueError("k_lens must be int32 [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    st = load_library().attn_fwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq,
+                                        Hkv, Sq, Sk, d, int(bool(causal)), float(scale),
+                                        _ptr(k_lens), _stream(stream))
+    _check(st, "attn_fwd_masked")
+    return out, lse
+
+
+def attn_fwd(q, k, v, causal: bool, scale: float, out=None, lse=None, return_lse: bool = True,
+             stream=None):
+    """attn_fwd_masked without key padding."""
+    return attn_fwd_masked(q, k, v, causal, scale, None, out, lse, return_lse, stream)
+
+
+def attn_decode_workspace_size(B: int, Hq: int, max_pages_per_seq: int, page_size: int,
+                               d: int) -> int:
+    return int(load_library().attn_decode_workspace_size(B, Hq, max_pages_per_seq, page_size, d))
+
+
+def attn_decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float, out=None,
+                      lse=None, workspace=None, return_lse: bool = True, stream=None):
+    """Single-query attention over a paged cache (see include/attn.h for layouts)."""
+    import torch
+    _require_cuda(q, k_cache, v_cache, block_table, seq_lens)
+    B, Hq, d = q.shape
+    num_pages, page_size, Hkv, dk = k_cache.shape
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or dk != d:
+        raise ValueError("cache shapes disagree")
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be int32 [B, max_pages_per_seq]")
+    if seq_lens.dtype != torch.int32 or tuple(seq_lens.shape) != (B,):
+        raise ValueError("seq_lens must be int32 [B]")
+    for t in (q, k_cache, v_cache, block_table, seq_lens):
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    max_pages = block_table.shape[1]
+    need = attn_decode_workspace_size(B, Hq, max_pages, page_size, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = load_library().attn_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                          _ptr(seq_lens), page_size, B, Hq, Hkv, d, max_pages,
+                                          num_pages, float(scale), _ptr(out), _ptr(lse),
+                                          _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "attn_decode_paged")
+    return out, lse
+
+
+def attn_get_device_error(stream=None):
+    """(status, flags): synchronises the stream, reads and clears the device error word."""
+    flags = ctypes.c_uint(0)
+    st = load_library().attn_get_device_error(_stream(stream), ctypes.byref(flags))
+    return st, int(flags.value)

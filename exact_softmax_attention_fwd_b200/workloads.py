@@ -1,0 +1,196 @@
+"""Seeded synthetic inputs shaped like the notes' workloads.
+
+This module only draws inputs (random numbers, lengths, page placements); it
+holds none of the attention arithmetic.  Both the CUDA path and the CPU
+oracle are fed the very same bf16 bytes produced here.
+
+Recipe (all on the host, ``torch.Generator().manual_seed(seed)``):
+  * Q, K, V: ``randn(float32) * value_scale`` rounded to bf16 (round to nearest
+    even), each tensor from its own seed offset so that shapes can change
+    without reshuffling the others.
+  * Key padding: per sequence, a pad p_b uniform in [0, floor(max_frac * Sk)]
+    keys is masked at the end (k_len = Sk - p_b); at least one p_b > 0.
+  * Paged decode: seq_lens uniform in [lo, hi]; the cache pool holds exactly
+    sum ceil(len/page) pages and a seeded random permutation gives the
+    physical page of each logical page; unused block-table slots are -1.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+# Seeds fixed per workload: config n uses 1000 + n, the padded variant 1100,
+# decode lengths 2000 and the page permutation 2001.
+SEED_PADDING = 1100
+SEED_DECODE_LENS = 2000
+SEED_DECODE_PERM = 2001
+
+
+@dataclass(frozen=True)
+class PrefillConfig:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    S: int
+    d: int
+    causal: bool
+    seed: int
+    value_scale: float = 1.0
+    padded: bool = False  # per-sequence key padding of 0-25% of Sk
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def flops(self) -> float:
+        """4*B*Hq*Sq*Sk*d, halved when causal (the notes' cost model)."""
+        f = 4.0 * self.B * self.Hq * self.S * self.S * self.d
+        return f / 2 if self.causal else f
+
+
+@dataclass(frozen=True)
+class DecodeConfig:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    page_size: int
+    len_lo: int
+    len_hi: int
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def max_pages_per_seq(self) -> int:
+        return -(-self.len_hi // self.page_size)
+
+
+CONFIGS = {
+    "tiny_mha": PrefillConfig("tiny_mha", B=1, Hq=2, Hkv=2, S=256, d=64, causal=False, seed=1001),
+    "mha_causal_2k": PrefillConfig("mha_causal_2k", B=4, Hq=16, Hkv=16, S=2048, d=128,
+                                   causal=True, seed=1002),
+    "gqa_causal_8k": PrefillConfig("gqa_causal_8k", B=2, Hq=32, Hkv=8, S=8192, d=128,
+                                   causal=True, seed=1003),
+    "gqa_causal_8k_padded": PrefillConfig("gqa_causal_8k_padded", B=2, Hq=32, Hkv=8, S=8192,
+                                          d=128, causal=True, seed=1003, padded=True),
+    "gqa_causal_32k": PrefillConfig("gqa_causal_32k", B=1, Hq=32, Hkv=8, S=32768, d=128,
+                                    causal=True, seed=1004, value_scale=0.5),
+    "paged_decode": DecodeConfig("paged_decode", B=64, Hq=32, Hkv=8, d=128, page_size=16,
+                                 len_lo=512, len_hi=8192, seed=1005),
+}
+
+
+def _gen(seed: int) -> torch.Generator:
+    g = torch.Generator()
+    g.manual_seed(int(seed))
+    return g
+
+
+def randn_bf16(shape, seed: int, value_scale: float = 1.0) -> torch.Tensor:
+    """i.i.d. N(0,1) * value_scale drawn in float32 on the host, rounded to bf16."""
+    x = torch.randn(*shape, generator=_gen(seed), dtype=torch.float32)
+    if value_scale != 1.0:
+        x.mul_(value_scale)
+    return x.to(torch.bfloat16)
+
+
+def prefill_inputs(B, Hq, Hkv, Sq, Sk, d, seed, value_scale=1.0):
+    """Q [B,Hq,Sq,d], K and V [B,Hkv,Sk,d] bf16 on the host."""
+    q = randn_bf16((B, Hq, Sq, d), seed * 16 + 0, value_scale)
+    k = randn_bf16((B, Hkv, Sk, d), seed * 16 + 1, value_scale)
+    v = randn_bf16((B, Hkv, Sk, d), seed * 16 + 2, value_scale)
+    return q, k, v
+
+
+def key_padding(B: int, Sk: int, seed: int = SEED_PADDING, max_frac: float = 0.25) -> torch.Tensor:
+    """k_lens [B] int32: Sk minus a pad uniform in [0, floor(max_frac*Sk)]; one pad > 0."""
+    hi = int(math.floor(max_frac * Sk))
+    g = _gen(seed)
+    pads = torch.randint(0, hi + 1, (B,), generator=g, dtype=torch.int64)
+    if hi > 0 and int(pads.max()) == 0:
+        pads[0] = hi
+    return (Sk - pads).to(torch.int32)
+
+
+def config_inputs(cfg: PrefillConfig):
+    """(q, k, v, k_lens or None) for a named prefill configuration."""
+    q, k, v = prefill_inputs(cfg.B, cfg.Hq, cfg.Hkv, cfg.S, cfg.S, cfg.d, cfg.seed,
+                             cfg.value_scale)
+    k_lens = key_padding(cfg.B, cfg.S) if cfg.padded else None
+    return q, k, v, k_lens
+
+
+@dataclass
+class PagedInputs:
+    q: torch.Tensor            # [B, Hq, d] bf16
+    k_cache: torch.Tensor      # [num_pages, page_size, Hkv, d] bf16
+    v_cache: torch.Tensor      # [num_pages, page_size, Hkv, d] bf16
+    block_table: torch.Tensor  # [B, max_pages_per_seq] int32, -1 = unused
+    seq_lens: torch.Tensor     # [B] int32
+    page_size: int
+    extra: dict = field(default_factory=dict)
+
+    @property
+    def num_pages(self) -> int:
+        return int(self.k_cache.shape[0])
+
+
+def decode_lengths(B: int, lo: int, hi: int, seed: int = SEED_DECODE_LENS) -> torch.Tensor:
+    return torch.randint(lo, hi + 1, (B,), generator=_gen(seed), dtype=torch.int64).to(torch.int32)
+
+
+def paged_inputs(seq_lens, Hq, Hkv, d, page_size, seed, max_pages_per_seq=None,
+                 perm_seed: int = SEED_DECODE_PERM, contiguous: bool = False,
+                 extra_pages: int = 0) -> PagedInputs:
+    """Paged cache holding exactly the pages the sequences need (+ extra_pages unused).
+
+    Physical page ids come from a seeded random permutation of the pool unless
+    ``contiguous`` (logical page i of sequence b then sits right after the
+    previous sequence's pages).
+    """
+    lens = torch.as_tensor(seq_lens, dtype=torch.int32).clone()
+    B = lens.shape[0]
+    pages_per = [(-(-int(n) // page_size)) for n in lens.tolist()]
+    need = sum(pages_per)
+    maxp = max_pages_per_seq if max_pages_per_seq is not None else max(pages_per + [1])
+    num_pages = need + extra_pages
+    if contiguous:
+        phys = torch.arange(num_pages, dtype=torch.int64)
+    else:
+        phys = torch.randperm(num_pages, generator=_gen(perm_seed))
+    table = torch.full((B, maxp), -1, dtype=torch.int32)
+    pos = 0
+    for b, n in enumerate(pages_per):
+        if n > maxp:
+            raise ValueError("sequence needs more pages than max_pages_per_seq")
+        table[b, :n] = phys[pos:pos + n].to(torch.int32)
+        pos += n
+    q = randn_bf16((B, Hq, d), seed * 16 + 3)
+    k_cache = randn_bf16((max(num_pages, 1), page_size, Hkv, d), seed * 16 + 4)
+    v_cache = randn_bf16((max(num_pages, 1), page_size, Hkv, d), seed * 16 + 5)
+    return PagedInputs(q, k_cache, v_cache, table, lens, page_size)
+
+
+def decode_config_inputs(cfg: DecodeConfig) -> PagedInputs:
+    lens = decode_lengths(cfg.B, cfg.len_lo, cfg.len_hi)
+    return paged_inputs(lens, cfg.Hq, cfg.Hkv, cfg.d, cfg.page_size, cfg.seed,
+                        max_pages_per_seq=cfg.max_pages_per_seq)
+
+
+def decode_kv_bytes(seq_lens, Hkv: int, d: int, elem_bytes: int = 2) -> int:
+    """K+V bytes of the attended tokens: sum(len) * Hkv * d * 2 (K and V)."""
+    return int(torch.as_tensor(seq_lens, dtype=torch.int64).sum()) * Hkv * d * elem_bytes * 2
+
+
+def sample_rows(B, Hq, Sq, n, seed) -> torch.Tensor:
+    """n distinct seeded flat row ids (b*Hq + hq)*Sq + i."""
+    total = B * Hq * Sq
+    n = min(n, total)
+    return torch.randperm(total, generator=_gen(seed))[:n].sort().values

@@ -1,0 +1,160 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) exact softmax attention library
+ * (libattn_b200.so).
+ *
+ * What is computed ("Attention Kernel", section "问题与成本"):
+ *     P = softmax(Q K^T * scale + M),   O = P V
+ * with Q [B, Hq, Sq, d] and K, V [B, Hkv, Sk, d].  Several query heads share
+ * one KV head (GQA); query head hq reads KV head hq / (Hq / Hkv).  The result
+ * is exact: the score matrix is consumed block by block with the online
+ * softmax (m, l, o) recurrence ("Attention Kernel", section "Online softmax")
+ * and never written to memory; "exact" means the same mathematics within
+ * floating-point rounding, not bitwise equality with another kernel.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are dense and contiguous (row-major in the order given).  q, k,
+ *     v, o, k_cache and v_cache hold bfloat16; lse holds float32; index
+ *     arrays hold int32.  Accumulation is float32.
+ *   - Every pointer argument except `workspace` sizes is a DEVICE pointer on
+ *     the current CUDA device.  The caller owns all memory; the library
+ *     allocates nothing per call and never synchronises the stream in a
+ *     launch.  Work is enqueued on `stream` and runs asynchronously.
+ *   - Tensor pointers must be 16-byte aligned (a TMA requirement).
+ *   - Masking: the additive mask M holds only 0 and -inf.  A key j is visible
+ *     to query row i of sequence b iff j < k_len[b] and, when causal,
+ *     j <= i + (k_len[b] - Sq) (causal diagonal aligned to the bottom right,
+ *     so Sq = 1 sees every key and a square problem gets the usual j <= i).
+ *   - A row with no visible key gets O = 0 and LSE = -inf (never NaN), as
+ *     the "Online softmax" section of "Attention Kernel" requires.
+ *   - LSE[b, h, i] = ln sum_j exp(scale * q_i . k_j) over the visible keys
+ *     (natural log), the statistic a backward pass recomputes P from.
+ *   - Return value: ATTN_OK, or an attn_status describing why nothing was
+ *     launched (arguments are checked on the host before any CUDA call) or
+ *     why the launch failed.  Faults found on the device (a block-table entry
+ *     outside the page pool, a timed-out internal wait) set a device error
+ *     word instead; read it with attn_get_device_error().
+ */
+#ifndef ATTN_B200_ATTN_H_
+#define ATTN_B200_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same underlying type as cudaStream_t / CUstream; NULL is the legacy default stream. */
+typedef struct CUstream_st* attn_stream_t;
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1, /* null pointer, bad extent, Hq % Hkv != 0, non-finite scale */
+  ATTN_ERR_UNSUPPORTED = 2, /* head dim, page size or group size outside what is built */
+  ATTN_ERR_ALIGNMENT = 3,   /* a tensor pointer is not 16-byte aligned */
+  ATTN_ERR_WORKSPACE = 4,   /* decode workspace missing or too small */
+  ATTN_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed (no device, launch error) */
+  ATTN_ERR_DEVICE = 6       /* attn_get_device_error(): the device error word was set */
+} attn_status;
+
+/* Bits of the device error word (attn_get_device_error's flags_out). */
+#define ATTN_DEVERR_WAIT_TIMEOUT 0x1u /* an internal pipeline wait exceeded its time limit */
+#define ATTN_DEVERR_BAD_PAGE 0x2u     /* a block-table entry outside [0, num_pages) was skipped */
+#define ATTN_DEVERR_BAD_LENGTH 0x4u   /* a k_len / seq_len outside its legal range was clamped */
+
+/*
+ * attn_fwd -- prefill / full-sequence attention forward.
+ * Source: "Attention Kernel", sections "问题与成本" (the operation and shapes),
+ * "Online softmax" (the recurrence and the zero-output contract) and
+ * "FlashAttention 的稳定基础" (whole-tile causal skipping, per-element
+ * predicates on boundary tiles, the saved log-sum-exp).
+ *
+ *   q   [B, Hq,  Sq, d] bf16      k, v [B, Hkv, Sk, d] bf16
+ *   o   [B, Hq,  Sq, d] bf16 (written)
+ *   lse [B, Hq,  Sq]    fp32 (written; may be NULL to skip it)
+ *   B, Hq, Hkv >= 1, Hq % Hkv == 0, Sq >= 1, Sk >= 0 (Sk = 0: every row is
+ *   empty), d in {64, 128}; causal in {0, 1}; scale finite (usually 1/sqrt(d)).
+ * Errors: INVALID_ARG, UNSUPPORTED (d), ALIGNMENT, CUDA.  Nothing is written
+ * when an error is returned before the launch.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+             int Hkv, int Sq, int Sk, int d, int causal, float scale, attn_stream_t stream);
+
+/*
+ * attn_fwd_masked -- attn_fwd with per-sequence key padding.
+ * Source: as attn_fwd, plus "Attention Kernel", section "正确性契约" (padding
+ * semantics and fully masked rows are part of the contract).
+ *   k_lens [B] int32 device array, nullable (NULL = Sk for every sequence):
+ *   sequence b sees only keys j < k_lens[b].  Values outside [0, Sk] are
+ *   clamped on the device and flagged with ATTN_DEVERR_BAD_LENGTH.
+ * Other arguments, layout and errors as attn_fwd.
+ */
+int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int Hq, int Hkv, int Sq, int Sk, int d, int causal, float scale,
+                    const int32_t* k_lens, attn_stream_t stream);
+
+/*
+ * attn_decode_workspace_size -- bytes of caller-owned device workspace that
+ * attn_decode_paged needs for the given capacity.
+ * Source: "Attention 算子加速史", section 4.1-4.2 (split-K decode: each split
+ * writes a partial output and its log-sum-exp; a light kernel merges them).
+ * The workspace holds float32 partial outputs [B, Hq, n_split, d] and float32
+ * partial log-sum-exps [B, Hq, n_split], n_split = ceil(max_pages_per_seq *
+ * page_size / split_tokens) with the library's fixed split length.
+ * Returns 0 for invalid arguments.
+ */
+size_t attn_decode_workspace_size(int B, int Hq, int max_pages_per_seq, int page_size, int d);
+
+/*
+ * attn_decode_paged -- single-query (Sq = 1) attention over a paged KV cache.
+ * Source: "Attention Kernel", section "Paged 与 ragged KV" (token t of a
+ * sequence lives in logical block t / page_size at offset t mod page_size;
+ * the block table maps the block to a physical page; the last page is
+ * partial) and "Prefill 与 decode 是两种 kernel"; "Attention 算子加速史",
+ * section 4 (split-KV decode with a log-sum-exp merge).
+ *
+ *   q            [B, Hq, d] bf16
+ *   k_cache      [num_pages, page_size, Hkv, d] bf16
+ *   v_cache      [num_pages, page_size, Hkv, d] bf16
+ *   block_table  [B, max_pages_per_seq] int32: physical page of each logical
+ *                page; entries past the sequence's last page are never read
+ *   seq_lens     [B] int32: tokens in each sequence (0 allowed: O = 0, LSE = -inf)
+ *   o            [B, Hq, d] bf16 (written)
+ *   lse          [B, Hq] fp32 (written; nullable)
+ *   workspace    device scratch of at least attn_decode_workspace_size(...)
+ *                bytes, 16-byte aligned; its contents are overwritten.
+ *   page_size a positive multiple of 16 (<= 256); d in {64, 128};
+ *   Hq / Hkv <= 8.
+ * Device-side faults: a page id outside [0, num_pages) is skipped (its tokens
+ * contribute nothing) and flags ATTN_DEVERR_BAD_PAGE; a seq_len outside
+ * [0, max_pages_per_seq * page_size] is clamped and flags
+ * ATTN_DEVERR_BAD_LENGTH.  The result is deterministic: the splits are merged
+ * in a fixed order with no atomics.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA.
+ */
+int attn_decode_paged(const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_table, const int32_t* seq_lens, int page_size, int B,
+                      int Hq, int Hkv, int d, int max_pages_per_seq, int num_pages, float scale,
+                      void* o, float* lse, void* workspace, size_t workspace_bytes,
+                      attn_stream_t stream);
+
+/*
+ * attn_get_device_error -- synchronise `stream`, read and clear the device
+ * error word of the current device.  Returns ATTN_OK when it was zero,
+ * ATTN_ERR_DEVICE when it was set (flags_out, nullable, receives the
+ * ATTN_DEVERR_* bits), or ATTN_ERR_CUDA if the read itself failed.
+ * The word is per device and shared by all streams and calls.
+ */
+int attn_get_device_error(attn_stream_t stream, unsigned int* flags_out);
+
+/* attn_strerror -- static description of an attn_status value. */
+const char* attn_strerror(int status);
+
+/* attn_split_tokens -- the fixed number of tokens per decode split. */
+int attn_split_tokens(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_ATTN_H_ */

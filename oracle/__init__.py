@@ -1,0 +1,185 @@
+"""CPU oracle for exact softmax attention -- TEST INFRASTRUCTURE ONLY.
+
+A plain double-precision C statement of what the attention path computes
+(``attn_oracle.c``), loaded through ctypes.  Only the tests, the smoke check
+and the benchmark's CPU-baseline / reference legs may import this package; the
+product path (the CUDA library and its Python binding) never does, and the
+two share no code.
+
+Sources followed (page title, section):
+  * "Attention Kernel" -- "问题与成本": O = softmax(QK^T/sqrt(d_h) + M) V with
+    Q [B, A, S_q, d_h] and K, V [B, A_kv, S_k, d_h] (GQA).
+  * "Attention Kernel" -- "Online softmax" and "Blockwise reference": the
+    (m, l, o) merge rule and the zero output for an all -inf row.
+  * "Attention Kernel" -- "Paged 与 ragged KV": block = floor(t/q), offset =
+    t mod q, physical page through the block table.
+
+Every function here is pinned by tests in ``tests/test_oracle_pins.py``
+against things other than itself (the notes' worked example evaluated with
+``torch.softmax``, closed forms, invariances, ``torch`` SDPA in float64 on
+tiny shapes).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+OK = 0
+ERR_ARG = 1
+ERR_TABLE = 2
+
+
+def build(force: bool = False) -> str:
+    """Compile ``attn_oracle.c`` into ``liboracle.so`` next to it (plain gcc)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c99", "-Wall", "-fPIC", "-shared", "-o", tmp, _SRC,
+           "-lm", "-lpthread"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I = ctypes.c_int
+            D = ctypes.c_double
+            L = ctypes.c_int64
+            lib.oracle_softmax_attend.argtypes = [P, I, P, I, I, P, P]
+            lib.oracle_softmax_attend.restype = I
+            lib.oracle_online_attend.argtypes = [P, I, P, I, I, I, P, P, P]
+            lib.oracle_online_attend.restype = I
+            lib.oracle_attn_fwd_rows.argtypes = [P, P, P, I, I, I, I, I, I, I, D, P, P, L,
+                                                 P, P, I]
+            lib.oracle_attn_fwd_rows.restype = I
+            lib.oracle_decode_paged.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, D, P, P, I]
+            lib.oracle_decode_paged.restype = I
+            _lib = lib
+    return _lib
+
+
+def _threads(n_threads):
+    return int(n_threads) if n_threads else (os.cpu_count() or 1)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _bits(x) -> np.ndarray:
+    """bf16 tensor (torch) or uint16 array -> contiguous uint16 numpy bit patterns."""
+    if isinstance(x, np.ndarray):
+        if x.dtype != np.uint16:
+            raise TypeError("expected bf16 bit patterns as uint16")
+        return np.ascontiguousarray(x)
+    import torch
+    if x.dtype != torch.bfloat16:
+        raise TypeError("expected a bfloat16 tensor")
+    return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy()
+                                .view(np.uint16))
+
+
+class OracleError(RuntimeError):
+    def __init__(self, status):
+        super().__init__(f"oracle returned status {status}")
+        self.status = status
+
+
+def softmax_attend(scores, values):
+    """softmax(scores) @ values for one row, plus its natural-log LSE."""
+    s = np.ascontiguousarray(scores, dtype=np.float64)
+    v = np.ascontiguousarray(values, dtype=np.float64)
+    if s.ndim != 1 or v.ndim != 2:
+        raise ValueError("scores must be 1-D and values 2-D")
+    o = np.zeros(v.shape[1], np.float64)
+    lse = np.zeros(1, np.float64)
+    st = _load().oracle_softmax_attend(_ptr(s), s.shape[0], _ptr(v), v.shape[0], v.shape[1],
+                                       _ptr(o), _ptr(lse))
+    if st != OK:
+        raise OracleError(st)
+    return o, float(lse[0])
+
+
+def online_attend(scores, values, block_size, block_order=None):
+    """The same row through the blockwise (m, l, o) recurrence."""
+    s = np.ascontiguousarray(scores, dtype=np.float64)
+    v = np.ascontiguousarray(values, dtype=np.float64)
+    if s.ndim != 1 or v.ndim != 2:
+        raise ValueError("scores must be 1-D and values 2-D")
+    order = None if block_order is None else np.ascontiguousarray(block_order, dtype=np.int32)
+    o = np.zeros(v.shape[1], np.float64)
+    lse = np.zeros(1, np.float64)
+    st = _load().oracle_online_attend(_ptr(s), s.shape[0], _ptr(v), v.shape[0], v.shape[1],
+                                      int(block_size), _ptr(order), _ptr(o), _ptr(lse))
+    if st != OK:
+        raise OracleError(st)
+    return o, float(lse[0])
+
+
+def attn_fwd(q, k, v, causal, scale, k_lens=None, rows=None, n_threads=None):
+    """Exact attention.  q [B,Hq,Sq,d], k/v [B,Hkv,Sk,d] bf16 (torch or uint16 bits).
+
+    ``rows``: optional flat row ids (b*Hq + hq)*Sq + i; default every row.
+    Returns (o, lse) as float64 arrays: o [n_rows, d] (or [B,Hq,Sq,d] when
+    ``rows`` is None) and lse [n_rows] (or [B,Hq,Sq]).
+    """
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, Hq, Sq, d = qb.shape
+    Bk, Hkv, Sk, dk = kb.shape
+    if kb.shape != vb.shape or Bk != B or dk != d:
+        raise ValueError("q/k/v shapes disagree")
+    kl = None if k_lens is None else np.ascontiguousarray(np.asarray(k_lens), dtype=np.int32)
+    r = None if rows is None else np.ascontiguousarray(np.asarray(rows), dtype=np.int64)
+    n = B * Hq * Sq if r is None else r.shape[0]
+    o = np.zeros((n, d), np.float64)
+    lse = np.zeros(n, np.float64)
+    st = _load().oracle_attn_fwd_rows(_ptr(qb), _ptr(kb), _ptr(vb), B, Hq, Hkv, Sq, Sk, d,
+                                      int(bool(causal)), float(scale), _ptr(kl), _ptr(r), n,
+                                      _ptr(o), _ptr(lse), _threads(n_threads))
+    if st != OK:
+        raise OracleError(st)
+    if r is None:
+        return o.reshape(B, Hq, Sq, d), lse.reshape(B, Hq, Sq)
+    return o, lse
+
+
+def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale, n_threads=None):
+    """Exact single-query attention over a paged cache.
+
+    q [B,Hq,d]; k_cache/v_cache [num_pages, page_size, Hkv, d] bf16;
+    block_table [B, max_pages] int32; seq_lens [B] int32.
+    Returns (o [B,Hq,d], lse [B,Hq]) float64.
+    """
+    qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
+    B, Hq, d = qb.shape
+    num_pages, page_size, Hkv, dk = kb.shape
+    if kb.shape != vb.shape or dk != d:
+        raise ValueError("cache shapes disagree")
+    tbl = np.ascontiguousarray(np.asarray(block_table), dtype=np.int32)
+    lens = np.ascontiguousarray(np.asarray(seq_lens), dtype=np.int32)
+    if tbl.ndim != 2 or tbl.shape[0] != B or lens.shape != (B,):
+        raise ValueError("block table / seq_lens shapes disagree")
+    o = np.zeros((B, Hq, d), np.float64)
+    lse = np.zeros((B, Hq), np.float64)
+    st = _load().oracle_decode_paged(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(tbl), _ptr(lens), B, Hq,
+                                     Hkv, d, page_size, tbl.shape[1], num_pages, float(scale),
+                                     _ptr(o), _ptr(lse), _threads(n_threads))
+    if st != OK:
+        raise OracleError(st)
+    return o, lse

@@ -1,0 +1,365 @@
+"""Pins for the CPU oracle: each checks it against something other than itself.
+
+* The worked example of "Attention Kernel", section "Blockwise reference":
+  the page states the blockwise result must equal softmax(score) @ value
+  (evaluated here with torch.softmax, a library routine), that an all -inf row
+  returns zeros, and that mismatched score/value rows are rejected.
+* Invariance of the (m, l, o) recurrence to block size and order ("Online
+  softmax": any block order gives the exact merge).
+* torch's scaled_dot_product_attention in float64 on tiny shapes (a library
+  routine), plus a long-double evaluation written differently
+  (exp(s - logsumexp)).
+* Closed forms: constant V, uniform weights, causal row 0, scale 0.
+* GQA == MHA with K/V repeated; key permutation invariance; paged == gathered
+  contiguous ("Attention Kernel", section "验证": a contiguous cache and a
+  random block table must agree).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_softmax_attention_fwd_b200 import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_example.json")
+NEG_INF = float("-inf")
+
+
+def _golden():
+    with open(GOLDEN) as f:
+        g = json.load(f)
+    score = [NEG_INF if s == "-inf" else float(s) for s in g["score"]]
+    value = np.array(g["value"], dtype=np.float64).reshape(g["value_shape"])
+    return g, score, value
+
+
+# --------------------------------------------------------------------------- worked example
+
+
+def test_worked_example_matches_torch_softmax():
+    g, score, value = _golden()
+    expected = (torch.softmax(torch.tensor(score, dtype=torch.float64), dim=0)
+                @ torch.tensor(value)).numpy()
+    o, lse = oracle.softmax_attend(score, value)
+    np.testing.assert_allclose(o, expected, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(g["expected_o"], expected, rtol=0, atol=1e-12)
+    lse_ref = torch.logsumexp(torch.tensor(score, dtype=torch.float64), dim=0).item()
+    assert abs(lse - lse_ref) < 1e-12
+    assert abs(g["expected_lse"] - lse_ref) < 1e-12
+
+
+def test_worked_example_blockwise_block2():
+    g, score, value = _golden()
+    o, lse = oracle.online_attend(score, value, g["block_size"])
+    np.testing.assert_allclose(o, g["expected_o"], rtol=0, atol=1e-12)
+    assert abs(lse - g["expected_lse"]) < 1e-12
+
+
+def test_all_masked_row_is_zero_not_nan():
+    _, _, value = _golden()
+    row = [NEG_INF] * 5
+    for o, lse in (oracle.softmax_attend(row, value), oracle.online_attend(row, value, 2)):
+        assert np.array_equal(o, np.zeros(3))
+        assert lse == NEG_INF
+
+
+def test_mismatched_rows_rejected():
+    _, score, _ = _golden()
+    for fn in (lambda: oracle.softmax_attend(score, np.zeros((6, 3))),
+               lambda: oracle.online_attend(score, np.zeros((6, 3)), 2)):
+        with pytest.raises(oracle.OracleError) as e:
+            fn()
+        assert e.value.status == oracle.ERR_ARG
+    with pytest.raises(oracle.OracleError):
+        oracle.online_attend(score, np.zeros((5, 3)), 0)
+
+
+# --------------------------------------------------------------------------- recurrence invariance
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_online_invariant_to_block_size_and_order(seed):
+    rng = np.random.default_rng(seed)
+    n, dv = 53, 7
+    s = rng.normal(0, 3, n)
+    s[rng.random(n) < 0.2] = NEG_INF
+    s[10:20] = NEG_INF  # a whole block with nothing finite for several sizes
+    v = rng.normal(0, 1, (n, dv))
+    o_ref, lse_ref = oracle.softmax_attend(s, v)
+    for bs in (1, 2, 3, 7, 16, 64, n):
+        nb = -(-n // bs)
+        orders = [None, list(range(nb))[::-1], list(rng.permutation(nb))]
+        for order in orders:
+            o, lse = oracle.online_attend(s, v, bs, order)
+            np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12)
+            assert abs(lse - lse_ref) < 1e-12
+
+
+def test_online_rejects_bad_order():
+    with pytest.raises(oracle.OracleError):
+        oracle.online_attend([0.0, 1.0, 2.0], np.zeros((3, 2)), 1, [0, 0, 1])
+
+
+# --------------------------------------------------------------------------- prefill pins
+
+
+def _visible_mask(Sq, Sk, causal, klen):
+    i = torch.arange(Sq)[:, None]
+    j = torch.arange(Sk)[None, :]
+    vis = (j < klen).expand(Sq, Sk)
+    if causal:
+        vis = vis & (j <= i + (klen - Sq))
+    return vis
+
+
+def _sdpa_reference(q, k, v, causal, scale, k_lens):
+    """torch SDPA (float64, CPU) with an explicit boolean mask; empty rows -> 0/-inf."""
+    B, Hq, Sq, d = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    g = Hq // Hkv
+    qd, kd, vd = q.double(), k.double().repeat_interleave(g, 1), v.double().repeat_interleave(g, 1)
+    o = torch.zeros(B, Hq, Sq, d, dtype=torch.float64)
+    lse = torch.full((B, Hq, Sq), NEG_INF, dtype=torch.float64)
+    for b in range(B):
+        kl = Sk if k_lens is None else int(k_lens[b])
+        vis = _visible_mask(Sq, Sk, causal, kl)
+        nonempty = vis.any(-1)
+        if Sk > 0 and nonempty.any():
+            ob = torch.nn.functional.scaled_dot_product_attention(
+                qd[b], kd[b], vd[b], attn_mask=vis, scale=scale)
+            o[b][:, nonempty] = ob[:, nonempty]
+            s = (qd[b] @ kd[b].transpose(-1, -2)) * scale
+            s = s.masked_fill(~vis, NEG_INF)
+            lse[b][:, nonempty] = torch.logsumexp(s, -1)[:, nonempty]
+    return o.numpy(), lse.numpy()
+
+
+def _longdouble_reference(q, k, v, causal, scale, k_lens):
+    """A differently written evaluation: weights exp(s - logsumexp(s)) in long double."""
+    B, Hq, Sq, d = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    g = Hq // Hkv
+    qn = q.double().numpy().astype(np.longdouble)
+    kn = k.double().numpy().astype(np.longdouble)
+    vn = v.double().numpy().astype(np.longdouble)
+    o = np.zeros((B, Hq, Sq, d), np.longdouble)
+    for b in range(B):
+        kl = Sk if k_lens is None else int(k_lens[b])
+        vis = _visible_mask(Sq, Sk, causal, kl).numpy()
+        for h in range(Hq):
+            for i in range(Sq):
+                js = np.nonzero(vis[i])[0]
+                if js.size == 0:
+                    continue
+                s = np.array([np.sum(qn[b, h, i] * kn[b, h // g, j]) * scale for j in js],
+                             dtype=np.longdouble)
+                mx = s.max()
+                lse = mx + np.log(np.sum(np.exp(s - mx)))
+                w = np.exp(s - lse)
+                o[b, h, i] = (w[:, None] * vn[b, h // g, js]).sum(0)
+    return o.astype(np.float64)
+
+
+TINY_CASES = [
+    # B, Hq, Hkv, Sq, Sk, d, causal, padded
+    (1, 1, 1, 1, 1, 1, False, False),
+    (1, 2, 1, 5, 7, 3, False, False),
+    (2, 4, 2, 6, 6, 4, True, False),
+    (2, 4, 1, 7, 7, 2, True, True),
+    (1, 3, 3, 4, 9, 4, True, False),   # Sq < Sk, bottom-right causal
+    (2, 2, 2, 8, 5, 3, True, True),    # Sq > Sk: leading rows fully masked
+    (1, 2, 2, 3, 0, 4, False, False),  # Sk = 0: every row empty
+]
+
+
+@pytest.mark.parametrize("case", TINY_CASES)
+def test_prefill_matches_torch_sdpa_tiny(case):
+    B, Hq, Hkv, Sq, Sk, d, causal, padded = case
+    q, k, v = workloads.prefill_inputs(B, Hq, Hkv, Sq, Sk, d, seed=7 + Sq + Sk)
+    k_lens = None
+    if padded:
+        k_lens = torch.tensor([max(0, Sk - 1 - b) for b in range(B)], dtype=torch.int32)
+    scale = 0.37
+    o, lse = oracle.attn_fwd(q, k, v, causal, scale, k_lens=k_lens)
+    o_ref, lse_ref = _sdpa_reference(q, k, v, causal, scale, k_lens)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12)
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isfinite(lse), fin)
+    np.testing.assert_allclose(lse[fin], lse_ref[fin], rtol=0, atol=1e-12)
+    assert np.all(o[~fin] == 0.0)
+    o_ld = _longdouble_reference(q, k, v, causal, scale, k_lens)
+    np.testing.assert_allclose(o, o_ld, rtol=0, atol=1e-12)
+
+
+def test_prefill_square_causal_matches_sdpa_is_causal():
+    q, k, v = workloads.prefill_inputs(2, 2, 2, 9, 9, 4, seed=11)
+    o, _ = oracle.attn_fwd(q, k, v, True, 0.5)
+    ref = torch.nn.functional.scaled_dot_product_attention(q.double(), k.double(), v.double(),
+                                                           is_causal=True, scale=0.5)
+    np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_prefill_constant_values():
+    q, k, _ = workloads.prefill_inputs(1, 2, 2, 6, 6, 8, seed=3)
+    v = torch.full((1, 2, 6, 8), 1.75, dtype=torch.bfloat16)
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd(q, k, v, causal, 0.3)
+        np.testing.assert_allclose(o, 1.75, rtol=0, atol=1e-12)
+        assert np.all(np.isfinite(lse))
+
+
+def test_prefill_uniform_weights_closed_form():
+    # q = 0 makes every visible score 0: O is the mean of the visible V rows and
+    # LSE = ln(number of visible keys).
+    _, k, v = workloads.prefill_inputs(1, 1, 1, 5, 5, 4, seed=5)
+    q = torch.zeros(1, 1, 5, 4, dtype=torch.bfloat16)
+    o, lse = oracle.attn_fwd(q, k, v, True, 1.0)
+    vd = v.double().numpy()[0, 0]
+    for i in range(5):
+        np.testing.assert_allclose(o[0, 0, i], vd[: i + 1].mean(0), rtol=0, atol=1e-12)
+        assert abs(lse[0, 0, i] - math.log(i + 1)) < 1e-12
+    # scale = 0 does the same for any q
+    q2, _, _ = workloads.prefill_inputs(1, 1, 1, 5, 5, 4, seed=6)
+    o2, lse2 = oracle.attn_fwd(q2, k, v, False, 0.0)
+    np.testing.assert_allclose(o2[0, 0], np.broadcast_to(vd.mean(0), (5, 4)), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse2, math.log(5), rtol=0, atol=1e-12)
+
+
+def test_prefill_causal_row0_sees_only_key0():
+    q, k, v = workloads.prefill_inputs(1, 2, 2, 4, 4, 8, seed=9)
+    o, lse = oracle.attn_fwd(q, k, v, True, 0.25)
+    for h in range(2):
+        np.testing.assert_allclose(o[0, h, 0], v.double().numpy()[0, h, 0], rtol=0, atol=1e-12)
+        s00 = 0.25 * float((q.double()[0, h, 0] * k.double()[0, h, 0]).sum())
+        assert abs(lse[0, h, 0] - s00) < 1e-12
+
+
+def test_prefill_gqa_equals_repeated_mha():
+    q, k, v = workloads.prefill_inputs(2, 8, 2, 6, 10, 4, seed=21)
+    o, lse = oracle.attn_fwd(q, k, v, True, 0.5)
+    o2, lse2 = oracle.attn_fwd(q, k.repeat_interleave(4, 1), v.repeat_interleave(4, 1), True, 0.5)
+    np.testing.assert_allclose(o, o2, rtol=0, atol=0)
+    np.testing.assert_allclose(lse, lse2, rtol=0, atol=0)
+
+
+def test_prefill_noncausal_key_permutation_invariance():
+    q, k, v = workloads.prefill_inputs(1, 2, 1, 4, 12, 4, seed=31)
+    perm = torch.randperm(12, generator=torch.Generator().manual_seed(0))
+    o, lse = oracle.attn_fwd(q, k, v, False, 0.5)
+    o2, lse2 = oracle.attn_fwd(q, k[:, :, perm].contiguous(), v[:, :, perm].contiguous(), False, 0.5)
+    np.testing.assert_allclose(o, o2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse2, rtol=0, atol=1e-12)
+
+
+def test_prefill_padding_equals_truncation_noncausal():
+    q, k, v = workloads.prefill_inputs(2, 2, 2, 5, 11, 4, seed=41)
+    k_lens = torch.tensor([7, 11], dtype=torch.int32)
+    o, lse = oracle.attn_fwd(q, k, v, False, 0.5, k_lens=k_lens)
+    for b, kl in enumerate(k_lens.tolist()):
+        ob, lb = oracle.attn_fwd(q[b:b + 1], k[b:b + 1, :, :kl].contiguous(),
+                                 v[b:b + 1, :, :kl].contiguous(), False, 0.5)
+        np.testing.assert_allclose(o[b], ob[0], rtol=0, atol=0)
+        np.testing.assert_allclose(lse[b], lb[0], rtol=0, atol=0)
+
+
+def test_prefill_bottom_right_padding_masks_leading_rows():
+    q, k, v = workloads.prefill_inputs(1, 1, 1, 8, 8, 4, seed=43)
+    o, lse = oracle.attn_fwd(q, k, v, True, 0.5, k_lens=torch.tensor([5], dtype=torch.int32))
+    # rows i < Sq - k_len = 3 have no visible key
+    assert np.all(o[0, 0, :3] == 0) and np.all(lse[0, 0, :3] == NEG_INF)
+    assert np.all(np.isfinite(lse[0, 0, 3:]))
+    # the last row sees exactly keys 0..4
+    ob, _ = oracle.attn_fwd(q[:, :, 7:8].contiguous(), k[:, :, :5].contiguous(),
+                            v[:, :, :5].contiguous(), False, 0.5)
+    np.testing.assert_allclose(o[0, 0, 7], ob[0, 0, 0], rtol=0, atol=0)
+
+
+def test_prefill_row_subset_matches_full():
+    q, k, v = workloads.prefill_inputs(2, 4, 2, 7, 9, 4, seed=51)
+    o, lse = oracle.attn_fwd(q, k, v, True, 0.5)
+    rows = workloads.sample_rows(2, 4, 7, 13, seed=1)
+    o_s, lse_s = oracle.attn_fwd(q, k, v, True, 0.5, rows=rows, n_threads=3)
+    np.testing.assert_array_equal(o_s, o.reshape(-1, 4)[rows.numpy()])
+    np.testing.assert_array_equal(lse_s, lse.reshape(-1)[rows.numpy()])
+
+
+def test_prefill_rejects_bad_args():
+    q, k, v = workloads.prefill_inputs(1, 3, 2, 2, 2, 4, seed=1)
+    with pytest.raises(oracle.OracleError):
+        oracle.attn_fwd(q, k, v, False, 1.0)  # Hq % Hkv != 0
+
+
+# --------------------------------------------------------------------------- paged decode pins
+
+
+def _gather_contiguous(inp, b, Hkv, d):
+    n = int(inp.seq_lens[b])
+    ks, vs = [], []
+    for t in range(n):
+        page = int(inp.block_table[b, t // inp.page_size])
+        ks.append(inp.k_cache[page, t % inp.page_size])
+        vs.append(inp.v_cache[page, t % inp.page_size])
+    if n == 0:
+        return (torch.zeros(1, Hkv, 0, d, dtype=torch.bfloat16),) * 2
+    return (torch.stack(ks, 1).unsqueeze(0).contiguous(),   # [1, Hkv, n, d]
+            torch.stack(vs, 1).unsqueeze(0).contiguous())
+
+
+def test_decode_paged_matches_prefill_on_gathered_kv():
+    lens = torch.tensor([1, 16, 17, 40, 0, 33], dtype=torch.int32)
+    Hq, Hkv, d = 8, 2, 4
+    inp = workloads.paged_inputs(lens, Hq, Hkv, d, page_size=16, seed=61, extra_pages=3)
+    o, lse = oracle.decode_paged(inp.q, inp.k_cache, inp.v_cache, inp.block_table, inp.seq_lens, 0.5)
+    for b in range(len(lens)):
+        kb, vb = _gather_contiguous(inp, b, Hkv, d)
+        if int(lens[b]) == 0:
+            assert np.all(o[b] == 0) and np.all(lse[b] == NEG_INF)
+            continue
+        ob, lb = oracle.attn_fwd(inp.q[b].reshape(1, Hq, 1, d).contiguous(), kb, vb, False, 0.5)
+        np.testing.assert_allclose(o[b], ob[0, :, 0], rtol=0, atol=0)
+        np.testing.assert_allclose(lse[b], lb[0, :, 0], rtol=0, atol=0)
+        # and against the library routine
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            inp.q[b].double().reshape(1, Hq, 1, d),
+            kb.double().repeat_interleave(Hq // Hkv, 1), vb.double().repeat_interleave(Hq // Hkv, 1),
+            scale=0.5)
+        np.testing.assert_allclose(o[b], ref[0, :, 0].numpy(), rtol=0, atol=1e-12)
+
+
+def test_decode_contiguous_vs_permuted_pages():
+    lens = torch.tensor([5, 31, 64], dtype=torch.int32)
+    a = workloads.paged_inputs(lens, 4, 2, 8, 16, seed=71, contiguous=True)
+    b = workloads.paged_inputs(lens, 4, 2, 8, 16, seed=71, contiguous=False)
+    # same logical cache content: move b's pages into a's physical order
+    kc = torch.empty_like(a.k_cache)
+    vc = torch.empty_like(a.v_cache)
+    for s in range(3):
+        for p in range(-(-int(lens[s]) // 16)):
+            kc[int(b.block_table[s, p])] = a.k_cache[int(a.block_table[s, p])]
+            vc[int(b.block_table[s, p])] = a.v_cache[int(a.block_table[s, p])]
+    oa, la = oracle.decode_paged(a.q, a.k_cache, a.v_cache, a.block_table, lens, 0.3)
+    ob, lb = oracle.decode_paged(a.q, kc, vc, b.block_table, lens, 0.3)
+    np.testing.assert_array_equal(oa, ob)
+    np.testing.assert_array_equal(la, lb)
+
+
+def test_decode_single_token_returns_v0():
+    inp = workloads.paged_inputs(torch.tensor([1], dtype=torch.int32), 4, 2, 8, 16, seed=81)
+    o, lse = oracle.decode_paged(inp.q, inp.k_cache, inp.v_cache, inp.block_table, inp.seq_lens, 0.5)
+    page = int(inp.block_table[0, 0])
+    for h in range(4):
+        np.testing.assert_allclose(o[0, h], inp.v_cache[page, 0, h // 2].double().numpy(),
+                                   rtol=0, atol=0)
+
+
+def test_decode_bad_page_id_reported():
+    inp = workloads.paged_inputs(torch.tensor([20], dtype=torch.int32), 2, 1, 4, 16, seed=91)
+    tbl = inp.block_table.clone()
+    tbl[0, 1] = inp.num_pages + 5
+    with pytest.raises(oracle.OracleError) as e:
+        oracle.decode_paged(inp.q, inp.k_cache, inp.v_cache, tbl, inp.seq_lens, 0.5)
+    assert e.value.status == oracle.ERR_TABLE
