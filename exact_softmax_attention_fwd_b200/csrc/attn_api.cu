@@ -1,0 +1,244 @@
+// attn_api.cu -- the C ABI declared in include/attn.h: argument checks on the
+// host (before any CUDA call), TMA descriptor construction, and the launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "attn.h"
+#include "decode_sm100.cuh"
+#include "prefill_sm100.cuh"
+#include "sm100_primitives.cuh"
+
+namespace attn_b200 {
+namespace {
+
+// Rows with no visible key at all (Sk = 0): O = 0, LSE = -inf.
+__global__ void fill_empty_rows_kernel(uint4* o, size_t n_vec16, float* lse, size_t n_rows) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t e = i; e < n_vec16; e += stride) o[e] = make_uint4(0u, 0u, 0u, 0u);
+  if (lse != nullptr)
+    for (size_t e = i; e < n_rows; e += stride) lse[e] = -INFINITY;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 map over a contiguous [planes, rows, D] tensor, box = 128 rows x 64
+// columns, 128-byte swizzle (the layout the tcgen05 descriptors expect).
+bool make_tile_map(CUtensorMap* map, const void* ptr, int D, long long rows, long long planes) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+template <int D, bool CAUSAL>
+int launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                   const CUtensorMap& mo, const PrefillParams& prm, cudaStream_t stream) {
+  using C = PrefillCfg<D>;
+  auto kern = attn_prefill_sm100_kernel<D, CAUSAL>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+      cudaSuccess)
+    return ATTN_ERR_CUDA;
+  dim3 grid(prm.n_qblocks, prm.Hq, prm.B);
+  kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, prm);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int check_prefill_args(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int Hq, int Hkv, int Sq, int Sk, int d, int causal, float scale,
+                       const int32_t* k_lens) {
+  if (q == nullptr || o == nullptr || (Sk > 0 && (k == nullptr || v == nullptr)))
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Sk < 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (B > 65535 || Hq > 65535) return ATTN_ERR_INVALID_ARG;  // grid extents
+  if (Sq > (1 << 30) || Sk > (1 << 30)) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(o) || (Sk > 0 && (!aligned16(k) || !aligned16(v))))
+    return ATTN_ERR_ALIGNMENT;
+  if ((lse != nullptr && !aligned4(lse)) || (k_lens != nullptr && !aligned4(k_lens)))
+    return ATTN_ERR_ALIGNMENT;
+  return ATTN_OK;
+}
+
+}  // namespace
+}  // namespace attn_b200
+
+using namespace attn_b200;
+
+extern "C" {
+
+const char* attn_strerror(int status) {
+  switch (status) {
+    case ATTN_OK: return "success";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration (head dim, page size or group size)";
+    case ATTN_ERR_ALIGNMENT: return "tensor pointer not 16-byte aligned";
+    case ATTN_ERR_WORKSPACE: return "decode workspace missing or too small";
+    case ATTN_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case ATTN_ERR_DEVICE: return "device error word set (bad page id, bad length or wait timeout)";
+    default: return "unknown status";
+  }
+}
+
+int attn_split_tokens(void) { return kSplitTokens; }
+
+int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int Hq, int Hkv, int Sq, int Sk, int d, int causal, float scale,
+                    const int32_t* k_lens, attn_stream_t stream_) {
+  const int st = check_prefill_args(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens);
+  if (st != ATTN_OK) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const long long rows_q = (long long)B * Hq * Sq;
+  if (Sk == 0) {
+    const size_t n_vec = (size_t)rows_q * d * 2 / 16;
+    const int threads = 256;
+    const long long want = ((long long)n_vec + threads - 1) / threads;
+    const int blocks = (int)(want < 4096 ? (want > 0 ? want : 1) : 4096);
+    fill_empty_rows_kernel<<<blocks, threads, 0, stream>>>(reinterpret_cast<uint4*>(o), n_vec, lse,
+                                                           (size_t)rows_q);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_tile_map(&mq, q, d, Sq, (long long)B * Hq) ||
+      !make_tile_map(&mk, k, d, Sk, (long long)B * Hkv) ||
+      !make_tile_map(&mv, v, d, Sk, (long long)B * Hkv) ||
+      !make_tile_map(&mo, o, d, Sq, (long long)B * Hq))
+    return ATTN_ERR_CUDA;
+  PrefillParams prm;
+  prm.lse = lse;
+  prm.k_lens = k_lens;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.Sq = Sq;
+  prm.Sk = Sk;
+  prm.group = Hq / Hkv;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.n_qblocks = (Sq + 255) / 256;
+  if (d == 128)
+    return causal ? launch_prefill<128, true>(mq, mk, mv, mo, prm, stream)
+                  : launch_prefill<128, false>(mq, mk, mv, mo, prm, stream);
+  return causal ? launch_prefill<64, true>(mq, mk, mv, mo, prm, stream)
+                : launch_prefill<64, false>(mq, mk, mv, mo, prm, stream);
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+             int Hkv, int Sq, int Sk, int d, int causal, float scale, attn_stream_t stream) {
+  return attn_fwd_masked(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, causal, scale, nullptr, stream);
+}
+
+size_t attn_decode_workspace_size(int B, int Hq, int max_pages_per_seq, int page_size, int d) {
+  if (B < 1 || Hq < 1 || max_pages_per_seq < 1 || page_size < 1 || d < 1) return 0;
+  const long long tokens = (long long)max_pages_per_seq * page_size;
+  const long long n_split = (tokens + kSplitTokens - 1) / kSplitTokens;
+  const long long parts = (long long)B * Hq * n_split;
+  const size_t o_bytes = (size_t)parts * d * sizeof(float);
+  const size_t lse_bytes = (size_t)parts * sizeof(float);
+  return o_bytes + ((lse_bytes + 255) / 256) * 256;
+}
+
+int attn_decode_paged(const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_table, const int32_t* seq_lens, int page_size, int B,
+                      int Hq, int Hkv, int d, int max_pages_per_seq, int num_pages, float scale,
+                      void* o, float* lse, void* workspace, size_t workspace_bytes,
+                      attn_stream_t stream_) {
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr ||
+      seq_lens == nullptr || o == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || max_pages_per_seq < 1 || num_pages < 1 ||
+      page_size < 1)
+    return ATTN_ERR_INVALID_ARG;
+  if (B > 65535 || Hkv > 65535 || (long long)max_pages_per_seq * page_size > (1ll << 30))
+    return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (page_size % 16 != 0 || page_size > 256) return ATTN_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 8) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      !aligned4(block_table) || !aligned4(seq_lens) || (lse != nullptr && !aligned4(lse)))
+    return ATTN_ERR_ALIGNMENT;
+  const size_t need = attn_decode_workspace_size(B, Hq, max_pages_per_seq, page_size, d);
+  if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
+
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const long long tokens = (long long)max_pages_per_seq * page_size;
+  DecodeParams prm;
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.k_cache = static_cast<const uint16_t*>(k_cache);
+  prm.v_cache = static_cast<const uint16_t*>(v_cache);
+  prm.block_table = block_table;
+  prm.seq_lens = seq_lens;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.page_size = page_size;
+  prm.max_pages = max_pages_per_seq;
+  prm.num_pages = num_pages;
+  prm.n_split = (int)((tokens + kSplitTokens - 1) / kSplitTokens);
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  const size_t parts = (size_t)B * Hq * prm.n_split;
+  prm.o_part = static_cast<float*>(workspace);
+  prm.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + parts * d * sizeof(float));
+  prm.o = static_cast<uint16_t*>(o);
+  prm.lse = lse;
+
+  dim3 grid_split((prm.n_split + 3) / 4, Hkv, B);
+  dim3 grid_merge((unsigned)(((long long)B * Hq + 3) / 4));
+  if (d == 128) {
+    attn_decode_split_kernel<128><<<grid_split, 128, 0, stream>>>(prm);
+    attn_decode_merge_kernel<128><<<grid_merge, 128, 0, stream>>>(prm);
+  } else {
+    attn_decode_split_kernel<64><<<grid_split, 128, 0, stream>>>(prm);
+    attn_decode_merge_kernel<64><<<grid_merge, 128, 0, stream>>>(prm);
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_get_device_error(attn_stream_t stream_, unsigned int* flags_out) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return ATTN_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof v) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero) != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  if (flags_out != nullptr) *flags_out = v;
+  return v == 0 ? ATTN_OK : ATTN_ERR_DEVICE;
+}
+
+}  // extern "C"

@@ -1,0 +1,331 @@
+// decode_sm100.cuh -- single-query attention over a paged KV cache, split
+// along the keys, plus the deterministic merge of the splits.
+//
+// Sources: "Attention Kernel", sections "Paged 与 ragged KV" (logical token t
+// lives in block t / page_size at offset t mod page_size; the block table
+// gives the physical page) and "Prefill 与 decode 是两种 kernel" (decode is
+// bound by KV bandwidth and indirect addressing); "Attention 算子加速史",
+// section 4.1-4.2 (split-K decode: each split writes a partial output and its
+// log-sum-exp, a light kernel merges them) and "Attention Kernel", section
+// "Online softmax" (the merge rule).
+//
+// Split kernel: one warp per (sequence b, KV head, split of kSplitTokens
+// tokens).  The warp serves all Hq/Hkv query heads that share the KV head
+// (GQA), 16 tokens at a time, with warp-level bf16 MMAs whose operands come
+// straight from global memory into registers -- no shared memory:
+//   S (heads x 16 tokens)  = q (16 padded heads x d) . K^T
+//   O^T (d x heads)       += V^T (d x 16 tokens) . P^T (16 tokens x heads)
+// The contraction index of each MMA may be permuted freely as long as both
+// operands use the same permutation, and an output index may be relabelled
+// if the write-back uses the same labels.  Both are chosen so that every
+// thread loads 16-byte contiguous pieces of K and V rows: for K a thread owns
+// a contiguous quarter of a row, for V a contiguous eighth of four rows.
+// The next 16 tokens' K (V) are requested as soon as the current K (V)
+// registers are consumed, so loads overlap the softmax and the other MMA.
+//
+// Merge kernel: one warp per (b, query head) combines the splits in a fixed
+// order: LSE = M + log2 sum_s 2^(lse_s - M), O = sum_s 2^(lse_s - LSE) o_s,
+// giving empty splits (lse = -inf) zero weight; no atomics, so the result is
+// the same on every run.  Partial log-sum-exps are kept in log2 units inside
+// the workspace; the final LSE is converted to the natural log.
+#pragma once
+
+#include "sm100_primitives.cuh"
+
+namespace attn_b200 {
+
+constexpr int kSplitTokens = 512;
+
+struct DecodeParams {
+  const uint16_t* q;        // [B, Hq, D]
+  const uint16_t* k_cache;  // [num_pages, page_size, Hkv, D]
+  const uint16_t* v_cache;
+  const int* block_table;   // [B, max_pages]
+  const int* seq_lens;      // [B]
+  float* o_part;            // [B, Hq, n_split, D]
+  float* lse_part;          // [B, Hq, n_split] (log2 units)
+  uint16_t* o;              // [B, Hq, D] bf16
+  float* lse;               // [B, Hq] or nullptr
+  int B, Hq, Hkv, group, page_size, max_pages, num_pages, n_split;
+  float scale_log2;
+};
+
+__device__ __forceinline__ int decode_clamped_len(const DecodeParams& p, int b, bool report) {
+  int len = p.seq_lens[b];
+  const long long cap = (long long)p.max_pages * p.page_size;
+  if (len < 0 || (long long)len > cap) {
+    if (report) flag_device_error(kDevErrBadLength);
+    len = len < 0 ? 0 : (int)cap;
+  }
+  return len;
+}
+
+template <int D>
+struct DecodeGroupRegs {
+  uint32_t k[2][D / 8];   // tokens nc*8 + g (nc = 0, 1): D/4 bf16 each
+  uint32_t v[4][D / 16];  // tokens 2tq, 2tq+1, 2tq+8, 2tq+9: D/8 bf16 each
+};
+
+template <int D>
+__device__ __forceinline__ bool decode_page_row(const DecodeParams& p, int b, int t0, int& page,
+                                                int& row) {
+  page = p.block_table[(size_t)b * p.max_pages + t0 / p.page_size];
+  row = t0 % p.page_size;
+  return page >= 0 && page < p.num_pages;
+}
+
+// K rows for 16 tokens starting at logical token t0 (page-relative row `row`).
+template <int D>
+__device__ __forceinline__ void decode_load_k(const DecodeParams& p, int page, int row, int kvh,
+                                              int g, int tq, int n_valid, uint32_t (&k)[2][D / 8]) {
+#pragma unroll
+  for (int nc = 0; nc < 2; ++nc) {
+    const int tok = nc * 8 + g;
+    if (tok < n_valid) {
+      const uint16_t* src = p.k_cache +
+                            (((size_t)page * p.page_size + row + tok) * p.Hkv + kvh) * D +
+                            (D / 4) * tq;
+#pragma unroll
+      for (int w = 0; w < D / 32; ++w) {
+        const uint4 x = ld_stream_v4(src + 8 * w);
+        k[nc][4 * w + 0] = x.x;
+        k[nc][4 * w + 1] = x.y;
+        k[nc][4 * w + 2] = x.z;
+        k[nc][4 * w + 3] = x.w;
+      }
+    } else {
+#pragma unroll
+      for (int w = 0; w < D / 8; ++w) k[nc][w] = 0u;
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void decode_load_v(const DecodeParams& p, int page, int row, int kvh,
+                                              int g, int tq, int n_valid, uint32_t (&v)[4][D / 16]) {
+#pragma unroll
+  for (int ti = 0; ti < 4; ++ti) {
+    const int tok = 2 * tq + (ti & 1) + 8 * (ti >> 1);
+    if (tok < n_valid) {
+      const uint16_t* src = p.v_cache +
+                            (((size_t)page * p.page_size + row + tok) * p.Hkv + kvh) * D +
+                            (D / 8) * g;
+#pragma unroll
+      for (int w = 0; w < D / 64; ++w) {
+        const uint4 x = ld_stream_v4(src + 8 * w);
+        v[ti][4 * w + 0] = x.x;
+        v[ti][4 * w + 1] = x.y;
+        v[ti][4 * w + 2] = x.z;
+        v[ti][4 * w + 3] = x.w;
+      }
+    } else {
+#pragma unroll
+      for (int w = 0; w < D / 16; ++w) v[ti][w] = 0u;  // masked tokens must not inject NaN
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) attn_decode_split_kernel(const DecodeParams p) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int split = blockIdx.x * 4 + warp;
+  const int kvh = blockIdx.y;
+  const int b = blockIdx.z;
+  if (split >= p.n_split) return;
+  const int len = decode_clamped_len(p, b, lane == 0 && split == 0 && kvh == 0);
+  const int t_begin = split * kSplitTokens;
+  if (t_begin >= len) return;  // the merge kernel never reads splits past the end
+  const int t_end = min(t_begin + kSplitTokens, len);
+
+  const int g = lane >> 2;   // MMA group id: head row of S / P, d-row block of V^T
+  const int tq = lane & 3;   // thread within the group
+  const int hq0 = kvh * p.group;
+
+  // q as the A operand of S = q K^T: row g = query head hq0 + g (rows g + 8 and
+  // heads beyond the group are zero padding); k-chunk kc holds
+  // d = (D/4)*tq + 4*kc + {0,1} (a0a1) and + {2,3} (a4a5).
+  uint32_t qa[D / 16][2];
+  if (g < p.group) {
+    const uint16_t* src = p.q + ((size_t)b * p.Hq + hq0 + g) * D + (D / 4) * tq;
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) {
+      const uint4 x = *reinterpret_cast<const uint4*>(src + 8 * w);
+      qa[2 * w][0] = x.x;
+      qa[2 * w][1] = x.y;
+      qa[2 * w + 1][0] = x.z;
+      qa[2 * w + 1][1] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int kc = 0; kc < D / 16; ++kc) qa[kc][0] = qa[kc][1] = 0u;
+  }
+
+  float c2 = p.scale_log2;
+  const bool scale_pos = c2 > 0.f;
+  if (!scale_pos) c2 = 1.f;
+  float m_run = -INFINITY;  // per head row g, log2 units
+  float l_run = 0.f;
+  float acc[D / 16][4];
+#pragma unroll
+  for (int mc = 0; mc < D / 16; ++mc) acc[mc][0] = acc[mc][1] = acc[mc][2] = acc[mc][3] = 0.f;
+
+  DecodeGroupRegs<D> cur;
+  int page, row;
+  bool page_ok = decode_page_row<D>(p, b, t_begin, page, row);
+  int n_valid = page_ok ? min(16, t_end - t_begin) : 0;
+  if (!page_ok && lane == 0) flag_device_error(kDevErrBadPage);
+  decode_load_k<D>(p, page, row, kvh, g, tq, n_valid, cur.k);
+  decode_load_v<D>(p, page, row, kvh, g, tq, n_valid, cur.v);
+
+#pragma unroll 1
+  for (int t0 = t_begin; t0 < t_end; t0 += 16) {
+    const int n_here = n_valid;
+    const int t1 = t0 + 16;
+    int page_n = 0, row_n = 0, n_next = 0;
+    if (t1 < t_end) {
+      const bool ok_n = decode_page_row<D>(p, b, t1, page_n, row_n);
+      if (!ok_n && lane == 0) flag_device_error(kDevErrBadPage);
+      n_next = ok_n ? min(16, t_end - t1) : 0;
+    }
+
+    // ---- S = q K^T (16 padded head rows x 16 tokens)
+    float sc[2][4];
+#pragma unroll
+    for (int nc = 0; nc < 2; ++nc) {
+      sc[nc][0] = sc[nc][1] = sc[nc][2] = sc[nc][3] = 0.f;
+#pragma unroll
+      for (int kc = 0; kc < D / 16; ++kc)
+        mma_m16n8k16_bf16(sc[nc], qa[kc][0], 0u, qa[kc][1], 0u, cur.k[nc][2 * kc],
+                          cur.k[nc][2 * kc + 1]);
+    }
+    if (t1 < t_end) decode_load_k<D>(p, page_n, row_n, kvh, g, tq, n_next, cur.k);
+
+    // ---- online softmax for head row g over this thread's 4 tokens
+    float s4[4] = {sc[0][0], sc[0][1], sc[1][0], sc[1][1]};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int tok = (e >> 1) * 8 + 2 * tq + (e & 1);
+      if (tok >= n_here) s4[e] = -INFINITY;
+      else if (!scale_pos) s4[e] *= p.scale_log2;
+    }
+    float mx = fmaxf(fmaxf(s4[0], s4[1]), fmaxf(s4[2], s4[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx * c2);
+    // nothing accumulated while m_run = -inf (also avoids -inf - -inf = NaN)
+    const float alpha = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_new);
+    const float base = (m_new == -INFINITY) ? 0.f : m_new;
+    float pr[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) pr[e] = ex2(fmaf(s4[e], c2, -base));
+    float rs = (pr[0] + pr[1]) + (pr[2] + pr[3]);
+    rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+    rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+    l_run = l_run * alpha + rs;
+    m_run = m_new;
+    const uint32_t pb0 = pack_bf16x2(pr[0], pr[1]);  // P^T rows 2tq, 2tq+1 (tokens), column g (head)
+    const uint32_t pb1 = pack_bf16x2(pr[2], pr[3]);  // tokens 2tq+8, 2tq+9
+
+    // ---- O^T += V^T P^T; accumulator columns are heads 2tq and 2tq+1
+    const float a_h0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
+    const float a_h1 = __shfl_sync(0xffffffffu, alpha, (2 * tq + 1) * 4);
+#pragma unroll
+    for (int mc = 0; mc < D / 16; ++mc) {
+      acc[mc][0] *= a_h0;
+      acc[mc][1] *= a_h1;
+      acc[mc][2] *= a_h0;
+      acc[mc][3] *= a_h1;
+      // A = V^T block: row g <-> d = (D/8)*g + 2*mc, row g+8 <-> d + 1;
+      // columns = tokens 2tq, 2tq+1 (a0a1, a2a3) and 2tq+8, 2tq+9 (a4a5, a6a7).
+      const uint32_t a01 = prmt(cur.v[0][mc], cur.v[1][mc], 0x5410u);
+      const uint32_t a23 = prmt(cur.v[0][mc], cur.v[1][mc], 0x7632u);
+      const uint32_t a45 = prmt(cur.v[2][mc], cur.v[3][mc], 0x5410u);
+      const uint32_t a67 = prmt(cur.v[2][mc], cur.v[3][mc], 0x7632u);
+      mma_m16n8k16_bf16(acc[mc], a01, a23, a45, a67, pb0, pb1);
+    }
+    if (t1 < t_end) decode_load_v<D>(p, page_n, row_n, kvh, g, tq, n_next, cur.v);
+    n_valid = n_next;
+  }
+
+  // ---- write this split's normalised partial output and its log2-sum-exp
+  const int h0 = 2 * tq, h1 = 2 * tq + 1;
+  const float l_h0 = __shfl_sync(0xffffffffu, l_run, h0 * 4);
+  const float l_h1 = __shfl_sync(0xffffffffu, l_run, h1 * 4);
+  const float inv0 = l_h0 > 0.f ? 1.f / l_h0 : 0.f;
+  const float inv1 = l_h1 > 0.f ? 1.f / l_h1 : 0.f;
+  const int dbase = (D / 8) * g;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int h = hh ? h1 : h0;
+    if (h >= p.group) continue;
+    const float inv = hh ? inv1 : inv0;
+    float* dst = p.o_part + (((size_t)b * p.Hq + hq0 + h) * p.n_split + split) * D + dbase;
+#pragma unroll
+    for (int mc = 0; mc < D / 16; mc += 2) {
+      float4 w;
+      w.x = acc[mc][hh] * inv;          // d = dbase + 2mc
+      w.y = acc[mc][2 + hh] * inv;      // d = dbase + 2mc + 1
+      w.z = acc[mc + 1][hh] * inv;      // d = dbase + 2mc + 2
+      w.w = acc[mc + 1][2 + hh] * inv;  // d = dbase + 2mc + 3
+      *reinterpret_cast<float4*>(dst + 2 * mc) = w;
+    }
+  }
+  if (tq == 0 && g < p.group) {
+    const float lse2 = l_run > 0.f ? m_run + lg2(l_run) : -INFINITY;
+    p.lse_part[((size_t)b * p.Hq + hq0 + g) * p.n_split + split] = lse2;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) attn_decode_merge_kernel(const DecodeParams p) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int pair = blockIdx.x * 4 + warp;  // b * Hq + hq
+  if (pair >= p.B * p.Hq) return;
+  const int b = pair / p.Hq;
+  const int len = decode_clamped_len(p, b, false);
+  const int ns = (len + kSplitTokens - 1) / kSplitTokens;
+  const float* lse_s = p.lse_part + (size_t)pair * p.n_split;
+  float mx = -INFINITY;
+  for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, lse_s[s]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  constexpr int PER = D / 32;  // output columns per lane
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  float wsum = 0.f;
+  if (mx != -INFINITY) {
+    const float* op = p.o_part + (size_t)pair * p.n_split * D + lane * PER;
+    for (int s = 0; s < ns; ++s) {  // fixed order: deterministic
+      const float w = ex2(lse_s[s] - mx);
+      wsum += w;
+      if (PER == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(op + (size_t)s * D);
+        acc[0] += w * x.x;
+        acc[1 % PER] += w * x.y;
+        acc[2 % PER] += w * x.z;
+        acc[3 % PER] += w * x.w;
+      } else {
+        const float2 x = *reinterpret_cast<const float2*>(op + (size_t)s * D);
+        acc[0] += w * x.x;
+        acc[1 % PER] += w * x.y;
+      }
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  uint16_t* dst = p.o + (size_t)pair * D + lane * PER;
+  if (PER == 4) {
+    uint2 w;
+    w.x = pack_bf16x2(acc[0] * inv, acc[1 % PER] * inv);
+    w.y = pack_bf16x2(acc[2 % PER] * inv, acc[3 % PER] * inv);
+    *reinterpret_cast<uint2*>(dst) = w;
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1 % PER] * inv);
+  }
+  if (p.lse != nullptr && lane == 0)
+    p.lse[pair] = wsum > 0.f ? (mx + lg2(wsum)) * 0.69314718055994531f : -INFINITY;
+}
+
+}  // namespace attn_b200

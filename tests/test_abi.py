@@ -1,0 +1,127 @@
+"""CPU checks of the C ABI: the library loads, exports every declared symbol, and
+rejects bad arguments on the host before touching CUDA (no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_softmax_attention_fwd_b200 import _binding as B
+from exact_softmax_attention_fwd_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(attn_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.load_library()
+
+
+def test_header_declares_expected_entry_points():
+    names = _declared_functions()
+    for n in ("attn_fwd", "attn_fwd_masked", "attn_decode_paged", "attn_decode_workspace_size",
+              "attn_get_device_error", "attn_strerror"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), f"{name} declared in attn.h but not exported"
+        assert name in B.SIGNATURES, f"{name} has no binding signature"
+
+
+def test_strerror_covers_codes(lib):
+    for code in range(0, 7):
+        s = lib.attn_strerror(code).decode()
+        assert s and s != "unknown status"
+    assert lib.attn_strerror(99).decode() == "unknown status"
+
+
+FAKE = 0x100000  # 16-byte aligned, never dereferenced: every call below fails validation
+
+
+def _fwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B_=1, Hq=2, Hkv=2, Sq=128, Sk=128, d=128,
+         causal=0, scale=0.1, k_lens=None):
+    return lib.attn_fwd_masked(q, k, v, o, lse, B_, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(o=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(B_=0), B.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), B.ATTN_ERR_INVALID_ARG),
+    (dict(Sq=0), B.ATTN_ERR_INVALID_ARG),
+    (dict(Sk=-1), B.ATTN_ERR_INVALID_ARG),
+    (dict(causal=2), B.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), B.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), B.ATTN_ERR_INVALID_ARG),
+    (dict(d=96), B.ATTN_ERR_UNSUPPORTED),
+    (dict(d=256), B.ATTN_ERR_UNSUPPORTED),
+    (dict(q=FAKE + 8), B.ATTN_ERR_ALIGNMENT),
+    (dict(v=FAKE + 2), B.ATTN_ERR_ALIGNMENT),
+    (dict(lse=FAKE + 2), B.ATTN_ERR_ALIGNMENT),
+    (dict(B_=70000), B.ATTN_ERR_INVALID_ARG),
+])
+def test_prefill_validation(lib, kw, status):
+    assert _fwd(lib, **kw) == status
+
+
+def test_prefill_plain_entry_validates_too(lib):
+    assert lib.attn_fwd(None, FAKE, FAKE, FAKE, None, 1, 1, 1, 1, 1, 64, 0, 1.0, None) == \
+        B.ATTN_ERR_INVALID_ARG
+
+
+def _dec(lib, q=FAKE, kc=FAKE, vc=FAKE, tbl=FAKE, lens=FAKE, ps=16, B_=2, Hq=8, Hkv=2, d=128,
+         maxp=4, npages=8, scale=0.1, o=FAKE, lse=None, ws=FAKE, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = lib.attn_decode_workspace_size(B_, Hq, maxp, ps, d) if B_ > 0 else 0
+    return lib.attn_decode_paged(q, kc, vc, tbl, lens, ps, B_, Hq, Hkv, d, maxp, npages, scale, o,
+                                 lse, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(tbl=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), B.ATTN_ERR_INVALID_ARG),
+    (dict(maxp=0), B.ATTN_ERR_INVALID_ARG),
+    (dict(npages=0), B.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), B.ATTN_ERR_INVALID_ARG),
+    (dict(ps=8), B.ATTN_ERR_UNSUPPORTED),
+    (dict(ps=24), B.ATTN_ERR_UNSUPPORTED),
+    (dict(d=80), B.ATTN_ERR_UNSUPPORTED),
+    (dict(Hq=32, Hkv=2), B.ATTN_ERR_UNSUPPORTED),
+    (dict(kc=FAKE + 4), B.ATTN_ERR_ALIGNMENT),
+    (dict(ws=None), B.ATTN_ERR_WORKSPACE),
+    (dict(ws_bytes=16), B.ATTN_ERR_WORKSPACE),
+    (dict(ws=FAKE + 8), B.ATTN_ERR_ALIGNMENT),
+])
+def test_decode_validation(lib, kw, status):
+    assert _dec(lib, **kw) == status
+
+
+def test_workspace_size_formula(lib):
+    split = lib.attn_split_tokens()
+    assert split > 0 and split % 16 == 0
+    B_, Hq, maxp, ps, d = 64, 32, 512, 16, 128
+    n_split = -(-(maxp * ps) // split)
+    parts = B_ * Hq * n_split
+    got = lib.attn_decode_workspace_size(B_, Hq, maxp, ps, d)
+    assert got >= parts * d * 4 + parts * 4
+    assert got <= parts * d * 4 + parts * 4 + 256
+    assert lib.attn_decode_workspace_size(0, 1, 1, 16, 128) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        B.attn_fwd(q, q, q, False, 0.1)
