@@ -1,0 +1,465 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-softmax-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--decode-workload NAME] [--no-e2e] [--no-cpu-baseline]
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  * prefill: attn_fwd on the named prefill workload (default mha_causal_2k:
+    B=4, H=16, S=2048, d=128, causal), and
+  * decode: attn_decode_paged (split kernel + merge kernel) on paged_decode
+    (B=64, Hq=32, Hkv=8, d=128, pages of 16, lengths U[512, 8192]).
+Each kernel is timed with CUDA events on the stream it is launched on; L2 is
+flushed (a 256 MiB write) before each timed kernel.  The headline `value` is
+prefill TFLOPS (FLOPs = 4*B*Hq*Sq*Sk*d, halved when causal) over all ranks;
+`decode` reports KV GB/s (K+V bytes of the attended tokens).  Under torchrun
+every rank runs the same per-GPU workload (weak scaling; the work units are
+independent, so there is no data-path collective) and times are the max over
+ranks.
+
+--impl reference times the CPU oracle (the only reference implementation this
+project has) on the host cores of rank 0, on a bounded seeded sample of the
+same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attn fwd TFLOPS (prefill) and decode KV GB/s on 1 B200, % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mha_causal_2k")
+    ap.add_argument("--decode-workload", default="paged_decode")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+def kernel_source_sha() -> str:
+    """Hash of the CUDA sources: ncu traffic figures are valid only for this hash."""
+    csrc = os.path.join(ROOT, "exact_softmax_attention_fwd_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key: str, config_name: str):
+    """Per-launch DRAM bytes of a kernel from profiles/traffic.json, if current."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    e = t.get(kernel_key, {}).get(config_name)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return float(e["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    def __init__(self, device, period_s: float = 0.02):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.ok = False
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self._nv = nv
+            self._h = None
+            try:  # NVML numbering can differ from CUDA's: match the PCI bus id
+                import torch
+                pr = torch.cuda.get_device_properties(device)
+                bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+                self._h = nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self._h = nv.nvmlDeviceGetHandleByIndex(device.index or 0)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self._h, nv.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self._nv = None
+        self._names = {
+            "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+            "hw_power_brake_slowdown": 0x80, "sw_power_cap": 0x4, "sync_boost": 0x10,
+            "gpu_idle": 0x1, "applications_clocks_setting": 0x2,
+        }
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except AttributeError:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                for name, bit in self._names.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"],
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------------------------- reference arm
+
+
+def run_reference(args, world, rank):
+    """Time the CPU oracle on a bounded sample of the prefill workload (rank 0 only)."""
+    if rank != 0:
+        return None
+    import torch
+
+    import oracle
+    from exact_softmax_attention_fwd_b200 import workloads as W
+    cfg = W.CONFIGS[args.workload]
+    q, k, v, k_lens = W.config_inputs(cfg)
+    n_rows = 4096  # rows per step: a few seconds of the host's cores
+    threads = os.cpu_count() or 1
+    oracle.build()
+    times, flops = [], []
+    for step in range(args.warmup + args.steps):
+        rows = W.sample_rows(cfg.B, cfg.Hq, cfg.S, n_rows, seed=5000 + step)
+        i = (rows % cfg.S).double()
+        vis = (i + 1) if cfg.causal else torch.full_like(i, float(cfg.S))
+        f = float(4.0 * cfg.d * vis.sum())
+        t0 = time.perf_counter()
+        oracle.attn_fwd(q, k, v, cfg.causal, cfg.scale, k_lens=k_lens, rows=rows, n_threads=threads)
+        dt = time.perf_counter() - t0
+        if step >= args.warmup:
+            times.append(dt)
+            flops.append(f)
+    value = sum(flops) / sum(times) / 1e12
+    ms = 1e3 * sum(times) / len(times)
+    sample = f"{n_rows} seeded rows of {cfg.name} per step (of {cfg.B * cfg.Hq * cfg.S})"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(cfg, None),
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    return line
+
+
+# --------------------------------------------------------------------------- our arm
+
+
+def config_dict(cfg, dcfg):
+    d = {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "Sq": cfg.S, "Sk": cfg.S,
+         "d": cfg.d, "causal": cfg.causal, "inputs": "bf16 N(0,1) seeded",
+         "l2": "flushed before every timed kernel (256 MiB write)"}
+    if dcfg is not None:
+        d["decode_workload"] = dcfg.name
+        d["decode"] = {"B": dcfg.B, "Hq": dcfg.Hq, "Hkv": dcfg.Hkv, "d": dcfg.d,
+                       "page_size": dcfg.page_size, "seq_lens": f"U[{dcfg.len_lo},{dcfg.len_hi}]"}
+    return d
+
+
+def cpu_baseline_leg(cfg, q, k, v, k_lens):
+    """The oracle on a bounded sample of the prefill workload (about 10-30 s of CPU)."""
+    import torch
+
+    import oracle
+    from exact_softmax_attention_fwd_b200 import workloads as W
+    threads = os.cpu_count() or 1
+    # size the sample from a short calibration run
+    rows = W.sample_rows(cfg.B, cfg.Hq, cfg.S, 512, seed=77)
+    t0 = time.perf_counter()
+    oracle.attn_fwd(q, k, v, cfg.causal, cfg.scale, k_lens=k_lens, rows=rows, n_threads=threads)
+    t_cal = time.perf_counter() - t0
+    n = int(max(512, min(cfg.B * cfg.Hq * cfg.S, 512 * 12.0 / max(t_cal, 1e-3))))
+    rows = W.sample_rows(cfg.B, cfg.Hq, cfg.S, n, seed=78)
+    i = (rows % cfg.S).double()
+    vis = (i + 1) if cfg.causal else torch.full_like(i, float(cfg.S))
+    flops = float(4.0 * cfg.d * vis.sum())
+    t0 = time.perf_counter()
+    oracle.attn_fwd(q, k, v, cfg.causal, cfg.scale, k_lens=k_lens, rows=rows, n_threads=threads)
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+            "sample": f"{rows.numel()} seeded query rows of {cfg.name} ({dt:.1f} s)"}
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    from exact_softmax_attention_fwd_b200 import (attn_decode_paged, attn_decode_workspace_size,
+                                                  attn_fwd_masked, attn_get_device_error)
+    from exact_softmax_attention_fwd_b200 import workloads as W
+
+    dev = torch.device("cuda", local if world > 1 else 0)
+    peaks = load_peaks()
+    cfg = W.CONFIGS[args.workload]
+    dcfg = None if args.no_decode else W.CONFIGS[args.decode_workload]
+
+    # ---- inputs resident in HBM before the timed region
+    q_h, k_h, v_h, kl_h = W.config_inputs(cfg)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    k_lens = None if kl_h is None else kl_h.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((cfg.B, cfg.Hq, cfg.S), dtype=torch.float32, device=dev)
+    flops = cfg.flops()
+    if dcfg is not None:
+        dinp = W.decode_config_inputs(dcfg)
+        dq, dk, dv = dinp.q.to(dev), dinp.k_cache.to(dev), dinp.v_cache.to(dev)
+        dtbl, dlens = dinp.block_table.to(dev), dinp.seq_lens.to(dev)
+        ws = torch.empty(attn_decode_workspace_size(dcfg.B, dcfg.Hq, dcfg.max_pages_per_seq,
+                                                    dcfg.page_size, dcfg.d),
+                         dtype=torch.uint8, device=dev)
+        do = torch.empty((dcfg.B, dcfg.Hq, dcfg.d), dtype=torch.bfloat16, device=dev)
+        dlse = torch.empty((dcfg.B, dcfg.Hq), dtype=torch.float32, device=dev)
+        kv_bytes = W.decode_kv_bytes(dinp.seq_lens, dcfg.Hkv, dcfg.d)
+        table_bytes = int(sum(-(-int(n) // dcfg.page_size) for n in dinp.seq_lens.tolist())) * 4
+        decode_bytes = (kv_bytes + 2 * dq.numel() * 2 + table_bytes + dlens.numel() * 4
+                        + dlse.numel() * 4)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def prefill():
+        attn_fwd_masked(q, k, v, cfg.causal, cfg.scale, k_lens=k_lens, out=o, lse=lse)
+
+    def decode():
+        attn_decode_paged(dq, dk, dv, dtbl, dlens, dcfg.scale, out=do, lse=dlse, workspace=ws)
+
+    def step(evs=None):
+        flush.fill_(1.0)
+        if evs is not None:
+            evs[0].record(stream)
+        prefill()
+        if evs is not None:
+            evs[1].record(stream)
+        if dcfg is not None:
+            flush.fill_(2.0)
+            if evs is not None:
+                evs[2].record(stream)
+            decode()
+            if evs is not None:
+                evs[3].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    st, fl = attn_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word set during warm-up: {fl:#x}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_all0 = torch.cuda.Event(enable_timing=True)
+    t_all1 = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with sampler:
+        t_all0.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        t_all1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    st, fl = attn_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word set in the timed region: {fl:#x}")
+
+    pre_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    pre_avg = max_over_ranks(sum(pre_ms) / len(pre_ms), world)
+    step_ms = max_over_ranks(t_all0.elapsed_time(t_all1) / args.steps, world)
+    value = world * flops / (pre_avg * 1e-3) / 1e12
+    achieved = flops / (pre_avg * 1e-3) / 1e12
+    traffic = ncu_traffic("attn_prefill_sm100_kernel", cfg.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": config_dict(cfg, dcfg),
+        "roofline": {"bound": "tensor", "achieved": achieved,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                     "kernel": "attn_prefill_sm100_kernel",
+                     "peak_source": f"{peaks['source']} bf16 burst (kernel timed alone)",
+                     "per_launch_flops": flops, "median_ms": statistics.median(pre_ms)},
+    }
+    launches_per_step = 1
+    if dcfg is not None:
+        dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
+        dec_avg = max_over_ranks(sum(dec_ms) / len(dec_ms), world)
+        gbs = decode_bytes / (dec_avg * 1e-3) / 1e9
+        dtraffic = ncu_traffic("attn_decode_split_kernel", dcfg.name)
+        line["decode"] = {
+            "value": world * gbs, "unit": "GB/s", "ms": dec_avg,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": dtraffic,
+                         "kernel": "attn_decode_split_kernel + attn_decode_merge_kernel",
+                         "peak_source": f"{peaks['source']} copy bandwidth",
+                         "algorithmic_bytes": decode_bytes, "median_ms": statistics.median(dec_ms)},
+        }
+        launches_per_step += 2
+    line["gpu_launches"] = launches_per_step * args.steps
+    line["clocks"] = sampler.summary()
+
+    if not args.no_e2e:
+        line["e2e"] = e2e_leg(args, cfg, q_h, k_h, v_h, kl_h, dev, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_leg(cfg, q_h, k_h, v_h, kl_h)
+    return line if rank == 0 else None
+
+
+def e2e_leg(args, cfg, q_h, k_h, v_h, kl_h, dev, world):
+    """Same metric through the public call with host buffers: H2D of q/k/v from pinned
+    memory, the prefill kernel, D2H of O and LSE -- all inside the timed region."""
+    import torch
+
+    from exact_softmax_attention_fwd_b200 import attn_fwd_masked
+    qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    op = torch.empty_like(q_h).pin_memory()
+    lp = torch.empty((cfg.B, cfg.Hq, cfg.S), dtype=torch.float32).pin_memory()
+    q, k, v = torch.empty_like(qp, device=dev), torch.empty_like(kp, device=dev), torch.empty_like(
+        vp, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((cfg.B, cfg.Hq, cfg.S), dtype=torch.float32, device=dev)
+    kl = None if kl_h is None else kl_h.to(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def one():
+        q.copy_(qp, non_blocking=True)
+        k.copy_(kp, non_blocking=True)
+        v.copy_(vp, non_blocking=True)
+        attn_fwd_masked(q, k, v, cfg.causal, cfg.scale, k_lens=kl, out=o, lse=lse)
+        op.copy_(o, non_blocking=True)
+        lp.copy_(lse, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize(dev)
+    n = max(5, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    for _ in range(n):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1) / n, world)
+    h2d = (qp.numel() + kp.numel() + vp.numel()) * 2
+    d2h = op.numel() * 2 + lp.numel() * 4
+    return {"value": world * cfg.flops() / (ms * 1e-3) / 1e12, "unit": "TFLOPS",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        # the oracle runs on rank 0's host cores; other ranks have nothing to do
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        line = run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), 0)
+        print(json.dumps(line), flush=True)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        line = run_ours(args, world, rank, local)
+        if line is not None and rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

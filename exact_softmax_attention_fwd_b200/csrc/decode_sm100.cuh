@@ -165,7 +165,8 @@ __global__ void __launch_bounds__(128) attn_decode_split_kernel(const DecodePara
   const bool scale_pos = c2 > 0.f;
   if (!scale_pos) c2 = 1.f;
   float m_run = -INFINITY;  // per head row g, log2 units
-  float l_run = 0.f;
+  float l_run = 0.f;   // sum of P (f32): the LSE
+  float lr_run = 0.f;  // sum of bf16(P): normalises O
   float acc[D / 16][4];
 #pragma unroll
   for (int mc = 0; mc < D / 16; ++mc) acc[mc][0] = acc[mc][1] = acc[mc][2] = acc[mc][3] = 0.f;
@@ -219,13 +220,19 @@ __global__ void __launch_bounds__(128) attn_decode_split_kernel(const DecodePara
     float pr[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) pr[e] = ex2(fmaf(s4[e], c2, -base));
-    float rs = (pr[0] + pr[1]) + (pr[2] + pr[3]);
-    rs += __shfl_xor_sync(0xffffffffu, rs, 1);
-    rs += __shfl_xor_sync(0xffffffffu, rs, 2);
-    l_run = l_run * alpha + rs;
-    m_run = m_new;
     const uint32_t pb0 = pack_bf16x2(pr[0], pr[1]);  // P^T rows 2tq, 2tq+1 (tokens), column g (head)
     const uint32_t pb1 = pack_bf16x2(pr[2], pr[3]);  // tokens 2tq+8, 2tq+9
+    // row sums over the f32 P (for the LSE) and over the bf16-rounded P that
+    // the MMA consumes (normalises O)
+    float rs = (pr[0] + pr[1]) + (pr[2] + pr[3]);
+    float rr = sum_f32x2(add_f32x2(bf16x2_to_f32x2(pb0), bf16x2_to_f32x2(pb1)));
+    rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+    rr += __shfl_xor_sync(0xffffffffu, rr, 1);
+    rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+    rr += __shfl_xor_sync(0xffffffffu, rr, 2);
+    l_run = l_run * alpha + rs;
+    lr_run = lr_run * alpha + rr;
+    m_run = m_new;
 
     // ---- O^T += V^T P^T; accumulator columns are heads 2tq and 2tq+1
     const float a_h0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
@@ -250,8 +257,8 @@ __global__ void __launch_bounds__(128) attn_decode_split_kernel(const DecodePara
 
   // ---- write this split's normalised partial output and its log2-sum-exp
   const int h0 = 2 * tq, h1 = 2 * tq + 1;
-  const float l_h0 = __shfl_sync(0xffffffffu, l_run, h0 * 4);
-  const float l_h1 = __shfl_sync(0xffffffffu, l_run, h1 * 4);
+  const float l_h0 = __shfl_sync(0xffffffffu, lr_run, h0 * 4);
+  const float l_h1 = __shfl_sync(0xffffffffu, lr_run, h1 * 4);
   const float inv0 = l_h0 > 0.f ? 1.f / l_h0 : 0.f;
   const float inv1 = l_h1 > 0.f ? 1.f / l_h1 : 0.f;
   const int dbase = (D / 8) * g;

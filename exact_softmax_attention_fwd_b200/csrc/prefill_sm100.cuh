@@ -310,7 +310,8 @@ __global__ void __launch_bounds__(320, 1)
     const bool scale_pos = c2 > 0.f;
     if (!scale_pos) c2 = 1.f;  // scores are pre-multiplied below instead
     float m_run = -INFINITY;   // exponent base (log2 units)
-    float l_run = 0.f;
+    float l_run = 0.f;         // sum of P (f32)
+    float lr_run = 0.f;        // sum of bf16(P)
     bool ok = true;
 
     for (int j = 0; j < n; ++j) {
@@ -363,7 +364,11 @@ __global__ void __launch_bounds__(320, 1)
         m_run = m_tile;
       }
       const float base = (m_run == -INFINITY) ? 0.f : m_run;
-      float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+      // Two row sums: l over the f32 P (gives the LSE) and lr over the
+      // bf16-rounded P that the PV MMA consumes (normalises O, so that the
+      // weights applied to V sum to one exactly as used).
+      float l0 = 0.f, l1 = 0.f;
+      uint64_t r01 = 0ull, r23 = 0ull;  // f32x2 partial sums of the rounded P
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
@@ -374,16 +379,17 @@ __global__ void __launch_bounds__(320, 1)
           const float p1 = ex2(fmaf(s[cc + 1], c2, -base));
           const float p2 = ex2(fmaf(s[cc + 2], c2, -base));
           const float p3 = ex2(fmaf(s[cc + 3], c2, -base));
-          l0 += p0;
-          l1 += p1;
-          l2 += p2;
-          l3 += p3;
+          l0 += p0 + p1;
+          l1 += p2 + p3;
           pk[c / 2] = pack_bf16x2(p0, p1);
           pk[c / 2 + 1] = pack_bf16x2(p2, p3);
+          r01 = add_f32x2(r01, bf16x2_to_f32x2(pk[c / 2]));
+          r23 = add_f32x2(r23, bf16x2_to_f32x2(pk[c / 2 + 1]));
         }
         tmem_st32(t_s + 32 * half, pk);  // P columns [32*half, 32*half + 32)
       }
-      l_run = l_run * alpha + ((l0 + l1) + (l2 + l3));
+      l_run = l_run * alpha + (l0 + l1);
+      lr_run = lr_run * alpha + (sum_f32x2(r01) + sum_f32x2(r23));
       // Rescale the accumulator when any row of this warp moved its base.  The
       // MMA that last wrote O_i completed before S_i(j) was signalled.
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -407,7 +413,7 @@ __global__ void __launch_bounds__(320, 1)
       if (n > 0 && ok) ok = mbar_wait_warp(bar(C::B_OFULL + i), 0, abort_flag);
       tc_fence_after_sync();
       const bool has_o = (n > 0) && ok;
-      const float inv = (l_run > 0.f) ? (1.f / l_run) : 0.f;
+      const float inv = (lr_run > 0.f) ? (1.f / lr_run) : 0.f;
       uint8_t* stage = sbase_ptr + C::OFF_Q + i * C::TILE_BYTES;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {

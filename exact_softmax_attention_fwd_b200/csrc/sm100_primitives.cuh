@@ -66,6 +66,26 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Packed pair of f32 in one 64-bit register (sm_100 f32x2 arithmetic).
+// bf16x2 -> f32x2 is exact: a bf16 is the upper half of an f32.
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t pk) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(pk << 16), "r"(pk & 0xffff0000u));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ float sum_f32x2(uint64_t a) {
+  uint32_t lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(a));
+  return __uint_as_float(lo) + __uint_as_float(hi);
+}
+
 // ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------

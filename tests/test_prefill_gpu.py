@@ -148,8 +148,22 @@ def test_unusual_scales(scale):
 
 
 def test_large_magnitude_scores_stay_finite():
-    # large logits exercise the lazy rescale (the base moves by more than 8)
-    _full_case(1, 2, 2, 256, 512, 128, False, seed=13, value_scale=3.0)
+    # Inputs 3x unit scale: logits with std ~9 exercise the lazy rescale (the
+    # exponent base moves by more than 8).  Outside the unit-scale regime the
+    # absolute 1e-2 bar does not apply; the bound here follows from the
+    # arithmetic: rounding O to bf16 costs up to 2^-8 |O|, and rounding P to
+    # bf16 (weights normalised by the rounded sum) up to 2^-8 max|V|.
+    q, k, v = W.prefill_inputs(1, 2, 2, 256, 512, 128, seed=13, value_scale=3.0)
+    o, lse = _run(q, k, v, False, 1 / math.sqrt(128))
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, False, 1 / math.sqrt(128))
+    og = o.double().numpy()
+    assert np.isfinite(og).all() and np.isfinite(lse.numpy()).all()
+    vmax = float(v.abs().max())
+    bound = 2.0 ** -8 * np.abs(o_ref) + 2.0 ** -8 * vmax + 1e-3
+    assert np.all(np.abs(og - o_ref) <= bound)
+    rel_rms = np.linalg.norm(og - o_ref) / np.linalg.norm(o_ref)
+    assert rel_rms <= 5e-3
+    assert np.abs(lse.numpy() - lse_ref).max() <= 1e-3
 
 
 def test_worked_example_embedded():
