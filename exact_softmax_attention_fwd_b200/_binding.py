@@ -39,6 +39,8 @@ SIGNATURES = {
     "attn_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P,
                                _SZ, _P]),
+    "attn_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P,
+                                       _P, _P]),
     "attn_get_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
     "attn_strerror": (ctypes.c_char_p, [_I]),
     "attn_split_tokens": (_I, []),
@@ -169,6 +171,46 @@ def attn_decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float, 
                                           num_pages, float(scale), _ptr(out), _ptr(lse),
                                           _ptr(workspace), ws_bytes, _stream(stream))
     _check(st, "attn_decode_paged")
+    return out, lse
+
+
+# Size of the library's static decode scratch area (ATTN_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def attn_decode_paged_noalloc(q, k_cache, v_cache, block_table, seq_lens, scale, out=None,
+                              lse=None, return_lse: bool = True, stream=None):
+    """attn_decode_paged for callers that may not allocate device memory.
+
+    The library keeps the split partials in its own static device scratch area
+    (NOALLOC_SCRATCH_BYTES per GPU), so no workspace is passed and the C call
+    allocates nothing.  Only `out`/`lse` are created here when not supplied --
+    callers that cannot allocate pass their own.  Calls that overlap on the GPU
+    share that scratch area and race; serialise them.  The first call on a
+    device caches the area's address: make it before any stream capture.
+    """
+    import torch
+    _require_cuda(q, k_cache, v_cache, block_table, seq_lens)
+    B, Hq, d = q.shape
+    num_pages, page_size, Hkv, dk = k_cache.shape
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or dk != d:
+        raise ValueError("cache shapes disagree")
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be int32 [B, max_pages_per_seq]")
+    if seq_lens.dtype != torch.int32 or tuple(seq_lens.shape) != (B,):
+        raise ValueError("seq_lens must be int32 [B]")
+    for t in (q, k_cache, v_cache, block_table, seq_lens):
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    st = load_library().attn_decode_paged_noalloc(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens), page_size, B,
+        Hq, Hkv, d, block_table.shape[1], num_pages, float(scale), _ptr(out), _ptr(lse),
+        _stream(stream))
+    _check(st, "attn_decode_paged_noalloc")
     return out, lse
 
 

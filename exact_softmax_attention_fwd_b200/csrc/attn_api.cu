@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "attn.h"
 #include "decode_sm100.cuh"
@@ -242,3 +243,54 @@ int attn_get_device_error(attn_stream_t stream_, unsigned int* flags_out) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode for callers that may not allocate device memory (see attn.h): the
+// split partials go to a file-scope device array instead of a workspace.
+// ---------------------------------------------------------------------------
+namespace attn_b200 {
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+// In host code `g_noalloc_scratch` names a host-side stand-in, not device
+// memory; the kernels must be given the address cudaGetSymbolAddress returns,
+// which is looked up once per device (with that device current) and cached.
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_device_ptr[kMaxDevices] = {};
+
+int noalloc_scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_device_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return ATTN_ERR_CUDA;
+    g_noalloc_device_ptr[dev] = p;
+  }
+  *out = g_noalloc_device_ptr[dev];
+  return ATTN_OK;
+}
+
+}  // namespace
+}  // namespace attn_b200
+
+extern "C" int attn_decode_paged_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                         const int32_t* block_table, const int32_t* seq_lens,
+                                         int page_size, int B, int Hq, int Hkv, int d,
+                                         int max_pages_per_seq, int num_pages, float scale,
+                                         void* o, float* lse, attn_stream_t stream) {
+  // Size check first, on the host: nothing is launched for a problem that
+  // does not fit the static scratch area.
+  const size_t need = attn_decode_workspace_size(B, Hq, max_pages_per_seq, page_size, d);
+  if (need == 0) return ATTN_ERR_INVALID_ARG;
+  if (need > (size_t)ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const int st = attn_b200::noalloc_scratch_address(&scratch);
+  if (st != ATTN_OK) return st;
+  return attn_decode_paged(q, k_cache, v_cache, block_table, seq_lens, page_size, B, Hq, Hkv, d,
+                           max_pages_per_seq, num_pages, scale, o, lse, scratch,
+                           (size_t)ATTN_NOALLOC_SCRATCH_BYTES, stream);
+}

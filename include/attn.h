@@ -147,6 +147,41 @@ int attn_decode_paged(const void* q, const void* k_cache, const void* v_cache,
  */
 int attn_get_device_error(attn_stream_t stream, unsigned int* flags_out);
 
+/*
+ * attn_decode_paged_noalloc -- attn_decode_paged without a caller-supplied
+ * workspace, for callers that are not allowed to allocate device memory: code
+ * that runs inside a host framework which owns every device allocation (and
+ * so has no buffer of its own to lend as scratch), or a latency-critical path
+ * where cudaMalloc / cudaFree, which may synchronise the device, cannot be
+ * called.  The pages this library follows have no counterpart to this call;
+ * it exists only for such callers.
+ *
+ * The split partials live in one library-owned scratch area of
+ * ATTN_NOALLOC_SCRATCH_BYTES, a static device array that every GPU which
+ * loads the library holds until the process exits.  Nothing is allocated by
+ * this call.  Arguments, layouts and results are those of attn_decode_paged;
+ * the caller still provides q, the caches, the table, the lengths and the
+ * outputs.
+ *   - A problem whose attn_decode_workspace_size(...) exceeds
+ *     ATTN_NOALLOC_SCRATCH_BYTES is rejected with ATTN_ERR_WORKSPACE before
+ *     anything is launched.
+ *   - The first call on a device looks up the scratch area's device address
+ *     (with that device current) and caches it; make that first call before
+ *     any stream capture on that device.
+ *   - Every call on a device shares the same scratch area.  Calls whose
+ *     kernels overlap on the GPU (different streams, or different host
+ *     threads) race on it and produce garbage; serialise them.  Each call
+ *     writes every scratch byte it later reads, so nothing has to be cleared
+ *     between calls.
+ * Errors: as attn_decode_paged, plus ATTN_ERR_CUDA if the scratch address
+ * cannot be obtained.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int attn_decode_paged_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_table, const int32_t* seq_lens, int page_size,
+                              int B, int Hq, int Hkv, int d, int max_pages_per_seq, int num_pages,
+                              float scale, void* o, float* lse, attn_stream_t stream);
+
 /* attn_strerror -- static description of an attn_status value. */
 const char* attn_strerror(int status);
 
