@@ -44,14 +44,15 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D bf16 map over a contiguous [planes, rows, D] tensor, box = 128 rows x 64
-// columns, 128-byte swizzle (the layout the tcgen05 descriptors expect).
-bool make_tile_map(CUtensorMap* map, const void* ptr, int D, long long rows, long long planes) {
+// 3-D bf16 map over a contiguous [planes, rows, D] tensor, box = box_rows rows
+// x 64 columns, 128-byte swizzle (the layout the tcgen05 descriptors expect).
+bool make_tile_map(CUtensorMap* map, const void* ptr, int D, long long rows, long long planes,
+                   unsigned box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
   const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -62,6 +63,19 @@ bool make_tile_map(CUtensorMap* map, const void* ptr, int D, long long rows, lon
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 template <int D, bool CAUSAL>
 int launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                    const CUtensorMap& mo, const PrefillParams& prm, cudaStream_t stream) {
@@ -70,7 +84,11 @@ int launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
       cudaSuccess)
     return ATTN_ERR_CUDA;
-  dim3 grid(prm.n_qblocks, prm.Hq, prm.B);
+  // persistent: one CTA per SM (or fewer when there are fewer work units)
+  const long long units = (long long)prm.n_qblocks * prm.Hq * prm.B;
+  const int sms = sm_count();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  dim3 grid((unsigned)(units < sms ? units : sms));
   kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, prm);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -135,7 +153,7 @@ int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float*
   if (!make_tile_map(&mq, q, d, Sq, (long long)B * Hq) ||
       !make_tile_map(&mk, k, d, Sk, (long long)B * Hkv) ||
       !make_tile_map(&mv, v, d, Sk, (long long)B * Hkv) ||
-      !make_tile_map(&mo, o, d, Sq, (long long)B * Hq))
+      !make_tile_map(&mo, o, d, Sq, (long long)B * Hq, 32))
     return ATTN_ERR_CUDA;
   PrefillParams prm;
   prm.lse = lse;

@@ -6,15 +6,21 @@
 // "Online softmax"; "Attention 算子加速史", section 1.3), so the S_q x S_k
 // score matrix never leaves the chip.
 //
-// Organisation of one CTA (320 threads, one CTA per SM):
-//   * It owns two 128-row query tiles of one (batch, query head): rows
-//     [256*qb, 256*qb + 256).  The loop order is query tile outside, KV tiles
-//     inside, with the output accumulator resident on chip until one final
-//     write ("Attention 算子加速史", section 2.1).
-//   * warp 0, lane 0  -- TMA producer: the two Q tiles once, then K_j and V_j
-//     128-key tiles into a STAGES-deep ring guarded by full/empty mbarriers
-//     ("Attention 算子加速史", section 3.3: producer warp, mbarriers, double
-//     buffering; TMA as in section 3.1).  No multicast.
+// Persistent organisation: one CTA per SM (320 threads) walks a list of work
+// units.  A unit is two 128-row query tiles of one (batch, query head): rows
+// [256*qb, 256*qb + 256).  Units are ranked heaviest first (largest causal
+// q-block first) and dealt to the CTAs in a back-and-forth ("snake") order so
+// that every SM gets about the same number of KV tiles.  Inside a unit the
+// loop order is query tile outside, KV tiles inside, with the accumulator
+// resident on chip until one final write ("Attention 算子加速史", section 2.1).
+//
+//   * warp 0, lane 0  -- TMA producer: each unit's two Q tiles, then K_j and
+//     V_j 128-key tiles into a STAGES-deep ring guarded by full/empty
+//     mbarriers ("Attention 算子加速史", section 3.3: a producer warp,
+//     mbarriers and multi-buffering; TMA as in section 3.1).  A Q tile of the
+//     next unit is loaded as soon as the last MMA reading the current one
+//     retires, and K/V of the next unit stream in while the current unit
+//     finishes.  No multicast.
 //   * warp 1, lane 0  -- tcgen05 MMA issuer: S_i = Q_i K_j^T (SS form, both
 //     operands in shared memory) and O_i += P_i V_j (TS form, P read from
 //     tensor memory), ping-ponging between the two query tiles so that the
@@ -26,8 +32,9 @@
 //     Kernel", section "FlashAttention 的稳定基础"), update the running max,
 //     write P = 2^(S*scale*log2e - m) as bf16 back into TMEM over the S
 //     columns, rescale O in TMEM when the max moved, and hand P to the MMA
-//     warp.  The division by l happens once in the epilogue ("Attention
-//     算子加速史", section 2.2).
+//     warp.  The division by l happens once per unit ("Attention 算子加速史",
+//     section 2.2): each warp normalises its 32 rows, stages them (64 columns
+//     at a time) in its own 4 KB shared-memory buffer and stores them by TMA.
 //   * Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0 and O_1
 //     after them (d columns each); P_i aliases the first 64 columns of S_i.
 //
@@ -61,13 +68,16 @@ struct PrefillCfg {
   static constexpr int TILE_BYTES = BM * D * 2;  // bf16 128 x D tile (Q, K or V)
   static constexpr int CB_BYTES = 128 * 128;     // one 64-column block of a 128-row tile
   static constexpr int NCB = D / 64;             // 64-column blocks per tile
+  static constexpr int STG_BYTES = 32 * 128;     // per-warp epilogue staging: 32 rows x 64 cols
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_V + STAGES * TILE_BYTES;
+  static constexpr int OFF_STG = OFF_V + STAGES * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_STG + 8 * STG_BYTES;
   // barrier indices
-  static constexpr int B_QFULL = 0;
-  static constexpr int B_KFULL = 1;
+  static constexpr int B_QFULL = 0;                  // 2: Q_i landed
+  static constexpr int B_QFREE = B_QFULL + 2;        // 2: last MMA reading Q_i retired
+  static constexpr int B_KFULL = B_QFREE + 2;
   static constexpr int B_KEMPTY = B_KFULL + STAGES;
   static constexpr int B_VFULL = B_KEMPTY + STAGES;
   static constexpr int B_VEMPTY = B_VFULL + STAGES;
@@ -87,15 +97,50 @@ struct PrefillCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
-// Number of 128-key tiles query tile i (rows [row0, row0+127]) must visit, and
-// the largest key index visible to its first row (tiles beyond that need the
-// per-element predicate).
+// Number of 128-key tiles the query tile with first row `row0` must visit
+// (0 when the tile is past Sq or none of its rows sees a key).
 __device__ __forceinline__ int prefill_num_kv_tiles(int row0, int Sq, int klen, bool causal) {
   if (row0 >= Sq) return 0;
   const int last_row = min(row0 + 127, Sq - 1);
   long long lim = (long long)klen - 1;
   if (causal) lim = min(lim, (long long)last_row + (long long)klen - Sq);
   return lim < 0 ? 0 : (int)(lim / 128) + 1;
+}
+
+// One work unit: query rows [256*qb, 256*qb + 256) of head hq in sequence b.
+struct PrefillUnit {
+  int qb, hq, b;
+  int klen;        // visible keys of the sequence
+  int row0[2];     // first row of each query tile
+  int nkv[2];      // KV tiles each query tile visits
+};
+
+// The k-th unit of this CTA, or false when the CTA has no more work.  Ranks
+// are ordered heaviest first (q-blocks descending, heads inner) and dealt
+// back and forth across the CTAs: rank k*G + c for even k, k*G + G-1-c for odd.
+template <bool CAUSAL>
+__device__ __forceinline__ bool prefill_unit(const PrefillParams& p, int k, PrefillUnit& u) {
+  const long long G = gridDim.x;
+  const long long c = blockIdx.x;
+  const long long r = (long long)k * G + ((k & 1) ? (G - 1 - c) : c);
+  const long long HB = (long long)p.Hq * p.B;
+  if (r >= (long long)p.n_qblocks * HB) return false;
+  u.qb = p.n_qblocks - 1 - (int)(r / HB);
+  const int rem = (int)(r % HB);
+  u.hq = rem % p.Hq;
+  u.b = rem / p.Hq;
+  int klen = p.Sk;
+  if (p.k_lens != nullptr) {
+    klen = p.k_lens[u.b];
+    if (klen < 0 || klen > p.Sk) klen = klen < 0 ? 0 : p.Sk;  // flagged by the softmax warps
+  }
+  u.klen = klen;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    u.row0[i] = u.qb * 256 + i * 128;
+    u.nkv[i] = prefill_num_kv_tiles(u.row0[i], p.Sq, klen, CAUSAL);
+  }
+  return true;
 }
 
 template <int D, bool CAUSAL>
@@ -116,42 +161,20 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit: heaviest causal blocks first (longest processing time first)
-  const int qb = p.n_qblocks - 1 - (int)blockIdx.x;
-  const int hq = blockIdx.y;
-  const int b = blockIdx.z;
-  const int kvh = hq / p.group;
-  int klen = p.Sk;
-  if (p.k_lens != nullptr) {
-    klen = p.k_lens[b];
-    if (klen < 0 || klen > p.Sk) {
-      if (threadIdx.x == 0) flag_device_error(kDevErrBadLength);
-      klen = klen < 0 ? 0 : p.Sk;
-    }
-  }
-  // per query tile i in {0, 1}: first row and number of KV tiles to visit
-  const int row0_0 = qb * 256, row0_1 = qb * 256 + 128;
-  const int nkv_0 = prefill_num_kv_tiles(row0_0, p.Sq, klen, CAUSAL);
-  const int nkv_1 = prefill_num_kv_tiles(row0_1, p.Sq, klen, CAUSAL);
-  auto row0 = [&](int i) { return i ? row0_1 : row0_0; };
-  auto nkv = [&](int i) { return i ? nkv_1 : nkv_0; };
-  const int n_max = max(nkv_0, nkv_1);
-  const int q_head_row = b * p.Hq + hq;   // z coordinate in the Q / O maps
-  const int kv_head_row = b * p.Hkv + kvh;
-
   // ---- setup: barriers (thread 0), tensor memory (warp 1)
   if (threadIdx.x == 0) {
-    mbar_init(bar(C::B_QFULL), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(C::B_QFULL + i), 1);
+      mbar_init(bar(C::B_QFREE + i), 1);
+      mbar_init(bar(C::B_SFULL + i), 1);
+      mbar_init(bar(C::B_PFULL + i), 128);
+      mbar_init(bar(C::B_OFULL + i), 1);
+    }
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(bar(C::B_KFULL + s), 1);
       mbar_init(bar(C::B_KEMPTY + s), 1);
       mbar_init(bar(C::B_VFULL + s), 1);
       mbar_init(bar(C::B_VEMPTY + s), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(C::B_SFULL + i), 1);
-      mbar_init(bar(C::B_PFULL + i), 128);
-      mbar_init(bar(C::B_OFULL + i), 1);
     }
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
@@ -169,54 +192,66 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 0) {
     // ======================= TMA producer =======================
-    if (lane == 0 && n_max > 0) {
+    if (lane == 0) {
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_v);
-      uint32_t q_bytes = 0;
-#pragma unroll
-      for (int i = 0; i < 2; ++i)
-        if (nkv(i) > 0) q_bytes += C::TILE_BYTES;
-      mbar_arrive_expect_tx(bar(C::B_QFULL), q_bytes);
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        if (nkv(i) == 0) continue;
+      uint32_t q_loads0 = 0, q_loads1 = 0;  // Q tiles loaded so far, per tile slot
+      uint32_t kv = 0;                      // K/V tiles issued so far (ring position)
+      bool ok = true;
+      auto load_q = [&](const PrefillUnit& u, int i) -> bool {
+        uint32_t& n = i ? q_loads1 : q_loads0;
+        if (n > 0 && !mbar_wait(bar(C::B_QFREE + i), (n - 1) & 1u, abort_flag)) return false;
+        mbar_arrive_expect_tx(bar(C::B_QFULL + i), C::TILE_BYTES);
         for (int cb = 0; cb < C::NCB; ++cb)
           tma_load_3d(sbase + C::OFF_Q + i * C::TILE_BYTES + cb * C::CB_BYTES, &tm_q,
-                      bar(C::B_QFULL), 64 * cb, row0(i), q_head_row);
-      }
-      int loaded = 0;  // KV tiles whose loads were issued
-      for (int j = 0; j < n_max; ++j) {
-        const int s = j % C::STAGES;
-        const uint32_t ph = (uint32_t)(j / C::STAGES) & 1u;
-        if (!mbar_wait(bar(C::B_KEMPTY + s), ph ^ 1u, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::TILE_BYTES);
-        for (int cb = 0; cb < C::NCB; ++cb)
-          tma_load_3d(sbase + C::OFF_K + s * C::TILE_BYTES + cb * C::CB_BYTES, &tm_k,
-                      bar(C::B_KFULL + s), 64 * cb, j * 128, kv_head_row);
-        if (!mbar_wait(bar(C::B_VEMPTY + s), ph ^ 1u, abort_flag)) {
-          loaded = -(j + 1);  // K_j issued, V_j not
-          break;
+                      bar(C::B_QFULL + i), 64 * cb, u.row0[i], u.b * p.Hq + u.hq);
+        ++n;
+        return true;
+      };
+      PrefillUnit u;
+      for (int k = 0; ok && prefill_unit<CAUSAL>(p, k, u); ++k) {
+        const int n_max = max(u.nkv[0], u.nkv[1]);
+        const int kv_row = u.b * p.Hkv + u.hq / p.group;
+        // Q_0 first (its slot frees first under a causal mask), then the first
+        // K tile, then Q_1, so that no wait on Q_1 holds back the K/V stream.
+        if (u.nkv[0] > 0 && !(ok = load_q(u, 0))) break;
+        for (int j = 0; j < n_max; ++j, ++kv) {
+          const int s = kv % C::STAGES;
+          const uint32_t ph = (kv / C::STAGES) & 1u;
+          if (!(ok = mbar_wait(bar(C::B_KEMPTY + s), ph ^ 1u, abort_flag))) break;
+          mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::TILE_BYTES);
+          for (int cb = 0; cb < C::NCB; ++cb)
+            tma_load_3d(sbase + C::OFF_K + s * C::TILE_BYTES + cb * C::CB_BYTES, &tm_k,
+                        bar(C::B_KFULL + s), 64 * cb, j * 128, kv_row);
+          if (j == 0 && u.nkv[1] > 0 && !(ok = load_q(u, 1))) {
+            ++kv;  // K_0 of this unit was issued
+            break;
+          }
+          if (!(ok = mbar_wait(bar(C::B_VEMPTY + s), ph ^ 1u, abort_flag))) {
+            ++kv;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE_BYTES);
+          for (int cb = 0; cb < C::NCB; ++cb)
+            tma_load_3d(sbase + C::OFF_V + s * C::TILE_BYTES + cb * C::CB_BYTES, &tm_v,
+                        bar(C::B_VFULL + s), 64 * cb, j * 128, kv_row);
         }
-        mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE_BYTES);
-        for (int cb = 0; cb < C::NCB; ++cb)
-          tma_load_3d(sbase + C::OFF_V + s * C::TILE_BYTES + cb * C::CB_BYTES, &tm_v,
-                      bar(C::B_VFULL + s), 64 * cb, j * 128, kv_head_row);
-        loaded = j + 1;
       }
       // Drain: never leave the CTA with copies still landing in shared memory.
-      mbar_wait(bar(C::B_QFULL), 0, nullptr);
-      const int nk = loaded >= 0 ? loaded : -loaded;
-      const int nv = loaded >= 0 ? loaded : -loaded - 1;
-      for (int j = (nk > C::STAGES ? nk - C::STAGES : 0); j < nk; ++j)
-        mbar_wait(bar(C::B_KFULL + j % C::STAGES), (uint32_t)(j / C::STAGES) & 1u, nullptr);
-      for (int j = (nv > C::STAGES ? nv - C::STAGES : 0); j < nv; ++j)
-        mbar_wait(bar(C::B_VFULL + j % C::STAGES), (uint32_t)(j / C::STAGES) & 1u, nullptr);
+      // (On an abort the last K may lack its V; waiting on a V phase that was
+      // never armed would only run into the time limit, so V is skipped then.)
+      if (q_loads0 > 0) mbar_wait(bar(C::B_QFULL + 0), (q_loads0 - 1) & 1u, nullptr);
+      if (q_loads1 > 0) mbar_wait(bar(C::B_QFULL + 1), (q_loads1 - 1) & 1u, nullptr);
+      for (uint32_t j = (kv > C::STAGES ? kv - C::STAGES : 0); j < kv; ++j) {
+        mbar_wait(bar(C::B_KFULL + j % C::STAGES), (j / C::STAGES) & 1u, nullptr);
+        if (ok) mbar_wait(bar(C::B_VFULL + j % C::STAGES), (j / C::STAGES) & 1u, nullptr);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ======================= tcgen05 MMA issuer =======================
-    if (lane == 0 && n_max > 0) {
+    if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
       // S_i = Q_i K^T over d in steps of 16 (32 bytes inside a 128-byte swizzled row,
@@ -242,46 +277,67 @@ __global__ void __launch_bounds__(320, 1)
                   (accumulate || ks > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(bar(C::B_QFULL), 0, abort_flag);
-      if (ok) ok = mbar_wait(bar(C::B_KFULL + 0), 0, abort_flag);
-      if (ok) {
-        tc_fence_after_sync();
+      uint32_t kv = 0;                  // ring position
+      uint32_t q_waits0 = 0, q_waits1 = 0;  // Q_FULL phases consumed per tile slot
+      uint32_t p_waits0 = 0, p_waits1 = 0;  // P_FULL phases consumed per tile slot
+      bool ok = true;
+      PrefillUnit u;
+      for (int k = 0; ok && prefill_unit<CAUSAL>(p, k, u); ++k) {
+        const int n_max = max(u.nkv[0], u.nkv[1]);
+        if (n_max == 0) continue;
+        // prologue: S_i(0) for each participating tile
+        {
+          const int s = kv % C::STAGES;
+          if (!(ok = mbar_wait(bar(C::B_KFULL + s), (kv / C::STAGES) & 1u, abort_flag))) break;
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          if (nkv(i) == 0) continue;
-          issue_qk(i, 0);
-          umma_commit(bar(C::B_SFULL + i));
-        }
-        umma_commit(bar(C::B_KEMPTY + 0));
-      }
-      for (int j = 0; ok && j < n_max; ++j) {
-        const int s = j % C::STAGES;
-        const uint32_t ph = (uint32_t)(j / C::STAGES) & 1u;
-        const int s1 = (j + 1) % C::STAGES;
-        const uint32_t ph1 = (uint32_t)((j + 1) / C::STAGES) & 1u;
-        if (!(ok = mbar_wait(bar(C::B_VFULL + s), ph, abort_flag))) break;
-        bool k_next = false;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          if (!ok) break;
-          if (j >= nkv(i)) continue;
-          if (!(ok = mbar_wait(bar(C::B_PFULL + i), (uint32_t)j & 1u, abort_flag))) break;
-          tc_fence_after_sync();
-          issue_pv(i, s, j > 0);
-          if (j + 1 < nkv(i)) {
-            if (!k_next) {
-              if (!(ok = mbar_wait(bar(C::B_KFULL + s1), ph1, abort_flag))) break;
-              tc_fence_after_sync();
-              k_next = true;
-            }
-            issue_qk(i, s1);
+          for (int i = 0; i < 2; ++i) {
+            if (!ok) break;
+            if (u.nkv[i] == 0) continue;
+            uint32_t& qw = i ? q_waits1 : q_waits0;
+            if (!(ok = mbar_wait(bar(C::B_QFULL + i), qw & 1u, abort_flag))) break;
+            ++qw;
+            tc_fence_after_sync();
+            issue_qk(i, s);
             umma_commit(bar(C::B_SFULL + i));
-          } else {
-            umma_commit(bar(C::B_OFULL + i));
+            if (u.nkv[i] == 1) umma_commit(bar(C::B_QFREE + i));  // Q_i read for the last time
           }
+          if (!ok) break;
+          umma_commit(bar(C::B_KEMPTY + s));
         }
-        umma_commit(bar(C::B_VEMPTY + s));
-        if (k_next) umma_commit(bar(C::B_KEMPTY + s1));
+        for (int j = 0; ok && j < n_max; ++j) {
+          const uint32_t idx = kv + j;
+          const int s = idx % C::STAGES;
+          const int s1 = (idx + 1) % C::STAGES;
+          if (!(ok = mbar_wait(bar(C::B_VFULL + s), (idx / C::STAGES) & 1u, abort_flag))) break;
+          bool k_next = false;
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            if (!ok) break;
+            if (j >= u.nkv[i]) continue;
+            uint32_t& pw = i ? p_waits1 : p_waits0;
+            if (!(ok = mbar_wait(bar(C::B_PFULL + i), pw & 1u, abort_flag))) break;
+            ++pw;
+            tc_fence_after_sync();
+            issue_pv(i, s, j > 0);
+            if (j + 1 < u.nkv[i]) {
+              if (!k_next) {
+                if (!(ok = mbar_wait(bar(C::B_KFULL + s1), ((idx + 1) / C::STAGES) & 1u,
+                                     abort_flag)))
+                  break;
+                tc_fence_after_sync();
+                k_next = true;
+              }
+              issue_qk(i, s1);
+              umma_commit(bar(C::B_SFULL + i));
+              if (j + 2 == u.nkv[i]) umma_commit(bar(C::B_QFREE + i));
+            } else {
+              umma_commit(bar(C::B_OFULL + i));
+            }
+          }
+          umma_commit(bar(C::B_VEMPTY + s));
+          if (k_next) umma_commit(bar(C::B_KEMPTY + s1));
+        }
+        kv += n_max;
       }
       // Drain: every MMA issued above has completed before TMEM is released.
       umma_commit(bar(C::B_DRAIN));
@@ -290,167 +346,196 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     // ======================= softmax warpgroups =======================
-    const int i = (warp - 2) >> 2;       // query tile of this warpgroup
+    const int i = (warp - 2) >> 2;       // query tile slot of this warpgroup
     const int quarter = warp & 3;        // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;   // row within the tile
-    const int row = row0(i) + r;
-    const int n = nkv(i);
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t t_s = tmem + lane_off + C::tmem_s(i);
     const uint32_t t_o = tmem + lane_off + C::tmem_o(i);
-    const long long koff = (long long)klen - p.Sq;
-    // largest visible key of this row, and of the tile's first row
-    long long lim_row = (long long)klen - 1;
-    long long lim_tile = lim_row;
-    if (CAUSAL) {
-      lim_row = min(lim_row, (long long)row + koff);
-      lim_tile = min(lim_tile, (long long)row0(i) + koff);
-    }
+    const uint32_t stg = sbase + C::OFF_STG + (warp - 2) * C::STG_BYTES;
+    uint8_t* stg_ptr = sbase_ptr + C::OFF_STG + (warp - 2) * C::STG_BYTES;
     float c2 = p.scale_log2;
     const bool scale_pos = c2 > 0.f;
     if (!scale_pos) c2 = 1.f;  // scores are pre-multiplied below instead
-    float m_run = -INFINITY;   // exponent base (log2 units)
-    float l_run = 0.f;         // sum of P (f32)
-    float lr_run = 0.f;        // sum of bf16(P)
+    uint32_t s_waits = 0, o_waits = 0;
+    bool stores_pending = false;
     bool ok = true;
+    PrefillUnit u;
+    for (int k = 0; ok && prefill_unit<CAUSAL>(p, k, u); ++k) {
+      const int row0 = i ? u.row0[1] : u.row0[0];
+      if (row0 >= p.Sq) continue;  // this tile slot holds no rows in this unit
+      const int n = i ? u.nkv[1] : u.nkv[0];
+      const int row = row0 + r;
+      const int q_head_row = u.b * p.Hq + u.hq;
+      if (p.k_lens != nullptr && r == 0) {
+        const int kl = p.k_lens[u.b];
+        if (kl < 0 || kl > p.Sk) flag_device_error(kDevErrBadLength);
+      }
+      // largest visible key of this row, and of the tile's first row
+      const long long koff = (long long)u.klen - p.Sq;
+      long long lim_row = (long long)u.klen - 1;
+      long long lim_tile = lim_row;
+      if (CAUSAL) {
+        lim_row = min(lim_row, (long long)row + koff);
+        lim_tile = min(lim_tile, (long long)row0 + koff);
+      }
+      float m_run = -INFINITY;   // exponent base (log2 units)
+      float l_run = 0.f;         // sum of P (f32)
+      float lr_run = 0.f;        // sum of bf16(P)
 
-    for (int j = 0; j < n; ++j) {
-      if (!(ok = mbar_wait_warp(bar(C::B_SFULL + i), (uint32_t)j & 1u, abort_flag))) break;
-      tc_fence_after_sync();
-      float s[128];
-      {
-        uint32_t u0[32], u1[32], u2[32], u3[32];
-        tmem_ld32(t_s, u0);
-        tmem_ld32(t_s + 32, u1);
-        tmem_ld32(t_s + 64, u2);
-        tmem_ld32(t_s + 96, u3);
-        tmem_ld_wait();
-        reg_fence32(u0);
-        reg_fence32(u1);
-        reg_fence32(u2);
-        reg_fence32(u3);
+      for (int j = 0; j < n; ++j) {
+        if (!(ok = mbar_wait_warp(bar(C::B_SFULL + i), s_waits & 1u, abort_flag))) break;
+        ++s_waits;
+        tc_fence_after_sync();
+        float s[128];
+        {
+          uint32_t u0[32], u1[32], u2[32], u3[32];
+          tmem_ld32(t_s, u0);
+          tmem_ld32(t_s + 32, u1);
+          tmem_ld32(t_s + 64, u2);
+          tmem_ld32(t_s + 96, u3);
+          tmem_ld_wait();
+          reg_fence32(u0);
+          reg_fence32(u1);
+          reg_fence32(u2);
+          reg_fence32(u3);
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          s[k] = __uint_as_float(u0[k]);
-          s[32 + k] = __uint_as_float(u1[k]);
-          s[64 + k] = __uint_as_float(u2[k]);
-          s[96 + k] = __uint_as_float(u3[k]);
+          for (int e = 0; e < 32; ++e) {
+            s[e] = __uint_as_float(u0[e]);
+            s[32 + e] = __uint_as_float(u1[e]);
+            s[64 + e] = __uint_as_float(u2[e]);
+            s[96 + e] = __uint_as_float(u3[e]);
+          }
         }
-      }
-      if ((long long)j * 128 + 127 > lim_tile) {
-        // boundary tile: per-element predicate
-        const long long lim_local = lim_row - (long long)j * 128;
+        if ((long long)j * 128 + 127 > lim_tile) {
+          // boundary tile: per-element predicate, in 32-bit once clamped to the tile
+          const long long ll = lim_row - (long long)j * 128;
+          const int lim_local = ll < -1 ? -1 : (ll > 127 ? 127 : (int)ll);
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if ((long long)c > lim_local) s[c] = -INFINITY;
-      }
-      if (!scale_pos) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          s[c] = (s[c] == -INFINITY) ? -INFINITY : s[c] * p.scale_log2;
-      }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, s[c]);
-        mx1 = fmaxf(mx1, s[c + 1]);
-        mx2 = fmaxf(mx2, s[c + 2]);
-        mx3 = fmaxf(mx3, s[c + 3]);
-      }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c2;
-      float alpha = 1.f;
-      if (m_tile > m_run + 8.f) {  // also true for the first finite max
-        alpha = ex2(m_run - m_tile);
-        m_run = m_tile;
-      }
-      const float base = (m_run == -INFINITY) ? 0.f : m_run;
-      // Two row sums: l over the f32 P (gives the LSE) and lr over the
-      // bf16-rounded P that the PV MMA consumes (normalises O, so that the
-      // weights applied to V sum to one exactly as used).
-      float l0 = 0.f, l1 = 0.f;
-      uint64_t r01 = 0ull, r23 = 0ull;  // f32x2 partial sums of the rounded P
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-          const int cc = 64 * half + c;
-          const float p0 = ex2(fmaf(s[cc], c2, -base));
-          const float p1 = ex2(fmaf(s[cc + 1], c2, -base));
-          const float p2 = ex2(fmaf(s[cc + 2], c2, -base));
-          const float p3 = ex2(fmaf(s[cc + 3], c2, -base));
-          l0 += p0 + p1;
-          l1 += p2 + p3;
-          pk[c / 2] = pack_bf16x2(p0, p1);
-          pk[c / 2 + 1] = pack_bf16x2(p2, p3);
-          r01 = add_f32x2(r01, bf16x2_to_f32x2(pk[c / 2]));
-          r23 = add_f32x2(r23, bf16x2_to_f32x2(pk[c / 2 + 1]));
+          for (int c = 0; c < 128; ++c)
+            if (c > lim_local) s[c] = -INFINITY;
         }
-        tmem_st32(t_s + 32 * half, pk);  // P columns [32*half, 32*half + 32)
-      }
-      l_run = l_run * alpha + (l0 + l1);
-      lr_run = lr_run * alpha + (sum_f32x2(r01) + sum_f32x2(r23));
-      // Rescale the accumulator when any row of this warp moved its base.  The
-      // MMA that last wrote O_i completed before S_i(j) was signalled.
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!scale_pos) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            s[c] = (s[c] == -INFINITY) ? -INFINITY : s[c] * p.scale_log2;
+        }
+        // row max: four chains of 3-input maxes
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int c = 4; c < 128; c += 8) {
+          mx0 = max3f(mx0, s[c], s[c + 1]);
+          mx1 = max3f(mx1, s[c + 2], s[c + 3]);
+          mx2 = max3f(mx2, s[c + 4], s[c + 5]);
+          mx3 = max3f(mx3, s[c + 6], s[c + 7]);
+        }
+        const float m_tile = max3f(fmaxf(mx0, mx1), mx2, mx3) * c2;
+        float alpha = 1.f;
+        if (m_tile > m_run + 8.f) {  // also true for the first finite max
+          alpha = ex2(m_run - m_tile);
+          m_run = m_tile;
+        }
+        const float base = (m_run == -INFINITY) ? 0.f : m_run;
+        // P = 2^(s*c2 - base) two columns at a time (packed f32x2 FMA), two row
+        // sums: l over the f32 P (gives the LSE) and lr over the bf16-rounded P
+        // that the PV MMA consumes (normalises O, so the weights applied to V
+        // sum to one exactly as used).
+        const uint64_t c2x2 = f32x2(c2, c2);
+        const uint64_t nbx2 = f32x2(-base, -base);
+        uint64_t la = 0ull, lb = 0ull;                 // f32x2 partial sums of P
+        float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;  // partial sums of bf16(P)
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int cc = 64 * half + 2 * e;
+            float x0, x1, x2, x3;
+            split_f32x2(fma_f32x2(f32x2(s[cc], s[cc + 1]), c2x2, nbx2), x0, x1);
+            split_f32x2(fma_f32x2(f32x2(s[cc + 2], s[cc + 3]), c2x2, nbx2), x2, x3);
+            const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+            pk[e] = pack_bf16x2(p0, p1);
+            pk[e + 1] = pack_bf16x2(p2, p3);
+            la = add_f32x2(la, f32x2(p0, p1));
+            lb = add_f32x2(lb, f32x2(p2, p3));
+            add_bf16x2_halves(pk[e], r0, r1);
+            add_bf16x2_halves(pk[e + 1], r2, r3);
+          }
+          tmem_st32(t_s + 32 * half, pk);  // P columns [32*half, 32*half + 32)
+        }
+        l_run = l_run * alpha + (sum_f32x2(la) + sum_f32x2(lb));
+        lr_run = lr_run * alpha + ((r0 + r1) + (r2 + r3));
+        // Rescale the accumulator when any row of this warp moved its base.  The
+        // MMA that last wrote O_i completed before S_i(j) was signalled.
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
-          uint32_t u[32];
-          tmem_ld32_sync(t_o + c, u);
+          for (int c = 0; c < D; c += 32) {
+            uint32_t v[32];
+            tmem_ld32_sync(t_o + c, v);
 #pragma unroll
-          for (int k = 0; k < 32; ++k) u[k] = __float_as_uint(__uint_as_float(u[k]) * alpha);
-          tmem_st32(t_o + c, u);
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+            tmem_st32(t_o + c, v);
+          }
         }
+        tmem_st_wait();
+        tc_fence_before_sync();
+        mbar_arrive(bar(C::B_PFULL + i));
       }
-      tmem_st_wait();
-      tc_fence_before_sync();
-      mbar_arrive(bar(C::B_PFULL + i));
-    }
+      if (!ok) break;
 
-    // ---- epilogue: O = o / l -> bf16, staged through this tile's Q buffer
-    // (free once its last MMA completed) and stored with TMA; LSE per row.
-    if (row0(i) < p.Sq) {
-      if (n > 0 && ok) ok = mbar_wait_warp(bar(C::B_OFULL + i), 0, abort_flag);
+      // ---- epilogue: O = o / l -> bf16; each warp stages its 32 rows, 64
+      // columns at a time, in its own buffer and stores them by TMA; LSE per row.
+      const bool has_o = n > 0;
+      if (has_o) {
+        if (!(ok = mbar_wait_warp(bar(C::B_OFULL + i), o_waits & 1u, abort_flag))) break;
+        ++o_waits;
+      }
       tc_fence_after_sync();
-      const bool has_o = (n > 0) && ok;
       const float inv = (lr_run > 0.f) ? (1.f / lr_run) : 0.f;
-      uint8_t* stage = sbase_ptr + C::OFF_Q + i * C::TILE_BYTES;
+      const bool warp_has_rows = row0 + quarter * 32 < p.Sq;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        uint32_t u[32];
-        if (has_o) {
-          tmem_ld32_sync(t_o + c, u);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) u[k] = 0u;
+      for (int cb = 0; cb < C::NCB; ++cb) {
+        if (stores_pending) {  // the previous store must have read the buffer
+          if (lane == 0) tma_store_wait_read_all();
+          __syncwarp();
+          stores_pending = false;
         }
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int dcol = c + 8 * q4;        // first of 8 columns in this 16-byte chunk
-          const int cb = dcol >> 6;           // 64-column block
-          const int chunk = (dcol & 63) >> 3; // 16-byte chunk within the 128-byte row
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(u[8 * q4 + 0]) * inv, __uint_as_float(u[8 * q4 + 1]) * inv);
-          w.y = pack_bf16x2(__uint_as_float(u[8 * q4 + 2]) * inv, __uint_as_float(u[8 * q4 + 3]) * inv);
-          w.z = pack_bf16x2(__uint_as_float(u[8 * q4 + 4]) * inv, __uint_as_float(u[8 * q4 + 5]) * inv);
-          w.w = pack_bf16x2(__uint_as_float(u[8 * q4 + 6]) * inv, __uint_as_float(u[8 * q4 + 7]) * inv);
-          *reinterpret_cast<uint4*>(stage + cb * C::CB_BYTES + r * 128 +
-                                    ((chunk ^ (r & 7)) << 4)) = w;
+        for (int half = 0; half < 2; ++half) {
+          uint32_t v[32];
+          if (has_o) {
+            tmem_ld32_sync(t_o + 64 * cb + 32 * half, v);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          }
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int chunk = 4 * half + q4;  // 16-byte chunk within the 128-byte row
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * inv, __uint_as_float(v[8 * q4 + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv, __uint_as_float(v[8 * q4 + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv, __uint_as_float(v[8 * q4 + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv, __uint_as_float(v[8 * q4 + 7]) * inv);
+            *reinterpret_cast<uint4*>(stg_ptr + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = w;
+          }
         }
-      }
-      fence_proxy_async_smem();
-      named_barrier_sync(1 + i, 128);
-      if (warp == 2 + 4 * i && lane == 0 && !*abort_flag) {
-        for (int cb = 0; cb < C::NCB; ++cb)
-          tma_store_3d(&tm_o, smem_u32(stage) + cb * C::CB_BYTES, 64 * cb, row0(i), q_head_row);
-        tma_store_commit();
-        tma_store_wait_read_all();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && warp_has_rows && !*abort_flag) {
+          tma_store_3d(&tm_o, stg, 64 * cb, row0 + quarter * 32, q_head_row);
+          tma_store_commit();
+        }
+        stores_pending = true;
       }
       if (p.lse != nullptr && row < p.Sq) {
         const float lse = (l_run > 0.f) ? (m_run + lg2(l_run)) * 0.69314718055994531f : -INFINITY;
         p.lse[(size_t)q_head_row * p.Sq + row] = lse;
       }
     }
+    // all of this warp's output stores complete before the CTA exits
+    if (lane == 0) tma_store_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before_sync();
