@@ -6,7 +6,7 @@
 // "Online softmax"; "Attention 算子加速史", section 1.3), so the S_q x S_k
 // score matrix never leaves the chip.
 //
-// Persistent organisation: one CTA per SM (320 threads) walks a list of work
+// Persistent organisation: one CTA per SM (384 threads) walks a list of work
 // units.  A unit is two 128-row query tiles of one (batch, query head): rows
 // [256*qb, 256*qb + 256).  Units are ranked heaviest first (largest causal
 // q-block first) and dealt to the CTAs in a back-and-forth ("snake") order so
@@ -25,7 +25,8 @@
 //     operands in shared memory) and O_i += P_i V_j (TS form, P read from
 //     tensor memory), ping-ponging between the two query tiles so that the
 //     tensor core works on one tile while the other tile's softmax runs.
-//   * warps 2-5 and 6-9 -- one softmax warpgroup per query tile; thread r of
+//   * warps 2-3       -- idle (they complete the first warpgroup).
+//   * warps 4-7 and 8-11 -- one softmax warpgroup per query tile; thread r of
 //     a warpgroup owns row r (= TMEM lane r).  Per KV tile: load the S row
 //     from TMEM, apply the causal / key-length predicate (boundary tiles
 //     only; tiles that are wholly masked are never visited -- "Attention
@@ -37,6 +38,10 @@
 //     at a time) in its own 4 KB shared-memory buffer and stores them by TMA.
 //   * Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0 and O_1
 //     after them (d columns each); P_i aliases the first 64 columns of S_i.
+//   * Registers: the kernel is built for 168 per thread (384 x 168 = 64512);
+//     the producer/MMA warpgroup gives 112 of each thread's registers back
+//     (setmaxnreg 56) and each softmax warpgroup takes 56 more (224):
+//     128 x (56 + 224 + 224) = 64512, so the increase never waits.
 //
 // Rescaling is lazy: the max used as the exponent base only moves when the
 // new row max exceeds it by more than 8 (log2 units), so P <= 2^8.  The final
@@ -92,7 +97,12 @@ struct PrefillCfg {
   // TMEM columns of S_i (P_i aliases its first 64) and of O_i
   __host__ __device__ static constexpr uint32_t tmem_s(int i) { return i ? 128u : 0u; }
   __host__ __device__ static constexpr uint32_t tmem_o(int i) { return i ? 256u + D : 256u; }
-  static constexpr int NUM_THREADS = 320;
+  static constexpr int NUM_THREADS = 384;
+  static constexpr uint32_t REGS_LAUNCH = 168;  // = 65536 / 384 rounded down to a multiple of 8
+  static constexpr uint32_t REGS_PRODUCER = 56;
+  static constexpr uint32_t REGS_SOFTMAX = 224;
+  static_assert(128 * (REGS_PRODUCER + 2 * REGS_SOFTMAX) <= NUM_THREADS * REGS_LAUNCH,
+                "register reallocation must fit the launch allocation");
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -144,7 +154,7 @@ __device__ __forceinline__ bool prefill_unit(const PrefillParams& p, int k, Pref
 }
 
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                               const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v,
@@ -190,7 +200,12 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  // Each register reallocation sits inside the branch of the warpgroup that
+  // makes it, so that the compiler sees every role's code reachable only under
+  // its own register budget.
+  if (warp < 4) {
+    warpgroup_reg_dealloc<C::REGS_PRODUCER>();
+    if (warp == 0) {
     // ======================= TMA producer =======================
     if (lane == 0) {
       tma_prefetch_map(&tm_q);
@@ -257,8 +272,8 @@ __global__ void __launch_bounds__(320, 1)
       // S_i = Q_i K^T over d in steps of 16 (32 bytes inside a 128-byte swizzled row,
       // 64-column blocks 16 KB apart).
       auto issue_qk = [&](int i, int stage) {
-        const uint32_t qa = sbase + C::OFF_Q + i * C::TILE_BYTES;
-        const uint32_t ka = sbase + C::OFF_K + stage * C::TILE_BYTES;
+        const uint32_t qa = opaque_u32(sbase + C::OFF_Q + i * C::TILE_BYTES);
+        const uint32_t ka = opaque_u32(sbase + C::OFF_K + stage * C::TILE_BYTES);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * C::CB_BYTES + (ks & 3) * 32;
@@ -269,10 +284,11 @@ __global__ void __launch_bounds__(320, 1)
       // O_i (+)= P_i V over the 128 keys in steps of 16: P from TMEM (8 columns
       // per step), V as an MN-major operand (16 keys = 2048 bytes per step).
       auto issue_pv = [&](int i, int stage, bool accumulate) {
-        const uint32_t va = sbase + C::OFF_V + stage * C::TILE_BYTES;
+        const uint32_t va = opaque_u32(sbase + C::OFF_V + stage * C::TILE_BYTES);
+        const uint32_t ts = opaque_u32(tmem + C::tmem_s(i));
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          umma_ts(tmem + C::tmem_o(i), tmem + C::tmem_s(i) + ks * 8,
+          umma_ts(tmem + C::tmem_o(i), ts + ks * 8,
                   smem_desc_sw128(va + ks * 2048, C::CB_BYTES, 1024), idesc_pv,
                   (accumulate || ks > 0) ? 1u : 0u);
         }
@@ -344,16 +360,18 @@ __global__ void __launch_bounds__(320, 1)
       mbar_wait(bar(C::B_DRAIN), 0, nullptr);
     }
     __syncwarp();
+    }  // warps 2-3: nothing to do
   } else {
+    warpgroup_reg_alloc<C::REGS_SOFTMAX>();
     // ======================= softmax warpgroups =======================
-    const int i = (warp - 2) >> 2;       // query tile slot of this warpgroup
+    const int i = (warp - 4) >> 2;       // query tile slot of this warpgroup
     const int quarter = warp & 3;        // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;   // row within the tile
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t t_s = tmem + lane_off + C::tmem_s(i);
     const uint32_t t_o = tmem + lane_off + C::tmem_o(i);
-    const uint32_t stg = sbase + C::OFF_STG + (warp - 2) * C::STG_BYTES;
-    uint8_t* stg_ptr = sbase_ptr + C::OFF_STG + (warp - 2) * C::STG_BYTES;
+    const uint32_t stg = sbase + C::OFF_STG + (warp - 4) * C::STG_BYTES;
+    uint8_t* stg_ptr = sbase_ptr + C::OFF_STG + (warp - 4) * C::STG_BYTES;
     float c2 = p.scale_log2;
     const bool scale_pos = c2 > 0.f;
     if (!scale_pos) c2 = 1.f;  // scores are pre-multiplied below instead

@@ -166,8 +166,10 @@ __device__ __forceinline__ bool mbar_test_sleep(uint32_t bar, uint32_t parity, u
 // Slow path of a bounded wait.  Gives up (returning false) when the CTA's abort
 // flag is raised by another thread, or after kWaitTimeoutNs, in which case it
 // records the timeout and raises the abort flag itself.  With abort_flag ==
-// nullptr only the time limit applies (used to drain in-flight copies).
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
+// nullptr only the time limit applies (used to drain in-flight copies).  It is
+// inlined: a call would pin the caller to the kernel-wide register budget,
+// which a warpgroup that raised its budget with setmaxnreg cannot use.
+__device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
                                             volatile int* abort_flag) {
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
@@ -194,6 +196,26 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
   int ok = 0;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Returns x unchanged but opaque to the optimiser, so that values derived from
+// it are recomputed where they are used instead of being hoisted (and kept
+// live in registers) across a long loop.
+__device__ __forceinline__ uint32_t opaque_u32(uint32_t x) {
+  asm volatile("" : "+r"(x));
+  return x;
+}
+
+// Register reallocation between warpgroups (all four warps of a warpgroup
+// execute the same instruction).  The counts must add up to what the CTA was
+// launched with, or an increase waits forever: see the prefill kernel.
+template <uint32_t N>
+__device__ __forceinline__ void warpgroup_reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void warpgroup_reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ---------------------------------------------------------------------------
