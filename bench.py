@@ -177,14 +177,24 @@ def dist_setup(args):
     return world, rank, local
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The largest x over all ranks (times are reported as the slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, ms_per_rank: float, world: int,
+                       device: str = "cuda"):
+    """Whole-job throughput under weak scaling: every rank processes the same
+    number of independent units; the job takes as long as its slowest rank.
+    Returns (units of all ranks per second, slowest rank's ms)."""
+    ms = max_over_ranks(ms_per_rank, world, device)
+    return world * units_per_rank / (ms * 1e-3), ms
 
 
 def barrier(world: int):
@@ -357,9 +367,9 @@ def run_ours(args, world, rank, local):
         raise RuntimeError(f"device error word set in the timed region: {fl:#x}")
 
     pre_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    pre_avg = max_over_ranks(sum(pre_ms) / len(pre_ms), world)
+    flops_per_s, pre_avg = weak_scaling_value(flops, sum(pre_ms) / len(pre_ms), world)
     step_ms = max_over_ranks(t_all0.elapsed_time(t_all1) / args.steps, world)
-    value = world * flops / (pre_avg * 1e-3) / 1e12
+    value = flops_per_s / 1e12
     achieved = flops / (pre_avg * 1e-3) / 1e12
     traffic = ncu_traffic("attn_prefill_sm100_kernel", cfg.name)
     line = {
@@ -377,11 +387,11 @@ def run_ours(args, world, rank, local):
     launches_per_step = 1
     if dcfg is not None:
         dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
-        dec_avg = max_over_ranks(sum(dec_ms) / len(dec_ms), world)
+        bytes_per_s, dec_avg = weak_scaling_value(decode_bytes, sum(dec_ms) / len(dec_ms), world)
         gbs = decode_bytes / (dec_avg * 1e-3) / 1e9
         dtraffic = ncu_traffic("attn_decode_split_kernel", dcfg.name)
         line["decode"] = {
-            "value": world * gbs, "unit": "GB/s", "ms": dec_avg,
+            "value": bytes_per_s / 1e9, "unit": "GB/s", "ms": dec_avg,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": dtraffic,
                          "kernel": "attn_decode_split_kernel + attn_decode_merge_kernel",
