@@ -166,6 +166,26 @@ def test_large_magnitude_scores_stay_finite():
     assert np.abs(lse.numpy() - lse_ref).max() <= 1e-3
 
 
+@pytest.mark.parametrize("d,causal", [(128, False), (128, True), (64, True)])
+def test_scores_rising_across_key_tiles(d, causal):
+    # Key tiles scaled 1, 2.5, 5, 12: from tile to tile a row's max grows by
+    # less than 8, by 8..16 and by more than 16 (log2 units), so the exponent
+    # base stays put, moves one step late, and (for the last tile) the tile is
+    # recomputed against its own max.  Error bound as in the test above.
+    q, k, v = W.prefill_inputs(1, 2, 1, 512, 512, d, seed=29)
+    f = torch.tensor([1.0, 2.5, 5.0, 12.0]).repeat_interleave(128).view(1, 1, 512, 1)
+    k = (k.float() * f).to(torch.bfloat16)
+    scale = 1 / math.sqrt(d)
+    o, lse = _run(q, k, v, causal, scale)
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, causal, scale)
+    og = o.double().numpy()
+    assert np.isfinite(og).all() and np.isfinite(lse.numpy()).all()
+    bound = 2.0 ** -8 * np.abs(o_ref) + 2.0 ** -8 * float(v.abs().max()) + 1e-3
+    assert np.all(np.abs(og - o_ref) <= bound)
+    assert np.linalg.norm(og - o_ref) / np.linalg.norm(o_ref) <= 5e-3
+    assert np.abs(lse.numpy() - lse_ref).max() <= 1e-3
+
+
 def test_worked_example_embedded():
     # "Attention Kernel", section "Blockwise reference": scores [1, -inf, 3, -2, 0]
     # against values arange(15) as 5 x 3.  Embedded with d = 64, q = e0,
