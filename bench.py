@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-ragged", action="store_true")
+    ap.add_argument("--ragged-workload", default="ragged_gqa_causal")
     return ap.parse_args()
 
 
@@ -402,11 +404,70 @@ def run_ours(args, world, rank, local):
     line["gpu_launches"] = launches_per_step * args.steps
     line["clocks"] = sampler.summary()
 
+    if not args.no_ragged:
+        line["ragged"] = ragged_leg(args, dev, world, peaks)
     if not args.no_e2e:
         line["e2e"] = e2e_leg(args, cfg, q_h, k_h, v_h, kl_h, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_leg(cfg, q_h, k_h, v_h, kl_h)
     return line if rank == 0 else None
+
+
+def ragged_leg(args, dev, world, peaks):
+    """Prefill over a packed ragged batch (attn_fwd_varlen: the unit-list kernel and
+    the prefill kernel), timed on its own after the headline region: inputs resident,
+    L2 flushed before each call, CUDA events around each call, max over ranks."""
+    import torch
+
+    from exact_softmax_attention_fwd_b200 import (attn_fwd_varlen,
+                                                  attn_fwd_varlen_workspace_size,
+                                                  attn_get_device_error)
+    from exact_softmax_attention_fwd_b200 import workloads as W
+
+    rc = W.CONFIGS[args.ragged_workload]
+    q_h, k_h, v_h, cu_q_h, cu_k_h, lens = W.varlen_config_inputs(rc)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    cu_q, cu_k = cu_q_h.to(dev), cu_k_h.to(dev)
+    max_q = int(lens.max())
+    ws = torch.empty(attn_fwd_varlen_workspace_size(rc.B, q.shape[0], max_q), dtype=torch.uint8,
+                     device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((rc.Hq, q.shape[0]), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def one():
+        attn_fwd_varlen(q, k, v, cu_q, cu_k, max_q, rc.causal, rc.scale, out=o, lse=lse,
+                        workspace=ws)
+
+    for _ in range(3):
+        flush.fill_(1.0)
+        one()
+    torch.cuda.synchronize(dev)
+    n = max(5, min(args.steps, 50))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    barrier(world)
+    for e0, e1 in evs:
+        flush.fill_(1.0)
+        e0.record(stream)
+        one()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    st, fl = attn_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word set in the ragged leg: {fl:#x}")
+    ms = [a.elapsed_time(b) for a, b in evs]
+    flops = rc.flops(lens)
+    flops_per_s, avg = weak_scaling_value(flops, sum(ms) / len(ms), world)
+    achieved = flops / (avg * 1e-3) / 1e12
+    return {"workload": rc.name, "value": flops_per_s / 1e12, "unit": "TFLOPS", "ms": avg,
+            "median_ms": statistics.median(ms), "calls": n, "gpu_launches_per_call": 2,
+            "sequences": rc.B, "total_tokens": int(q.shape[0]),
+            "lengths": f"uniform {rc.len_lo}..{rc.len_hi} (seed {rc.seed})",
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "per_call_flops": flops}}
 
 
 def e2e_leg(args, cfg, q_h, k_h, v_h, kl_h, dev, world):

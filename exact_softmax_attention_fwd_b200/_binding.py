@@ -36,6 +36,9 @@ _SZ = ctypes.c_size_t
 SIGNATURES = {
     "attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "attn_fwd_masked": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P]),
+    "attn_fwd_varlen_workspace_size": (_SZ, [_I, ctypes.c_longlong, _I]),
+    "attn_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, ctypes.c_longlong,
+                             ctypes.c_longlong, _I, _I, _I, _F, _P, _SZ, _P]),
     "attn_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P,
                                _SZ, _P]),
@@ -134,6 +137,47 @@ def attn_fwd(q, k, v, causal: bool, scale: float, out=None, lse=None, return_lse
              stream=None):
     """attn_fwd_masked without key padding."""
     return attn_fwd_masked(q, k, v, causal, scale, None, out, lse, return_lse, stream)
+
+
+def attn_fwd_varlen_workspace_size(B: int, total_q: int, max_seqlen_q: int) -> int:
+    return int(load_library().attn_fwd_varlen_workspace_size(B, total_q, max_seqlen_q))
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, causal: bool,
+                    scale: float, out=None, lse=None, workspace=None, return_lse: bool = True,
+                    stream=None):
+    """Prefill over a ragged batch: q [total_q, Hq, d], k/v [total_k, Hkv, d] bf16, packed;
+    cu_seqlens_q/k int32 [B+1] on the device.  Returns O [total_q, Hq, d], LSE [Hq, total_q]."""
+    import torch
+    _require_cuda(q, k, v, cu_seqlens_q, cu_seqlens_k)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError("q, k, v must be contiguous 3-d bfloat16 tensors")
+    total_q, Hq, d = q.shape
+    total_k, Hkv, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or dk != d:
+        raise ValueError("q/k/v shapes disagree")
+    for t in (cu_seqlens_q, cu_seqlens_k):
+        if t.dtype != torch.int32 or t.dim() != 1 or not t.is_contiguous():
+            raise ValueError("cu_seqlens must be contiguous int32 [B+1]")
+    if cu_seqlens_q.shape != cu_seqlens_k.shape or cu_seqlens_q.shape[0] < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both be [B+1], B >= 1")
+    B = cu_seqlens_q.shape[0] - 1
+    need = attn_fwd_varlen_workspace_size(B, total_q, max_seqlen_q)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = load_library().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                        _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, Hq, Hkv,
+                                        total_q, total_k, int(max_seqlen_q), d,
+                                        int(bool(causal)), float(scale), _ptr(workspace),
+                                        ws_bytes, _stream(stream))
+    _check(st, "attn_fwd_varlen")
+    return out, lse
 
 
 def attn_decode_workspace_size(B: int, Hq: int, max_pages_per_seq: int, page_size: int,

@@ -12,6 +12,7 @@
 #include "decode_sm100.cuh"
 #include "prefill_sm100.cuh"
 #include "sm100_primitives.cuh"
+#include "varlen_schedule.cuh"
 
 namespace attn_b200 {
 namespace {
@@ -60,6 +61,22 @@ bool make_tile_map(CUtensorMap* map, const void* ptr, int D, long long rows, lon
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 map over a packed token-major [tokens, heads, D] tensor, box = 128
+// tokens of one head x 64 columns, 128-byte swizzle: the same shared-memory
+// tile as make_tile_map gives (128 rows of 128 bytes).
+bool make_token_map(CUtensorMap* map, const void* ptr, int D, long long heads, long long tokens) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)tokens};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
@@ -76,16 +93,18 @@ int sm_count() {
   return cached[dev];
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool VARLEN = false>
 int launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                   const CUtensorMap& mo, const PrefillParams& prm, cudaStream_t stream) {
+                   const CUtensorMap& mo, const PrefillParams& prm, cudaStream_t stream,
+                   long long max_units = 0) {
   using C = PrefillCfg<D>;
-  auto kern = attn_prefill_sm100_kernel<D, CAUSAL>;
+  auto kern = attn_prefill_sm100_kernel<D, CAUSAL, VARLEN>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
       cudaSuccess)
     return ATTN_ERR_CUDA;
   // persistent: one CTA per SM (or fewer when there are fewer work units)
-  const long long units = (long long)prm.n_qblocks * prm.Hq * prm.B;
+  const long long units =
+      VARLEN ? max_units * prm.Hq : (long long)prm.n_qblocks * prm.Hq * prm.B;
   const int sms = sm_count();
   if (sms <= 0) return ATTN_ERR_CUDA;
   dim3 grid((unsigned)(units < sms ? units : sms));
@@ -110,6 +129,10 @@ int check_prefill_args(const void* q, const void* k, const void* v, void* o, flo
     return ATTN_ERR_ALIGNMENT;
   return ATTN_OK;
 }
+
+// Units of a ragged batch: sum over sequences of ceil(len_q / 256) is at most
+// total_q / 256 + B for non-overlapping ranges; one more for rounding.
+long long varlen_max_units(int B, long long total_q) { return total_q / 256 + B + 1; }
 
 }  // namespace
 }  // namespace attn_b200
@@ -156,6 +179,7 @@ int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float*
       !make_tile_map(&mo, o, d, Sq, (long long)B * Hq, 32))
     return ATTN_ERR_CUDA;
   PrefillParams prm;
+  std::memset(&prm, 0, sizeof(prm));
   prm.lse = lse;
   prm.k_lens = k_lens;
   prm.B = B;
@@ -171,6 +195,88 @@ int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float*
                   : launch_prefill<128, false>(mq, mk, mv, mo, prm, stream);
   return causal ? launch_prefill<64, true>(mq, mk, mv, mo, prm, stream)
                 : launch_prefill<64, false>(mq, mk, mv, mo, prm, stream);
+}
+
+size_t attn_fwd_varlen_workspace_size(int B, long long total_q, int max_seqlen_q) {
+  if (B < 1 || total_q < 0 || total_q > 0x7fffffffLL || max_seqlen_q < 1 ||
+      max_seqlen_q > kVarlenMaxLevels * 256)
+    return 0;
+  return 16 + 8 * (size_t)varlen_max_units(B, total_q);
+}
+
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B, int Hq,
+                    int Hkv, long long total_q, long long total_k, int max_seqlen_q, int d,
+                    int causal, float scale, void* workspace, size_t workspace_bytes,
+                    attn_stream_t stream_) {
+  if (q == nullptr || o == nullptr || cu_seqlens_q == nullptr || cu_seqlens_k == nullptr ||
+      (total_k > 0 && (k == nullptr || v == nullptr)))
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq > 65535) return ATTN_ERR_INVALID_ARG;
+  if (total_q < 0 || total_k < 0 || total_q > 0x7fffffffLL || total_k > 0x7fffffffLL)
+    return ATTN_ERR_INVALID_ARG;
+  if (max_seqlen_q < 1 || max_seqlen_q > kVarlenMaxLevels * 256) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(o) || (total_k > 0 && (!aligned16(k) || !aligned16(v))))
+    return ATTN_ERR_ALIGNMENT;
+  if ((lse != nullptr && !aligned4(lse)) || !aligned4(cu_seqlens_q) || !aligned4(cu_seqlens_k))
+    return ATTN_ERR_ALIGNMENT;
+  const size_t need = attn_fwd_varlen_workspace_size(B, total_q, max_seqlen_q);
+  if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (total_q == 0) return ATTN_OK;  // no query token: nothing to write
+  if (total_k == 0) {  // no key anywhere: every query row is empty
+    const size_t n_vec = (size_t)total_q * Hq * d * 2 / 16;
+    const int threads = 256;
+    const long long want = ((long long)n_vec + threads - 1) / threads;
+    const int blocks = (int)(want < 4096 ? (want > 0 ? want : 1) : 4096);
+    fill_empty_rows_kernel<<<blocks, threads, 0, stream>>>(reinterpret_cast<uint4*>(o), n_vec, lse,
+                                                           (size_t)total_q * Hq);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+  // 1. the unit list (heaviest first) in the workspace
+  int* unit_count = static_cast<int*>(workspace);
+  int2* units = reinterpret_cast<int2*>(static_cast<char*>(workspace) + 16);
+  const long long max_units = varlen_max_units(B, total_q);
+  const int n_levels = (max_seqlen_q + 255) / 256;
+  const size_t sched_smem = (size_t)(2 * n_levels + 32) * sizeof(int);
+  if (cudaFuncSetAttribute(attn_varlen_schedule_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sched_smem) !=
+      cudaSuccess)
+    return ATTN_ERR_CUDA;
+  attn_varlen_schedule_kernel<<<1, 1024, sched_smem, stream>>>(
+      cu_seqlens_q, cu_seqlens_k, B, (int)total_q, (int)total_k, max_seqlen_q, units, unit_count,
+      (int)max_units);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  // 2. the prefill kernel over packed token-major tensors
+  CUtensorMap mq, mk, mv;
+  if (!make_token_map(&mq, q, d, Hq, total_q) || !make_token_map(&mk, k, d, Hkv, total_k) ||
+      !make_token_map(&mv, v, d, Hkv, total_k))
+    return ATTN_ERR_CUDA;
+  PrefillParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.lse = lse;
+  prm.k_lens = nullptr;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.o = static_cast<uint16_t*>(o);
+  prm.cu_q = cu_seqlens_q;
+  prm.cu_k = cu_seqlens_k;
+  prm.units = units;
+  prm.unit_count = unit_count;
+  prm.total_q = (int)total_q;
+  // the output map is unused by the ragged path (rows are stored one by one)
+  if (d == 128)
+    return causal ? launch_prefill<128, true, true>(mq, mk, mv, mq, prm, stream, max_units)
+                  : launch_prefill<128, false, true>(mq, mk, mv, mq, prm, stream, max_units);
+  return causal ? launch_prefill<64, true, true>(mq, mk, mv, mq, prm, stream, max_units)
+                : launch_prefill<64, false, true>(mq, mk, mv, mq, prm, stream, max_units);
 }
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,

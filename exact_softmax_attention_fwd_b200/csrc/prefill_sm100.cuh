@@ -57,12 +57,20 @@
 namespace attn_b200 {
 
 struct PrefillParams {
-  float* lse;           // [B, Hq, Sq] or nullptr
-  const int* k_lens;    // [B] or nullptr
+  float* lse;           // [B, Hq, Sq] (ragged: [Hq, total_q]) or nullptr
+  const int* k_lens;    // [B] or nullptr (fixed-length batches only)
   int B, Hq, Hkv, Sq, Sk;
   int group;            // Hq / Hkv
   float scale_log2;     // scale * log2(e)
   int n_qblocks;        // ceil(Sq / 256)
+  // ragged batches: packed token-major tensors, cumulative sequence lengths
+  // and the unit list written by attn_varlen_schedule_kernel
+  uint16_t* o;          // [total_q, Hq, d] bf16
+  const int* cu_q;      // [B + 1]
+  const int* cu_k;      // [B + 1]
+  const int2* units;    // (sequence, query block), heaviest first
+  const int* unit_count;
+  int total_q;
 };
 
 template <int D>
@@ -120,7 +128,10 @@ __device__ __forceinline__ int prefill_num_kv_tiles(int row0, int Sq, int klen, 
 // One work unit: query rows [256*qb, 256*qb + 256) of head hq in sequence b.
 struct PrefillUnit {
   int qb, hq, b;
+  int sq;          // query rows of the sequence
   int klen;        // visible keys of the sequence
+  int q_tok0;      // ragged batches: packed index of the sequence's first query
+  int k_tok0;      //   and first key token (0 otherwise)
   int row0[2];     // first row of each query tile
   int nkv[2];      // KV tiles each query tile visits
 };
@@ -128,32 +139,48 @@ struct PrefillUnit {
 // The k-th unit of this CTA, or false when the CTA has no more work.  Ranks
 // are ordered heaviest first (q-blocks descending, heads inner) and dealt
 // back and forth across the CTAs: rank k*G + c for even k, k*G + G-1-c for odd.
-template <bool CAUSAL>
+// For a ragged batch the (sequence, q-block) order comes from the unit list.
+template <bool CAUSAL, bool VARLEN>
 __device__ __forceinline__ bool prefill_unit(const PrefillParams& p, int k, PrefillUnit& u) {
   const long long G = gridDim.x;
   const long long c = blockIdx.x;
   const long long r = (long long)k * G + ((k & 1) ? (G - 1 - c) : c);
-  const long long HB = (long long)p.Hq * p.B;
-  if (r >= (long long)p.n_qblocks * HB) return false;
-  u.qb = p.n_qblocks - 1 - (int)(r / HB);
-  const int rem = (int)(r % HB);
-  u.hq = rem % p.Hq;
-  u.b = rem / p.Hq;
-  int klen = p.Sk;
-  if (p.k_lens != nullptr) {
-    klen = p.k_lens[u.b];
-    if (klen < 0 || klen > p.Sk) klen = klen < 0 ? 0 : p.Sk;  // flagged by the softmax warps
+  if (VARLEN) {
+    if (r >= (long long)__ldg(p.unit_count) * p.Hq) return false;
+    const int2 e = __ldg(&p.units[r / p.Hq]);
+    u.hq = (int)(r % p.Hq);
+    u.b = e.x;
+    u.qb = e.y;
+    u.q_tok0 = __ldg(p.cu_q + u.b);
+    u.k_tok0 = __ldg(p.cu_k + u.b);
+    u.sq = __ldg(p.cu_q + u.b + 1) - u.q_tok0;  // listed sequences passed the
+    u.klen = __ldg(p.cu_k + u.b + 1) - u.k_tok0;  // schedule kernel's checks
+  } else {
+    const long long HB = (long long)p.Hq * p.B;
+    if (r >= (long long)p.n_qblocks * HB) return false;
+    u.qb = p.n_qblocks - 1 - (int)(r / HB);
+    const int rem = (int)(r % HB);
+    u.hq = rem % p.Hq;
+    u.b = rem / p.Hq;
+    int klen = p.Sk;
+    if (p.k_lens != nullptr) {
+      klen = p.k_lens[u.b];
+      if (klen < 0 || klen > p.Sk) klen = klen < 0 ? 0 : p.Sk;  // flagged by the softmax warps
+    }
+    u.klen = klen;
+    u.sq = p.Sq;
+    u.q_tok0 = 0;
+    u.k_tok0 = 0;
   }
-  u.klen = klen;
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     u.row0[i] = u.qb * 256 + i * 128;
-    u.nkv[i] = prefill_num_kv_tiles(u.row0[i], p.Sq, klen, CAUSAL);
+    u.nkv[i] = prefill_num_kv_tiles(u.row0[i], u.sq, u.klen, CAUSAL);
   }
   return true;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(384, 1)
     attn_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                               const __grid_constant__ CUtensorMap tm_k,
@@ -218,16 +245,19 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t& n = i ? q_loads1 : q_loads0;
         if (n > 0 && !mbar_wait(bar(C::B_QFREE + i), (n - 1) & 1u, abort_flag)) return false;
         mbar_arrive_expect_tx(bar(C::B_QFULL + i), C::TILE_BYTES);
+        // fixed-length maps are (d, Sq, B*Hq); ragged ones (d, Hq, total_q)
         for (int cb = 0; cb < C::NCB; ++cb)
           tma_load_3d(sbase + C::OFF_Q + i * C::TILE_BYTES + cb * C::CB_BYTES, &tm_q,
-                      bar(C::B_QFULL + i), 64 * cb, u.row0[i], u.b * p.Hq + u.hq);
+                      bar(C::B_QFULL + i), 64 * cb, VARLEN ? u.hq : u.row0[i],
+                      VARLEN ? u.q_tok0 + u.row0[i] : u.b * p.Hq + u.hq);
         ++n;
         return true;
       };
       PrefillUnit u;
-      for (int k = 0; ok && prefill_unit<CAUSAL>(p, k, u); ++k) {
+      for (int k = 0; ok && prefill_unit<CAUSAL, VARLEN>(p, k, u); ++k) {
         const int n_max = max(u.nkv[0], u.nkv[1]);
-        const int kv_row = u.b * p.Hkv + u.hq / p.group;
+        const int kvh = u.hq / p.group;
+        const int kv_row = u.b * p.Hkv + kvh;
         // Q_0 first (its slot frees first under a causal mask), then the first
         // K tile, then Q_1, so that no wait on Q_1 holds back the K/V stream.
         if (u.nkv[0] > 0 && !(ok = load_q(u, 0))) break;
@@ -238,7 +268,8 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::TILE_BYTES);
           for (int cb = 0; cb < C::NCB; ++cb)
             tma_load_3d(sbase + C::OFF_K + s * C::TILE_BYTES + cb * C::CB_BYTES, &tm_k,
-                        bar(C::B_KFULL + s), 64 * cb, j * 128, kv_row);
+                        bar(C::B_KFULL + s), 64 * cb, VARLEN ? kvh : j * 128,
+                        VARLEN ? u.k_tok0 + j * 128 : kv_row);
           if (j == 0 && u.nkv[1] > 0 && !(ok = load_q(u, 1))) {
             ++kv;  // K_0 of this unit was issued
             break;
@@ -250,7 +281,8 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE_BYTES);
           for (int cb = 0; cb < C::NCB; ++cb)
             tma_load_3d(sbase + C::OFF_V + s * C::TILE_BYTES + cb * C::CB_BYTES, &tm_v,
-                        bar(C::B_VFULL + s), 64 * cb, j * 128, kv_row);
+                        bar(C::B_VFULL + s), 64 * cb, VARLEN ? kvh : j * 128,
+                        VARLEN ? u.k_tok0 + j * 128 : kv_row);
         }
       }
       // Drain: never leave the CTA with copies still landing in shared memory.
@@ -298,7 +330,7 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t p_waits0 = 0, p_waits1 = 0;  // P_FULL phases consumed per tile slot
       bool ok = true;
       PrefillUnit u;
-      for (int k = 0; ok && prefill_unit<CAUSAL>(p, k, u); ++k) {
+      for (int k = 0; ok && prefill_unit<CAUSAL, VARLEN>(p, k, u); ++k) {
         const int n_max = max(u.nkv[0], u.nkv[1]);
         if (n_max == 0) continue;
         // prologue: S_i(0) for each participating tile
@@ -379,18 +411,18 @@ __global__ void __launch_bounds__(384, 1)
     bool stores_pending = false;
     bool ok = true;
     PrefillUnit u;
-    for (int k = 0; ok && prefill_unit<CAUSAL>(p, k, u); ++k) {
+    for (int k = 0; ok && prefill_unit<CAUSAL, VARLEN>(p, k, u); ++k) {
       const int row0 = i ? u.row0[1] : u.row0[0];
-      if (row0 >= p.Sq) continue;  // this tile slot holds no rows in this unit
+      if (row0 >= u.sq) continue;  // this tile slot holds no rows in this unit
       const int n = i ? u.nkv[1] : u.nkv[0];
       const int row = row0 + r;
       const int q_head_row = u.b * p.Hq + u.hq;
-      if (p.k_lens != nullptr && r == 0) {
+      if (!VARLEN && p.k_lens != nullptr && r == 0) {
         const int kl = p.k_lens[u.b];
         if (kl < 0 || kl > p.Sk) flag_device_error(kDevErrBadLength);
       }
       // largest visible key of this row, and of the tile's first row
-      const long long koff = (long long)u.klen - p.Sq;
+      const long long koff = (long long)u.klen - u.sq;
       long long lim_row = (long long)u.klen - 1;
       long long lim_tile = lim_row;
       if (CAUSAL) {
@@ -510,45 +542,82 @@ __global__ void __launch_bounds__(384, 1)
       }
       tc_fence_after_sync();
       const float inv = (lr_run > 0.f) ? (1.f / lr_run) : 0.f;
-      const bool warp_has_rows = row0 + quarter * 32 < p.Sq;
-#pragma unroll 1
-      for (int cb = 0; cb < C::NCB; ++cb) {
-        if (stores_pending) {  // the previous store must have read the buffer
-          if (lane == 0) tma_store_wait_read_all();
-          __syncwarp();
-          stores_pending = false;
+      if constexpr (VARLEN) {
+        // A TMA box could reach into the next sequence's rows, so each thread
+        // writes its own row: d accumulator columns read from TMEM in one
+        // batch, normalised, stored as 2d contiguous bytes in 16-byte pieces.
+        uint32_t v[D / 32][32];
+        if (has_o) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) tmem_ld32(t_o + 32 * c, v[c]);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) reg_fence32(v[c]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[c][e] = 0u;
         }
+        if (row < u.sq) {
+          const size_t tok = (size_t)u.q_tok0 + row;
+          uint4* dst = reinterpret_cast<uint4*>(p.o + (tok * p.Hq + u.hq) * D);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t v[32];
-          if (has_o) {
-            tmem_ld32_sync(t_o + 64 * cb + 32 * half, v);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = 0u;
-          }
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int chunk = 4 * half + q4;  // 16-byte chunk within the 128-byte row
+          for (int q8 = 0; q8 < D / 8; ++q8) {  // 8 bf16 = 16 bytes per store
+            const uint32_t* x = &v[q8 >> 2][(q8 & 3) * 8];
             uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * inv, __uint_as_float(v[8 * q4 + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv, __uint_as_float(v[8 * q4 + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv, __uint_as_float(v[8 * q4 + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv, __uint_as_float(v[8 * q4 + 7]) * inv);
-            *reinterpret_cast<uint4*>(stg_ptr + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = w;
+            w.x = pack_bf16x2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv);
+            dst[q8] = w;
+          }
+          if (p.lse != nullptr) {
+            const float lse = (l_run > 0.f) ? (m_run + lg2(l_run)) * 0.69314718055994531f : -INFINITY;
+            p.lse[(size_t)u.hq * p.total_q + tok] = lse;
           }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && warp_has_rows && !*abort_flag) {
-          tma_store_3d(&tm_o, stg, 64 * cb, row0 + quarter * 32, q_head_row);
-          tma_store_commit();
+      } else {
+        const bool warp_has_rows = row0 + quarter * 32 < p.Sq;
+#pragma unroll 1
+        for (int cb = 0; cb < C::NCB; ++cb) {
+          if (stores_pending) {  // the previous store must have read the buffer
+            if (lane == 0) tma_store_wait_read_all();
+            __syncwarp();
+            stores_pending = false;
+          }
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t v[32];
+            if (has_o) {
+              tmem_ld32_sync(t_o + 64 * cb + 32 * half, v);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = 0u;
+            }
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const int chunk = 4 * half + q4;  // 16-byte chunk within the 128-byte row
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * inv, __uint_as_float(v[8 * q4 + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv, __uint_as_float(v[8 * q4 + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv, __uint_as_float(v[8 * q4 + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv, __uint_as_float(v[8 * q4 + 7]) * inv);
+              *reinterpret_cast<uint4*>(stg_ptr + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = w;
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && warp_has_rows && !*abort_flag) {  // rows past Sq are clipped by the map
+            tma_store_3d(&tm_o, stg, 64 * cb, row0 + quarter * 32, q_head_row);
+            tma_store_commit();
+          }
+          stores_pending = true;
         }
-        stores_pending = true;
-      }
-      if (p.lse != nullptr && row < p.Sq) {
-        const float lse = (l_run > 0.f) ? (m_run + lg2(l_run)) * 0.69314718055994531f : -INFINITY;
-        p.lse[(size_t)q_head_row * p.Sq + row] = lse;
+        if (p.lse != nullptr && row < p.Sq) {
+          const float lse = (l_run > 0.f) ? (m_run + lg2(l_run)) * 0.69314718055994531f : -INFINITY;
+          p.lse[(size_t)q_head_row * p.Sq + row] = lse;
+        }
       }
     }
     // all of this warp's output stores complete before the CTA exits

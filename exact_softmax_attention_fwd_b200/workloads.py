@@ -13,6 +13,8 @@ Recipe (all on the host, ``torch.Generator().manual_seed(seed)``):
   * Paged decode: seq_lens uniform in [lo, hi]; the cache pool holds exactly
     sum ceil(len/page) pages and a seeded random permutation gives the
     physical page of each logical page; unused block-table slots are -1.
+  * Ragged (packed) batches: per-sequence lengths uniform in [lo, hi]; Q, K,
+    V drawn packed token-major [total, H, d]; cumulative lengths int32 [B+1].
 """
 from __future__ import annotations
 
@@ -72,6 +74,35 @@ class DecodeConfig:
         return -(-self.len_hi // self.page_size)
 
 
+@dataclass(frozen=True)
+class VarlenConfig:
+    """A ragged batch: B sequences with len_q = len_k uniform in [len_lo, len_hi]."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    causal: bool
+    len_lo: int
+    len_hi: int
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def lengths(self) -> torch.Tensor:
+        g = _gen(self.seed)
+        return torch.randint(self.len_lo, self.len_hi + 1, (self.B,), generator=g,
+                             dtype=torch.int64).to(torch.int32)
+
+    def flops(self, lengths=None) -> float:
+        """sum over sequences of 4*Hq*len^2*d, halved when causal."""
+        lens = (self.lengths() if lengths is None else lengths).to(torch.float64)
+        f = float(4.0 * self.Hq * self.d * (lens * lens).sum())
+        return f / 2 if self.causal else f
+
+
 CONFIGS = {
     "tiny_mha": PrefillConfig("tiny_mha", B=1, Hq=2, Hkv=2, S=256, d=64, causal=False, seed=1001),
     "mha_causal_2k": PrefillConfig("mha_causal_2k", B=4, Hq=16, Hkv=16, S=2048, d=128,
@@ -84,6 +115,9 @@ CONFIGS = {
                                     causal=True, seed=1004, value_scale=0.5),
     "paged_decode": DecodeConfig("paged_decode", B=64, Hq=32, Hkv=8, d=128, page_size=16,
                                  len_lo=512, len_hi=8192, seed=1005),
+    # the GQA shapes of gqa_causal_8k, as a ragged batch of mixed lengths
+    "ragged_gqa_causal": VarlenConfig("ragged_gqa_causal", B=16, Hq=32, Hkv=8, d=128,
+                                      causal=True, len_lo=128, len_hi=8192, seed=1200),
 }
 
 
@@ -194,3 +228,26 @@ def sample_rows(B, Hq, Sq, n, seed) -> torch.Tensor:
     total = B * Hq * Sq
     n = min(n, total)
     return torch.randperm(total, generator=_gen(seed))[:n].sort().values
+
+
+def cu_seqlens(lengths) -> torch.Tensor:
+    """Cumulative lengths int32 [B+1] (leading 0) of an int tensor or list of lengths."""
+    lens = torch.as_tensor(lengths, dtype=torch.int64)
+    return torch.cat([torch.zeros(1, dtype=torch.int64), torch.cumsum(lens, 0)]).to(torch.int32)
+
+
+def varlen_inputs(lens_q, lens_k, Hq: int, Hkv: int, d: int, seed: int, value_scale: float = 1.0):
+    """Packed q [sum lens_q, Hq, d], k/v [sum lens_k, Hkv, d] bf16 and cu_seqlens_q/k int32."""
+    cu_q, cu_k = cu_seqlens(lens_q), cu_seqlens(lens_k)
+    tq, tk = int(cu_q[-1]), int(cu_k[-1])
+    q = randn_bf16((tq, Hq, d), seed * 16 + 0, value_scale)
+    k = randn_bf16((tk, Hkv, d), seed * 16 + 1, value_scale)
+    v = randn_bf16((tk, Hkv, d), seed * 16 + 2, value_scale)
+    return q, k, v, cu_q, cu_k
+
+
+def varlen_config_inputs(cfg: VarlenConfig):
+    """(q, k, v, cu_q, cu_k, lengths) for a named ragged configuration."""
+    lens = cfg.lengths()
+    q, k, v, cu_q, cu_k = varlen_inputs(lens, lens, cfg.Hq, cfg.Hkv, cfg.d, cfg.seed)
+    return q, k, v, cu_q, cu_k, lens

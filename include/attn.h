@@ -52,7 +52,7 @@ typedef enum {
   ATTN_ERR_INVALID_ARG = 1, /* null pointer, bad extent, Hq % Hkv != 0, non-finite scale */
   ATTN_ERR_UNSUPPORTED = 2, /* head dim, page size or group size outside what is built */
   ATTN_ERR_ALIGNMENT = 3,   /* a tensor pointer is not 16-byte aligned */
-  ATTN_ERR_WORKSPACE = 4,   /* decode workspace missing or too small */
+  ATTN_ERR_WORKSPACE = 4,   /* decode / varlen workspace missing or too small */
   ATTN_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed (no device, launch error) */
   ATTN_ERR_DEVICE = 6       /* attn_get_device_error(): the device error word was set */
 } attn_status;
@@ -60,7 +60,7 @@ typedef enum {
 /* Bits of the device error word (attn_get_device_error's flags_out). */
 #define ATTN_DEVERR_WAIT_TIMEOUT 0x1u /* an internal pipeline wait exceeded its time limit */
 #define ATTN_DEVERR_BAD_PAGE 0x2u     /* a block-table entry outside [0, num_pages) was skipped */
-#define ATTN_DEVERR_BAD_LENGTH 0x4u   /* a k_len / seq_len outside its legal range was clamped */
+#define ATTN_DEVERR_BAD_LENGTH 0x4u   /* a k_len / seq_len / cu_seqlens entry outside its legal range */
 
 /*
  * attn_fwd -- prefill / full-sequence attention forward.
@@ -92,6 +92,53 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
 int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                     int Hq, int Hkv, int Sq, int Sk, int d, int causal, float scale,
                     const int32_t* k_lens, attn_stream_t stream);
+
+/*
+ * attn_fwd_varlen_workspace_size -- bytes of caller-owned device workspace
+ * that attn_fwd_varlen needs: the list of (sequence, 256-row query block)
+ * work units the call schedules.  total_q is the number of packed query
+ * tokens, B the number of sequences, max_seqlen_q an upper bound on any
+ * sequence's query length.  Returns 0 for invalid arguments.
+ */
+size_t attn_fwd_varlen_workspace_size(int B, long long total_q, int max_seqlen_q);
+
+/*
+ * attn_fwd_varlen -- prefill attention over a ragged batch of packed
+ * sequences, described by cumulative sequence lengths instead of padding.
+ * Source: "Attention Kernel", section "Paged 与 ragged KV" (a ragged batch is
+ * not padded into a rectangle; cumulative sequence lengths give each
+ * sequence's range, and the offset type, empty sequences and accesses across
+ * sequence boundaries are part of the correctness contract), with the
+ * operation, masking and outputs of attn_fwd.
+ *
+ *   q   [total_q, Hq,  d] bf16   sequence b owns tokens [cu_q[b], cu_q[b+1])
+ *   k,v [total_k, Hkv, d] bf16   sequence b owns tokens [cu_k[b], cu_k[b+1])
+ *   o   [total_q, Hq,  d] bf16 (written for every token that belongs to a sequence)
+ *   lse [Hq, total_q]     fp32 (written likewise; nullable)
+ *   cu_seqlens_q, cu_seqlens_k  [B + 1] int32 device arrays: cu[0] = 0,
+ *       non-decreasing, cu_q[B] <= total_q, cu_k[B] <= total_k.  Sequence
+ *       lengths may be 0: an empty query range produces nothing, and a query
+ *       range with an empty key range gets O = 0, LSE = -inf.
+ *   Within sequence b the mask is attn_fwd's with Sq = len_q(b) and
+ *   k_len = Sk = len_k(b) (causal diagonal aligned to the bottom right).
+ *   Keys of other sequences are never visible.  A tile that straddles a
+ *   boundary reads a neighbour's rows, which then get weight exactly 0, so
+ *   inputs must be finite for that to leave the result untouched.
+ *   max_seqlen_q >= every len_q(b), at most 2^21; B >= 1; Hq % Hkv == 0;
+ *   d in {64, 128}; causal in {0, 1}; scale finite.
+ *   workspace    device scratch of at least
+ *                attn_fwd_varlen_workspace_size(B, total_q, max_seqlen_q)
+ *                bytes, 16-byte aligned; overwritten.
+ * Device-side faults: offsets that decrease, exceed the totals or give a
+ * query length above max_seqlen_q make that sequence empty (nothing of it
+ * is written) and flag ATTN_DEVERR_BAD_LENGTH.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA.
+ */
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B, int Hq,
+                    int Hkv, long long total_q, long long total_k, int max_seqlen_q, int d,
+                    int causal, float scale, void* workspace, size_t workspace_bytes,
+                    attn_stream_t stream);
 
 /*
  * attn_decode_workspace_size -- bytes of caller-owned device workspace that

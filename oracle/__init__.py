@@ -12,7 +12,8 @@ Sources followed (page title, section):
   * "Attention Kernel" -- "Online softmax" and "Blockwise reference": the
     (m, l, o) merge rule and the zero output for an all -inf row.
   * "Attention Kernel" -- "Paged 与 ragged KV": block = floor(t/q), offset =
-    t mod q, physical page through the block table.
+    t mod q, physical page through the block table; a ragged batch is a list
+    of sequences given by cumulative lengths, each attended on its own.
 
 Every function here is pinned by tests in ``tests/test_oracle_pins.py``
 against things other than itself (the notes' worked example evaluated with
@@ -156,6 +157,48 @@ def attn_fwd(q, k, v, causal, scale, k_lens=None, rows=None, n_threads=None):
         raise OracleError(st)
     if r is None:
         return o.reshape(B, Hq, Sq, d), lse.reshape(B, Hq, Sq)
+    return o, lse
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, causal, scale, n_threads=None):
+    """Exact attention over a ragged batch ("Attention Kernel", "Paged 与 ragged KV").
+
+    q [total_q, Hq, d], k/v [total_k, Hkv, d] bf16 (torch or uint16 bits),
+    packed; sequence b owns query tokens [cu_q[b], cu_q[b+1]) and key tokens
+    [cu_k[b], cu_k[b+1]).  Each sequence is attended on its own, exactly as
+    ``attn_fwd`` with B = 1, Sq = len_q, Sk = len_k (bottom-right causal
+    diagonal); nothing crosses a sequence boundary.
+    Returns (o [total_q, Hq, d], lse [Hq, total_q]) as float64 arrays; rows
+    that belong to no sequence stay NaN.
+    """
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    total_q, Hq, d = qb.shape
+    total_k, Hkv, dk = kb.shape
+    if kb.shape != vb.shape or dk != d:
+        raise ValueError("q/k/v shapes disagree")
+    cq = np.asarray(cu_seqlens_q, dtype=np.int64)
+    ck = np.asarray(cu_seqlens_k, dtype=np.int64)
+    if cq.shape != ck.shape or cq.ndim != 1 or cq.shape[0] < 2:
+        raise ValueError("cu_seqlens must both be [B+1]")
+    o = np.full((total_q, Hq, d), np.nan)
+    lse = np.full((Hq, total_q), np.nan)
+    for b in range(cq.shape[0] - 1):
+        q0, q1, k0, k1 = int(cq[b]), int(cq[b + 1]), int(ck[b]), int(ck[b + 1])
+        if not (0 <= q0 <= q1 <= total_q and 0 <= k0 <= k1 <= total_k):
+            raise ValueError(f"sequence {b}: offsets out of range")
+        if q1 == q0:
+            continue
+        # [len, H, d] -> [1, H, len, d]
+        qs = np.ascontiguousarray(qb[q0:q1].transpose(1, 0, 2))[None]
+        if k1 == k0:  # no key: every row is empty
+            o[q0:q1] = 0.0
+            lse[:, q0:q1] = -np.inf
+            continue
+        ks = np.ascontiguousarray(kb[k0:k1].transpose(1, 0, 2))[None]
+        vs = np.ascontiguousarray(vb[k0:k1].transpose(1, 0, 2))[None]
+        ob, lb = attn_fwd(qs, ks, vs, causal, scale, n_threads=n_threads)
+        o[q0:q1] = ob[0].transpose(1, 0, 2)
+        lse[:, q0:q1] = lb[0]
     return o, lse
 
 

@@ -28,8 +28,9 @@ def lib():
 
 def test_header_declares_expected_entry_points():
     names = _declared_functions()
-    for n in ("attn_fwd", "attn_fwd_masked", "attn_decode_paged", "attn_decode_workspace_size",
-              "attn_get_device_error", "attn_strerror"):
+    for n in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_fwd_varlen_workspace_size",
+              "attn_decode_paged", "attn_decode_workspace_size", "attn_get_device_error",
+              "attn_strerror"):
         assert n in names
 
 
@@ -106,6 +107,51 @@ def _dec(lib, q=FAKE, kc=FAKE, vc=FAKE, tbl=FAKE, lens=FAKE, ps=16, B_=2, Hq=8, 
 ])
 def test_decode_validation(lib, kw, status):
     assert _dec(lib, **kw) == status
+
+
+def _var(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, cq=FAKE, ck=FAKE, B_=3, Hq=8, Hkv=2,
+         tq=1000, tk=1000, maxq=512, d=128, causal=1, scale=0.1, ws=FAKE, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = lib.attn_fwd_varlen_workspace_size(B_, tq, maxq) if B_ > 0 else 0
+    return lib.attn_fwd_varlen(q, k, v, o, lse, cq, ck, B_, Hq, Hkv, tq, tk, maxq, d, causal,
+                               scale, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(cq=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(ck=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(k=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(B_=0), B.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), B.ATTN_ERR_INVALID_ARG),
+    (dict(tq=-1), B.ATTN_ERR_INVALID_ARG),
+    (dict(tk=1 << 31), B.ATTN_ERR_INVALID_ARG),
+    (dict(maxq=0), B.ATTN_ERR_INVALID_ARG),
+    (dict(maxq=(1 << 21) + 1, ws_bytes=1 << 20), B.ATTN_ERR_INVALID_ARG),
+    (dict(causal=3), B.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), B.ATTN_ERR_INVALID_ARG),
+    (dict(d=96), B.ATTN_ERR_UNSUPPORTED),
+    (dict(o=FAKE + 8), B.ATTN_ERR_ALIGNMENT),
+    (dict(cq=FAKE + 2), B.ATTN_ERR_ALIGNMENT),
+    (dict(ws=None), B.ATTN_ERR_WORKSPACE),
+    (dict(ws_bytes=16), B.ATTN_ERR_WORKSPACE),
+    (dict(ws=FAKE + 8), B.ATTN_ERR_ALIGNMENT),
+])
+def test_varlen_validation(lib, kw, status):
+    assert _var(lib, **kw) == status
+
+
+def test_varlen_empty_batch_launches_nothing(lib):
+    # total_q = 0: nothing to compute, returns OK without touching a pointer
+    assert _var(lib, tq=0) == B.ATTN_OK
+
+
+def test_varlen_workspace_size_formula(lib):
+    # one 16-byte header plus one int2 per possible (sequence, 256-row block)
+    for B_, tq in ((1, 0), (16, 60592), (3, 1000)):
+        assert lib.attn_fwd_varlen_workspace_size(B_, tq, 8192) == 16 + 8 * (tq // 256 + B_ + 1)
+    assert lib.attn_fwd_varlen_workspace_size(0, 10, 10) == 0
+    assert lib.attn_fwd_varlen_workspace_size(1, 10, 0) == 0
 
 
 def test_workspace_size_formula(lib):

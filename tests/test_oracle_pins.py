@@ -363,3 +363,90 @@ def test_decode_bad_page_id_reported():
     with pytest.raises(oracle.OracleError) as e:
         oracle.decode_paged(inp.q, inp.k_cache, inp.v_cache, tbl, inp.seq_lens, 0.5)
     assert e.value.status == oracle.ERR_TABLE
+
+
+# --------------------------------------------------------------------------- ragged batches
+# "Attention Kernel", section "Paged 与 ragged KV": a ragged batch is a list of
+# sequences given by cumulative lengths; nothing crosses a sequence boundary.
+
+
+def _packed(x):
+    """[B, H, S, d] -> packed token-major [B*S, H, d]."""
+    B, H, S, d = x.shape
+    return x.permute(0, 2, 1, 3).reshape(B * S, H, d).contiguous()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_equal_lengths_equals_batched(causal):
+    B, Hq, Hkv, S, d = 3, 4, 2, 23, 8
+    q, k, v = workloads.prefill_inputs(B, Hq, Hkv, S, S, d, seed=41)
+    cu = workloads.cu_seqlens([S] * B)
+    o, lse = oracle.attn_fwd_varlen(_packed(q), _packed(k), _packed(v), cu, cu, causal, 0.3)
+    ob, lb = oracle.attn_fwd(q, k, v, causal, 0.3)
+    np.testing.assert_array_equal(o, ob.transpose(0, 2, 1, 3).reshape(B * S, Hq, d))
+    np.testing.assert_array_equal(lse, lb.transpose(1, 0, 2).reshape(Hq, B * S))
+
+
+def test_varlen_sequences_do_not_see_each_other():
+    # changing every token of sequence 1 leaves sequences 0 and 2 bit-identical
+    lens = [7, 12, 5]
+    q, k, v, cu_q, cu_k = workloads.varlen_inputs(lens, lens, 2, 1, 4, seed=43)
+    o, lse = oracle.attn_fwd_varlen(q, k, v, cu_q, cu_k, True, 0.5)
+    k2, v2 = k.clone(), v.clone()
+    k2[7:19] = -k2[7:19] * 3
+    v2[7:19] = v2[7:19] + 7
+    o2, lse2 = oracle.attn_fwd_varlen(q, k2, v2, cu_q, cu_k, True, 0.5)
+    for a, b in ((0, 7), (19, 24)):
+        np.testing.assert_array_equal(o[a:b], o2[a:b])
+        np.testing.assert_array_equal(lse[:, a:b], lse2[:, a:b])
+    assert not np.array_equal(o[7:19], o2[7:19])
+
+
+def test_varlen_empty_query_and_key_ranges():
+    # sequence 1 has no query (nothing written: NaN), sequence 2 no key (O = 0, LSE = -inf)
+    lens_q, lens_k = [4, 0, 3], [4, 6, 0]
+    q, k, v, cu_q, cu_k = workloads.varlen_inputs(lens_q, lens_k, 2, 2, 4, seed=47)
+    o, lse = oracle.attn_fwd_varlen(q, k, v, cu_q, cu_k, False, 0.5)
+    assert np.isfinite(o[:4]).all() and np.isfinite(lse[:, :4]).all()
+    assert np.array_equal(o[4:7], np.zeros((3, 2, 4)))
+    assert np.isneginf(lse[:, 4:7]).all()
+
+
+def test_varlen_worked_example_masked_key_is_the_next_sequence():
+    # The worked example with its -inf key realised as a sequence boundary: the
+    # row sees keys [1, 3, -2, 0] (values as in the golden file, reordered);
+    # the key after them, with value [3, 4, 5], is the first key of the next
+    # sequence and must not contribute.
+    g, _, value = _golden()
+    d = 4
+    s = [1.0, 3.0, -2.0, 0.0, 5.0]
+    rows = [0, 2, 3, 4, 1]  # golden value rows for those keys
+    q = torch.zeros(2, 1, d, dtype=torch.bfloat16)
+    q[:, 0, 0] = 1.0
+    k = torch.zeros(5, 1, d, dtype=torch.bfloat16)
+    v = torch.zeros(5, 1, d, dtype=torch.bfloat16)
+    for j in range(5):
+        k[j, 0, 0] = s[j]
+        v[j, 0, :3] = torch.tensor(value[rows[j]], dtype=torch.bfloat16)
+    cu_q = torch.tensor([0, 1, 2], dtype=torch.int32)
+    cu_k = torch.tensor([0, 4, 5], dtype=torch.int32)
+    o, lse = oracle.attn_fwd_varlen(q, k, v, cu_q, cu_k, False, 1.0)
+    np.testing.assert_allclose(o[0, 0, :3], g["expected_o"], rtol=0, atol=1e-12)
+    assert abs(lse[0, 0] - g["expected_lse"]) < 1e-12
+    np.testing.assert_allclose(o[1, 0, :3], value[1], rtol=0, atol=0)  # one key: O = its value
+    assert lse[0, 1] == 5.0
+
+
+def test_varlen_bottom_right_causal_last_row_sees_every_key():
+    # len_q < len_k: the last query row of a causal sequence sees all of its
+    # keys, so it equals the non-causal result; the first row sees
+    # len_k - len_q + 1 keys.
+    lens_q, lens_k = [3, 5], [9, 5]
+    q, k, v, cu_q, cu_k = workloads.varlen_inputs(lens_q, lens_k, 2, 1, 4, seed=53)
+    oc, lc = oracle.attn_fwd_varlen(q, k, v, cu_q, cu_k, True, 0.7)
+    on, ln = oracle.attn_fwd_varlen(q, k, v, cu_q, cu_k, False, 0.7)
+    np.testing.assert_array_equal(oc[2], on[2])
+    np.testing.assert_array_equal(oc[7], on[7])
+    # first row of sequence 0 == non-causal attention over its first 7 keys
+    o7, l7 = oracle.attn_fwd_varlen(q[:1], k[:7], v[:7], [0, 1], [0, 7], False, 0.7)
+    np.testing.assert_array_equal(oc[0], o7[0])
