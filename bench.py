@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-ragged", action="store_true")
     ap.add_argument("--ragged-workload", default="ragged_gqa_causal")
+    ap.add_argument("--no-paged-prefill", action="store_true")
+    ap.add_argument("--paged-prefill-workload", default="paged_prefill_gqa")
     return ap.parse_args()
 
 
@@ -406,11 +408,77 @@ def run_ours(args, world, rank, local):
 
     if not args.no_ragged:
         line["ragged"] = ragged_leg(args, dev, world, peaks)
+    if not args.no_paged_prefill:
+        line["paged_prefill"] = paged_prefill_leg(args, dev, world, peaks)
     if not args.no_e2e:
         line["e2e"] = e2e_leg(args, cfg, q_h, k_h, v_h, kl_h, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_leg(cfg, q_h, k_h, v_h, kl_h)
     return line if rank == 0 else None
+
+
+def _timed_calls(args, dev, world, one):
+    """Warm up, then time n calls of `one` (L2 flushed before each, CUDA events on the
+    launch stream around each); returns the per-call milliseconds."""
+    import torch
+
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(3):
+        flush.fill_(1.0)
+        one()
+    torch.cuda.synchronize(dev)
+    n = max(5, min(args.steps, 50))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    barrier(world)
+    for e0, e1 in evs:
+        flush.fill_(1.0)
+        e0.record(stream)
+        one()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def paged_prefill_leg(args, dev, world, peaks):
+    """Chunked prefill over a paged cache (attn_fwd_paged: the unit-list kernel and the
+    prefill kernel reading K/V page by page), timed on its own like the ragged leg."""
+    import torch
+
+    from exact_softmax_attention_fwd_b200 import (attn_fwd_paged, attn_fwd_varlen_workspace_size,
+                                                  attn_get_device_error)
+    from exact_softmax_attention_fwd_b200 import workloads as W
+
+    pc = W.CONFIGS[args.paged_prefill_workload]
+    q_h, cu_q_h, cache, lq, lk = W.paged_prefill_config_inputs(pc)
+    q, cu_q = q_h.to(dev), cu_q_h.to(dev)
+    kc, vc = cache.k_cache.to(dev), cache.v_cache.to(dev)
+    tbl, lens = cache.block_table.to(dev), cache.seq_lens.to(dev)
+    max_q = int(lq.max())
+    ws = torch.empty(attn_fwd_varlen_workspace_size(pc.B, q.shape[0], max_q), dtype=torch.uint8,
+                     device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((pc.Hq, q.shape[0]), dtype=torch.float32, device=dev)
+
+    def one():
+        attn_fwd_paged(q, kc, vc, tbl, cu_q, lens, max_q, True, pc.scale, out=o, lse=lse,
+                       workspace=ws)
+
+    ms = _timed_calls(args, dev, world, one)
+    st, fl = attn_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word set in the paged-prefill leg: {fl:#x}")
+    flops = pc.flops()
+    flops_per_s, avg = weak_scaling_value(flops, sum(ms) / len(ms), world)
+    achieved = flops / (avg * 1e-3) / 1e12
+    return {"workload": pc.name, "value": flops_per_s / 1e12, "unit": "TFLOPS", "ms": avg,
+            "median_ms": statistics.median(ms), "calls": len(ms), "gpu_launches_per_call": 2,
+            "sequences": pc.B, "new_tokens": int(q.shape[0]), "page_size": pc.page_size,
+            "keys": f"cached uniform {pc.cached_lo}..{pc.cached_hi} + {pc.new_tokens} new (seed {pc.seed})",
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "per_call_flops": flops}}
 
 
 def ragged_leg(args, dev, world, peaks):

@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     attn_decode_workspace_size,
     attn_fwd,
     attn_fwd_masked,
+    attn_fwd_paged,
     attn_fwd_varlen,
     attn_fwd_varlen_workspace_size,
     attn_get_device_error,

@@ -39,6 +39,8 @@ SIGNATURES = {
     "attn_fwd_varlen_workspace_size": (_SZ, [_I, ctypes.c_longlong, _I]),
     "attn_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, ctypes.c_longlong,
                              ctypes.c_longlong, _I, _I, _I, _F, _P, _SZ, _P]),
+    "attn_fwd_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_longlong, _I, _I,
+                            _I, _I, _I, _F, _P, _P, _P, _SZ, _P]),
     "attn_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P,
                                _SZ, _P]),
@@ -177,6 +179,46 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, caus
                                         int(bool(causal)), float(scale), _ptr(workspace),
                                         ws_bytes, _stream(stream))
     _check(st, "attn_fwd_varlen")
+    return out, lse
+
+
+def attn_fwd_paged(q, k_cache, v_cache, block_table, cu_seqlens_q, seq_lens_k, max_seqlen_q: int,
+                   causal: bool, scale: float, out=None, lse=None, workspace=None,
+                   return_lse: bool = True, stream=None):
+    """Prefill/append of packed queries q [total_q, Hq, d] over a paged cache
+    [num_pages, page_size, Hkv, d]; returns O [total_q, Hq, d], LSE [Hq, total_q]."""
+    import torch
+    _require_cuda(q, k_cache, v_cache, block_table, cu_seqlens_q, seq_lens_k)
+    for t in (q, k_cache, v_cache):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("q and the caches must be contiguous bfloat16")
+    if q.dim() != 3 or k_cache.dim() != 4 or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("q [total_q, Hq, d]; caches [num_pages, page_size, Hkv, d]")
+    total_q, Hq, d = q.shape
+    num_pages, page_size, Hkv, dk = k_cache.shape
+    if dk != d:
+        raise ValueError("head dims disagree")
+    B = cu_seqlens_q.shape[0] - 1
+    for t, shape in ((cu_seqlens_q, (B + 1,)), (seq_lens_k, (B,))):
+        if t.dtype != torch.int32 or tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError("cu_seqlens_q int32 [B+1], seq_lens_k int32 [B]")
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != B \
+            or not block_table.is_contiguous():
+        raise ValueError("block_table must be contiguous int32 [B, max_pages_per_seq]")
+    need = attn_fwd_varlen_workspace_size(B, total_q, max_seqlen_q)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = load_library().attn_fwd_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                       _ptr(cu_seqlens_q), _ptr(seq_lens_k), page_size, B, Hq,
+                                       Hkv, total_q, int(max_seqlen_q), block_table.shape[1],
+                                       num_pages, d, int(bool(causal)), float(scale), _ptr(out),
+                                       _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "attn_fwd_paged")
     return out, lse
 
 

@@ -61,15 +61,18 @@ bool make_tile_map(CUtensorMap* map, const void* ptr, int D, long long rows, lon
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D bf16 map over a packed token-major [tokens, heads, D] tensor, box = 128
-// tokens of one head x 64 columns, 128-byte swizzle: the same shared-memory
-// tile as make_tile_map gives (128 rows of 128 bytes).
-bool make_token_map(CUtensorMap* map, const void* ptr, int D, long long heads, long long tokens) {
+// 3-D bf16 map over a packed token-major [tokens, heads, D] tensor, box =
+// box_rows tokens of one head x 64 columns, 128-byte swizzle: with 128 rows the
+// same shared-memory tile as make_tile_map gives (128 rows of 128 bytes); a
+// paged pool [num_pages, page_size, heads, D] is such a tensor with
+// num_pages * page_size tokens, read one page (box_rows = page_size) at a time.
+bool make_token_map(CUtensorMap* map, const void* ptr, int D, long long heads, long long tokens,
+                    unsigned box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)tokens};
   const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
-  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t box[3] = {64, 1, box_rows};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -93,12 +96,13 @@ int sm_count() {
   return cached[dev];
 }
 
-template <int D, bool CAUSAL, bool VARLEN = false>
+template <int D, bool CAUSAL, int LAYOUT = kLayoutDense>
 int launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                    const CUtensorMap& mo, const PrefillParams& prm, cudaStream_t stream,
                    long long max_units = 0) {
   using C = PrefillCfg<D>;
-  auto kern = attn_prefill_sm100_kernel<D, CAUSAL, VARLEN>;
+  constexpr bool VARLEN = LAYOUT != kLayoutDense;
+  auto kern = attn_prefill_sm100_kernel<D, CAUSAL, LAYOUT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
       cudaSuccess)
     return ATTN_ERR_CUDA;
@@ -241,15 +245,16 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   int* unit_count = static_cast<int*>(workspace);
   int2* units = reinterpret_cast<int2*>(static_cast<char*>(workspace) + 16);
   const long long max_units = varlen_max_units(B, total_q);
-  const int n_levels = (max_seqlen_q + 255) / 256;
+  int shift, n_levels;
+  varlen_levels(total_k, shift, n_levels);  // total_k bounds every key range
   const size_t sched_smem = (size_t)(2 * n_levels + 32) * sizeof(int);
   if (cudaFuncSetAttribute(attn_varlen_schedule_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sched_smem) !=
       cudaSuccess)
     return ATTN_ERR_CUDA;
   attn_varlen_schedule_kernel<<<1, 1024, sched_smem, stream>>>(
-      cu_seqlens_q, cu_seqlens_k, B, (int)total_q, (int)total_k, max_seqlen_q, units, unit_count,
-      (int)max_units);
+      cu_seqlens_q, cu_seqlens_k, nullptr, B, (int)total_q, (int)total_k, max_seqlen_q, 0, causal,
+      shift, n_levels, units, unit_count, (int)max_units);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   // 2. the prefill kernel over packed token-major tensors
   CUtensorMap mq, mk, mv;
@@ -273,10 +278,86 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   prm.total_q = (int)total_q;
   // the output map is unused by the ragged path (rows are stored one by one)
   if (d == 128)
-    return causal ? launch_prefill<128, true, true>(mq, mk, mv, mq, prm, stream, max_units)
-                  : launch_prefill<128, false, true>(mq, mk, mv, mq, prm, stream, max_units);
-  return causal ? launch_prefill<64, true, true>(mq, mk, mv, mq, prm, stream, max_units)
-                : launch_prefill<64, false, true>(mq, mk, mv, mq, prm, stream, max_units);
+    return causal ? launch_prefill<128, true, kLayoutRagged>(mq, mk, mv, mq, prm, stream, max_units)
+                  : launch_prefill<128, false, kLayoutRagged>(mq, mk, mv, mq, prm, stream, max_units);
+  return causal ? launch_prefill<64, true, kLayoutRagged>(mq, mk, mv, mq, prm, stream, max_units)
+                : launch_prefill<64, false, kLayoutRagged>(mq, mk, mv, mq, prm, stream, max_units);
+}
+
+int attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache,
+                   const int32_t* block_table, const int32_t* cu_seqlens_q,
+                   const int32_t* seq_lens_k, int page_size, int B, int Hq, int Hkv,
+                   long long total_q, int max_seqlen_q, int max_pages_per_seq, int num_pages, int d,
+                   int causal, float scale, void* o, float* lse, void* workspace,
+                   size_t workspace_bytes, attn_stream_t stream_) {
+  if (q == nullptr || o == nullptr || k_cache == nullptr || v_cache == nullptr ||
+      block_table == nullptr || cu_seqlens_q == nullptr || seq_lens_k == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq > 65535) return ATTN_ERR_INVALID_ARG;
+  if (total_q < 0 || total_q > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  if (max_seqlen_q < 1 || max_seqlen_q > kVarlenMaxLevels * 256) return ATTN_ERR_INVALID_ARG;
+  if (max_pages_per_seq < 1 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
+  if ((long long)max_pages_per_seq * page_size > 0x7fffffffLL ||
+      (long long)num_pages * page_size > 0x7fffffffLL)
+    return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128)
+    return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(k_cache) || !aligned16(v_cache))
+    return ATTN_ERR_ALIGNMENT;
+  if ((lse != nullptr && !aligned4(lse)) || !aligned4(cu_seqlens_q) || !aligned4(seq_lens_k) ||
+      !aligned4(block_table))
+    return ATTN_ERR_ALIGNMENT;
+  const size_t need = attn_fwd_varlen_workspace_size(B, total_q, max_seqlen_q);
+  if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (total_q == 0) return ATTN_OK;
+  int* unit_count = static_cast<int*>(workspace);
+  int2* units = reinterpret_cast<int2*>(static_cast<char*>(workspace) + 16);
+  const long long max_units = varlen_max_units(B, total_q);
+  const int max_keys = max_pages_per_seq * page_size;
+  int shift, n_levels;
+  varlen_levels(max_keys, shift, n_levels);
+  const size_t sched_smem = (size_t)(2 * n_levels + 32) * sizeof(int);
+  if (cudaFuncSetAttribute(attn_varlen_schedule_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sched_smem) !=
+      cudaSuccess)
+    return ATTN_ERR_CUDA;
+  attn_varlen_schedule_kernel<<<1, 1024, sched_smem, stream>>>(
+      cu_seqlens_q, nullptr, seq_lens_k, B, (int)total_q, 0, max_seqlen_q, max_keys, causal,
+      shift, n_levels, units, unit_count, (int)max_units);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  CUtensorMap mq, mk, mv;
+  if (!make_token_map(&mq, q, d, Hq, total_q) ||
+      !make_token_map(&mk, k_cache, d, Hkv, (long long)num_pages * page_size, page_size) ||
+      !make_token_map(&mv, v_cache, d, Hkv, (long long)num_pages * page_size, page_size))
+    return ATTN_ERR_CUDA;
+  PrefillParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.lse = lse;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.o = static_cast<uint16_t*>(o);
+  prm.cu_q = cu_seqlens_q;
+  prm.seq_lens_k = seq_lens_k;
+  prm.block_table = block_table;
+  prm.max_pages = max_pages_per_seq;
+  prm.page_size = page_size;
+  prm.num_pages = num_pages;
+  prm.units = units;
+  prm.unit_count = unit_count;
+  prm.total_q = (int)total_q;
+  if (d == 128)
+    return causal ? launch_prefill<128, true, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units)
+                  : launch_prefill<128, false, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units);
+  return causal ? launch_prefill<64, true, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units)
+                : launch_prefill<64, false, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units);
 }
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,

@@ -52,6 +52,8 @@
 // falls back to 0 while the running max is -inf, so P = 2^-inf = 0 and l = 0.
 #pragma once
 
+#include <climits>
+
 #include "sm100_primitives.cuh"
 
 namespace attn_b200 {
@@ -67,7 +69,11 @@ struct PrefillParams {
   // and the unit list written by attn_varlen_schedule_kernel
   uint16_t* o;          // [total_q, Hq, d] bf16
   const int* cu_q;      // [B + 1]
-  const int* cu_k;      // [B + 1]
+  const int* cu_k;      // [B + 1] (ragged K/V) or nullptr (paged K/V)
+  // paged K/V: [num_pages, page_size, Hkv, d] caches addressed by a block table
+  const int* seq_lens_k;    // [B] keys of each sequence
+  const int* block_table;   // [B, max_pages]
+  int max_pages, page_size, num_pages;
   const int2* units;    // (sequence, query block), heaviest first
   const int* unit_count;
   int total_q;
@@ -115,6 +121,13 @@ struct PrefillCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
+// Tensor layouts of a prefill kernel instantiation: dense [B, H, S, d]; a
+// ragged batch of packed token-major [tokens, H, d] tensors; or packed
+// queries over a paged K/V cache.
+constexpr int kLayoutDense = 0;
+constexpr int kLayoutRagged = 1;
+constexpr int kLayoutPaged = 2;
+
 // Number of 128-key tiles the query tile with first row `row0` must visit
 // (0 when the tile is past Sq or none of its rows sees a key).
 __device__ __forceinline__ int prefill_num_kv_tiles(int row0, int Sq, int klen, bool causal) {
@@ -140,8 +153,9 @@ struct PrefillUnit {
 // are ordered heaviest first (q-blocks descending, heads inner) and dealt
 // back and forth across the CTAs: rank k*G + c for even k, k*G + G-1-c for odd.
 // For a ragged batch the (sequence, q-block) order comes from the unit list.
-template <bool CAUSAL, bool VARLEN>
+template <bool CAUSAL, int LAYOUT>
 __device__ __forceinline__ bool prefill_unit(const PrefillParams& p, int k, PrefillUnit& u) {
+  constexpr bool VARLEN = LAYOUT != kLayoutDense;
   const long long G = gridDim.x;
   const long long c = blockIdx.x;
   const long long r = (long long)k * G + ((k & 1) ? (G - 1 - c) : c);
@@ -152,9 +166,14 @@ __device__ __forceinline__ bool prefill_unit(const PrefillParams& p, int k, Pref
     u.b = e.x;
     u.qb = e.y;
     u.q_tok0 = __ldg(p.cu_q + u.b);
-    u.k_tok0 = __ldg(p.cu_k + u.b);
     u.sq = __ldg(p.cu_q + u.b + 1) - u.q_tok0;  // listed sequences passed the
-    u.klen = __ldg(p.cu_k + u.b + 1) - u.k_tok0;  // schedule kernel's checks
+    if (LAYOUT == kLayoutPaged) {                  // schedule kernel's checks
+      u.k_tok0 = 0;
+      u.klen = __ldg(p.seq_lens_k + u.b);
+    } else {
+      u.k_tok0 = __ldg(p.cu_k + u.b);
+      u.klen = __ldg(p.cu_k + u.b + 1) - u.k_tok0;
+    }
   } else {
     const long long HB = (long long)p.Hq * p.B;
     if (r >= (long long)p.n_qblocks * HB) return false;
@@ -180,13 +199,15 @@ __device__ __forceinline__ bool prefill_unit(const PrefillParams& p, int k, Pref
   return true;
 }
 
-template <int D, bool CAUSAL, bool VARLEN>
+template <int D, bool CAUSAL, int LAYOUT>
 __global__ void __launch_bounds__(384, 1)
     attn_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                               const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v,
                               const __grid_constant__ CUtensorMap tm_o, const PrefillParams p) {
   using C = PrefillCfg<D>;
+  constexpr bool VARLEN = LAYOUT != kLayoutDense;
+  constexpr bool PAGED = LAYOUT == kLayoutPaged;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
@@ -216,6 +237,15 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
     mbar_init_fence();
+    fence_proxy_async_smem();
+  }
+  if (PAGED) {
+    // K/V rows of a tile that no page fills (past the sequence's last page, or
+    // a skipped page id) keep what the ring held before: zeros at first, then
+    // earlier cache rows -- finite either way, and masked to weight 0.
+    uint4* ring = reinterpret_cast<uint4*>(sbase_ptr + C::OFF_K);
+    for (int x = threadIdx.x; x < 2 * C::STAGES * C::TILE_BYTES / 16; x += C::NUM_THREADS)
+      ring[x] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
   }
   if (warp == 1) {
@@ -254,10 +284,15 @@ __global__ void __launch_bounds__(384, 1)
         return true;
       };
       PrefillUnit u;
-      for (int k = 0; ok && prefill_unit<CAUSAL, VARLEN>(p, k, u); ++k) {
+      for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT>(p, k, u); ++k) {
         const int n_max = max(u.nkv[0], u.nkv[1]);
         const int kvh = u.hq / p.group;
         const int kv_row = u.b * p.Hkv + kvh;
+        if (PAGED) {  // warp 2 streams paged K/V; this thread only loads Q
+          if (u.nkv[0] > 0 && !(ok = load_q(u, 0))) break;
+          if (u.nkv[1] > 0 && !(ok = load_q(u, 1))) break;
+          continue;
+        }
         // Q_0 first (its slot frees first under a causal mask), then the first
         // K tile, then Q_1, so that no wait on Q_1 holds back the K/V stream.
         if (u.nkv[0] > 0 && !(ok = load_q(u, 0))) break;
@@ -290,6 +325,62 @@ __global__ void __launch_bounds__(384, 1)
       // never armed would only run into the time limit, so V is skipped then.)
       if (q_loads0 > 0) mbar_wait(bar(C::B_QFULL + 0), (q_loads0 - 1) & 1u, nullptr);
       if (q_loads1 > 0) mbar_wait(bar(C::B_QFULL + 1), (q_loads1 - 1) & 1u, nullptr);
+      for (uint32_t j = (kv > C::STAGES ? kv - C::STAGES : 0); j < kv; ++j) {
+        mbar_wait(bar(C::B_KFULL + j % C::STAGES), (j / C::STAGES) & 1u, nullptr);
+        if (ok) mbar_wait(bar(C::B_VFULL + j % C::STAGES), (j / C::STAGES) & 1u, nullptr);
+      }
+    }
+    __syncwarp();
+  } else if (PAGED && warp == 2) {
+    // ================ paged K/V loader (all 32 lanes) ================
+    // The 128-key tile j is 128 / page_size (<= 8) pages.  Lane t reads the
+    // block-table entry of page t and issues that page's TMA boxes (page_size
+    // rows of one KV head per 64-column block), so a tile's copies go out in
+    // one pass of the warp.  The pool [num_pages, page_size, Hkv, d] is read as
+    // the token-major tensor [num_pages * page_size, Hkv, d] (page p starts at
+    // token p * page_size).  The barrier's byte count (valid pages, counted by
+    // a ballot) is set by lane 0 before any copy is issued.
+    constexpr int kNoPage = INT_MIN;  // past the sequence's last page
+    uint32_t kv = 0;                  // K/V tiles issued so far (ring position)
+    bool ok = true;
+    PrefillUnit u;
+    for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT>(p, k, u); ++k) {
+      const int n_max = max(u.nkv[0], u.nkv[1]);
+      const int kvh = u.hq / p.group;
+      const int ppt = 128 / p.page_size;
+      const int n_lp = (u.klen + p.page_size - 1) / p.page_size;  // <= max_pages
+      const int* tbl = p.block_table + (size_t)u.b * p.max_pages;
+      const uint32_t row_off = (uint32_t)(lane * p.page_size * 128);
+      for (int j = 0; j < n_max; ++j, ++kv) {
+        const int s = kv % C::STAGES;
+        const uint32_t ph = (kv / C::STAGES) & 1u;
+        const int lp = j * ppt + lane;
+        const int phys = (lane < ppt && lp < n_lp) ? __ldg(tbl + lp) : kNoPage;
+        const bool valid = phys >= 0 && phys < p.num_pages;
+        if (phys != kNoPage && !valid) flag_device_error(kDevErrBadPage);  // skipped: its
+        const uint32_t bytes = (uint32_t)__popc(__ballot_sync(0xffffffffu, valid)) *  // keys read
+                               (uint32_t)(p.page_size * 128 * C::NCB);  // as earlier finite rows
+        if (!(ok = mbar_wait_warp(bar(C::B_KEMPTY + s), ph ^ 1u, abort_flag))) break;
+        if (lane == 0) mbar_arrive_expect_tx(bar(C::B_KFULL + s), bytes);
+        __syncwarp();
+        if (valid)
+          for (int cb = 0; cb < C::NCB; ++cb)
+            tma_load_3d(sbase + C::OFF_K + s * C::TILE_BYTES + cb * C::CB_BYTES + row_off, &tm_k,
+                        bar(C::B_KFULL + s), 64 * cb, kvh, phys * p.page_size);
+        if (!(ok = mbar_wait_warp(bar(C::B_VEMPTY + s), ph ^ 1u, abort_flag))) {
+          ++kv;  // K of this tile was issued
+          break;
+        }
+        if (lane == 0) mbar_arrive_expect_tx(bar(C::B_VFULL + s), bytes);
+        __syncwarp();
+        if (valid)
+          for (int cb = 0; cb < C::NCB; ++cb)
+            tma_load_3d(sbase + C::OFF_V + s * C::TILE_BYTES + cb * C::CB_BYTES + row_off, &tm_v,
+                        bar(C::B_VFULL + s), 64 * cb, kvh, phys * p.page_size);
+      }
+    }
+    // Drain as the producer does: no copy may still be landing at exit.
+    if (lane == 0) {
       for (uint32_t j = (kv > C::STAGES ? kv - C::STAGES : 0); j < kv; ++j) {
         mbar_wait(bar(C::B_KFULL + j % C::STAGES), (j / C::STAGES) & 1u, nullptr);
         if (ok) mbar_wait(bar(C::B_VFULL + j % C::STAGES), (j / C::STAGES) & 1u, nullptr);
@@ -330,7 +421,7 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t p_waits0 = 0, p_waits1 = 0;  // P_FULL phases consumed per tile slot
       bool ok = true;
       PrefillUnit u;
-      for (int k = 0; ok && prefill_unit<CAUSAL, VARLEN>(p, k, u); ++k) {
+      for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT>(p, k, u); ++k) {
         const int n_max = max(u.nkv[0], u.nkv[1]);
         if (n_max == 0) continue;
         // prologue: S_i(0) for each participating tile
@@ -411,7 +502,7 @@ __global__ void __launch_bounds__(384, 1)
     bool stores_pending = false;
     bool ok = true;
     PrefillUnit u;
-    for (int k = 0; ok && prefill_unit<CAUSAL, VARLEN>(p, k, u); ++k) {
+    for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT>(p, k, u); ++k) {
       const int row0 = i ? u.row0[1] : u.row0[0];
       if (row0 >= u.sq) continue;  // this tile slot holds no rows in this unit
       const int n = i ? u.nkv[1] : u.nkv[0];

@@ -4,37 +4,64 @@
 // by cumulative sequence lengths instead of being padded into a rectangle.
 // The prefill kernel's work unit is (sequence b, 256-row query block qb, query
 // head); this kernel lists the (b, qb) pairs so that the persistent prefill
-// kernel can deal them out heaviest first: query blocks in descending qb
-// (under a causal mask a block's KV work grows with its index), sequences of
-// the same qb in arbitrary order.  The order only affects which CTA computes a
-// unit, never its result, so the output stays bitwise deterministic.
+// kernel can deal them out heaviest first.  A unit's weight is the number of
+// 128-key tiles its two query tiles visit (the kernel's own visibility rule),
+// so that long and short sequences, square prefill and appends to a long
+// cache are all ordered by the work they carry.  Units of equal weight come in
+// arbitrary order; the order only decides which CTA computes a unit, never its
+// result, so the output stays bitwise deterministic.
 //
-// One CTA of 1024 threads, a counting sort by qb:
-//   cnt[L]  = number of sequences whose last query block is L
-//   c[L]    = number of sequences with more than L blocks   (suffix sum of cnt)
-//   off[L]  = first list position of level L = sum of c over levels above L
-// then each (b, L) takes position off[L] + atomicAdd(cursor[L], 1).
+// One CTA of 1024 threads, a counting sort by weight level
+// (level = weight >> shift, at most kVarlenMaxLevels levels):
+//   cnt[L]  = number of units of level L
+//   off[L]  = first list position of level L = number of units above level L
+// then each unit takes position off[L] + atomicAdd(cursor[L], 1).
 // A sequence whose offsets decrease, leave [0, total] or exceed max_seqlen_q
-// is left out and flagged (ATTN_DEVERR_BAD_LENGTH).
+// (or, over a paged cache, whose key length exceeds the block table) is left
+// out and flagged (ATTN_DEVERR_BAD_LENGTH).
 #pragma once
 
 #include "sm100_primitives.cuh"
 
 namespace attn_b200 {
 
-constexpr int kVarlenMaxLevels = 8192;  // max_seqlen_q <= 2^21
+constexpr int kVarlenMaxLevels = 8192;  // counting-sort levels (shared memory: 2 ints each)
 
-// Query blocks of sequence b, or 0 (flagged) when its offsets are not valid.
-__device__ __forceinline__ int varlen_seq_blocks(const int* cu_q, const int* cu_k, int b,
-                                                 int total_q, int total_k, int max_seqlen_q) {
-  const int q0 = cu_q[b], q1 = cu_q[b + 1], k0 = cu_k[b], k1 = cu_k[b + 1];
-  const bool bad = q0 < 0 || q1 < q0 || q1 > total_q || k0 < 0 || k1 < k0 || k1 > total_k ||
-                   q1 - q0 > max_seqlen_q;
-  if (bad) {
-    flag_device_error(kDevErrBadLength);
-    return 0;
+// Query rows and keys of sequence b, or false (flagged) when its offsets are
+// not valid.
+// Keys come either as packed ranges (cu_k) or, for a paged cache, as lengths
+// (seq_lens_k, at most max_keys = the block table's capacity).
+__device__ __forceinline__ bool varlen_seq_lengths(const int* cu_q, const int* cu_k,
+                                                   const int* seq_lens_k, int b, int total_q,
+                                                   int total_k, int max_seqlen_q, int max_keys,
+                                                   int& len_q, int& len_k) {
+  const int q0 = cu_q[b], q1 = cu_q[b + 1];
+  bool bad = q0 < 0 || q1 < q0 || q1 > total_q || q1 - q0 > max_seqlen_q;
+  if (cu_k != nullptr) {
+    const int k0 = cu_k[b], k1 = cu_k[b + 1];
+    bad = bad || k0 < 0 || k1 < k0 || k1 > total_k;
+    len_k = k1 - k0;
+  } else {
+    len_k = seq_lens_k[b];
+    bad = bad || len_k < 0 || len_k > max_keys;
   }
-  return (q1 - q0 + 255) / 256;
+  len_q = q1 - q0;
+  if (bad) flag_device_error(kDevErrBadLength);
+  return !bad;
+}
+
+// 128-key tiles the two query tiles of block qb visit (as prefill_num_kv_tiles).
+__device__ __forceinline__ int varlen_unit_weight(int qb, int len_q, int len_k, bool causal) {
+  int w = 0;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int row0 = qb * 256 + i * 128;
+    if (row0 >= len_q) continue;
+    long long lim = (long long)len_k - 1;
+    if (causal) lim = min(lim, (long long)min(row0 + 127, len_q - 1) + len_k - len_q);
+    if (lim >= 0) w += (int)(lim / 128) + 1;
+  }
+  return w;
 }
 
 // a[0..n) := suffix sums of a (inclusive, or exclusive when `exclusive`),
@@ -77,37 +104,56 @@ __device__ __forceinline__ void block_suffix_sum(int* a, int n, bool exclusive, 
 
 // Writes unit_count and units[0 .. unit_count) (at most max_units entries).
 __global__ void __launch_bounds__(1024, 1)
-    attn_varlen_schedule_kernel(const int* cu_q, const int* cu_k, int B, int total_q, int total_k,
-                                int max_seqlen_q, int2* units, int* unit_count, int max_units) {
+    attn_varlen_schedule_kernel(const int* cu_q, const int* cu_k, const int* seq_lens_k, int B,
+                                int total_q, int total_k, int max_seqlen_q, int max_keys,
+                                int causal, int level_shift, int n_levels, int2* units,
+                                int* unit_count, int max_units) {
   extern __shared__ int sh[];
-  const int n_levels = (max_seqlen_q + 255) / 256;
-  int* lev = sh;                // cnt, then c, then off / cursors
-  int* cnt_copy = sh + n_levels;  // c kept for the total
+  int* lev = sh;                  // counts, then first positions / cursors
+  int* cnt_copy = sh + n_levels;  // counts kept for the total
   int* warp_sums = sh + 2 * n_levels;
   for (int L = threadIdx.x; L < n_levels; L += blockDim.x) lev[L] = 0;
   __syncthreads();
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
-    const int nqb = varlen_seq_blocks(cu_q, cu_k, b, total_q, total_k, max_seqlen_q);
-    if (nqb > 0) atomicAdd(&lev[nqb - 1], 1);
+    int lq, lk;
+    if (!varlen_seq_lengths(cu_q, cu_k, seq_lens_k, b, total_q, total_k, max_seqlen_q, max_keys,
+                            lq, lk))
+      continue;
+    for (int qb = 0; qb * 256 < lq; ++qb) {
+      const int L = min(varlen_unit_weight(qb, lq, lk, causal != 0) >> level_shift, n_levels - 1);
+      atomicAdd(&lev[L], 1);
+    }
   }
   __syncthreads();
-  block_suffix_sum(lev, n_levels, false, warp_sums);  // lev[L] = c[L]
   for (int L = threadIdx.x; L < n_levels; L += blockDim.x) cnt_copy[L] = lev[L];
   __syncthreads();
-  block_suffix_sum(lev, n_levels, true, warp_sums);   // lev[L] = off[L]
+  block_suffix_sum(lev, n_levels, true, warp_sums);  // lev[L] = units above level L
   if (threadIdx.x == 0) {
-    const long long total = (long long)lev[0] + cnt_copy[0];  // off[0] + c[0]
+    const long long total = (long long)lev[0] + cnt_copy[0];
     if (total > max_units) flag_device_error(kDevErrBadLength);  // overlapping ranges
     *unit_count = (int)(total < max_units ? total : max_units);
   }
   __syncthreads();
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
-    const int nqb = varlen_seq_blocks(cu_q, cu_k, b, total_q, total_k, max_seqlen_q);
-    for (int L = 0; L < nqb; ++L) {
+    int lq, lk;
+    if (!varlen_seq_lengths(cu_q, cu_k, seq_lens_k, b, total_q, total_k, max_seqlen_q, max_keys,
+                            lq, lk))
+      continue;
+    for (int qb = 0; qb * 256 < lq; ++qb) {
+      const int L = min(varlen_unit_weight(qb, lq, lk, causal != 0) >> level_shift, n_levels - 1);
       const int pos = atomicAdd(&lev[L], 1);
-      if (pos < max_units) units[pos] = make_int2(b, L);
+      if (pos < max_units) units[pos] = make_int2(b, qb);
     }
   }
+}
+
+// Counting-sort levels for weights up to 2 * ceil(max_keys / 128): the shift
+// that keeps them within kVarlenMaxLevels, and the level count.
+inline void varlen_levels(long long max_keys, int& shift, int& n_levels) {
+  const long long max_weight = 2 * ((max_keys + 127) / 128);
+  shift = 0;
+  while ((max_weight >> shift) + 1 > kVarlenMaxLevels) ++shift;
+  n_levels = (int)(max_weight >> shift) + 1;
 }
 
 }  // namespace attn_b200

@@ -103,6 +103,41 @@ class VarlenConfig:
         return f / 2 if self.causal else f
 
 
+@dataclass(frozen=True)
+class PagedPrefillConfig:
+    """Appending new_tokens query tokens to each of B sequences whose cache already
+    holds cached tokens (uniform in [cached_lo, cached_hi]); K/V live in pages."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    page_size: int
+    new_tokens: int
+    cached_lo: int
+    cached_hi: int
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def lengths(self):
+        """(lens_q, lens_k) int32 [B]: new tokens and cached + new tokens per sequence."""
+        g = _gen(self.seed)
+        cached = torch.randint(self.cached_lo, self.cached_hi + 1, (self.B,), generator=g,
+                               dtype=torch.int64)
+        lq = torch.full((self.B,), self.new_tokens, dtype=torch.int64)
+        return lq.to(torch.int32), (cached + lq).to(torch.int32)
+
+    def flops(self) -> float:
+        """4*Hq*d per visible (query, key) pair; a query at offset i of a sequence
+        with len_k keys sees len_k - len_q + i + 1 of them (causal)."""
+        lq, lk = (t.to(torch.float64) for t in self.lengths())
+        pairs = (lq * (lk - lq) + lq * (lq + 1) / 2).sum()
+        return float(4.0 * self.Hq * self.d * pairs)
+
+
 CONFIGS = {
     "tiny_mha": PrefillConfig("tiny_mha", B=1, Hq=2, Hkv=2, S=256, d=64, causal=False, seed=1001),
     "mha_causal_2k": PrefillConfig("mha_causal_2k", B=4, Hq=16, Hkv=16, S=2048, d=128,
@@ -115,6 +150,10 @@ CONFIGS = {
                                     causal=True, seed=1004, value_scale=0.5),
     "paged_decode": DecodeConfig("paged_decode", B=64, Hq=32, Hkv=8, d=128, page_size=16,
                                  len_lo=512, len_hi=8192, seed=1005),
+    # chunked prefill: 1024 new tokens appended to caches of 0..7168 tokens
+    "paged_prefill_gqa": PagedPrefillConfig("paged_prefill_gqa", B=8, Hq=32, Hkv=8, d=128,
+                                            page_size=16, new_tokens=1024, cached_lo=0,
+                                            cached_hi=7168, seed=1300),
     # the GQA shapes of gqa_causal_8k, as a ragged batch of mixed lengths
     "ragged_gqa_causal": VarlenConfig("ragged_gqa_causal", B=16, Hq=32, Hkv=8, d=128,
                                       causal=True, len_lo=128, len_hi=8192, seed=1200),
@@ -251,3 +290,20 @@ def varlen_config_inputs(cfg: VarlenConfig):
     lens = cfg.lengths()
     q, k, v, cu_q, cu_k = varlen_inputs(lens, lens, cfg.Hq, cfg.Hkv, cfg.d, cfg.seed)
     return q, k, v, cu_q, cu_k, lens
+
+
+def paged_prefill_inputs(lens_q, lens_k, Hq: int, Hkv: int, d: int, page_size: int, seed: int,
+                         contiguous: bool = False, max_pages_per_seq=None):
+    """(q packed [sum lens_q, Hq, d], cu_seqlens_q, PagedInputs holding the K/V pages,
+    block table and seq_lens = lens_k).  The cache is drawn as in ``paged_inputs``."""
+    cache = paged_inputs(lens_k, 1, Hkv, d, page_size, seed, max_pages_per_seq=max_pages_per_seq,
+                         contiguous=contiguous)
+    cu_q = cu_seqlens(lens_q)
+    q = randn_bf16((int(cu_q[-1]), Hq, d), seed * 16 + 6)
+    return q, cu_q, cache
+
+
+def paged_prefill_config_inputs(cfg: PagedPrefillConfig):
+    lq, lk = cfg.lengths()
+    q, cu_q, cache = paged_prefill_inputs(lq, lk, cfg.Hq, cfg.Hkv, cfg.d, cfg.page_size, cfg.seed)
+    return q, cu_q, cache, lq, lk

@@ -141,6 +141,47 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
                     attn_stream_t stream);
 
 /*
+ * attn_fwd_paged -- prefill / append over a paged KV cache: new query tokens
+ * of a ragged batch attend to their sequence's keys in a page pool.
+ * Source: "Attention Kernel", section "Paged 与 ragged KV" (token t of a
+ * sequence lives in logical page t / page_size at offset t mod page_size; the
+ * block table maps it to a physical page; the last page is partial; ragged
+ * queries by cumulative lengths), with the operation and masking of attn_fwd.
+ *
+ *   q            [total_q, Hq, d] bf16, packed: sequence b owns query tokens
+ *                [cu_q[b], cu_q[b+1])
+ *   k_cache      [num_pages, page_size, Hkv, d] bf16
+ *   v_cache      [num_pages, page_size, Hkv, d] bf16
+ *   block_table  [B, max_pages_per_seq] int32 physical page of each logical
+ *                page; entries past a sequence's last page are never read
+ *   cu_seqlens_q [B + 1] int32 (as attn_fwd_varlen)
+ *   seq_lens_k   [B] int32 keys of each sequence (cached + new), at most
+ *                max_pages_per_seq * page_size
+ *   o            [total_q, Hq, d] bf16 (written for tokens of a sequence)
+ *   lse          [Hq, total_q] fp32 (nullable)
+ *   Masking is attn_fwd's with Sq = len_q(b), k_len = seq_lens_k[b]: with
+ *   causal = 1 the queries are the last len_q positions of the sequence
+ *   (query i sees keys j <= i + seq_lens_k[b] - len_q), which is appending
+ *   len_q new tokens to a cache that already holds them.
+ *   page_size in {16, 32, 64, 128}; d in {64, 128}; Hq % Hkv == 0;
+ *   max_seqlen_q in [1, 2^21]; workspace as attn_fwd_varlen (size from
+ *   attn_fwd_varlen_workspace_size(B, total_q, max_seqlen_q)).
+ *   Whole pages are read, so every slot of a referenced page must hold finite
+ *   values (slots past a sequence's length get weight exactly 0).
+ * Device-side faults: a page id outside [0, num_pages) is skipped and flags
+ * ATTN_DEVERR_BAD_PAGE; query offsets as attn_fwd_varlen, and a seq_lens_k
+ * outside [0, max_pages_per_seq * page_size], make that sequence empty and
+ * flag ATTN_DEVERR_BAD_LENGTH.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA.
+ */
+int attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache,
+                   const int32_t* block_table, const int32_t* cu_seqlens_q,
+                   const int32_t* seq_lens_k, int page_size, int B, int Hq, int Hkv,
+                   long long total_q, int max_seqlen_q, int max_pages_per_seq, int num_pages, int d,
+                   int causal, float scale, void* o, float* lse, void* workspace,
+                   size_t workspace_bytes, attn_stream_t stream);
+
+/*
  * attn_decode_workspace_size -- bytes of caller-owned device workspace that
  * attn_decode_paged needs for the given capacity.
  * Source: "Attention 算子加速史", section 4.1-4.2 (split-K decode: each split

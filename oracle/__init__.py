@@ -160,7 +160,8 @@ def attn_fwd(q, k, v, causal, scale, k_lens=None, rows=None, n_threads=None):
     return o, lse
 
 
-def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, causal, scale, n_threads=None):
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, causal, scale, n_threads=None,
+                    tokens=None):
     """Exact attention over a ragged batch ("Attention Kernel", "Paged 与 ragged KV").
 
     q [total_q, Hq, d], k/v [total_k, Hkv, d] bf16 (torch or uint16 bits),
@@ -169,7 +170,9 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, causal, scale, n_thread
     ``attn_fwd`` with B = 1, Sq = len_q, Sk = len_k (bottom-right causal
     diagonal); nothing crosses a sequence boundary.
     Returns (o [total_q, Hq, d], lse [Hq, total_q]) as float64 arrays; rows
-    that belong to no sequence stay NaN.
+    that belong to no sequence stay NaN.  ``tokens``: optional packed query
+    token ids; then only those are evaluated (every head) and the result is
+    (o [n, Hq, d], lse [Hq, n]) in that order.
     """
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     total_q, Hq, d = qb.shape
@@ -180,13 +183,33 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, causal, scale, n_thread
     ck = np.asarray(cu_seqlens_k, dtype=np.int64)
     if cq.shape != ck.shape or cq.ndim != 1 or cq.shape[0] < 2:
         raise ValueError("cu_seqlens must both be [B+1]")
-    o = np.full((total_q, Hq, d), np.nan)
-    lse = np.full((Hq, total_q), np.nan)
+    tok = None if tokens is None else np.asarray(tokens, dtype=np.int64)
+    n_out = total_q if tok is None else tok.shape[0]
+    o = np.full((n_out, Hq, d), np.nan)
+    lse = np.full((Hq, n_out), np.nan)
     for b in range(cq.shape[0] - 1):
         q0, q1, k0, k1 = int(cq[b]), int(cq[b + 1]), int(ck[b]), int(ck[b + 1])
         if not (0 <= q0 <= q1 <= total_q and 0 <= k0 <= k1 <= total_k):
             raise ValueError(f"sequence {b}: offsets out of range")
         if q1 == q0:
+            continue
+        if tok is not None:  # only the requested tokens of this sequence
+            sel = np.nonzero((tok >= q0) & (tok < q1))[0]
+            if sel.size == 0:
+                continue
+            qs = np.ascontiguousarray(qb[q0:q1].transpose(1, 0, 2))[None]
+            if k1 == k0:
+                o[sel] = 0.0
+                lse[:, sel] = -np.inf
+                continue
+            ks = np.ascontiguousarray(kb[k0:k1].transpose(1, 0, 2))[None]
+            vs = np.ascontiguousarray(vb[k0:k1].transpose(1, 0, 2))[None]
+            n = q1 - q0
+            i = tok[sel] - q0
+            rows = (np.arange(Hq)[:, None] * n + i[None, :]).reshape(-1)  # head-major
+            orow, lrow = attn_fwd(qs, ks, vs, causal, scale, rows=rows, n_threads=n_threads)
+            o[sel] = orow.reshape(Hq, sel.size, d).transpose(1, 0, 2)
+            lse[:, sel] = lrow.reshape(Hq, sel.size)
             continue
         # [len, H, d] -> [1, H, len, d]
         qs = np.ascontiguousarray(qb[q0:q1].transpose(1, 0, 2))[None]
@@ -200,6 +223,35 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, causal, scale, n_thread
         o[q0:q1] = ob[0].transpose(1, 0, 2)
         lse[:, q0:q1] = lb[0]
     return o, lse
+
+
+def attn_fwd_paged(q, k_cache, v_cache, block_table, cu_seqlens_q, seq_lens_k, causal, scale,
+                   n_threads=None, tokens=None):
+    """Packed queries over a paged cache ("Attention Kernel", "Paged 与 ragged KV").
+
+    Key token t of sequence b is k_cache[block_table[b][t // page_size], t % page_size]
+    (likewise V).  The keys of each sequence are gathered that way and the
+    sequence is attended with ``attn_fwd_varlen`` (bottom-right causal
+    diagonal: the queries are the last len_q positions).
+    Returns (o [total_q, Hq, d], lse [Hq, total_q]) float64; rows of no sequence NaN.
+    """
+    kc, vc = _bits(k_cache), _bits(v_cache)
+    num_pages, page_size, Hkv, d = kc.shape
+    tbl = np.asarray(block_table, dtype=np.int64)
+    lens = np.asarray(seq_lens_k, dtype=np.int64)
+    ks, vs, cu_k = [], [], [0]
+    for b in range(lens.shape[0]):
+        t = np.arange(int(lens[b]))
+        pages = tbl[b, t // page_size]
+        if (pages < 0).any() or (pages >= num_pages).any():
+            raise OracleError(ERR_TABLE)
+        ks.append(kc[pages, t % page_size])
+        vs.append(vc[pages, t % page_size])
+        cu_k.append(cu_k[-1] + int(lens[b]))
+    kp = np.concatenate(ks) if ks else np.zeros((0, Hkv, d), np.uint16)
+    vp = np.concatenate(vs) if vs else np.zeros((0, Hkv, d), np.uint16)
+    return attn_fwd_varlen(q, kp, vp, cu_seqlens_q, cu_k, causal, scale, n_threads=n_threads,
+                           tokens=tokens)
 
 
 def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale, n_threads=None):

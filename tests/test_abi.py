@@ -29,6 +29,7 @@ def lib():
 def test_header_declares_expected_entry_points():
     names = _declared_functions()
     for n in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_fwd_varlen_workspace_size",
+              "attn_fwd_paged",
               "attn_decode_paged", "attn_decode_workspace_size", "attn_get_device_error",
               "attn_strerror"):
         assert n in names
@@ -152,6 +153,36 @@ def test_varlen_workspace_size_formula(lib):
         assert lib.attn_fwd_varlen_workspace_size(B_, tq, 8192) == 16 + 8 * (tq // 256 + B_ + 1)
     assert lib.attn_fwd_varlen_workspace_size(0, 10, 10) == 0
     assert lib.attn_fwd_varlen_workspace_size(1, 10, 0) == 0
+
+
+def _pp(lib, q=FAKE, kc=FAKE, vc=FAKE, tbl=FAKE, cq=FAKE, lk=FAKE, ps=16, B_=2, Hq=8, Hkv=2,
+        tq=500, maxq=300, maxp=64, npages=100, d=128, causal=1, scale=0.1, o=FAKE, lse=None,
+        ws=FAKE, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = lib.attn_fwd_varlen_workspace_size(B_, tq, maxq) if B_ > 0 else 0
+    return lib.attn_fwd_paged(q, kc, vc, tbl, cq, lk, ps, B_, Hq, Hkv, tq, maxq, maxp, npages, d,
+                              causal, scale, o, lse, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(tbl=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(lk=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), B.ATTN_ERR_INVALID_ARG),
+    (dict(maxp=0), B.ATTN_ERR_INVALID_ARG),
+    (dict(npages=0), B.ATTN_ERR_INVALID_ARG),
+    (dict(maxq=0), B.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), B.ATTN_ERR_INVALID_ARG),
+    (dict(ps=8), B.ATTN_ERR_UNSUPPORTED),
+    (dict(ps=48), B.ATTN_ERR_UNSUPPORTED),
+    (dict(ps=256), B.ATTN_ERR_UNSUPPORTED),
+    (dict(d=80), B.ATTN_ERR_UNSUPPORTED),
+    (dict(kc=FAKE + 4), B.ATTN_ERR_ALIGNMENT),
+    (dict(tbl=FAKE + 2), B.ATTN_ERR_ALIGNMENT),
+    (dict(ws_bytes=8), B.ATTN_ERR_WORKSPACE),
+])
+def test_paged_prefill_validation(lib, kw, status):
+    assert _pp(lib, **kw) == status
 
 
 def test_workspace_size_formula(lib):

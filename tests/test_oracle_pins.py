@@ -450,3 +450,76 @@ def test_varlen_bottom_right_causal_last_row_sees_every_key():
     # first row of sequence 0 == non-causal attention over its first 7 keys
     o7, l7 = oracle.attn_fwd_varlen(q[:1], k[:7], v[:7], [0, 1], [0, 7], False, 0.7)
     np.testing.assert_array_equal(oc[0], o7[0])
+
+
+# --------------------------------------------------------------------------- paged prefill
+# "Attention Kernel", section "Paged 与 ragged KV": key token t of a sequence is
+# at offset t mod page_size of the physical page block_table[b][t // page_size].
+
+
+def test_paged_prefill_contiguous_pages_equal_ragged():
+    lens_q, lens_k = [5, 3, 0, 9], [21, 3, 7, 40]
+    q, cu_q, c = workloads.paged_prefill_inputs(lens_q, lens_k, 4, 2, 8, 16, seed=83,
+                                                contiguous=True)
+    o, lse = oracle.attn_fwd_paged(q, c.k_cache, c.v_cache, c.block_table, cu_q, c.seq_lens,
+                                   True, 0.4)
+    # with contiguous placement the keys of sequence b are the pool's rows in order
+    pool_k = c.k_cache.reshape(-1, 2, 8)
+    pool_v = c.v_cache.reshape(-1, 2, 8)
+    starts = [0]
+    for n in lens_k:
+        starts.append(starts[-1] + 16 * (-(-n // 16)))
+    ks = torch.cat([pool_k[starts[b]:starts[b] + lens_k[b]] for b in range(4)])
+    vs = torch.cat([pool_v[starts[b]:starts[b] + lens_k[b]] for b in range(4)])
+    o2, l2 = oracle.attn_fwd_varlen(q, ks, vs, cu_q, workloads.cu_seqlens(lens_k), True, 0.4)
+    np.testing.assert_array_equal(np.nan_to_num(o, nan=7.0), np.nan_to_num(o2, nan=7.0))
+    np.testing.assert_array_equal(np.nan_to_num(lse, nan=7.0), np.nan_to_num(l2, nan=7.0))
+
+
+def test_paged_prefill_permuted_pages_equal_contiguous():
+    lens_q, lens_k = [4, 6], [50, 33]
+    q, cu_q, cc = workloads.paged_prefill_inputs(lens_q, lens_k, 2, 1, 4, 16, seed=89,
+                                                 contiguous=True)
+    _, _, cp = workloads.paged_prefill_inputs(lens_q, lens_k, 2, 1, 4, 16, seed=89)
+    # move the contiguous pool's pages to the permuted placement
+    k2 = torch.empty_like(cc.k_cache)
+    v2 = torch.empty_like(cc.v_cache)
+    for b in range(2):
+        n = -(-lens_k[b] // 16)
+        for lp in range(n):
+            k2[cp.block_table[b, lp]] = cc.k_cache[cc.block_table[b, lp]]
+            v2[cp.block_table[b, lp]] = cc.v_cache[cc.block_table[b, lp]]
+    a = oracle.attn_fwd_paged(q, cc.k_cache, cc.v_cache, cc.block_table, cu_q, cc.seq_lens, True,
+                              0.5)
+    b_ = oracle.attn_fwd_paged(q, k2, v2, cp.block_table, cu_q, cp.seq_lens, True, 0.5)
+    np.testing.assert_array_equal(a[0], b_[0])
+    np.testing.assert_array_equal(a[1], b_[1])
+
+
+def test_paged_prefill_single_token_equals_decode_oracle():
+    # one new token per sequence sees every key: the C decode oracle's result
+    lens_k = [1, 17, 64, 100]
+    q, cu_q, c = workloads.paged_prefill_inputs([1] * 4, lens_k, 4, 2, 16, 16, seed=97)
+    o, lse = oracle.attn_fwd_paged(q, c.k_cache, c.v_cache, c.block_table, cu_q, c.seq_lens,
+                                   True, 0.3)
+    od, ld = oracle.decode_paged(q, c.k_cache, c.v_cache, c.block_table, c.seq_lens, 0.3)
+    np.testing.assert_allclose(o, od, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ld.T, rtol=0, atol=1e-12)
+
+
+def test_paged_prefill_bad_page_is_reported():
+    q, cu_q, c = workloads.paged_prefill_inputs([2], [20], 2, 1, 4, 16, seed=101)
+    tbl = c.block_table.clone()
+    tbl[0, 1] = c.k_cache.shape[0]
+    with pytest.raises(oracle.OracleError):
+        oracle.attn_fwd_paged(q, c.k_cache, c.v_cache, tbl, cu_q, c.seq_lens, True, 0.3)
+
+
+def test_varlen_token_subset_equals_full_evaluation():
+    lens_q, lens_k = [9, 0, 14, 3], [12, 5, 14, 0]
+    q, k, v, cu_q, cu_k = workloads.varlen_inputs(lens_q, lens_k, 3, 1, 4, seed=137)
+    o, lse = oracle.attn_fwd_varlen(q, k, v, cu_q, cu_k, True, 0.6)
+    tok = np.array([25, 0, 8, 9, 13, 24, 22])
+    os_, ls_ = oracle.attn_fwd_varlen(q, k, v, cu_q, cu_k, True, 0.6, tokens=tok)
+    np.testing.assert_array_equal(os_, o[tok])
+    np.testing.assert_array_equal(ls_, lse[:, tok])
