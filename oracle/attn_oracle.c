@@ -35,6 +35,10 @@
  *   - Causal alignment is bottom-right: with k_len keys visible to sequence
  *     b, key j is visible to query row i iff j < k_len and, when causal,
  *     j <= i + (k_len - Sq).
+ *   - Programmable masks ("Attention Kernel", section "可编程 mask"), both
+ *     with causal: a sliding window w > 0 keeps only the w keys ending at the
+ *     row's position p = i + (k_len - Sq), i.e. j > p - w; a prefix P > 0
+ *     makes keys j < P visible to every row (prefix-LM).  Not both at once.
  *
  * Inputs to the attention routines are bf16 bit patterns (uint16); this
  * file widens them to double itself (a bf16 value is the top half of an
@@ -174,7 +178,7 @@ int oracle_online_attend(const double* s, int n_scores, const double* v,
 
 typedef struct {
   const uint16_t *q, *k, *v;
-  int B, Hq, Hkv, Sq, Sk, d, causal;
+  int B, Hq, Hkv, Sq, Sk, d, causal, window, prefix;
   double scale;
   const int32_t* k_lens;
   const int64_t* rows; /* flat row ids (b*Hq + hq)*Sq + i, or NULL = all */
@@ -214,9 +218,13 @@ static int prefill_row(const prefill_job* J, int64_t r, prefill_scratch* W) {
   }
   const uint16_t* qp = J->q + (((size_t)b * J->Hq + hq) * J->Sq + i) * d;
   for (int t = 0; t < d; ++t) W->qrow[t] = bf16_to_double(qp[t]);
-  int64_t offset = (int64_t)klen - J->Sq; /* bottom-right causal alignment */
+  int64_t pos = (int64_t)i + ((int64_t)klen - J->Sq); /* bottom-right causal alignment */
   for (int j = 0; j < J->Sk; ++j) {
-    int visible = j < klen && (!J->causal || (int64_t)j <= (int64_t)i + offset);
+    int visible = j < klen;
+    if (J->causal) {
+      visible = visible && ((int64_t)j <= pos || (int64_t)j < J->prefix);
+      if (J->window > 0) visible = visible && (int64_t)j > pos - J->window;
+    }
     if (!visible) {
       W->s[j] = -INFINITY;
       continue;
@@ -254,12 +262,16 @@ static void* prefill_worker(void* arg) {
  * gives the number of leading keys visible per sequence.  Work is split over
  * n_threads POSIX threads by rows; each row is computed independently.
  */
-int oracle_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                         int B, int Hq, int Hkv, int Sq, int Sk, int d, int causal,
-                         double scale, const int32_t* k_lens, const int64_t* rows,
-                         int64_t n_rows, double* o, double* lse, int n_threads) {
+int oracle_attn_fwd_rows_masked(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                int B, int Hq, int Hkv, int Sq, int Sk, int d, int causal,
+                                double scale, const int32_t* k_lens, int window, int prefix,
+                                const int64_t* rows, int64_t n_rows, double* o, double* lse,
+                                int n_threads) {
   if (!q || (Sk > 0 && (!k || !v)) || !o || !lse || B < 1 || Hq < 1 || Hkv < 1 ||
       Sq < 1 || Sk < 0 || d < 1 || Hq % Hkv != 0 || n_rows < 0 || !isfinite(scale))
+    return ORACLE_ERR_ARG;
+  if (window < 0 || prefix < 0 || (window > 0 && prefix > 0) ||
+      ((window > 0 || prefix > 0) && !causal))
     return ORACLE_ERR_ARG;
   if (!rows && n_rows != (int64_t)B * Hq * Sq) return ORACLE_ERR_ARG;
   if (n_threads < 1) n_threads = 1;
@@ -276,6 +288,7 @@ int oracle_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v
     J->q = q; J->k = k; J->v = v;
     J->B = B; J->Hq = Hq; J->Hkv = Hkv; J->Sq = Sq; J->Sk = Sk; J->d = d;
     J->causal = causal; J->scale = scale; J->k_lens = k_lens;
+    J->window = window; J->prefix = prefix;
     J->rows = rows; J->n_rows = n_rows; J->o = o; J->lse = lse;
     J->begin = n_rows * w / n_threads;
     J->end = n_rows * (w + 1) / n_threads;
@@ -290,6 +303,15 @@ int oracle_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v
   free(jobs);
   free(th);
   return status;
+}
+
+/* oracle_attn_fwd_rows_masked without a window or prefix. */
+int oracle_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                         int B, int Hq, int Hkv, int Sq, int Sk, int d, int causal,
+                         double scale, const int32_t* k_lens, const int64_t* rows,
+                         int64_t n_rows, double* o, double* lse, int n_threads) {
+  return oracle_attn_fwd_rows_masked(q, k, v, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens, 0, 0,
+                                     rows, n_rows, o, lse, n_threads);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -523,3 +523,85 @@ def test_varlen_token_subset_equals_full_evaluation():
     os_, ls_ = oracle.attn_fwd_varlen(q, k, v, cu_q, cu_k, True, 0.6, tokens=tok)
     np.testing.assert_array_equal(os_, o[tok])
     np.testing.assert_array_equal(ls_, lse[:, tok])
+
+
+# --------------------------------------------------------------------------- programmable masks
+# "Attention Kernel", section "可编程 mask": causal, sliding window, document
+# boundaries, prefix-LM.  Window w: the row at key position p sees keys (p-w, p];
+# prefix P: keys below P are visible to every row (both with the causal mask).
+
+
+def _sdpa_masked(q, k, v, scale, visible):
+    """torch SDPA in float64 with an explicit boolean mask [Sq, Sk] (True = visible)."""
+    g = q.shape[1] // k.shape[1]
+    kk = k.double().repeat_interleave(g, dim=1)
+    vv = v.double().repeat_interleave(g, dim=1)
+    o = torch.nn.functional.scaled_dot_product_attention(q.double(), kk, vv, attn_mask=visible,
+                                                         scale=scale)
+    s = torch.einsum("bhqd,bhkd->bhqk", q.double(), kk) * scale
+    lse = torch.logsumexp(s.masked_fill(~visible, float("-inf")), dim=-1)
+    return o.numpy(), lse.numpy()
+
+
+@pytest.mark.parametrize("Sq,Sk,window", [(9, 9, 3), (5, 12, 4), (12, 12, 1), (7, 7, 20)])
+def test_sliding_window_against_sdpa(Sq, Sk, window):
+    q, k, v = workloads.prefill_inputs(1, 4, 2, Sq, Sk, 8, seed=139)
+    o, lse = oracle.attn_fwd(q, k, v, True, 0.4, window=window)
+    i = torch.arange(Sq)[:, None] + (Sk - Sq)
+    j = torch.arange(Sk)[None, :]
+    vis = (j <= i) & (j > i - window)  # every row keeps at least its diagonal key
+    ro, rl = _sdpa_masked(q, k, v, 0.4, vis)
+    np.testing.assert_allclose(o, ro, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, rl, rtol=0, atol=1e-12)
+
+
+def test_window_one_is_the_diagonal_key_and_wide_window_is_causal():
+    q, k, v = workloads.prefill_inputs(1, 2, 1, 11, 11, 8, seed=149)
+    o, lse = oracle.attn_fwd(q, k, v, True, 0.3, window=1)
+    vv = v.double().numpy()[0, 0]
+    s = (q.double() @ k.double().transpose(-1, -2)).numpy()[0] * 0.3
+    for h in range(2):
+        np.testing.assert_allclose(o[0, h], vv, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[0, h], np.diagonal(s[h]), rtol=0, atol=1e-12)
+    oc, lc = oracle.attn_fwd(q, k, v, True, 0.3)
+    ow, lw = oracle.attn_fwd(q, k, v, True, 0.3, window=11)
+    np.testing.assert_array_equal(oc, ow)
+    np.testing.assert_array_equal(lc, lw)
+
+
+@pytest.mark.parametrize("prefix", [1, 4, 9])
+def test_prefix_lm_against_sdpa(prefix):
+    q, k, v = workloads.prefill_inputs(1, 2, 2, 9, 9, 8, seed=151)
+    o, lse = oracle.attn_fwd(q, k, v, True, 0.5, prefix=prefix)
+    i = torch.arange(9)[:, None]
+    j = torch.arange(9)[None, :]
+    ro, rl = _sdpa_masked(q, k, v, 0.5, (j <= i) | (j < prefix))
+    np.testing.assert_allclose(o, ro, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, rl, rtol=0, atol=1e-12)
+    if prefix >= 9:  # every key visible: non-causal attention
+        on, ln = oracle.attn_fwd(q, k, v, False, 0.5)
+        np.testing.assert_array_equal(o, on)
+
+
+def test_window_and_prefix_together_are_rejected():
+    q, k, v = workloads.prefill_inputs(1, 1, 1, 4, 4, 8, seed=157)
+    with pytest.raises(oracle.OracleError):
+        oracle.attn_fwd(q, k, v, True, 0.5, window=2, prefix=2)
+    with pytest.raises(oracle.OracleError):
+        oracle.attn_fwd(q, k, v, False, 0.5, window=2)
+
+
+def test_document_mask_is_the_ragged_batch_of_its_documents():
+    # a sequence of three documents, each attending causally within itself, is
+    # the ragged batch of the documents (cumulative lengths at the boundaries)
+    docs = [5, 8, 3]
+    q, k, v, cu, _ = workloads.varlen_inputs(docs, docs, 2, 1, 8, seed=163)
+    o, lse = oracle.attn_fwd_varlen(q, k, v, cu, cu, True, 0.4)
+    doc = torch.repeat_interleave(torch.arange(3), torch.tensor(docs))
+    i = torch.arange(16)[:, None]
+    j = torch.arange(16)[None, :]
+    vis = (doc[:, None] == doc[None, :]) & (j <= i)
+    ro, rl = _sdpa_masked(q.permute(1, 0, 2)[None], k.permute(1, 0, 2)[None],
+                          v.permute(1, 0, 2)[None], 0.4, vis)
+    np.testing.assert_allclose(o, ro[0].transpose(1, 0, 2), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, rl[0], rtol=0, atol=1e-12)
