@@ -14,6 +14,7 @@ from ._binding import (  # noqa: F401
     attn_fwd_paged,
     attn_fwd_varlen,
     attn_fwd_varlen_workspace_size,
+    attn_fwd_window,
     attn_get_device_error,
     attn_strerror,
     library_path,

@@ -36,6 +36,7 @@ _SZ = ctypes.c_size_t
 SIGNATURES = {
     "attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "attn_fwd_masked": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P]),
+    "attn_fwd_window": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _I, _I, _P]),
     "attn_fwd_varlen_workspace_size": (_SZ, [_I, ctypes.c_longlong, _I]),
     "attn_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, ctypes.c_longlong,
                              ctypes.c_longlong, _I, _I, _I, _F, _P, _SZ, _P]),
@@ -139,6 +140,32 @@ def attn_fwd(q, k, v, causal: bool, scale: float, out=None, lse=None, return_lse
              stream=None):
     """attn_fwd_masked without key padding."""
     return attn_fwd_masked(q, k, v, causal, scale, None, out, lse, return_lse, stream)
+
+
+def attn_fwd_window(q, k, v, scale: float, window: int = 0, prefix: int = 0, k_lens=None,
+                    out=None, lse=None, return_lse: bool = True, stream=None):
+    """Causal prefill with a sliding window (window > 0) or a prefix-LM mask (prefix > 0);
+    q [B,Hq,Sq,d], k/v [B,Hkv,Sk,d] bf16 CUDA tensors (layouts as attn_fwd_masked)."""
+    import torch
+    _require_cuda(q, k, v, k_lens)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bfloat16")
+    B, Hq, Sq, d = q.shape
+    Bk, Hkv, Sk, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or dk != d:
+        raise ValueError("q/k/v shapes disagree")
+    if k_lens is not None and (k_lens.dtype != torch.int32 or tuple(k_lens.shape) != (B,)):
+        raise ValueError("k_lens must be int32 [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    st = load_library().attn_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq,
+                                        Hkv, Sq, Sk, d, float(scale), _ptr(k_lens), int(window),
+                                        int(prefix), _stream(stream))
+    _check(st, "attn_fwd_window")
+    return out, lse
 
 
 def attn_fwd_varlen_workspace_size(B: int, total_q: int, max_seqlen_q: int) -> int:

@@ -96,13 +96,13 @@ int sm_count() {
   return cached[dev];
 }
 
-template <int D, bool CAUSAL, int LAYOUT = kLayoutDense>
+template <int D, bool CAUSAL, int LAYOUT = kLayoutDense, bool MASKS = false>
 int launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                    const CUtensorMap& mo, const PrefillParams& prm, cudaStream_t stream,
                    long long max_units = 0) {
   using C = PrefillCfg<D>;
   constexpr bool VARLEN = LAYOUT != kLayoutDense;
-  auto kern = attn_prefill_sm100_kernel<D, CAUSAL, LAYOUT>;
+  auto kern = attn_prefill_sm100_kernel<D, CAUSAL, LAYOUT, MASKS>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
       cudaSuccess)
     return ATTN_ERR_CUDA;
@@ -138,34 +138,10 @@ int check_prefill_args(const void* q, const void* k, const void* v, void* o, flo
 // total_q / 256 + B for non-overlapping ranges; one more for rounding.
 long long varlen_max_units(int B, long long total_q) { return total_q / 256 + B + 1; }
 
-}  // namespace
-}  // namespace attn_b200
-
-using namespace attn_b200;
-
-extern "C" {
-
-const char* attn_strerror(int status) {
-  switch (status) {
-    case ATTN_OK: return "success";
-    case ATTN_ERR_INVALID_ARG: return "invalid argument";
-    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration (head dim, page size or group size)";
-    case ATTN_ERR_ALIGNMENT: return "tensor pointer not 16-byte aligned";
-    case ATTN_ERR_WORKSPACE: return "decode workspace missing or too small";
-    case ATTN_ERR_CUDA: return "CUDA runtime or driver call failed";
-    case ATTN_ERR_DEVICE: return "device error word set (bad page id, bad length or wait timeout)";
-    default: return "unknown status";
-  }
-}
-
-int attn_split_tokens(void) { return kSplitTokens; }
-
-int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                    int Hq, int Hkv, int Sq, int Sk, int d, int causal, float scale,
-                    const int32_t* k_lens, attn_stream_t stream_) {
-  const int st = check_prefill_args(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens);
-  if (st != ATTN_OK) return st;
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+// Dense fixed-length prefill with optional key lengths, sliding window and prefix.
+int prefill_dense(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                  int Hkv, int Sq, int Sk, int d, int causal, float scale, const int32_t* k_lens,
+                  int window, int prefix, cudaStream_t stream) {
   const long long rows_q = (long long)B * Hq * Sq;
   if (Sk == 0) {
     const size_t n_vec = (size_t)rows_q * d * 2 / 16;
@@ -194,11 +170,56 @@ int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float*
   prm.group = Hq / Hkv;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.n_qblocks = (Sq + 255) / 256;
+  prm.window = window;
+  prm.prefix = prefix;
+  if (window > 0 || prefix > 0)  // causal only (checked by the caller)
+    return d == 128 ? launch_prefill<128, true, kLayoutDense, true>(mq, mk, mv, mo, prm, stream)
+                    : launch_prefill<64, true, kLayoutDense, true>(mq, mk, mv, mo, prm, stream);
   if (d == 128)
     return causal ? launch_prefill<128, true>(mq, mk, mv, mo, prm, stream)
                   : launch_prefill<128, false>(mq, mk, mv, mo, prm, stream);
   return causal ? launch_prefill<64, true>(mq, mk, mv, mo, prm, stream)
                 : launch_prefill<64, false>(mq, mk, mv, mo, prm, stream);
+}
+}  // namespace
+}  // namespace attn_b200
+
+using namespace attn_b200;
+
+extern "C" {
+
+const char* attn_strerror(int status) {
+  switch (status) {
+    case ATTN_OK: return "success";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration (head dim, page size or group size)";
+    case ATTN_ERR_ALIGNMENT: return "tensor pointer not 16-byte aligned";
+    case ATTN_ERR_WORKSPACE: return "decode workspace missing or too small";
+    case ATTN_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case ATTN_ERR_DEVICE: return "device error word set (bad page id, bad length or wait timeout)";
+    default: return "unknown status";
+  }
+}
+
+int attn_split_tokens(void) { return kSplitTokens; }
+
+int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int Hq, int Hkv, int Sq, int Sk, int d, int causal, float scale,
+                    const int32_t* k_lens, attn_stream_t stream) {
+  const int st = check_prefill_args(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens);
+  if (st != ATTN_OK) return st;
+  return prefill_dense(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens, 0, 0,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int Hq, int Hkv, int Sq, int Sk, int d, float scale, const int32_t* k_lens,
+                    int window, int prefix, attn_stream_t stream) {
+  const int st = check_prefill_args(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, 1, scale, k_lens);
+  if (st != ATTN_OK) return st;
+  if (window < 0 || prefix < 0 || (window > 0 && prefix > 0)) return ATTN_ERR_INVALID_ARG;
+  return prefill_dense(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, 1, scale, k_lens, window, prefix,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t attn_fwd_varlen_workspace_size(int B, long long total_q, int max_seqlen_q) {
@@ -254,7 +275,7 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
     return ATTN_ERR_CUDA;
   attn_varlen_schedule_kernel<<<1, 1024, sched_smem, stream>>>(
       cu_seqlens_q, cu_seqlens_k, nullptr, B, (int)total_q, (int)total_k, max_seqlen_q, 0, causal,
-      shift, n_levels, units, unit_count, (int)max_units);
+      0, 0, shift, n_levels, units, unit_count, (int)max_units);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   // 2. the prefill kernel over packed token-major tensors
   CUtensorMap mq, mk, mv;
@@ -328,7 +349,7 @@ int attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache,
     return ATTN_ERR_CUDA;
   attn_varlen_schedule_kernel<<<1, 1024, sched_smem, stream>>>(
       cu_seqlens_q, nullptr, seq_lens_k, B, (int)total_q, 0, max_seqlen_q, max_keys, causal,
-      shift, n_levels, units, unit_count, (int)max_units);
+      0, 0, shift, n_levels, units, unit_count, (int)max_units);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   CUtensorMap mq, mk, mv;
   if (!make_token_map(&mq, q, d, Hq, total_q) ||

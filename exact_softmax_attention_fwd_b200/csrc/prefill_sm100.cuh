@@ -65,6 +65,9 @@ struct PrefillParams {
   int group;            // Hq / Hkv
   float scale_log2;     // scale * log2(e)
   int n_qblocks;        // ceil(Sq / 256)
+  // programmable masks (causal only; 0 = off): a row at key position p sees
+  // keys (p - window, p] (sliding window), or keys below prefix as well (prefix-LM)
+  int window, prefix;
   // ragged batches: packed token-major tensors, cumulative sequence lengths
   // and the unit list written by attn_varlen_schedule_kernel
   uint16_t* o;          // [total_q, Hq, d] bf16
@@ -128,14 +131,28 @@ constexpr int kLayoutDense = 0;
 constexpr int kLayoutRagged = 1;
 constexpr int kLayoutPaged = 2;
 
-// Number of 128-key tiles the query tile with first row `row0` must visit
-// (0 when the tile is past Sq or none of its rows sees a key).
-__device__ __forceinline__ int prefill_num_kv_tiles(int row0, int Sq, int klen, bool causal) {
-  if (row0 >= Sq) return 0;
+// The 128-key tiles [lo, hi) the query tile with first row `row0` must visit
+// (lo == hi: none).  A row at key position pos = i + (klen - Sq) (bottom-right
+// causal alignment) sees keys [max(0, pos - window + 1), max(pos, prefix - 1)]
+// within [0, klen) when causal (window / prefix 0 = off), all of [0, klen)
+// otherwise; tiles outside the union over the tile's rows are skipped whole
+// ("Attention Kernel", section "可编程 mask": block-level skipping, then an
+// element-wise rule inside the tiles left).
+__device__ __forceinline__ void prefill_kv_range(int row0, int Sq, int klen, bool causal,
+                                                 int window, int prefix, int& lo, int& hi) {
+  lo = hi = 0;
+  if (row0 >= Sq) return;
+  const long long off = (long long)klen - Sq;
   const int last_row = min(row0 + 127, Sq - 1);
-  long long lim = (long long)klen - 1;
-  if (causal) lim = min(lim, (long long)last_row + (long long)klen - Sq);
-  return lim < 0 ? 0 : (int)(lim / 128) + 1;
+  long long top = (long long)klen - 1;  // largest key any row of the tile sees
+  long long bot = 0;                    // smallest
+  if (causal) {
+    top = min(top, max((long long)last_row + off, (long long)prefix - 1));
+    if (window > 0) bot = max(0LL, (long long)row0 + off - window + 1);
+  }
+  if (top < bot) return;
+  lo = (int)(bot / 128);
+  hi = (int)(top / 128) + 1;
 }
 
 // One work unit: query rows [256*qb, 256*qb + 256) of head hq in sequence b.
@@ -146,14 +163,19 @@ struct PrefillUnit {
   int q_tok0;      // ragged batches: packed index of the sequence's first query
   int k_tok0;      //   and first key token (0 otherwise)
   int row0[2];     // first row of each query tile
-  int nkv[2];      // KV tiles each query tile visits
+  int kv_begin[2];  // KV tiles [kv_begin, kv_end) each query tile visits
+  int kv_end[2];
+  int kv_first;    // the unit's K/V stream: tiles [kv_first, kv_last)
+  int kv_last;
 };
 
 // The k-th unit of this CTA, or false when the CTA has no more work.  Ranks
 // are ordered heaviest first (q-blocks descending, heads inner) and dealt
 // back and forth across the CTAs: rank k*G + c for even k, k*G + G-1-c for odd.
 // For a ragged batch the (sequence, q-block) order comes from the unit list.
-template <bool CAUSAL, int LAYOUT>
+// MASKS: the instantiation honours p.window / p.prefix; without it both are
+// the constant 0, so every range starts at tile 0 and the extra bounds fold away.
+template <bool CAUSAL, int LAYOUT, bool MASKS>
 __device__ __forceinline__ bool prefill_unit(const PrefillParams& p, int k, PrefillUnit& u) {
   constexpr bool VARLEN = LAYOUT != kLayoutDense;
   const long long G = gridDim.x;
@@ -191,15 +213,23 @@ __device__ __forceinline__ bool prefill_unit(const PrefillParams& p, int k, Pref
     u.q_tok0 = 0;
     u.k_tok0 = 0;
   }
+  u.kv_first = INT_MAX;
+  u.kv_last = 0;
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     u.row0[i] = u.qb * 256 + i * 128;
-    u.nkv[i] = prefill_num_kv_tiles(u.row0[i], u.sq, u.klen, CAUSAL);
+    prefill_kv_range(u.row0[i], u.sq, u.klen, CAUSAL, MASKS ? p.window : 0,
+                     MASKS ? p.prefix : 0, u.kv_begin[i], u.kv_end[i]);
+    if (u.kv_end[i] > u.kv_begin[i]) {
+      u.kv_first = min(u.kv_first, u.kv_begin[i]);
+      u.kv_last = max(u.kv_last, u.kv_end[i]);
+    }
   }
+  if (u.kv_last == 0) u.kv_first = 0;
   return true;
 }
 
-template <int D, bool CAUSAL, int LAYOUT>
+template <int D, bool CAUSAL, int LAYOUT, bool MASKS>
 __global__ void __launch_bounds__(384, 1)
     attn_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                               const __grid_constant__ CUtensorMap tm_k,
@@ -284,19 +314,19 @@ __global__ void __launch_bounds__(384, 1)
         return true;
       };
       PrefillUnit u;
-      for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT>(p, k, u); ++k) {
-        const int n_max = max(u.nkv[0], u.nkv[1]);
+      for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT, MASKS>(p, k, u); ++k) {
+        const bool has0 = u.kv_end[0] > u.kv_begin[0], has1 = u.kv_end[1] > u.kv_begin[1];
         const int kvh = u.hq / p.group;
         const int kv_row = u.b * p.Hkv + kvh;
         if (PAGED) {  // warp 2 streams paged K/V; this thread only loads Q
-          if (u.nkv[0] > 0 && !(ok = load_q(u, 0))) break;
-          if (u.nkv[1] > 0 && !(ok = load_q(u, 1))) break;
+          if (has0 && !(ok = load_q(u, 0))) break;
+          if (has1 && !(ok = load_q(u, 1))) break;
           continue;
         }
         // Q_0 first (its slot frees first under a causal mask), then the first
         // K tile, then Q_1, so that no wait on Q_1 holds back the K/V stream.
-        if (u.nkv[0] > 0 && !(ok = load_q(u, 0))) break;
-        for (int j = 0; j < n_max; ++j, ++kv) {
+        if (has0 && !(ok = load_q(u, 0))) break;
+        for (int j = u.kv_first; j < u.kv_last; ++j, ++kv) {
           const int s = kv % C::STAGES;
           const uint32_t ph = (kv / C::STAGES) & 1u;
           if (!(ok = mbar_wait(bar(C::B_KEMPTY + s), ph ^ 1u, abort_flag))) break;
@@ -305,7 +335,7 @@ __global__ void __launch_bounds__(384, 1)
             tma_load_3d(sbase + C::OFF_K + s * C::TILE_BYTES + cb * C::CB_BYTES, &tm_k,
                         bar(C::B_KFULL + s), 64 * cb, VARLEN ? kvh : j * 128,
                         VARLEN ? u.k_tok0 + j * 128 : kv_row);
-          if (j == 0 && u.nkv[1] > 0 && !(ok = load_q(u, 1))) {
+          if (j == u.kv_first && has1 && !(ok = load_q(u, 1))) {
             ++kv;  // K_0 of this unit was issued
             break;
           }
@@ -344,14 +374,13 @@ __global__ void __launch_bounds__(384, 1)
     uint32_t kv = 0;                  // K/V tiles issued so far (ring position)
     bool ok = true;
     PrefillUnit u;
-    for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT>(p, k, u); ++k) {
-      const int n_max = max(u.nkv[0], u.nkv[1]);
+    for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT, MASKS>(p, k, u); ++k) {
       const int kvh = u.hq / p.group;
       const int ppt = 128 / p.page_size;
       const int n_lp = (u.klen + p.page_size - 1) / p.page_size;  // <= max_pages
       const int* tbl = p.block_table + (size_t)u.b * p.max_pages;
       const uint32_t row_off = (uint32_t)(lane * p.page_size * 128);
-      for (int j = 0; j < n_max; ++j, ++kv) {
+      for (int j = u.kv_first; j < u.kv_last; ++j, ++kv) {
         const int s = kv % C::STAGES;
         const uint32_t ph = (kv / C::STAGES) & 1u;
         const int lp = j * ppt + lane;
@@ -421,44 +450,63 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t p_waits0 = 0, p_waits1 = 0;  // P_FULL phases consumed per tile slot
       bool ok = true;
       PrefillUnit u;
-      for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT>(p, k, u); ++k) {
-        const int n_max = max(u.nkv[0], u.nkv[1]);
-        if (n_max == 0) continue;
-        // prologue: S_i(0) for each participating tile
+      for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT, MASKS>(p, k, u); ++k) {
+        const int jb = u.kv_first, je = u.kv_last;  // the unit's K/V stream
+        if (je <= jb) continue;
+        // prologue: S_i(jb) for each tile whose range starts at the stream's start
         {
           const int s = kv % C::STAGES;
           if (!(ok = mbar_wait(bar(C::B_KFULL + s), (kv / C::STAGES) & 1u, abort_flag))) break;
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (!ok) break;
-            if (u.nkv[i] == 0) continue;
+            if (u.kv_begin[i] != jb || u.kv_end[i] <= jb) continue;
             uint32_t& qw = i ? q_waits1 : q_waits0;
             if (!(ok = mbar_wait(bar(C::B_QFULL + i), qw & 1u, abort_flag))) break;
             ++qw;
             tc_fence_after_sync();
             issue_qk(i, s);
             umma_commit(bar(C::B_SFULL + i));
-            if (u.nkv[i] == 1) umma_commit(bar(C::B_QFREE + i));  // Q_i read for the last time
+            if (u.kv_end[i] == jb + 1) umma_commit(bar(C::B_QFREE + i));  // Q_i read for the last time
           }
           if (!ok) break;
           umma_commit(bar(C::B_KEMPTY + s));
         }
-        for (int j = 0; ok && j < n_max; ++j) {
-          const uint32_t idx = kv + j;
+        for (int j = jb; ok && j < je; ++j) {
+          const uint32_t idx = kv + (uint32_t)(j - jb);
           const int s = idx % C::STAGES;
           const int s1 = (idx + 1) % C::STAGES;
           if (!(ok = mbar_wait(bar(C::B_VFULL + s), (idx / C::STAGES) & 1u, abort_flag))) break;
-          bool k_next = false;
+          bool k_next = false;  // K_(j+1) seen to have landed
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (!ok) break;
-            if (j >= u.nkv[i]) continue;
+            const int b0 = u.kv_begin[i], e0 = u.kv_end[i];
+            if (j < b0 || j >= e0) {
+              // a tile whose range starts one K/V tile later gets its first S now
+              if (MASKS && j + 1 == b0 && b0 < e0) {
+                if (!k_next) {
+                  if (!(ok = mbar_wait(bar(C::B_KFULL + s1), ((idx + 1) / C::STAGES) & 1u,
+                                       abort_flag)))
+                    break;
+                  k_next = true;
+                }
+                uint32_t& qw = i ? q_waits1 : q_waits0;
+                if (!(ok = mbar_wait(bar(C::B_QFULL + i), qw & 1u, abort_flag))) break;
+                ++qw;
+                tc_fence_after_sync();
+                issue_qk(i, s1);
+                umma_commit(bar(C::B_SFULL + i));
+                if (e0 == b0 + 1) umma_commit(bar(C::B_QFREE + i));
+              }
+              continue;
+            }
             uint32_t& pw = i ? p_waits1 : p_waits0;
             if (!(ok = mbar_wait(bar(C::B_PFULL + i), pw & 1u, abort_flag))) break;
             ++pw;
             tc_fence_after_sync();
-            issue_pv(i, s, j > 0);
-            if (j + 1 < u.nkv[i]) {
+            issue_pv(i, s, j > b0);
+            if (j + 1 < e0) {
               if (!k_next) {
                 if (!(ok = mbar_wait(bar(C::B_KFULL + s1), ((idx + 1) / C::STAGES) & 1u,
                                      abort_flag)))
@@ -468,7 +516,7 @@ __global__ void __launch_bounds__(384, 1)
               }
               issue_qk(i, s1);
               umma_commit(bar(C::B_SFULL + i));
-              if (j + 2 == u.nkv[i]) umma_commit(bar(C::B_QFREE + i));
+              if (j + 2 == e0) umma_commit(bar(C::B_QFREE + i));
             } else {
               umma_commit(bar(C::B_OFULL + i));
             }
@@ -476,7 +524,7 @@ __global__ void __launch_bounds__(384, 1)
           umma_commit(bar(C::B_VEMPTY + s));
           if (k_next) umma_commit(bar(C::B_KEMPTY + s1));
         }
-        kv += n_max;
+        kv += (uint32_t)(je - jb);
       }
       // Drain: every MMA issued above has completed before TMEM is released.
       umma_commit(bar(C::B_DRAIN));
@@ -502,29 +550,38 @@ __global__ void __launch_bounds__(384, 1)
     bool stores_pending = false;
     bool ok = true;
     PrefillUnit u;
-    for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT>(p, k, u); ++k) {
+    for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT, MASKS>(p, k, u); ++k) {
       const int row0 = i ? u.row0[1] : u.row0[0];
       if (row0 >= u.sq) continue;  // this tile slot holds no rows in this unit
-      const int n = i ? u.nkv[1] : u.nkv[0];
+      const int kb = i ? u.kv_begin[1] : u.kv_begin[0];  // this tile's KV tiles [kb, ke)
+      const int ke = i ? u.kv_end[1] : u.kv_end[0];
       const int row = row0 + r;
       const int q_head_row = u.b * p.Hq + u.hq;
       if (!VARLEN && p.k_lens != nullptr && r == 0) {
         const int kl = p.k_lens[u.b];
         if (kl < 0 || kl > p.Sk) flag_device_error(kDevErrBadLength);
       }
-      // largest visible key of this row, and of the tile's first row
+      // visible keys of this row: [lo_row, hi_row]; a tile needs the per-element
+      // rule unless every row of it sees all of it (j*128 >= lo_tile and
+      // j*128 + 127 <= hi_tile, the tightest bounds over its rows)
       const long long koff = (long long)u.klen - u.sq;
-      long long lim_row = (long long)u.klen - 1;
-      long long lim_tile = lim_row;
+      const int last_row = min(row0 + 127, u.sq - 1);
+      long long hi_row = (long long)u.klen - 1, hi_tile = hi_row;
+      long long lo_row = 0, lo_tile = 0;
+      const int prefix = MASKS ? p.prefix : 0, window = MASKS ? p.window : 0;
       if (CAUSAL) {
-        lim_row = min(lim_row, (long long)row + koff);
-        lim_tile = min(lim_tile, (long long)row0 + koff);
+        hi_row = min(hi_row, max((long long)row + koff, (long long)prefix - 1));
+        hi_tile = min(hi_tile, max((long long)row0 + koff, (long long)prefix - 1));
+        if (window > 0) {
+          lo_row = max(0LL, (long long)row + koff - window + 1);
+          lo_tile = max(0LL, (long long)last_row + koff - window + 1);
+        }
       }
       float m_run = -INFINITY;   // exponent base (log2 units)
       float l_run = 0.f;         // sum of P (f32)
       float lr_run = 0.f;        // sum of bf16(P)
 
-      for (int j = 0; j < n; ++j) {
+      for (int j = kb; j < ke; ++j) {
         if (!(ok = mbar_wait_warp(bar(C::B_SFULL + i), s_waits & 1u, abort_flag))) break;
         ++s_waits;
         tc_fence_after_sync();
@@ -548,13 +605,15 @@ __global__ void __launch_bounds__(384, 1)
             s[96 + e] = __uint_as_float(u3[e]);
           }
         }
-        if ((long long)j * 128 + 127 > lim_tile) {
+        if ((long long)j * 128 + 127 > hi_tile || (MASKS && (long long)j * 128 < lo_tile)) {
           // boundary tile: per-element predicate, in 32-bit once clamped to the tile
-          const long long ll = lim_row - (long long)j * 128;
-          const int lim_local = ll < -1 ? -1 : (ll > 127 ? 127 : (int)ll);
+          const long long hl = hi_row - (long long)j * 128;
+          const long long ll = lo_row - (long long)j * 128;
+          const int hi_local = hl < -1 ? -1 : (hl > 127 ? 127 : (int)hl);
+          const int lo_local = ll < 0 ? 0 : (ll > 128 ? 128 : (int)ll);
 #pragma unroll
           for (int c = 0; c < 128; ++c)
-            if (c > lim_local) s[c] = -INFINITY;
+            if (c > hi_local || (MASKS && c < lo_local)) s[c] = -INFINITY;
         }
         if (!scale_pos) {
 #pragma unroll
@@ -608,7 +667,7 @@ __global__ void __launch_bounds__(384, 1)
         lr_run = lr_run * alpha + ((r0 + r1) + (r2 + r3));
         // Rescale the accumulator when any row of this warp moved its base.  The
         // MMA that last wrote O_i completed before S_i(j) was signalled.
-        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (j > kb && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
           for (int c = 0; c < D; c += 32) {
             uint32_t v[32];
@@ -626,7 +685,7 @@ __global__ void __launch_bounds__(384, 1)
 
       // ---- epilogue: O = o / l -> bf16; each warp stages its 32 rows, 64
       // columns at a time, in its own buffer and stores them by TMA; LSE per row.
-      const bool has_o = n > 0;
+      const bool has_o = ke > kb;
       if (has_o) {
         if (!(ok = mbar_wait_warp(bar(C::B_OFULL + i), o_waits & 1u, abort_flag))) break;
         ++o_waits;

@@ -21,6 +21,7 @@
 // out and flagged (ATTN_DEVERR_BAD_LENGTH).
 #pragma once
 
+#include "prefill_sm100.cuh"
 #include "sm100_primitives.cuh"
 
 namespace attn_b200 {
@@ -50,16 +51,15 @@ __device__ __forceinline__ bool varlen_seq_lengths(const int* cu_q, const int* c
   return !bad;
 }
 
-// 128-key tiles the two query tiles of block qb visit (as prefill_num_kv_tiles).
-__device__ __forceinline__ int varlen_unit_weight(int qb, int len_q, int len_k, bool causal) {
+// 128-key tiles the two query tiles of block qb visit (prefill_kv_range).
+__device__ __forceinline__ int varlen_unit_weight(int qb, int len_q, int len_k, bool causal,
+                                                  int window, int prefix) {
   int w = 0;
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const int row0 = qb * 256 + i * 128;
-    if (row0 >= len_q) continue;
-    long long lim = (long long)len_k - 1;
-    if (causal) lim = min(lim, (long long)min(row0 + 127, len_q - 1) + len_k - len_q);
-    if (lim >= 0) w += (int)(lim / 128) + 1;
+    int lo, hi;
+    prefill_kv_range(qb * 256 + i * 128, len_q, len_k, causal, window, prefix, lo, hi);
+    w += hi - lo;
   }
   return w;
 }
@@ -106,7 +106,8 @@ __device__ __forceinline__ void block_suffix_sum(int* a, int n, bool exclusive, 
 __global__ void __launch_bounds__(1024, 1)
     attn_varlen_schedule_kernel(const int* cu_q, const int* cu_k, const int* seq_lens_k, int B,
                                 int total_q, int total_k, int max_seqlen_q, int max_keys,
-                                int causal, int level_shift, int n_levels, int2* units,
+                                int causal, int window, int prefix, int level_shift,
+                                int n_levels, int2* units,
                                 int* unit_count, int max_units) {
   extern __shared__ int sh[];
   int* lev = sh;                  // counts, then first positions / cursors
@@ -120,7 +121,7 @@ __global__ void __launch_bounds__(1024, 1)
                             lq, lk))
       continue;
     for (int qb = 0; qb * 256 < lq; ++qb) {
-      const int L = min(varlen_unit_weight(qb, lq, lk, causal != 0) >> level_shift, n_levels - 1);
+      const int L = min(varlen_unit_weight(qb, lq, lk, causal != 0, window, prefix) >> level_shift, n_levels - 1);
       atomicAdd(&lev[L], 1);
     }
   }
@@ -140,7 +141,7 @@ __global__ void __launch_bounds__(1024, 1)
                             lq, lk))
       continue;
     for (int qb = 0; qb * 256 < lq; ++qb) {
-      const int L = min(varlen_unit_weight(qb, lq, lk, causal != 0) >> level_shift, n_levels - 1);
+      const int L = min(varlen_unit_weight(qb, lq, lk, causal != 0, window, prefix) >> level_shift, n_levels - 1);
       const int pos = atomicAdd(&lev[L], 1);
       if (pos < max_units) units[pos] = make_int2(b, qb);
     }

@@ -94,6 +94,27 @@ int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float*
                     const int32_t* k_lens, attn_stream_t stream);
 
 /*
+ * attn_fwd_window -- causal prefill with a sliding window or a prefix-LM mask.
+ * Source: "Attention Kernel", section "可编程 mask" (masks such as a sliding
+ * window or a prefix-LM rule: block-level sparsity decides which tiles are
+ * skipped entirely, an element-wise rule handles the tiles that remain).
+ *   A query row i has key position p = i + (k_len[b] - Sq) (the causal
+ *   diagonal aligned to the bottom right, as attn_fwd_masked) and sees:
+ *     window > 0: keys p - window < j <= p (at most `window` keys ending at
+ *                 its diagonal);
+ *     prefix > 0: keys j <= p and every key j < prefix (prefix-LM);
+ *     window = prefix = 0: keys j <= p (attn_fwd_masked with causal = 1);
+ *   always within j < k_len[b].  window and prefix may not both be > 0.
+ *   Key tiles outside a row block's visible range are skipped at both ends.
+ * Other arguments, layouts and errors as attn_fwd_masked (INVALID_ARG also
+ * for a negative window or prefix, or both > 0).  Document masks are ragged
+ * batches (attn_fwd_varlen with one range per document).
+ */
+int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int Hq, int Hkv, int Sq, int Sk, int d, float scale, const int32_t* k_lens,
+                    int window, int prefix, attn_stream_t stream);
+
+/*
  * attn_fwd_varlen_workspace_size -- bytes of caller-owned device workspace
  * that attn_fwd_varlen needs: the list of (sequence, 256-row query block)
  * work units the call schedules.  total_q is the number of packed query

@@ -29,7 +29,7 @@ def lib():
 def test_header_declares_expected_entry_points():
     names = _declared_functions()
     for n in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_fwd_varlen_workspace_size",
-              "attn_fwd_paged",
+              "attn_fwd_paged", "attn_fwd_window",
               "attn_decode_paged", "attn_decode_workspace_size", "attn_get_device_error",
               "attn_strerror"):
         assert n in names
@@ -108,6 +108,19 @@ def _dec(lib, q=FAKE, kc=FAKE, vc=FAKE, tbl=FAKE, lens=FAKE, ps=16, B_=2, Hq=8, 
 ])
 def test_decode_validation(lib, kw, status):
     assert _dec(lib, **kw) == status
+
+
+@pytest.mark.parametrize("window,prefix,status", [
+    (-1, 0, B.ATTN_ERR_INVALID_ARG), (0, -1, B.ATTN_ERR_INVALID_ARG),
+    (16, 16, B.ATTN_ERR_INVALID_ARG)])
+def test_window_validation(lib, window, prefix, status):
+    assert lib.attn_fwd_window(FAKE, FAKE, FAKE, FAKE, None, 1, 2, 2, 128, 128, 128, 0.1, None,
+                               window, prefix, None) == status
+    # the common checks still come first
+    assert lib.attn_fwd_window(None, FAKE, FAKE, FAKE, None, 1, 2, 2, 128, 128, 128, 0.1, None,
+                               16, 0, None) == B.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_window(FAKE, FAKE, FAKE, FAKE, None, 1, 2, 2, 128, 128, 96, 0.1, None,
+                               16, 0, None) == B.ATTN_ERR_UNSUPPORTED
 
 
 def _var(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, cq=FAKE, ck=FAKE, B_=3, Hq=8, Hkv=2,
