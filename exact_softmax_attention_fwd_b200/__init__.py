@@ -7,6 +7,7 @@ first call does, and raises if the library is missing or no GPU is present.
 """
 from ._binding import (  # noqa: F401
     AttnError,
+    attn_fwd_block_sparse,
     attn_decode_paged,
     attn_decode_workspace_size,
     attn_fwd,

@@ -37,6 +37,8 @@ SIGNATURES = {
     "attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "attn_fwd_masked": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P]),
     "attn_fwd_window": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _I, _I, _P]),
+    "attn_fwd_block_sparse": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _I,
+                                   _P]),
     "attn_fwd_varlen_workspace_size": (_SZ, [_I, ctypes.c_longlong, _I]),
     "attn_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, ctypes.c_longlong,
                              ctypes.c_longlong, _I, _I, _I, _F, _P, _SZ, _P]),
@@ -165,6 +167,37 @@ def attn_fwd_window(q, k, v, scale: float, window: int = 0, prefix: int = 0, k_l
                                         Hkv, Sq, Sk, d, float(scale), _ptr(k_lens), int(window),
                                         int(prefix), _stream(stream))
     _check(st, "attn_fwd_window")
+    return out, lse
+
+
+def attn_fwd_block_sparse(q, k, v, block_mask, causal: bool, scale: float, k_lens=None,
+                          out=None, lse=None, return_lse: bool = True, stream=None):
+    """Prefill with a block-sparse mask: block_mask uint8 [B, 1 or Hq, ceil(Sq/128),
+    ceil(Sk/128)] on the device (0 = the 128 x 128 block is skipped)."""
+    import torch
+    _require_cuda(q, k, v, k_lens, block_mask)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bfloat16")
+    B, Hq, Sq, d = q.shape
+    Bk, Hkv, Sk, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or dk != d:
+        raise ValueError("q/k/v shapes disagree")
+    if block_mask.dtype != torch.uint8 or not block_mask.is_contiguous() or block_mask.dim() != 4 \
+            or block_mask.shape[0] != B or block_mask.shape[1] not in (1, Hq) \
+            or block_mask.shape[2] != -(-Sq // 128) or block_mask.shape[3] != -(-Sk // 128):
+        raise ValueError("block_mask must be contiguous uint8 [B, 1 or Hq, ceil(Sq/128), ceil(Sk/128)]")
+    if k_lens is not None and (k_lens.dtype != torch.int32 or tuple(k_lens.shape) != (B,)):
+        raise ValueError("k_lens must be int32 [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    st = load_library().attn_fwd_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B,
+                                              Hq, Hkv, Sq, Sk, d, int(bool(causal)), float(scale),
+                                              _ptr(k_lens), _ptr(block_mask), block_mask.shape[1],
+                                              _stream(stream))
+    _check(st, "attn_fwd_block_sparse")
     return out, lse
 
 

@@ -138,10 +138,12 @@ int check_prefill_args(const void* q, const void* k, const void* v, void* o, flo
 // total_q / 256 + B for non-overlapping ranges; one more for rounding.
 long long varlen_max_units(int B, long long total_q) { return total_q / 256 + B + 1; }
 
-// Dense fixed-length prefill with optional key lengths, sliding window and prefix.
+// Dense fixed-length prefill with optional key lengths, sliding window, prefix
+// and block mask.
 int prefill_dense(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                   int Hkv, int Sq, int Sk, int d, int causal, float scale, const int32_t* k_lens,
-                  int window, int prefix, cudaStream_t stream) {
+                  int window, int prefix, const uint8_t* block_mask, int mask_heads,
+                  cudaStream_t stream) {
   const long long rows_q = (long long)B * Hq * Sq;
   if (Sk == 0) {
     const size_t n_vec = (size_t)rows_q * d * 2 / 16;
@@ -172,9 +174,17 @@ int prefill_dense(const void* q, const void* k, const void* v, void* o, float* l
   prm.n_qblocks = (Sq + 255) / 256;
   prm.window = window;
   prm.prefix = prefix;
-  if (window > 0 || prefix > 0)  // causal only (checked by the caller)
-    return d == 128 ? launch_prefill<128, true, kLayoutDense, true>(mq, mk, mv, mo, prm, stream)
-                    : launch_prefill<64, true, kLayoutDense, true>(mq, mk, mv, mo, prm, stream);
+  prm.block_mask = block_mask;
+  prm.mask_heads = mask_heads;
+  prm.n_qt = (Sq + 127) / 128;
+  prm.n_kt = (Sk + 127) / 128;
+  if (window > 0 || prefix > 0 || block_mask != nullptr) {  // window / prefix need causal
+    if (d == 128)
+      return causal ? launch_prefill<128, true, kLayoutDense, true>(mq, mk, mv, mo, prm, stream)
+                    : launch_prefill<128, false, kLayoutDense, true>(mq, mk, mv, mo, prm, stream);
+    return causal ? launch_prefill<64, true, kLayoutDense, true>(mq, mk, mv, mo, prm, stream)
+                  : launch_prefill<64, false, kLayoutDense, true>(mq, mk, mv, mo, prm, stream);
+  }
   if (d == 128)
     return causal ? launch_prefill<128, true>(mq, mk, mv, mo, prm, stream)
                   : launch_prefill<128, false>(mq, mk, mv, mo, prm, stream);
@@ -209,7 +219,7 @@ int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float*
   const int st = check_prefill_args(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens);
   if (st != ATTN_OK) return st;
   return prefill_dense(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens, 0, 0,
-                       reinterpret_cast<cudaStream_t>(stream));
+                       nullptr, 1, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -219,7 +229,18 @@ int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float*
   if (st != ATTN_OK) return st;
   if (window < 0 || prefix < 0 || (window > 0 && prefix > 0)) return ATTN_ERR_INVALID_ARG;
   return prefill_dense(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, 1, scale, k_lens, window, prefix,
-                       reinterpret_cast<cudaStream_t>(stream));
+                       nullptr, 1, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                          int Hq, int Hkv, int Sq, int Sk, int d, int causal, float scale,
+                          const int32_t* k_lens, const uint8_t* block_mask, int mask_heads,
+                          attn_stream_t stream) {
+  const int st = check_prefill_args(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens);
+  if (st != ATTN_OK) return st;
+  if (block_mask == nullptr || (mask_heads != 1 && mask_heads != Hq)) return ATTN_ERR_INVALID_ARG;
+  return prefill_dense(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens, 0, 0,
+                       block_mask, mask_heads, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t attn_fwd_varlen_workspace_size(int B, long long total_q, int max_seqlen_q) {

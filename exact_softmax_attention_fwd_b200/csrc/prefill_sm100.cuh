@@ -68,6 +68,10 @@ struct PrefillParams {
   // programmable masks (causal only; 0 = off): a row at key position p sees
   // keys (p - window, p] (sliding window), or keys below prefix as well (prefix-LM)
   int window, prefix;
+  // block-sparse mask (MASKS instantiations; nullable): uint8 [B, mask_heads,
+  // n_qt, n_kt] over 128 x 128 (query tile, key tile) blocks, 0 = skipped
+  const uint8_t* block_mask;
+  int mask_heads, n_qt, n_kt;
   // ragged batches: packed token-major tensors, cumulative sequence lengths
   // and the unit list written by attn_varlen_schedule_kernel
   uint16_t* o;          // [total_q, Hq, d] bf16
@@ -120,6 +124,8 @@ struct PrefillCfg {
   static constexpr uint32_t REGS_SOFTMAX = 224;
   static_assert(128 * (REGS_PRODUCER + 2 * REGS_SOFTMAX) <= NUM_THREADS * REGS_LAUNCH,
                 "register reallocation must fit the launch allocation");
+  static_assert(128 * ((REGS_PRODUCER + 16) + 2 * (REGS_SOFTMAX - 16)) <= NUM_THREADS * REGS_LAUNCH,
+                "the masked split must fit too");
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -153,6 +159,17 @@ __device__ __forceinline__ void prefill_kv_range(int row0, int Sq, int klen, boo
   if (top < bot) return;
   lo = (int)(bot / 128);
   hi = (int)(top / 128) + 1;
+}
+
+// Whether key tile kb is computed for the query tile starting at row0: inside
+// the tile's range [kbeg, kend) and, with a block mask, not switched off.
+__device__ __forceinline__ bool prefill_block_on(const PrefillParams& p, int b, int hq, int row0,
+                                                 int kbeg, int kend, int kb) {
+  if (kb < kbeg || kb >= kend) return false;
+  if (p.block_mask == nullptr) return true;
+  const size_t h = p.mask_heads == 1 ? 0 : (size_t)hq;
+  return __ldg(p.block_mask + ((((size_t)b * p.mask_heads + h) * p.n_qt + row0 / 128) * p.n_kt +
+                               kb)) != 0;
 }
 
 // One work unit: query rows [256*qb, 256*qb + 256) of head hq in sequence b.
@@ -220,6 +237,15 @@ __device__ __forceinline__ bool prefill_unit(const PrefillParams& p, int k, Pref
     u.row0[i] = u.qb * 256 + i * 128;
     prefill_kv_range(u.row0[i], u.sq, u.klen, CAUSAL, MASKS ? p.window : 0,
                      MASKS ? p.prefix : 0, u.kv_begin[i], u.kv_end[i]);
+    if (MASKS && p.block_mask != nullptr) {
+      // tighten the range to its first and last computed block, so that a
+      // tile with no block left has an empty range (and no Q load)
+      int lo = u.kv_begin[i], hi = u.kv_end[i];
+      while (lo < hi && !prefill_block_on(p, u.b, u.hq, u.row0[i], lo, hi, lo)) ++lo;
+      while (hi > lo && !prefill_block_on(p, u.b, u.hq, u.row0[i], lo, hi, hi - 1)) --hi;
+      u.kv_begin[i] = lo < hi ? lo : 0;
+      u.kv_end[i] = lo < hi ? hi : 0;
+    }
     if (u.kv_end[i] > u.kv_begin[i]) {
       u.kv_first = min(u.kv_first, u.kv_begin[i]);
       u.kv_last = max(u.kv_last, u.kv_end[i]);
@@ -291,7 +317,8 @@ __global__ void __launch_bounds__(384, 1)
   // makes it, so that the compiler sees every role's code reachable only under
   // its own register budget.
   if (warp < 4) {
-    warpgroup_reg_dealloc<C::REGS_PRODUCER>();
+    // the masked instantiations keep more stream state in the MMA warp
+    warpgroup_reg_dealloc<MASKS ? C::REGS_PRODUCER + 16 : C::REGS_PRODUCER>();
     if (warp == 0) {
     // ======================= TMA producer =======================
     if (lane == 0) {
@@ -326,7 +353,12 @@ __global__ void __launch_bounds__(384, 1)
         // Q_0 first (its slot frees first under a causal mask), then the first
         // K tile, then Q_1, so that no wait on Q_1 holds back the K/V stream.
         if (has0 && !(ok = load_q(u, 0))) break;
-        for (int j = u.kv_first; j < u.kv_last; ++j, ++kv) {
+        for (int j = u.kv_first; j < u.kv_last; ++j) {
+          // with a block mask, key tiles no query tile of the unit computes are not streamed
+          if (MASKS && p.block_mask != nullptr &&
+              !prefill_block_on(p, u.b, u.hq, u.row0[0], u.kv_begin[0], u.kv_end[0], j) &&
+              !prefill_block_on(p, u.b, u.hq, u.row0[1], u.kv_begin[1], u.kv_end[1], j))
+            continue;
           const int s = kv % C::STAGES;
           const uint32_t ph = (kv / C::STAGES) & 1u;
           if (!(ok = mbar_wait(bar(C::B_KEMPTY + s), ph ^ 1u, abort_flag))) break;
@@ -348,6 +380,7 @@ __global__ void __launch_bounds__(384, 1)
             tma_load_3d(sbase + C::OFF_V + s * C::TILE_BYTES + cb * C::CB_BYTES, &tm_v,
                         bar(C::B_VFULL + s), 64 * cb, VARLEN ? kvh : j * 128,
                         VARLEN ? u.k_tok0 + j * 128 : kv_row);
+          ++kv;
         }
       }
       // Drain: never leave the CTA with copies still landing in shared memory.
@@ -472,6 +505,62 @@ __global__ void __launch_bounds__(384, 1)
           if (!ok) break;
           umma_commit(bar(C::B_KEMPTY + s));
         }
+        if (MASKS && p.block_mask != nullptr) {
+          // Block-sparse stream: the key tiles some query tile computes, in
+          // order.  Per stream tile kb: PV for each tile computing kb, then the
+          // QK of each tile that computes the next stream tile.
+          auto on = [&](int i, int kb) {
+            return prefill_block_on(p, u.b, u.hq, u.row0[i], u.kv_begin[i], u.kv_end[i], kb);
+          };
+          auto next_pos = [&](int kb) {
+            for (int x = kb + 1; x < je; ++x)
+              if (on(0, x) || on(1, x)) return x;
+            return -1;
+          };
+          uint32_t pos = 0;
+          for (int kb = jb; ok && kb >= 0; ++pos) {
+            const int kbn = next_pos(kb);
+            const uint32_t idx = kv + pos;
+            const int s = idx % C::STAGES;
+            const int s1 = (idx + 1) % C::STAGES;
+            if (!(ok = mbar_wait(bar(C::B_VFULL + s), (idx / C::STAGES) & 1u, abort_flag))) break;
+            bool k_next = false;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              if (!ok) break;
+              if (on(i, kb)) {
+                uint32_t& pw = i ? p_waits1 : p_waits0;
+                if (!(ok = mbar_wait(bar(C::B_PFULL + i), pw & 1u, abort_flag))) break;
+                ++pw;
+                tc_fence_after_sync();
+                issue_pv(i, s, kb > u.kv_begin[i]);
+                if (kb == u.kv_end[i] - 1) umma_commit(bar(C::B_OFULL + i));
+              }
+              if (kbn >= 0 && on(i, kbn)) {
+                if (!k_next) {
+                  if (!(ok = mbar_wait(bar(C::B_KFULL + s1), ((idx + 1) / C::STAGES) & 1u,
+                                       abort_flag)))
+                    break;
+                  k_next = true;
+                }
+                if (kbn == u.kv_begin[i]) {  // this tile's first S: its Q must have landed
+                  uint32_t& qw = i ? q_waits1 : q_waits0;
+                  if (!(ok = mbar_wait(bar(C::B_QFULL + i), qw & 1u, abort_flag))) break;
+                  ++qw;
+                }
+                tc_fence_after_sync();
+                issue_qk(i, s1);
+                umma_commit(bar(C::B_SFULL + i));
+                if (kbn == u.kv_end[i] - 1) umma_commit(bar(C::B_QFREE + i));
+              }
+            }
+            umma_commit(bar(C::B_VEMPTY + s));
+            if (k_next) umma_commit(bar(C::B_KEMPTY + s1));
+            kb = kbn;
+          }
+          kv += pos;
+          continue;
+        }
         for (int j = jb; ok && j < je; ++j) {
           const uint32_t idx = kv + (uint32_t)(j - jb);
           const int s = idx % C::STAGES;
@@ -533,7 +622,7 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
     }  // warps 2-3: nothing to do
   } else {
-    warpgroup_reg_alloc<C::REGS_SOFTMAX>();
+    warpgroup_reg_alloc<MASKS ? C::REGS_SOFTMAX - 16 : C::REGS_SOFTMAX>();
     // ======================= softmax warpgroups =======================
     const int i = (warp - 4) >> 2;       // query tile slot of this warpgroup
     const int quarter = warp & 3;        // TMEM lane quarter this warp may access
@@ -582,6 +671,8 @@ __global__ void __launch_bounds__(384, 1)
       float lr_run = 0.f;        // sum of bf16(P)
 
       for (int j = kb; j < ke; ++j) {
+        if (MASKS && p.block_mask != nullptr && !prefill_block_on(p, u.b, u.hq, row0, kb, ke, j))
+          continue;  // a block the mask switches off: no S, no P for it
         if (!(ok = mbar_wait_warp(bar(C::B_SFULL + i), s_waits & 1u, abort_flag))) break;
         ++s_waits;
         tc_fence_after_sync();

@@ -108,11 +108,30 @@ int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float*
  *   Key tiles outside a row block's visible range are skipped at both ends.
  * Other arguments, layouts and errors as attn_fwd_masked (INVALID_ARG also
  * for a negative window or prefix, or both > 0).  Document masks are ragged
- * batches (attn_fwd_varlen with one range per document).
+ * batches (attn_fwd_varlen with one range per document); block-sparse masks
+ * are attn_fwd_block_sparse.
  */
 int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                     int Hq, int Hkv, int Sq, int Sk, int d, float scale, const int32_t* k_lens,
                     int window, int prefix, attn_stream_t stream);
+
+/*
+ * attn_fwd_block_sparse -- prefill with a block-sparse mask.
+ * Source: "Attention Kernel", section "可编程 mask" (block-level sparsity
+ * decides which tiles are skipped entirely; the element-wise rule -- here the
+ * causal / key-length one of attn_fwd_masked -- handles the tiles left).
+ *   block_mask  uint8 [B, mask_heads, ceil(Sq/128), ceil(Sk/128)] device
+ *               array (mask_heads 1: shared by all query heads, or Hq): entry
+ *               [b][h][i/128][j/128] == 0 hides key j from query row i of
+ *               head h; such 128 x 128 blocks are never loaded or computed.
+ *   Rows left without a visible key get O = 0, LSE = -inf.
+ * Other arguments, layouts and errors as attn_fwd_masked (INVALID_ARG also
+ * for a NULL mask or mask_heads not in {1, Hq}).
+ */
+int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                          int Hq, int Hkv, int Sq, int Sk, int d, int causal, float scale,
+                          const int32_t* k_lens, const uint8_t* block_mask, int mask_heads,
+                          attn_stream_t stream);
 
 /*
  * attn_fwd_varlen_workspace_size -- bytes of caller-owned device workspace

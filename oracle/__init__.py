@@ -72,6 +72,9 @@ def _load():
             lib.oracle_attn_fwd_rows_masked.argtypes = [P, P, P, I, I, I, I, I, I, I, D, P, I, I,
                                                         P, L, P, P, I]
             lib.oracle_attn_fwd_rows_masked.restype = I
+            lib.oracle_attn_fwd_rows_blocks.argtypes = [P, P, P, I, I, I, I, I, I, I, D, P, I, I,
+                                                        P, I, P, L, P, P, I]
+            lib.oracle_attn_fwd_rows_blocks.restype = I
             lib.oracle_decode_paged.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, D, P, P, I]
             lib.oracle_decode_paged.restype = I
             _lib = lib
@@ -136,12 +139,15 @@ def online_attend(scores, values, block_size, block_order=None):
     return o, float(lse[0])
 
 
-def attn_fwd(q, k, v, causal, scale, k_lens=None, rows=None, n_threads=None, window=0, prefix=0):
+def attn_fwd(q, k, v, causal, scale, k_lens=None, rows=None, n_threads=None, window=0, prefix=0,
+             block_mask=None):
     """Exact attention.  q [B,Hq,Sq,d], k/v [B,Hkv,Sk,d] bf16 (torch or uint16 bits).
 
     ``window`` > 0 (causal only): a row at key position p sees keys (p - window, p];
     ``prefix`` > 0 (causal only): keys below ``prefix`` are visible to every row
     ("Attention Kernel", section "可编程 mask"; not both at once).
+    ``block_mask``: optional uint8 [B, 1 or Hq, ceil(Sq/128), ceil(Sk/128)]; a
+    zero entry hides every (row, key) pair of that 128 x 128 block.
 
     ``rows``: optional flat row ids (b*Hq + hq)*Sq + i; default every row.
     Returns (o, lse) as float64 arrays: o [n_rows, d] (or [B,Hq,Sq,d] when
@@ -157,10 +163,17 @@ def attn_fwd(q, k, v, causal, scale, k_lens=None, rows=None, n_threads=None, win
     n = B * Hq * Sq if r is None else r.shape[0]
     o = np.zeros((n, d), np.float64)
     lse = np.zeros(n, np.float64)
-    st = _load().oracle_attn_fwd_rows_masked(_ptr(qb), _ptr(kb), _ptr(vb), B, Hq, Hkv, Sq, Sk, d,
+    bm, mh = None, 1
+    if block_mask is not None:
+        bm = np.ascontiguousarray(np.asarray(block_mask), dtype=np.uint8)
+        if bm.ndim != 4 or bm.shape[0] != B or bm.shape[1] not in (1, Hq) or \
+                bm.shape[2] != -(-Sq // 128) or bm.shape[3] != -(-Sk // 128):
+            raise ValueError("block_mask must be uint8 [B, 1 or Hq, ceil(Sq/128), ceil(Sk/128)]")
+        mh = bm.shape[1]
+    st = _load().oracle_attn_fwd_rows_blocks(_ptr(qb), _ptr(kb), _ptr(vb), B, Hq, Hkv, Sq, Sk, d,
                                              int(bool(causal)), float(scale), _ptr(kl),
-                                             int(window), int(prefix), _ptr(r), n, _ptr(o),
-                                             _ptr(lse), _threads(n_threads))
+                                             int(window), int(prefix), _ptr(bm), mh, _ptr(r), n,
+                                             _ptr(o), _ptr(lse), _threads(n_threads))
     if st != OK:
         raise OracleError(st)
     if r is None:

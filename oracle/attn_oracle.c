@@ -39,6 +39,9 @@
  *     with causal: a sliding window w > 0 keeps only the w keys ending at the
  *     row's position p = i + (k_len - Sq), i.e. j > p - w; a prefix P > 0
  *     makes keys j < P visible to every row (prefix-LM).  Not both at once.
+ *     A block mask (uint8 [B, mask_heads, ceil(Sq/128), ceil(Sk/128)],
+ *     mask_heads 1 or Hq) hides every key j of query row i whose block
+ *     entry [b][h][i/128][j/128] is 0 (block-sparse attention).
  *
  * Inputs to the attention routines are bf16 bit patterns (uint16); this
  * file widens them to double itself (a bf16 value is the top half of an
@@ -178,7 +181,8 @@ int oracle_online_attend(const double* s, int n_scores, const double* v,
 
 typedef struct {
   const uint16_t *q, *k, *v;
-  int B, Hq, Hkv, Sq, Sk, d, causal, window, prefix;
+  int B, Hq, Hkv, Sq, Sk, d, causal, window, prefix, mask_heads;
+  const uint8_t* block_mask;
   double scale;
   const int32_t* k_lens;
   const int64_t* rows; /* flat row ids (b*Hq + hq)*Sq + i, or NULL = all */
@@ -225,6 +229,12 @@ static int prefill_row(const prefill_job* J, int64_t r, prefill_scratch* W) {
       visible = visible && ((int64_t)j <= pos || (int64_t)j < J->prefix);
       if (J->window > 0) visible = visible && (int64_t)j > pos - J->window;
     }
+    if (J->block_mask) {
+      int64_t n_qt = (J->Sq + 127) / 128, n_kt = (J->Sk + 127) / 128;
+      int64_t h = J->mask_heads == 1 ? 0 : hq;
+      visible = visible &&
+                J->block_mask[(((int64_t)b * J->mask_heads + h) * n_qt + i / 128) * n_kt + j / 128];
+    }
     if (!visible) {
       W->s[j] = -INFINITY;
       continue;
@@ -262,17 +272,18 @@ static void* prefill_worker(void* arg) {
  * gives the number of leading keys visible per sequence.  Work is split over
  * n_threads POSIX threads by rows; each row is computed independently.
  */
-int oracle_attn_fwd_rows_masked(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+int oracle_attn_fwd_rows_blocks(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                 int B, int Hq, int Hkv, int Sq, int Sk, int d, int causal,
                                 double scale, const int32_t* k_lens, int window, int prefix,
-                                const int64_t* rows, int64_t n_rows, double* o, double* lse,
-                                int n_threads) {
+                                const uint8_t* block_mask, int mask_heads, const int64_t* rows,
+                                int64_t n_rows, double* o, double* lse, int n_threads) {
   if (!q || (Sk > 0 && (!k || !v)) || !o || !lse || B < 1 || Hq < 1 || Hkv < 1 ||
       Sq < 1 || Sk < 0 || d < 1 || Hq % Hkv != 0 || n_rows < 0 || !isfinite(scale))
     return ORACLE_ERR_ARG;
   if (window < 0 || prefix < 0 || (window > 0 && prefix > 0) ||
       ((window > 0 || prefix > 0) && !causal))
     return ORACLE_ERR_ARG;
+  if (block_mask && mask_heads != 1 && mask_heads != Hq) return ORACLE_ERR_ARG;
   if (!rows && n_rows != (int64_t)B * Hq * Sq) return ORACLE_ERR_ARG;
   if (n_threads < 1) n_threads = 1;
   if ((int64_t)n_threads > n_rows) n_threads = n_rows > 0 ? (int)n_rows : 1;
@@ -289,6 +300,7 @@ int oracle_attn_fwd_rows_masked(const uint16_t* q, const uint16_t* k, const uint
     J->B = B; J->Hq = Hq; J->Hkv = Hkv; J->Sq = Sq; J->Sk = Sk; J->d = d;
     J->causal = causal; J->scale = scale; J->k_lens = k_lens;
     J->window = window; J->prefix = prefix;
+    J->block_mask = block_mask; J->mask_heads = mask_heads;
     J->rows = rows; J->n_rows = n_rows; J->o = o; J->lse = lse;
     J->begin = n_rows * w / n_threads;
     J->end = n_rows * (w + 1) / n_threads;
@@ -303,6 +315,16 @@ int oracle_attn_fwd_rows_masked(const uint16_t* q, const uint16_t* k, const uint
   free(jobs);
   free(th);
   return status;
+}
+
+/* oracle_attn_fwd_rows_blocks without a block mask. */
+int oracle_attn_fwd_rows_masked(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                int B, int Hq, int Hkv, int Sq, int Sk, int d, int causal,
+                                double scale, const int32_t* k_lens, int window, int prefix,
+                                const int64_t* rows, int64_t n_rows, double* o, double* lse,
+                                int n_threads) {
+  return oracle_attn_fwd_rows_blocks(q, k, v, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens,
+                                     window, prefix, NULL, 1, rows, n_rows, o, lse, n_threads);
 }
 
 /* oracle_attn_fwd_rows_masked without a window or prefix. */

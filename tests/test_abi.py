@@ -29,7 +29,7 @@ def lib():
 def test_header_declares_expected_entry_points():
     names = _declared_functions()
     for n in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_fwd_varlen_workspace_size",
-              "attn_fwd_paged", "attn_fwd_window",
+              "attn_fwd_paged", "attn_fwd_window", "attn_fwd_block_sparse",
               "attn_decode_paged", "attn_decode_workspace_size", "attn_get_device_error",
               "attn_strerror"):
         assert n in names
@@ -121,6 +121,13 @@ def test_window_validation(lib, window, prefix, status):
                                16, 0, None) == B.ATTN_ERR_INVALID_ARG
     assert lib.attn_fwd_window(FAKE, FAKE, FAKE, FAKE, None, 1, 2, 2, 128, 128, 96, 0.1, None,
                                16, 0, None) == B.ATTN_ERR_UNSUPPORTED
+
+
+def test_block_sparse_validation(lib):
+    args = (FAKE, FAKE, FAKE, FAKE, None, 1, 4, 2, 128, 128, 128, 1, 0.1, None)
+    assert lib.attn_fwd_block_sparse(*args, None, 1, None) == B.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_block_sparse(*args, FAKE, 2, None) == B.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_block_sparse(None, *args[1:], FAKE, 1, None) == B.ATTN_ERR_INVALID_ARG
 
 
 def _var(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, cq=FAKE, ck=FAKE, B_=3, Hq=8, Hkv=2,

@@ -82,3 +82,72 @@ def test_sliding_window_8k_sampled_rows():
     o_ref, lse_ref = oracle.attn_fwd(q, k, v, True, c.scale, rows=rows, window=1024)
     check(o.reshape(-1, c.d)[rows], o_ref, lse.reshape(-1)[rows], lse_ref,
           what="gqa_causal_8k window 1024 sampled rows")
+
+
+# ------------------------------------------------------------------ block-sparse masks
+
+from exact_softmax_attention_fwd_b200 import attn_fwd_block_sparse  # noqa: E402
+
+
+def _blocks(B, heads, Sq, Sk, density, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.rand(B, heads, -(-Sq // 128), -(-Sk // 128), generator=g) < density).to(torch.uint8)
+
+
+def _run_bs(q, k, v, bm, causal, scale, k_lens=None):
+    kl = None if k_lens is None else k_lens.to(DEV)
+    o, lse = attn_fwd_block_sparse(q.to(DEV), k.to(DEV), v.to(DEV), bm.to(DEV), causal, scale,
+                                   k_lens=kl)
+    torch.cuda.synchronize()
+    st, flags = attn_get_device_error()
+    assert st == 0, f"device error flags {flags:#x}"
+    return o.cpu(), lse.cpu()
+
+
+BS_CASES = [
+    # (B, Hq, Hkv, Sq, Sk, d, causal, heads, density)
+    (1, 4, 2, 700, 700, 128, True, 1, 0.5),
+    (2, 4, 4, 513, 900, 64, False, 4, 0.3),
+    (1, 8, 2, 1000, 1000, 128, True, 8, 0.7),
+    (1, 2, 1, 300, 1300, 128, False, 1, 0.2),
+]
+
+
+@pytest.mark.parametrize("case", BS_CASES, ids=[str(c) for c in BS_CASES])
+def test_block_sparse_parity(case):
+    B, Hq, Hkv, Sq, Sk, d, causal, heads, density = case
+    q, k, v = W.prefill_inputs(B, Hq, Hkv, Sq, Sk, d, seed=199)
+    bm = _blocks(B, heads, Sq, Sk, density, seed=211)
+    scale = 1 / math.sqrt(d)
+    o, lse = _run_bs(q, k, v, bm, causal, scale)
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, causal, scale, block_mask=bm)
+    check(o, o_ref, lse, lse_ref, what=f"block sparse {case}")
+
+
+def test_block_sparse_band_with_key_padding():
+    B, Hq, Hkv, S, d = 2, 4, 2, 900, 128
+    q, k, v = W.prefill_inputs(B, Hq, Hkv, S, S, d, seed=223)
+    n = -(-S // 128)
+    t = torch.arange(n)
+    bm = ((t[:, None] - t[None, :]).abs() <= 1).to(torch.uint8).view(1, 1, n, n).repeat(B, 1, 1, 1)
+    k_lens = torch.tensor([900, 400], dtype=torch.int32)
+    o, lse = _run_bs(q, k, v, bm, True, 0.09, k_lens)
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, True, 0.09, k_lens=k_lens, block_mask=bm)
+    check(o, o_ref, lse, lse_ref, what="block band + key padding")
+
+
+def test_block_sparse_all_ones_bitwise_and_empty_tiles():
+    q, k, v = W.prefill_inputs(1, 4, 2, 600, 600, 128, seed=227)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    for causal in (False, True):
+        ones = torch.ones(1, 1, 5, 5, dtype=torch.uint8, device=DEV)
+        a = attn_fwd_masked(qd, kd, vd, causal, 0.1)
+        b = attn_fwd_block_sparse(qd, kd, vd, ones, causal, 0.1)
+        assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]), causal
+    bm = torch.ones(1, 4, 5, 5, dtype=torch.uint8)
+    bm[0, 2, 1, :] = 0  # head 2, query rows 128..255: nothing visible
+    bm[0, 1, :, 0] = 0
+    o, lse = _run_bs(q, k, v, bm, False, 0.1)
+    assert torch.all(o[0, 2, 128:256] == 0) and torch.isneginf(lse[0, 2, 128:256]).all()
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, False, 0.1, block_mask=bm)
+    check(o, o_ref, lse, lse_ref, what="block sparse with empty tiles")

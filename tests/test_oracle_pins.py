@@ -605,3 +605,41 @@ def test_document_mask_is_the_ragged_batch_of_its_documents():
                           v.permute(1, 0, 2)[None], 0.4, vis)
     np.testing.assert_allclose(o, ro[0].transpose(1, 0, 2), rtol=0, atol=1e-12)
     np.testing.assert_allclose(lse, rl[0], rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- block-sparse masks
+# "Attention Kernel", section "可编程 mask": block-level sparsity decides which
+# tiles are skipped entirely.  A zero entry of the [B, 1 or H, Sq/128, Sk/128]
+# block mask hides the whole 128 x 128 block.
+
+
+@pytest.mark.parametrize("causal,heads", [(False, 1), (True, 4)])
+def test_block_mask_against_sdpa(causal, heads):
+    B, Hq, Hkv, Sq, Sk, d = 1, 4, 2, 300, 420, 8
+    q, k, v = workloads.prefill_inputs(B, Hq, Hkv, Sq, Sk, d, seed=191)
+    g = torch.Generator().manual_seed(193)
+    bm = (torch.rand(B, heads, 3, 4, generator=g) < 0.6).to(torch.uint8)
+    bm[..., 0] = 1  # every row keeps its first key block
+    o, lse = oracle.attn_fwd(q, k, v, causal, 0.3, block_mask=bm)
+    blk = bm.repeat_interleave(128, 2).repeat_interleave(128, 3)[:, :, :Sq, :Sk].bool()
+    vis = blk.expand(B, Hq, Sq, Sk)
+    if causal:
+        i = torch.arange(Sq)[:, None] + (Sk - Sq)
+        vis = vis & (torch.arange(Sk)[None, :] <= i)
+    ro, rl = _sdpa_masked(q, k, v, 0.3, vis)
+    np.testing.assert_allclose(o, ro, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, rl, rtol=0, atol=1e-12)
+
+
+def test_block_mask_all_ones_is_no_mask_and_empty_rows_are_zero():
+    q, k, v = workloads.prefill_inputs(2, 2, 2, 200, 300, 8, seed=197)
+    ones = np.ones((2, 1, 2, 3), np.uint8)
+    a = oracle.attn_fwd(q, k, v, True, 0.5, block_mask=ones)
+    b_ = oracle.attn_fwd(q, k, v, True, 0.5)
+    np.testing.assert_array_equal(a[0], b_[0])
+    np.testing.assert_array_equal(a[1], b_[1])
+    bm = ones.copy()
+    bm[1, 0, 1, :] = 0  # sequence 1, query rows 128..199: no visible block
+    o, lse = oracle.attn_fwd(q, k, v, False, 0.5, block_mask=bm)
+    assert np.array_equal(o[1, :, 128:], np.zeros_like(o[1, :, 128:]))
+    assert np.isneginf(lse[1, :, 128:]).all()
