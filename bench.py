@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-ragged", action="store_true")
     ap.add_argument("--ragged-workload", default="ragged_gqa_causal")
+    ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--backward-workload", default="mha_causal_2k")
     ap.add_argument("--no-paged-prefill", action="store_true")
     ap.add_argument("--paged-prefill-workload", default="paged_prefill_gqa")
     return ap.parse_args()
@@ -410,6 +412,8 @@ def run_ours(args, world, rank, local):
         line["ragged"] = ragged_leg(args, dev, world, peaks)
     if not args.no_paged_prefill:
         line["paged_prefill"] = paged_prefill_leg(args, dev, world, peaks)
+    if not args.no_backward:
+        line["backward"] = backward_leg(args, dev, world, peaks)
     if not args.no_e2e:
         line["e2e"] = e2e_leg(args, cfg, q_h, k_h, v_h, kl_h, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -439,6 +443,47 @@ def _timed_calls(args, dev, world, one):
         e1.record(stream)
     torch.cuda.synchronize(dev)
     return [a.elapsed_time(b) for a, b in evs]
+
+
+def backward_leg(args, dev, world, peaks):
+    """The backward pass from the saved LSE (attn_bwd: the row-statistics kernel, the
+    dK/dV kernel and the dQ kernel) on a prefill workload, timed on its own: the
+    forward outputs are computed once before timing, inputs resident, L2 flushed
+    before each call.  FLOPs are the backward's five products (2.5x the forward's
+    count, halved when causal); the two-kernel design executes seven (3.5x)."""
+    import torch
+
+    from exact_softmax_attention_fwd_b200 import (attn_bwd, attn_bwd_workspace_size,
+                                                  attn_fwd_masked, attn_get_device_error)
+    from exact_softmax_attention_fwd_b200 import workloads as W
+
+    cfg = W.CONFIGS[args.backward_workload]
+    q_h, k_h, v_h, kl_h = W.config_inputs(cfg)
+    do_h = W.grad_output(cfg.B, cfg.Hq, cfg.S, cfg.d, seed=cfg.seed)
+    q, k, v, do = q_h.to(dev), k_h.to(dev), v_h.to(dev), do_h.to(dev)
+    kl = None if kl_h is None else kl_h.to(dev)
+    o, lse = attn_fwd_masked(q, k, v, cfg.causal, cfg.scale, k_lens=kl)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(attn_bwd_workspace_size(cfg.B, cfg.Hq, cfg.S), dtype=torch.uint8,
+                     device=dev)
+
+    def one():
+        attn_bwd(q, k, v, o, lse, do, cfg.causal, cfg.scale, k_lens=kl, dq=dq, dk=dk, dv=dv,
+                 workspace=ws)
+
+    ms = _timed_calls(args, dev, world, one)
+    st, fl = attn_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word set in the backward leg: {fl:#x}")
+    flops = 2.5 * cfg.flops()
+    flops_per_s, avg = weak_scaling_value(flops, sum(ms) / len(ms), world)
+    achieved = flops / (avg * 1e-3) / 1e12
+    return {"workload": cfg.name, "value": flops_per_s / 1e12, "unit": "TFLOPS", "ms": avg,
+            "median_ms": statistics.median(ms), "calls": len(ms), "gpu_launches_per_call": 3,
+            "flops_counted": "2.5x forward (dV, dP, dQ, dK and the recomputed S)",
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "per_call_flops": flops, "executed_flops_per_call": 3.5 * cfg.flops()}}
 
 
 def paged_prefill_leg(args, dev, world, peaks):

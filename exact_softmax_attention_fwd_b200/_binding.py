@@ -49,6 +49,9 @@ SIGNATURES = {
                                _SZ, _P]),
     "attn_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P,
                                        _P, _P]),
+    "attn_bwd_workspace_size": (_SZ, [_I, _I, _I]),
+    "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P,
+                      _SZ, _P]),
     "attn_get_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
     "attn_strerror": (ctypes.c_char_p, [_I]),
     "attn_split_tokens": (_I, []),
@@ -199,6 +202,44 @@ def attn_fwd_block_sparse(q, k, v, block_mask, causal: bool, scale: float, k_len
                                               _stream(stream))
     _check(st, "attn_fwd_block_sparse")
     return out, lse
+
+
+def attn_bwd_workspace_size(B: int, Hq: int, Sq: int) -> int:
+    return int(load_library().attn_bwd_workspace_size(B, Hq, Sq))
+
+
+def attn_bwd(q, k, v, o, lse, d_o, causal: bool, scale: float, k_lens=None, dq=None, dk=None,
+             dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of attn_fwd_masked.  q, o, d_o [B,Hq,Sq,d], k/v [B,Hkv,Sk,d] bf16; lse
+    [B,Hq,Sq] fp32 as the forward returned it for the same causal / scale / k_lens."""
+    import torch
+    _require_cuda(q, k, v, o, lse, d_o, k_lens, dq, dk, dv, workspace)
+    for t in (q, k, v, o, d_o):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("q, k, v, o, d_o must be contiguous bfloat16")
+    B, Hq, Sq, d = q.shape
+    Bk, Hkv, Sk, dk_ = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or dk_ != d:
+        raise ValueError("q/k/v shapes disagree")
+    if tuple(o.shape) != tuple(q.shape) or tuple(d_o.shape) != tuple(q.shape):
+        raise ValueError("o and d_o must have q's shape")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, Sq) or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous float32 [B, Hq, Sq]")
+    if k_lens is not None and (k_lens.dtype != torch.int32 or tuple(k_lens.shape) != (B,)):
+        raise ValueError("k_lens must be int32 [B]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = attn_bwd_workspace_size(B, Hq, Sq)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = load_library().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(d_o),
+                                 _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, Sq, Sk, d,
+                                 int(bool(causal)), float(scale), _ptr(k_lens), _ptr(workspace),
+                                 ws_bytes, _stream(stream))
+    _check(st, "attn_bwd")
+    return dq, dk, dv
 
 
 def attn_fwd_varlen_workspace_size(B: int, total_q: int, max_seqlen_q: int) -> int:

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "attn.h"
+#include "bwd_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "prefill_sm100.cuh"
 #include "sm100_primitives.cuh"
@@ -191,12 +192,102 @@ int prefill_dense(const void* q, const void* k, const void* v, void* o, float* l
   return causal ? launch_prefill<64, true>(mq, mk, mv, mo, prm, stream)
                 : launch_prefill<64, false>(mq, mk, mv, mo, prm, stream);
 }
+// Backward: the row-statistics pass, then dK/dV (one CTA per key tile and KV
+// head) and dQ (one CTA per query tile and query head), in stream order.
+template <int D, bool CAUSAL>
+int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mdo, const CUtensorMap& mk,
+               const CUtensorMap& mv, const BwdParams& prm, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  const long long prep_threads = (long long)prm.B * prm.Hq * prm.Sq_pad * (D / 8);
+  const long long prep_blocks = (prep_threads + 255) / 256;
+  const long long kv_units = (long long)prm.n_kt * prm.B * prm.Hkv;
+  const long long q_units = (long long)prm.n_qt * prm.B * prm.Hq;
+  if (prep_blocks > INT_MAX || kv_units > INT_MAX || q_units > INT_MAX) return ATTN_ERR_INVALID_ARG;
+  attn_bwd_prep_kernel<D><<<(unsigned)prep_blocks, 256, 0, stream>>>(prm);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  auto kv = attn_bwd_dkdv_kernel<D, CAUSAL>;
+  if (cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, C::KV_SMEM) !=
+      cudaSuccess)
+    return ATTN_ERR_CUDA;
+  kv<<<(unsigned)kv_units, C::NUM_THREADS, C::KV_SMEM, stream>>>(mq, mdo, mk, mv, prm);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  auto dq = attn_bwd_dq_kernel<D, CAUSAL>;
+  if (cudaFuncSetAttribute(dq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::Q_SMEM) !=
+      cudaSuccess)
+    return ATTN_ERR_CUDA;
+  dq<<<(unsigned)q_units, C::NUM_THREADS, C::Q_SMEM, stream>>>(mq, mdo, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+size_t bwd_workspace_bytes(int B, int Hq, int Sq) {
+  const size_t pad = ((size_t)Sq + 127) / 128 * 128;
+  return 2 * (size_t)B * Hq * pad * sizeof(float);
+}
 }  // namespace
 }  // namespace attn_b200
 
 using namespace attn_b200;
 
 extern "C" {
+
+size_t attn_bwd_workspace_size(int B, int Hq, int Sq) {
+  if (B < 1 || Hq < 1 || Sq < 1) return 0;
+  return bwd_workspace_bytes(B, Hq, Sq);
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* d_o, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk,
+             int d, int causal, float scale, const int32_t* k_lens, void* workspace,
+             size_t workspace_bytes, attn_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (o == nullptr || lse == nullptr || d_o == nullptr || dq == nullptr || workspace == nullptr ||
+      (Sk > 0 && (dk == nullptr || dv == nullptr)))
+    return ATTN_ERR_INVALID_ARG;
+  int st = check_prefill_args(q, k, v, dq, nullptr, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens);
+  if (st != ATTN_OK) return st;
+  if (!aligned16(o) || !aligned16(d_o) || !aligned16(workspace) || !aligned4(lse) ||
+      (Sk > 0 && (!aligned16(dk) || !aligned16(dv))))
+    return ATTN_ERR_ALIGNMENT;
+  if (workspace_bytes < bwd_workspace_bytes(B, Hq, Sq)) return ATTN_ERR_WORKSPACE;
+  if (Sk == 0) {  // no key: every output row is constant zero, so dQ = 0 (dK, dV are empty)
+    const size_t bytes = (size_t)B * Hq * Sq * d * 2;
+    return cudaMemsetAsync(dq, 0, bytes, stream) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+  CUtensorMap mq, mdo, mk, mv;
+  if (!make_tile_map(&mq, q, d, Sq, (long long)B * Hq) ||
+      !make_tile_map(&mdo, d_o, d, Sq, (long long)B * Hq) ||
+      !make_tile_map(&mk, k, d, Sk, (long long)B * Hkv) ||
+      !make_tile_map(&mv, v, d, Sk, (long long)B * Hkv))
+    return ATTN_ERR_CUDA;
+  BwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.o = static_cast<const uint16_t*>(o);
+  prm.d_o = static_cast<const uint16_t*>(d_o);
+  prm.lse = lse;
+  prm.Sq_pad = (Sq + 127) / 128 * 128;
+  prm.nlse2 = static_cast<float*>(workspace);
+  prm.dsum = prm.nlse2 + (size_t)B * Hq * prm.Sq_pad;
+  prm.k_lens = k_lens;
+  prm.dq = static_cast<uint16_t*>(dq);
+  prm.dk = static_cast<uint16_t*>(dk);
+  prm.dv = static_cast<uint16_t*>(dv);
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.Sq = Sq;
+  prm.Sk = Sk;
+  prm.group = Hq / Hkv;
+  prm.n_qt = prm.Sq_pad / 128;
+  prm.n_kt = (Sk + 127) / 128;
+  prm.scale = scale;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  if (d == 128)
+    return causal ? launch_bwd<128, true>(mq, mdo, mk, mv, prm, stream)
+                  : launch_bwd<128, false>(mq, mdo, mk, mv, prm, stream);
+  return causal ? launch_bwd<64, true>(mq, mdo, mk, mv, prm, stream)
+                : launch_bwd<64, false>(mq, mdo, mk, mv, prm, stream);
+}
+
 
 const char* attn_strerror(int status) {
   switch (status) {

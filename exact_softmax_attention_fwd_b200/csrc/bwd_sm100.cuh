@@ -1,0 +1,719 @@
+// bwd_sm100.cuh -- exact softmax attention backward for sm_100a.
+//
+// What it computes ("Attention Kernel", section "Backward 与重计算"): the
+// forward keeps no probability matrix, so the backward recomputes the local
+// probabilities from Q, K, the output O and the saved log-sum-exp, with the
+// forward's scale, mask and GQA head mapping:
+//     P  = exp(scale * Q K^T + M - LSE)          (row by row)
+//     dV = P^T dO          dP = dO V^T           D = rowsum(dO * O)
+//     dS = P * (dP - D)    dQ = scale * dS K     dK = scale * dS^T Q
+// ("Attention 算子加速史", FAQ Q1: recomputation trades FLOPs for HBM traffic.)
+// D = rowsum(dO * O) equals rowsum(P * dP) because O = P V.
+//
+// Three kernels, each output written by exactly one CTA, so results are
+// deterministic and no atomics are used (the contract in "Backward 与重计算"
+// asks that accumulation and writes be free of races):
+//   * attn_bwd_prep_kernel: per query row, D and -LSE*log2(e) into a workspace
+//     padded to whole 128-row tiles (padding rows get -inf and 0, so they
+//     recompute P = 0 without a predicate).
+//   * attn_bwd_dkdv_kernel: one CTA per (key tile, batch, KV head).  K and V
+//     stay in shared memory; Q, dO and their row statistics stream through a
+//     ring for every query head of the group and every query tile that sees
+//     the key tile.  Per query tile, four tcgen05 MMAs with the key tile as M:
+//       S^T = K Q^T, dP^T = V dO^T     (SS: both operands in shared memory)
+//       dV += P^T dO, dK += dS^T Q     (TS: P^T / dS^T read from tensor memory)
+//     so the transposed products land with keys on the TMEM lanes and need no
+//     transpose.  dV and dK accumulate in tensor memory across the whole loop.
+//   * attn_bwd_dq_kernel: one CTA per (query tile, batch, query head), K/V
+//     tiles streaming: S = Q K^T, dP = dO V^T (SS), dQ += dS K (TS).
+// Both compute kernels use the forward's organisation: warp 0 lane 0 issues
+// TMA copies (no multicast), warp 1 lane 0 issues the MMAs, and two
+// warpgroups (warps 4-7, 8-11) each own 64 of the 128 columns of every score
+// tile (thread r owns TMEM lane r).  A warpgroup packs its bf16 P or dS into
+// the first 32 columns of its own 64-column range, so the two warpgroups never
+// write a column the other still has to read; the TS MMAs read the operand
+// from those two 32-column runs.
+#pragma once
+
+#include "sm100_primitives.cuh"
+
+namespace attn_b200 {
+
+// 1-D bulk copy global -> shared (cp.async.bulk, no tensor map); completion is
+// counted in bytes on the mbarrier.  Both addresses 16-byte aligned, size a
+// multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+struct BwdParams {
+  const uint16_t* o;    // [B, Hq, Sq, d] forward output (bf16)
+  const uint16_t* d_o;  // [B, Hq, Sq, d] gradient of the output (bf16)
+  const float* lse;     // [B, Hq, Sq] forward log-sum-exp (natural log)
+  float* nlse2;         // [B*Hq, Sq_pad] workspace: -LSE*log2(e); -inf for empty and padding rows
+  float* dsum;          // [B*Hq, Sq_pad] workspace: rowsum(dO * O); 0 for padding rows
+  const int* k_lens;    // [B] or nullptr
+  uint16_t* dq;         // [B, Hq, Sq, d]
+  uint16_t* dk;         // [B, Hkv, Sk, d]
+  uint16_t* dv;         // [B, Hkv, Sk, d]
+  int B, Hq, Hkv, Sq, Sk, group, Sq_pad, n_qt, n_kt;
+  float scale, scale_log2;
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int TILE_BYTES = 128 * D * 2;  // a 128-row bf16 tile (Q, dO, K or V)
+  static constexpr int CB_BYTES = 128 * 128;      // one 64-column block of a tile
+  static constexpr int NCB = D / 64;
+  static constexpr int STAGES = (D == 64) ? 4 : 2;
+  static constexpr int STAT_BYTES = 1024;  // -LSE*log2(e) [128] then D [128] of a query tile
+  // ---- dK/dV kernel: K, V resident; Q, dO and statistics in a ring
+  static constexpr int KV_OFF_K = 0;
+  static constexpr int KV_OFF_V = TILE_BYTES;
+  static constexpr int KV_OFF_Q = 2 * TILE_BYTES;
+  static constexpr int KV_OFF_DO = KV_OFF_Q + STAGES * TILE_BYTES;
+  static constexpr int KV_OFF_ST = KV_OFF_DO + STAGES * TILE_BYTES;
+  static constexpr int KV_OFF_BAR = KV_OFF_ST + STAGES * STAT_BYTES;
+  static constexpr int KB_KV = 0;                  // K and V landed
+  static constexpr int KB_QF = 1;                  // STAGES: Q, dO, statistics landed
+  static constexpr int KB_QE = KB_QF + STAGES;     // STAGES: stage free (MMA + 256 threads)
+  static constexpr int KB_SF = KB_QE + STAGES;     // S^T in TMEM
+  static constexpr int KB_DPF = KB_SF + 1;         // dP^T in TMEM
+  static constexpr int KB_PF = KB_DPF + 1;         // P^T written (256 threads)
+  static constexpr int KB_DSF = KB_PF + 1;         // dS^T written (256 threads)
+  static constexpr int KB_ACC = KB_DSF + 1;        // every MMA retired
+  static constexpr int KB_NUM = KB_ACC + 1;
+  static constexpr int KV_OFF_MISC = KV_OFF_BAR + KB_NUM * 8;
+  static constexpr int KV_SMEM = KV_OFF_MISC + 16 + 1024;
+  // ---- dQ kernel: Q, dO resident; K, V in a ring
+  static constexpr int Q_OFF_Q = 0;
+  static constexpr int Q_OFF_DO = TILE_BYTES;
+  static constexpr int Q_OFF_K = 2 * TILE_BYTES;
+  static constexpr int Q_OFF_V = Q_OFF_K + STAGES * TILE_BYTES;
+  static constexpr int Q_OFF_BAR = Q_OFF_V + STAGES * TILE_BYTES;
+  static constexpr int QB_QF = 0;                  // Q and dO landed
+  static constexpr int QB_KVF = 1;                 // STAGES: K and V landed
+  static constexpr int QB_KVE = QB_KVF + STAGES;   // STAGES: stage free
+  static constexpr int QB_SF = QB_KVE + STAGES;    // 2: S in TMEM buffer 0 / 1
+  static constexpr int QB_DPF = QB_SF + 2;         // dP in TMEM
+  static constexpr int QB_DSF = QB_DPF + 1;        // dS written (256 threads)
+  static constexpr int QB_ACC = QB_DSF + 1;
+  static constexpr int QB_NUM = QB_ACC + 1;
+  static constexpr int Q_OFF_MISC = Q_OFF_BAR + QB_NUM * 8;
+  static constexpr int Q_SMEM = Q_OFF_MISC + 16 + 1024;
+  // ---- tensor memory (512 columns)
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t KV_TM_S = 0;        // S^T, then P^T (bf16) in its warpgroup runs
+  static constexpr uint32_t KV_TM_DP = 128;     // dP^T, then dS^T (bf16)
+  static constexpr uint32_t KV_TM_DV = 256;
+  static constexpr uint32_t KV_TM_DK = 256 + D;
+  static constexpr uint32_t Q_TM_S0 = 0, Q_TM_S1 = 128;
+  static constexpr uint32_t Q_TM_DP = 256;      // dP, then dS (bf16)
+  static constexpr uint32_t Q_TM_DQ = 384;
+  static constexpr int NUM_THREADS = 384;
+  static constexpr uint32_t REGS_PRODUCER = 72;
+  static constexpr uint32_t REGS_SOFTMAX = 208;
+  static_assert(128 * (REGS_PRODUCER + 2 * REGS_SOFTMAX) <= NUM_THREADS * 168,
+                "register reallocation must fit the launch allocation");
+  static_assert(KV_SMEM <= 232448 && Q_SMEM <= 232448, "shared memory");
+  static_assert(D == 64 || D == 128, "head dim");
+};
+
+// -inf for a masked element, x otherwise.
+__device__ __forceinline__ float bwd_keep(bool visible, float x) {
+  return visible ? x : -INFINITY;
+}
+
+// D = rowsum(dO * O) and -LSE*log2(e) for every padded query row.  D/8
+// threads per row, 8 elements each, reduced by shuffles.
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const BwdParams p) {
+  constexpr int TPR = D / 8;
+  const long long n_rows = (long long)p.B * p.Hq * p.Sq_pad;
+  const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long row = gt / TPR;
+  const int part = (int)(gt % TPR);
+  const bool valid = row < n_rows;
+  const long long bh = valid ? row / p.Sq_pad : 0;
+  const int i = valid ? (int)(row % p.Sq_pad) : 0;
+  const bool live = valid && i < p.Sq;
+  float acc = 0.f;
+  if (live) {
+    const size_t off = ((size_t)bh * p.Sq + i) * D + part * 8;
+    const uint4 a = ld_stream_v4(p.d_o + off);
+    const uint4 b = ld_stream_v4(p.o + off);
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+    const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc = fmaf(__uint_as_float(aw[e] << 16), __uint_as_float(bw[e] << 16), acc);
+      acc = fmaf(__uint_as_float(aw[e] & 0xFFFF0000u), __uint_as_float(bw[e] & 0xFFFF0000u), acc);
+    }
+  }
+#pragma unroll
+  for (int w = TPR / 2; w >= 1; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
+  if (valid && part == 0) {
+    float nl = -INFINITY;
+    if (live) {
+      const float l = p.lse[(size_t)bh * p.Sq + i];
+      nl = (l == -INFINITY) ? -INFINITY : -l * 1.4426950408889634f;
+    }
+    p.nlse2[row] = nl;
+    p.dsum[row] = live ? acc : 0.f;
+  }
+}
+
+// The valid key count of batch b (clamped and flagged when out of range).
+__device__ __forceinline__ int bwd_klen(const BwdParams& p, int b, bool report) {
+  if (p.k_lens == nullptr) return p.Sk;
+  int kl = __ldg(p.k_lens + b);
+  if (kl < 0 || kl > p.Sk) {
+    if (report) flag_device_error(kDevErrBadLength);
+    kl = kl < 0 ? 0 : p.Sk;
+  }
+  return kl;
+}
+
+// SS MMA over the head dimension: D[tm] = A B^T, A and B 128-row K-major tiles.
+template <int D>
+__device__ __forceinline__ void bwd_mma_ss(uint32_t d_tmem, uint32_t a, uint32_t b) {
+  using C = BwdCfg<D>;
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    const uint32_t off = (ks >> 2) * C::CB_BYTES + (ks & 3) * 32;
+    umma_ss(d_tmem, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b + off, 16, 1024), idesc,
+            ks > 0 ? 1u : 0u);
+  }
+}
+
+// TS MMA over 128 rows: D[tm] (+)= A B with A [128 x 128] bf16 in TMEM (its
+// columns 0-31 and 64-95: the two warpgroups' packed runs) and B a 128-row tile
+// used MN-major (its rows are the reduction index).
+template <int D>
+__device__ __forceinline__ void bwd_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b,
+                                           bool accumulate) {
+  using C = BwdCfg<D>;
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, true);
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    umma_ts(d_tmem, a_tmem + (ks >> 2) * 64 + (ks & 3) * 8,
+            smem_desc_sw128(b + ks * 2048, C::CB_BYTES, 1024), idesc,
+            (accumulate || ks > 0) ? 1u : 0u);
+  }
+}
+
+// Writes 32 fp32 values (times mul) as bf16 to a global row segment (16-byte stores).
+__device__ __forceinline__ void bwd_store32(uint16_t* dst, const uint32_t (&v)[32], float mul) {
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    uint4 w;
+    w.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * mul, __uint_as_float(v[8 * q4 + 1]) * mul);
+    w.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * mul, __uint_as_float(v[8 * q4 + 3]) * mul);
+    w.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * mul, __uint_as_float(v[8 * q4 + 5]) * mul);
+    w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * mul, __uint_as_float(v[8 * q4 + 7]) * mul);
+    reinterpret_cast<uint4*>(dst)[q4] = w;
+  }
+}
+
+// ===========================================================================
+// dK, dV: one CTA per (key tile kb, batch b, KV head).  Units are numbered key
+// tile major, so under a causal mask the heaviest key tiles (the first ones,
+// seen by the most query tiles) start first.
+// ===========================================================================
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                         const __grid_constant__ CUtensorMap tm_do,
+                         const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t* sbase_ptr = smem_raw + (sbase - raw_addr);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase_ptr + C::KV_OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase_ptr + C::KV_OFF_MISC + 4);
+  auto bar = [&](int i) -> uint32_t { return sbase + C::KV_OFF_BAR + 8u * (uint32_t)i; };
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- the unit and its query-tile range
+  const int bh_kv = blockIdx.x % (p.B * p.Hkv);
+  const int kb = blockIdx.x / (p.B * p.Hkv);
+  const int b = bh_kv / p.Hkv, kvh = bh_kv % p.Hkv;
+  const int klen = bwd_klen(p, b, threadIdx.x == 0);
+  const long long koff = (long long)klen - p.Sq;  // key j is visible to row i iff j <= i + koff
+  const int key0 = kb * 128;
+  int qt_lo = 0;
+  if (CAUSAL) {
+    const long long first_row = (long long)key0 - koff;  // the first row that sees key0
+    qt_lo = first_row <= 0 ? 0 : (int)min(first_row / 128, (long long)p.n_qt);
+  }
+  const int nq = (key0 >= klen) ? 0 : p.n_qt - qt_lo;
+  const int N = p.group * nq;  // (query head, query tile) iterations
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::KB_KV), 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(bar(C::KB_QF + s), 1);
+      mbar_init(bar(C::KB_QE + s), 1 + 256);
+    }
+    mbar_init(bar(C::KB_SF), 1);
+    mbar_init(bar(C::KB_DPF), 1);
+    mbar_init(bar(C::KB_PF), 256);
+    mbar_init(bar(C::KB_DSF), 256);
+    mbar_init(bar(C::KB_ACC), 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sK = sbase + C::KV_OFF_K, sV = sbase + C::KV_OFF_V;
+  auto sQ = [&](int s) { return sbase + C::KV_OFF_Q + (uint32_t)s * C::TILE_BYTES; };
+  auto sDO = [&](int s) { return sbase + C::KV_OFF_DO + (uint32_t)s * C::TILE_BYTES; };
+  auto sST = [&](int s) { return sbase + C::KV_OFF_ST + (uint32_t)s * C::STAT_BYTES; };
+
+  if (warp < 4) {
+    warpgroup_reg_dealloc<C::REGS_PRODUCER>();
+    if (warp == 0 && lane == 0 && N > 0) {
+      // ======================= TMA producer =======================
+      tma_prefetch_map(&tm_q);
+      tma_prefetch_map(&tm_do);
+      tma_prefetch_map(&tm_k);
+      tma_prefetch_map(&tm_v);
+      mbar_arrive_expect_tx(bar(C::KB_KV), 2 * C::TILE_BYTES);
+      for (int cb = 0; cb < C::NCB; ++cb) {
+        tma_load_3d(sK + cb * C::CB_BYTES, &tm_k, bar(C::KB_KV), 64 * cb, key0, bh_kv);
+        tma_load_3d(sV + cb * C::CB_BYTES, &tm_v, bar(C::KB_KV), 64 * cb, key0, bh_kv);
+      }
+      int issued = 0;
+      bool ok = true;
+      for (int n = 0; n < N; ++n) {
+        const int s = n % C::STAGES;
+        if (n >= C::STAGES &&
+            !(ok = mbar_wait(bar(C::KB_QE + s), ((n / C::STAGES) - 1) & 1u, abort_flag)))
+          break;
+        const int hq = kvh * p.group + n / nq;
+        const int qt = qt_lo + n % nq;
+        const int bh_q = b * p.Hq + hq;
+        mbar_arrive_expect_tx(bar(C::KB_QF + s), 2 * C::TILE_BYTES + C::STAT_BYTES);
+        for (int cb = 0; cb < C::NCB; ++cb) {
+          tma_load_3d(sQ(s) + cb * C::CB_BYTES, &tm_q, bar(C::KB_QF + s), 64 * cb, qt * 128, bh_q);
+          tma_load_3d(sDO(s) + cb * C::CB_BYTES, &tm_do, bar(C::KB_QF + s), 64 * cb, qt * 128,
+                      bh_q);
+        }
+        const size_t srow = (size_t)bh_q * p.Sq_pad + (size_t)qt * 128;
+        bulk_load(sST(s), p.nlse2 + srow, 512, bar(C::KB_QF + s));
+        bulk_load(sST(s) + 512, p.dsum + srow, 512, bar(C::KB_QF + s));
+        ++issued;
+      }
+      // Drain: no copy may still be landing when the CTA exits.
+      mbar_wait(bar(C::KB_KV), 0, nullptr);
+      for (int n = (issued > C::STAGES ? issued - C::STAGES : 0); n < issued; ++n)
+        mbar_wait(bar(C::KB_QF + n % C::STAGES), (n / C::STAGES) & 1u, nullptr);
+    } else if (warp == 1 && lane == 0 && N > 0) {
+      // ======================= tcgen05 MMA issuer =======================
+      const uint32_t tS = tmem + C::KV_TM_S, tDP = tmem + C::KV_TM_DP;
+      const uint32_t tDV = tmem + C::KV_TM_DV, tDK = tmem + C::KV_TM_DK;
+      bool ok = mbar_wait(bar(C::KB_KV), 0, abort_flag) && mbar_wait(bar(C::KB_QF), 0, abort_flag);
+      if (ok) {
+        tc_fence_after_sync();
+        bwd_mma_ss<D>(tS, sK, sQ(0));
+        umma_commit(bar(C::KB_SF));
+        bwd_mma_ss<D>(tDP, sV, sDO(0));
+        umma_commit(bar(C::KB_DPF));
+      }
+      for (int n = 0; ok && n < N; ++n) {
+        const int s = n % C::STAGES, s1 = (n + 1) % C::STAGES;
+        if (!(ok = mbar_wait(bar(C::KB_PF), n & 1u, abort_flag))) break;
+        tc_fence_after_sync();
+        bwd_mma_ts<D>(tDV, tS, sDO(s), n > 0);  // dV += P^T dO
+        if (n + 1 < N) {
+          // S^T of the next query tile: overwrites P^T only after the MMA above
+          // read it (MMAs of one thread run in issue order)
+          if (!(ok = mbar_wait(bar(C::KB_QF + s1), ((n + 1) / C::STAGES) & 1u, abort_flag))) break;
+          tc_fence_after_sync();
+          bwd_mma_ss<D>(tS, sK, sQ(s1));
+          umma_commit(bar(C::KB_SF));
+        }
+        if (!(ok = mbar_wait(bar(C::KB_DSF), n & 1u, abort_flag))) break;
+        tc_fence_after_sync();
+        bwd_mma_ts<D>(tDK, tDP, sQ(s), n > 0);  // dK += dS^T Q
+        umma_commit(bar(C::KB_QE + s));          // Q and dO of stage s read for the last time
+        if (n + 1 < N) {
+          bwd_mma_ss<D>(tDP, sV, sDO(s1));
+          umma_commit(bar(C::KB_DPF));
+        }
+      }
+      // every MMA retires before the epilogue reads TMEM and before TMEM is freed
+      umma_commit(bar(C::KB_ACC));
+      mbar_wait(bar(C::KB_ACC), 0, nullptr);
+    }
+    __syncwarp();
+  } else {
+    warpgroup_reg_alloc<C::REGS_SOFTMAX>();
+    // ======================= recompute warpgroups =======================
+    const int wg = (warp - 4) >> 2;      // query columns [64*wg, 64*wg + 64) of each tile
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;   // key row within the tile (TMEM lane)
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const int c0 = 64 * wg;
+    const uint32_t t_s = tmem + lane_off + C::KV_TM_S + c0;
+    const uint32_t t_dp = tmem + lane_off + C::KV_TM_DP + c0;
+    const int j = key0 + r;
+    const float c2 = p.scale_log2;
+    const uint64_t c2x2 = f32x2(c2, c2);
+    bool ok = true;
+    for (int n = 0; ok && n < N; ++n) {
+      const int s = n % C::STAGES;
+      const int qt = qt_lo + n % nq;
+      // columns c >= cmin are visible to this key (c relative to this warpgroup's run)
+      long long cm = (j >= klen) ? 64 : (CAUSAL ? (long long)j - koff - qt * 128 - c0 : 0);
+      const int cmin = (int)(cm < 0 ? 0 : (cm > 64 ? 64 : cm));
+      const bool edge = __any_sync(0xffffffffu, cmin > 0);
+      if (!(ok = mbar_wait_warp(bar(C::KB_SF), n & 1u, abort_flag))) break;
+      // the statistics arrived with Q (every thread observes the copy itself)
+      const bool st_ok = mbar_wait(bar(C::KB_QF + s), (n / C::STAGES) & 1u, abort_flag);
+      if (!(ok = __all_sync(0xffffffffu, st_ok))) break;
+      tc_fence_after_sync();
+      const float4* st = reinterpret_cast<const float4*>(sbase_ptr + C::KV_OFF_ST +
+                                                         s * C::STAT_BYTES);
+      float pr[64];
+      {
+        uint32_t a[32], bq[32];
+        tmem_ld32(t_s, a);
+        tmem_ld32(t_s + 32, bq);
+        tmem_ld_wait();
+        reg_fence32(a);
+        reg_fence32(bq);
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {  // columns 4e .. 4e+3
+          const float4 nl = st[(c0 >> 2) + e];
+          const int c = 4 * e;
+          const uint32_t s0 = c < 32 ? a[c] : bq[c - 32];
+          const uint32_t s1 = c < 32 ? a[c + 1] : bq[c - 31];
+          const uint32_t s2 = c < 32 ? a[c + 2] : bq[c - 30];
+          const uint32_t s3 = c < 32 ? a[c + 3] : bq[c - 29];
+          float x0, x1, x2, x3;
+          split_f32x2(fma_f32x2(f32x2(__uint_as_float(s0), __uint_as_float(s1)), c2x2,
+                                f32x2(nl.x, nl.y)), x0, x1);
+          split_f32x2(fma_f32x2(f32x2(__uint_as_float(s2), __uint_as_float(s3)), c2x2,
+                                f32x2(nl.z, nl.w)), x2, x3);
+          if (edge) {
+            x0 = bwd_keep(c >= cmin, x0);
+            x1 = bwd_keep(c + 1 >= cmin, x1);
+            x2 = bwd_keep(c + 2 >= cmin, x2);
+            x3 = bwd_keep(c + 3 >= cmin, x3);
+          }
+          pr[c] = ex2(x0);
+          pr[c + 1] = ex2(x1);
+          pr[c + 2] = ex2(x2);
+          pr[c + 3] = ex2(x3);
+          pk[2 * e] = pack_bf16x2(pr[c], pr[c + 1]);
+          pk[2 * e + 1] = pack_bf16x2(pr[c + 2], pr[c + 3]);
+        }
+        tmem_st32(t_s, pk);  // P^T into the first 32 columns of this warpgroup's run
+        tmem_st_wait();
+        tc_fence_before_sync();
+        mbar_arrive(bar(C::KB_PF));
+      }
+      if (!(ok = mbar_wait_warp(bar(C::KB_DPF), n & 1u, abort_flag))) break;
+      tc_fence_after_sync();
+      {
+        uint32_t a[32], bq[32];
+        tmem_ld32(t_dp, a);
+        tmem_ld32(t_dp + 32, bq);
+        tmem_ld_wait();
+        reg_fence32(a);
+        reg_fence32(bq);
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float4 dd = st[32 + (c0 >> 2) + e];  // D of columns 4e .. 4e+3
+          const int c = 4 * e;
+          const float d0 = __uint_as_float(c < 32 ? a[c] : bq[c - 32]) - dd.x;
+          const float d1 = __uint_as_float(c < 32 ? a[c + 1] : bq[c - 31]) - dd.y;
+          const float d2 = __uint_as_float(c < 32 ? a[c + 2] : bq[c - 30]) - dd.z;
+          const float d3 = __uint_as_float(c < 32 ? a[c + 3] : bq[c - 29]) - dd.w;
+          pk[2 * e] = pack_bf16x2(pr[c] * d0, pr[c + 1] * d1);
+          pk[2 * e + 1] = pack_bf16x2(pr[c + 2] * d2, pr[c + 3] * d3);
+        }
+        tmem_st32(t_dp, pk);  // dS^T into the first 32 columns of this warpgroup's run
+        tmem_st_wait();
+        tc_fence_before_sync();
+        mbar_arrive(bar(C::KB_DSF));
+      }
+      mbar_arrive(bar(C::KB_QE + s));  // this thread is done with stage s's statistics
+    }
+    // ---- epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (times scale)
+    bool have = N > 0;
+    if (have && ok) {
+      ok = mbar_wait_warp(bar(C::KB_ACC), 0, abort_flag);
+      tc_fence_after_sync();
+    }
+    if (!have || ok) {
+      const uint32_t t_acc = tmem + lane_off + (wg ? C::KV_TM_DK : C::KV_TM_DV);
+      uint16_t* out = (wg ? p.dk : p.dv) + ((size_t)bh_kv * p.Sk + (j < p.Sk ? j : 0)) * D;
+      const float mul = wg ? p.scale : 1.f;
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t v[32];
+        if (have) {
+          tmem_ld32_sync(t_acc + c, v);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
+        if (j < p.Sk) bwd_store32(out + c, v, mul);
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// ===========================================================================
+// dQ: one CTA per (query tile, batch, query head).  Units are numbered query
+// tile major from the last tile down, so under a causal mask the heaviest
+// tiles start first.
+// ===========================================================================
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_do,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t* sbase_ptr = smem_raw + (sbase - raw_addr);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase_ptr + C::Q_OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase_ptr + C::Q_OFF_MISC + 4);
+  auto bar = [&](int i) -> uint32_t { return sbase + C::Q_OFF_BAR + 8u * (uint32_t)i; };
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int bh_q = blockIdx.x % (p.B * p.Hq);
+  const int qt = p.n_qt - 1 - (int)(blockIdx.x / (p.B * p.Hq));
+  const int b = bh_q / p.Hq, hq = bh_q % p.Hq;
+  const int bh_kv = b * p.Hkv + hq / p.group;
+  const int klen = bwd_klen(p, b, threadIdx.x == 0);
+  const long long koff = (long long)klen - p.Sq;
+  const int row0 = qt * 128;
+  const int last_row = min(row0 + 127, p.Sq - 1);
+  long long max_key = (long long)klen - 1;  // the last key any row of the tile sees
+  if (CAUSAL) max_key = min(max_key, (long long)last_row + koff);
+  const int N = max_key < 0 ? 0 : (int)(max_key / 128) + 1;  // key tiles [0, N)
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::QB_QF), 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(bar(C::QB_KVF + s), 1);
+      mbar_init(bar(C::QB_KVE + s), 1);
+    }
+    mbar_init(bar(C::QB_SF), 1);
+    mbar_init(bar(C::QB_SF + 1), 1);
+    mbar_init(bar(C::QB_DPF), 1);
+    mbar_init(bar(C::QB_DSF), 256);
+    mbar_init(bar(C::QB_ACC), 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sQ = sbase + C::Q_OFF_Q, sDO = sbase + C::Q_OFF_DO;
+  auto sK = [&](int s) { return sbase + C::Q_OFF_K + (uint32_t)s * C::TILE_BYTES; };
+  auto sV = [&](int s) { return sbase + C::Q_OFF_V + (uint32_t)s * C::TILE_BYTES; };
+
+  if (warp < 4) {
+    warpgroup_reg_dealloc<C::REGS_PRODUCER>();
+    if (warp == 0 && lane == 0 && N > 0) {
+      // ======================= TMA producer =======================
+      tma_prefetch_map(&tm_q);
+      tma_prefetch_map(&tm_do);
+      tma_prefetch_map(&tm_k);
+      tma_prefetch_map(&tm_v);
+      mbar_arrive_expect_tx(bar(C::QB_QF), 2 * C::TILE_BYTES);
+      for (int cb = 0; cb < C::NCB; ++cb) {
+        tma_load_3d(sQ + cb * C::CB_BYTES, &tm_q, bar(C::QB_QF), 64 * cb, row0, bh_q);
+        tma_load_3d(sDO + cb * C::CB_BYTES, &tm_do, bar(C::QB_QF), 64 * cb, row0, bh_q);
+      }
+      int issued = 0;
+      bool ok = true;
+      for (int n = 0; n < N; ++n) {
+        const int s = n % C::STAGES;
+        if (n >= C::STAGES &&
+            !(ok = mbar_wait(bar(C::QB_KVE + s), ((n / C::STAGES) - 1) & 1u, abort_flag)))
+          break;
+        mbar_arrive_expect_tx(bar(C::QB_KVF + s), 2 * C::TILE_BYTES);
+        for (int cb = 0; cb < C::NCB; ++cb) {
+          tma_load_3d(sK(s) + cb * C::CB_BYTES, &tm_k, bar(C::QB_KVF + s), 64 * cb, n * 128, bh_kv);
+          tma_load_3d(sV(s) + cb * C::CB_BYTES, &tm_v, bar(C::QB_KVF + s), 64 * cb, n * 128, bh_kv);
+        }
+        ++issued;
+      }
+      mbar_wait(bar(C::QB_QF), 0, nullptr);
+      for (int n = (issued > C::STAGES ? issued - C::STAGES : 0); n < issued; ++n)
+        mbar_wait(bar(C::QB_KVF + n % C::STAGES), (n / C::STAGES) & 1u, nullptr);
+    } else if (warp == 1 && lane == 0 && N > 0) {
+      // ======================= tcgen05 MMA issuer =======================
+      const uint32_t tDP = tmem + C::Q_TM_DP, tDQ = tmem + C::Q_TM_DQ;
+      auto tS = [&](int n) { return tmem + ((n & 1) ? C::Q_TM_S1 : C::Q_TM_S0); };
+      bool ok = mbar_wait(bar(C::QB_QF), 0, abort_flag) && mbar_wait(bar(C::QB_KVF), 0, abort_flag);
+      if (ok) {
+        tc_fence_after_sync();
+        bwd_mma_ss<D>(tS(0), sQ, sK(0));
+        umma_commit(bar(C::QB_SF));
+        bwd_mma_ss<D>(tDP, sDO, sV(0));
+        umma_commit(bar(C::QB_DPF));
+      }
+      for (int n = 0; ok && n < N; ++n) {
+        const int s = n % C::STAGES, s1 = (n + 1) % C::STAGES;
+        if (n + 1 < N) {
+          if (!(ok = mbar_wait(bar(C::QB_KVF + s1), ((n + 1) / C::STAGES) & 1u, abort_flag))) break;
+          tc_fence_after_sync();
+          bwd_mma_ss<D>(tS(n + 1), sQ, sK(s1));
+          umma_commit(bar(C::QB_SF + ((n + 1) & 1)));
+        }
+        if (!(ok = mbar_wait(bar(C::QB_DSF), n & 1u, abort_flag))) break;
+        tc_fence_after_sync();
+        bwd_mma_ts<D>(tDQ, tDP, sK(s), n > 0);  // dQ += dS K
+        umma_commit(bar(C::QB_KVE + s));
+        if (n + 1 < N) {
+          // dP of the next key tile: overwrites dS only after the MMA above read it
+          bwd_mma_ss<D>(tDP, sDO, sV(s1));
+          umma_commit(bar(C::QB_DPF));
+        }
+      }
+      umma_commit(bar(C::QB_ACC));
+      mbar_wait(bar(C::QB_ACC), 0, nullptr);
+    }
+    __syncwarp();
+  } else {
+    warpgroup_reg_alloc<C::REGS_SOFTMAX>();
+    // ======================= recompute warpgroups =======================
+    const int wg = (warp - 4) >> 2;      // key columns [64*wg, 64*wg + 64) of each tile
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;   // query row within the tile (TMEM lane)
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const int c0 = 64 * wg;
+    const uint32_t t_dp = tmem + lane_off + C::Q_TM_DP + c0;
+    const int row = row0 + r;
+    const size_t srow = (size_t)bh_q * p.Sq_pad + row;
+    const float nl = p.nlse2[srow];
+    const float dd = p.dsum[srow];
+    const uint64_t c2x2 = f32x2(p.scale_log2, p.scale_log2);
+    const uint64_t nlx2 = f32x2(nl, nl);
+    // keys j < kend are visible to this row
+    long long kend = klen;
+    if (CAUSAL) kend = min(kend, (long long)row + koff + 1);
+    bool ok = true;
+    for (int n = 0; ok && n < N; ++n) {
+      const long long cm = kend - (long long)n * 128 - c0;  // visible iff c < cmax
+      const int cmax = (int)(cm < 0 ? 0 : (cm > 64 ? 64 : cm));
+      const bool edge = __any_sync(0xffffffffu, cmax < 64);
+      if (!(ok = mbar_wait_warp(bar(C::QB_SF + (n & 1)), (n >> 1) & 1u, abort_flag))) break;
+      tc_fence_after_sync();
+      const uint32_t t_s = tmem + lane_off + ((n & 1) ? C::Q_TM_S1 : C::Q_TM_S0) + c0;
+      float pr[64];
+      {
+        uint32_t a[32], bq[32];
+        tmem_ld32(t_s, a);
+        tmem_ld32(t_s + 32, bq);
+        tmem_ld_wait();
+        reg_fence32(a);
+        reg_fence32(bq);
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const uint32_t s0 = c < 32 ? a[c] : bq[c - 32];
+          const uint32_t s1 = c < 32 ? a[c + 1] : bq[c - 31];
+          float x0, x1;
+          split_f32x2(fma_f32x2(f32x2(__uint_as_float(s0), __uint_as_float(s1)), c2x2, nlx2), x0,
+                      x1);
+          if (edge) {
+            x0 = bwd_keep(c < cmax, x0);
+            x1 = bwd_keep(c + 1 < cmax, x1);
+          }
+          pr[c] = ex2(x0);
+          pr[c + 1] = ex2(x1);
+        }
+      }
+      if (!(ok = mbar_wait_warp(bar(C::QB_DPF), n & 1u, abort_flag))) break;
+      tc_fence_after_sync();
+      {
+        uint32_t a[32], bq[32];
+        tmem_ld32(t_dp, a);
+        tmem_ld32(t_dp + 32, bq);
+        tmem_ld_wait();
+        reg_fence32(a);
+        reg_fence32(bq);
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = 2 * e;
+          const float d0 = __uint_as_float(c < 32 ? a[c] : bq[c - 32]) - dd;
+          const float d1 = __uint_as_float(c < 32 ? a[c + 1] : bq[c - 31]) - dd;
+          pk[e] = pack_bf16x2(pr[c] * d0, pr[c + 1] * d1);
+        }
+        tmem_st32(t_dp, pk);  // dS into the first 32 columns of this warpgroup's run
+        tmem_st_wait();
+        tc_fence_before_sync();
+        mbar_arrive(bar(C::QB_DSF));
+      }
+    }
+    // ---- epilogue: each warpgroup writes half of the dQ row (times scale)
+    const bool have = N > 0;
+    if (have && ok) {
+      ok = mbar_wait_warp(bar(C::QB_ACC), 0, abort_flag);
+      tc_fence_after_sync();
+    }
+    if (!have || ok) {
+      constexpr int HALF = D / 2;
+      const uint32_t t_acc = tmem + lane_off + C::Q_TM_DQ + wg * HALF;
+      uint16_t* out = p.dq + ((size_t)bh_q * p.Sq + row) * D + wg * HALF;
+#pragma unroll
+      for (int c = 0; c < HALF; c += 32) {
+        uint32_t v[32];
+        if (have) {
+          tmem_ld32_sync(t_acc + c, v);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
+        if (row < p.Sq) bwd_store32(out + c, v, p.scale);
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace attn_b200

@@ -182,6 +182,11 @@ def prefill_inputs(B, Hq, Hkv, Sq, Sk, d, seed, value_scale=1.0):
     return q, k, v
 
 
+def grad_output(B, Hq, Sq, d, seed, value_scale=1.0):
+    """dO [B,Hq,Sq,d] bf16 on the host: the gradient a backward pass receives."""
+    return randn_bf16((B, Hq, Sq, d), seed * 16 + 3, value_scale)
+
+
 def key_padding(B: int, Sk: int, seed: int = SEED_PADDING, max_frac: float = 0.25) -> torch.Tensor:
     """k_lens [B] int32: Sk minus a pad uniform in [0, floor(max_frac*Sk)]; one pad > 0."""
     hi = int(math.floor(max_frac * Sk))

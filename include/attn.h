@@ -310,6 +310,47 @@ int attn_decode_paged_noalloc(const void* q, const void* k_cache, const void* v_
                               int B, int Hq, int Hkv, int d, int max_pages_per_seq, int num_pages,
                               float scale, void* o, float* lse, attn_stream_t stream);
 
+/*
+ * attn_bwd_workspace_size -- bytes of device workspace attn_bwd needs:
+ * 8 * B * Hq * ceil(Sq / 128) * 128 (two fp32 row statistics per query row,
+ * padded to whole 128-row tiles).  0 for invalid arguments.
+ */
+size_t attn_bwd_workspace_size(int B, int Hq, int Sq);
+
+/*
+ * attn_bwd -- backward pass of attn_fwd_masked, recomputing the probabilities
+ * from the saved log-sum-exp.
+ * Source: "Attention Kernel", section "Backward 与重计算" (the backward
+ * recomputes the local probabilities from Q, K, V, the output and the
+ * log-sum-exp, with the forward's softmax scale, mask and GQA head mapping,
+ * and its accumulation must be free of races); "Attention 算子加速史", FAQ Q1
+ * (recompute rather than store the attention matrix).
+ *   With P = softmax(scale * Q K^T + M) as in the forward and dO the gradient
+ *   of O, the call writes
+ *     dV = P^T dO,  dS = P * (dO V^T - rowsum(dO * O)),
+ *     dQ = scale * dS K,  dK = scale * dS^T Q,
+ *   dK and dV of a KV head summed over the query heads of its group.
+ *   q, o, d_o, dq [B, Hq, Sq, d] bf16    k, v, dk, dv [B, Hkv, Sk, d] bf16
+ *   lse [B, Hq, Sq] fp32: the forward's LSE for these q, k and mask
+ *   (-inf on rows with no visible key, whose gradients are zero).
+ *   o is the forward output for the same inputs; dq, dk, dv are written
+ *   (every element, including keys masked by k_lens, which get zero).
+ *   causal, scale, k_lens: exactly as given to attn_fwd_masked.
+ *   workspace: device memory of at least attn_bwd_workspace_size(B, Hq, Sq)
+ *   bytes, 16-byte aligned, owned by the caller; its contents on entry are
+ *   ignored and it must not be shared with a concurrent call.
+ *   Deterministic: every output element is written by one CTA in a fixed
+ *   order (no atomics), so repeated calls give identical bits.
+ * Errors: as attn_fwd_masked, plus INVALID_ARG for a NULL o, lse, d_o, dq or
+ * workspace (dk, dv when Sk > 0), ALIGNMENT (o, d_o, dq, dk, dv, workspace
+ * need 16 bytes, lse 4), WORKSPACE when workspace_bytes is too small.  Sk = 0
+ * only zero-fills dq.
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* d_o, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk,
+             int d, int causal, float scale, const int32_t* k_lens, void* workspace,
+             size_t workspace_bytes, attn_stream_t stream);
+
 /* attn_strerror -- static description of an attn_status value. */
 const char* attn_strerror(int status);
 

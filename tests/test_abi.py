@@ -31,7 +31,7 @@ def test_header_declares_expected_entry_points():
     for n in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_fwd_varlen_workspace_size",
               "attn_fwd_paged", "attn_fwd_window", "attn_fwd_block_sparse",
               "attn_decode_paged", "attn_decode_workspace_size", "attn_get_device_error",
-              "attn_strerror"):
+              "attn_bwd", "attn_bwd_workspace_size", "attn_strerror"):
         assert n in names
 
 
@@ -215,6 +215,45 @@ def test_workspace_size_formula(lib):
     assert got >= parts * d * 4 + parts * 4
     assert got <= parts * d * 4 + parts * 4 + 256
     assert lib.attn_decode_workspace_size(0, 1, 1, 16, 128) == 0
+
+
+def _bwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, do=FAKE, dq=FAKE, dk=FAKE, dv=FAKE,
+         B_=1, Hq=2, Hkv=1, Sq=200, Sk=300, d=128, causal=1, scale=0.1, k_lens=None, ws=FAKE,
+         ws_bytes=1 << 20):
+    return lib.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, B_, Hq, Hkv, Sq, Sk, d, causal, scale,
+                        k_lens, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(o=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(lse=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(do=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(dq=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(dk=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(ws=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(q=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), B.ATTN_ERR_INVALID_ARG),
+    (dict(Sq=0), B.ATTN_ERR_INVALID_ARG),
+    (dict(causal=3), B.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), B.ATTN_ERR_INVALID_ARG),
+    (dict(d=80), B.ATTN_ERR_UNSUPPORTED),
+    (dict(do=FAKE + 8), B.ATTN_ERR_ALIGNMENT),
+    (dict(dv=FAKE + 2), B.ATTN_ERR_ALIGNMENT),
+    (dict(o=FAKE + 4), B.ATTN_ERR_ALIGNMENT),
+    (dict(ws=FAKE + 8), B.ATTN_ERR_ALIGNMENT),
+    (dict(lse=FAKE + 2), B.ATTN_ERR_ALIGNMENT),
+    (dict(ws_bytes=2 * 2 * 256 * 4 - 1), B.ATTN_ERR_WORKSPACE),
+])
+def test_bwd_validation(lib, kw, status):
+    assert _bwd(lib, **kw) == status
+
+
+def test_bwd_workspace_size_formula(lib):
+    # two fp32 statistics per query row, rows padded to whole 128-row tiles
+    assert lib.attn_bwd_workspace_size(1, 2, 200) == 2 * 2 * 256 * 4
+    assert lib.attn_bwd_workspace_size(4, 16, 2048) == 2 * 64 * 2048 * 4
+    assert lib.attn_bwd_workspace_size(0, 1, 1) == 0
+    assert lib.attn_bwd_workspace_size(1, 1, 0) == 0
 
 
 def test_binding_refuses_cpu_tensors():
