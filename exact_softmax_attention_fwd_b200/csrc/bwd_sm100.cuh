@@ -24,15 +24,18 @@
 //       dV += P^T dO, dK += dS^T Q     (TS: P^T / dS^T read from tensor memory)
 //     so the transposed products land with keys on the TMEM lanes and need no
 //     transpose.  dV and dK accumulate in tensor memory across the whole loop.
+//     The S^T columns are released as soon as the recompute warps have read
+//     them, and P^T and dS^T both go into the dP^T columns, so the next tile's
+//     S^T runs on the tensor cores while this tile's P^T is computed.
 //   * attn_bwd_dq_kernel: one CTA per (query tile, batch, query head), K/V
 //     tiles streaming: S = Q K^T, dP = dO V^T (SS), dQ += dS K (TS).
 // Both compute kernels use the forward's organisation: warp 0 lane 0 issues
 // TMA copies (no multicast), warp 1 lane 0 issues the MMAs, and two
 // warpgroups (warps 4-7, 8-11) each own 64 of the 128 columns of every score
-// tile (thread r owns TMEM lane r).  A warpgroup packs its bf16 P or dS into
-// the first 32 columns of its own 64-column range, so the two warpgroups never
-// write a column the other still has to read; the TS MMAs read the operand
-// from those two 32-column runs.
+// tile (thread r owns TMEM lane r).  A warpgroup packs its bf16 operands into
+// its own 64-column range (32 columns each: dS, and in the dK/dV kernel P
+// after it), so the two warpgroups never write a column the other still has to
+// read; the TS MMAs read an operand from the two warpgroups' 32-column runs.
 #pragma once
 
 #include "sm100_primitives.cuh"
@@ -83,10 +86,10 @@ struct BwdCfg {
   static constexpr int KB_QF = 1;                  // STAGES: Q, dO, statistics landed
   static constexpr int KB_QE = KB_QF + STAGES;     // STAGES: stage free (MMA + 256 threads)
   static constexpr int KB_SF = KB_QE + STAGES;     // S^T in TMEM
-  static constexpr int KB_DPF = KB_SF + 1;         // dP^T in TMEM
-  static constexpr int KB_PF = KB_DPF + 1;         // P^T written (256 threads)
-  static constexpr int KB_DSF = KB_PF + 1;         // dS^T written (256 threads)
-  static constexpr int KB_ACC = KB_DSF + 1;        // every MMA retired
+  static constexpr int KB_SE = KB_SF + 1;          // S^T read by the recompute warps (256)
+  static constexpr int KB_DPF = KB_SE + 1;         // dP^T in TMEM
+  static constexpr int KB_PDS = KB_DPF + 1;        // P^T and dS^T written (256 threads)
+  static constexpr int KB_ACC = KB_PDS + 1;        // every MMA retired
   static constexpr int KB_NUM = KB_ACC + 1;
   static constexpr int KV_OFF_MISC = KV_OFF_BAR + KB_NUM * 8;
   static constexpr int KV_SMEM = KV_OFF_MISC + 16 + 1024;
@@ -108,16 +111,16 @@ struct BwdCfg {
   static constexpr int Q_SMEM = Q_OFF_MISC + 16 + 1024;
   // ---- tensor memory (512 columns)
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t KV_TM_S = 0;        // S^T, then P^T (bf16) in its warpgroup runs
-  static constexpr uint32_t KV_TM_DP = 128;     // dP^T, then dS^T (bf16)
+  static constexpr uint32_t KV_TM_S = 0;        // S^T
+  static constexpr uint32_t KV_TM_DP = 128;     // dP^T, then dS^T and P^T (bf16)
   static constexpr uint32_t KV_TM_DV = 256;
   static constexpr uint32_t KV_TM_DK = 256 + D;
   static constexpr uint32_t Q_TM_S0 = 0, Q_TM_S1 = 128;
   static constexpr uint32_t Q_TM_DP = 256;      // dP, then dS (bf16)
   static constexpr uint32_t Q_TM_DQ = 384;
   static constexpr int NUM_THREADS = 384;
-  static constexpr uint32_t REGS_PRODUCER = 72;
-  static constexpr uint32_t REGS_SOFTMAX = 208;
+  static constexpr uint32_t REGS_PRODUCER = 88;
+  static constexpr uint32_t REGS_SOFTMAX = 192;
   static_assert(128 * (REGS_PRODUCER + 2 * REGS_SOFTMAX) <= NUM_THREADS * 168,
                 "register reallocation must fit the launch allocation");
   static_assert(KV_SMEM <= 232448 && Q_SMEM <= 232448, "shared memory");
@@ -265,9 +268,9 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar(C::KB_QE + s), 1 + 256);
     }
     mbar_init(bar(C::KB_SF), 1);
+    mbar_init(bar(C::KB_SE), 256);
     mbar_init(bar(C::KB_DPF), 1);
-    mbar_init(bar(C::KB_PF), 256);
-    mbar_init(bar(C::KB_DSF), 256);
+    mbar_init(bar(C::KB_PDS), 256);
     mbar_init(bar(C::KB_ACC), 1);
     *abort_flag = 0;
     mbar_init_fence();
@@ -338,22 +341,22 @@ __global__ void __launch_bounds__(384, 1)
       }
       for (int n = 0; ok && n < N; ++n) {
         const int s = n % C::STAGES, s1 = (n + 1) % C::STAGES;
-        if (!(ok = mbar_wait(bar(C::KB_PF), n & 1u, abort_flag))) break;
-        tc_fence_after_sync();
-        bwd_mma_ts<D>(tDV, tS, sDO(s), n > 0);  // dV += P^T dO
         if (n + 1 < N) {
-          // S^T of the next query tile: overwrites P^T only after the MMA above
-          // read it (MMAs of one thread run in issue order)
+          // S^T of the next query tile, as soon as this tile's S^T has been read
+          if (!(ok = mbar_wait(bar(C::KB_SE), n & 1u, abort_flag))) break;
           if (!(ok = mbar_wait(bar(C::KB_QF + s1), ((n + 1) / C::STAGES) & 1u, abort_flag))) break;
           tc_fence_after_sync();
           bwd_mma_ss<D>(tS, sK, sQ(s1));
           umma_commit(bar(C::KB_SF));
         }
-        if (!(ok = mbar_wait(bar(C::KB_DSF), n & 1u, abort_flag))) break;
+        if (!(ok = mbar_wait(bar(C::KB_PDS), n & 1u, abort_flag))) break;
         tc_fence_after_sync();
-        bwd_mma_ts<D>(tDK, tDP, sQ(s), n > 0);  // dK += dS^T Q
-        umma_commit(bar(C::KB_QE + s));          // Q and dO of stage s read for the last time
+        bwd_mma_ts<D>(tDV, tDP + 32, sDO(s), n > 0);  // dV += P^T dO
+        bwd_mma_ts<D>(tDK, tDP, sQ(s), n > 0);        // dK += dS^T Q
+        umma_commit(bar(C::KB_QE + s));  // Q and dO of stage s read for the last time
         if (n + 1 < N) {
+          // dP^T of the next tile overwrites P^T and dS^T only after the two MMAs
+          // above read them (MMAs of one thread run in issue order)
           bwd_mma_ss<D>(tDP, sV, sDO(s1));
           umma_commit(bar(C::KB_DPF));
         }
@@ -385,13 +388,9 @@ __global__ void __launch_bounds__(384, 1)
       const int cmin = (int)(cm < 0 ? 0 : (cm > 64 ? 64 : cm));
       const bool edge = __any_sync(0xffffffffu, cmin > 0);
       if (!(ok = mbar_wait_warp(bar(C::KB_SF), n & 1u, abort_flag))) break;
-      // the statistics arrived with Q (every thread observes the copy itself)
-      const bool st_ok = mbar_wait(bar(C::KB_QF + s), (n / C::STAGES) & 1u, abort_flag);
-      if (!(ok = __all_sync(0xffffffffu, st_ok))) break;
       tc_fence_after_sync();
-      const float4* st = reinterpret_cast<const float4*>(sbase_ptr + C::KV_OFF_ST +
-                                                         s * C::STAT_BYTES);
       float pr[64];
+      uint32_t pk_p[32];
       {
         uint32_t a[32], bq[32];
         tmem_ld32(t_s, a);
@@ -399,7 +398,13 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld_wait();
         reg_fence32(a);
         reg_fence32(bq);
-        uint32_t pk[32];
+        tc_fence_before_sync();
+        mbar_arrive(bar(C::KB_SE));  // S^T read: the next tile's S^T may overwrite it
+        // the statistics arrived with Q (every thread observes the copy itself)
+        const bool st_ok = mbar_wait(bar(C::KB_QF + s), (n / C::STAGES) & 1u, abort_flag);
+        if (!(ok = __all_sync(0xffffffffu, st_ok))) break;
+        const float4* st = reinterpret_cast<const float4*>(sbase_ptr + C::KV_OFF_ST +
+                                                           s * C::STAT_BYTES);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {  // columns 4e .. 4e+3
           const float4 nl = st[(c0 >> 2) + e];
@@ -423,39 +428,40 @@ __global__ void __launch_bounds__(384, 1)
           pr[c + 1] = ex2(x1);
           pr[c + 2] = ex2(x2);
           pr[c + 3] = ex2(x3);
-          pk[2 * e] = pack_bf16x2(pr[c], pr[c + 1]);
-          pk[2 * e + 1] = pack_bf16x2(pr[c + 2], pr[c + 3]);
+          pk_p[2 * e] = pack_bf16x2(pr[c], pr[c + 1]);
+          pk_p[2 * e + 1] = pack_bf16x2(pr[c + 2], pr[c + 3]);
         }
-        tmem_st32(t_s, pk);  // P^T into the first 32 columns of this warpgroup's run
-        tmem_st_wait();
-        tc_fence_before_sync();
-        mbar_arrive(bar(C::KB_PF));
       }
       if (!(ok = mbar_wait_warp(bar(C::KB_DPF), n & 1u, abort_flag))) break;
       tc_fence_after_sync();
       {
-        uint32_t a[32], bq[32];
-        tmem_ld32(t_dp, a);
-        tmem_ld32(t_dp + 32, bq);
-        tmem_ld_wait();
-        reg_fence32(a);
-        reg_fence32(bq);
+        const float4* st = reinterpret_cast<const float4*>(sbase_ptr + C::KV_OFF_ST +
+                                                           s * C::STAT_BYTES);
         uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float4 dd = st[32 + (c0 >> 2) + e];  // D of columns 4e .. 4e+3
-          const int c = 4 * e;
-          const float d0 = __uint_as_float(c < 32 ? a[c] : bq[c - 32]) - dd.x;
-          const float d1 = __uint_as_float(c < 32 ? a[c + 1] : bq[c - 31]) - dd.y;
-          const float d2 = __uint_as_float(c < 32 ? a[c + 2] : bq[c - 30]) - dd.z;
-          const float d3 = __uint_as_float(c < 32 ? a[c + 3] : bq[c - 29]) - dd.w;
-          pk[2 * e] = pack_bf16x2(pr[c] * d0, pr[c + 1] * d1);
-          pk[2 * e + 1] = pack_bf16x2(pr[c + 2] * d2, pr[c + 3] * d3);
+        for (int h = 0; h < 2; ++h) {  // dP^T columns [32h, 32h + 32) of this warpgroup's run
+          uint32_t a[32];
+          tmem_ld32(t_dp + 32 * h, a);
+          tmem_ld_wait();
+          reg_fence32(a);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 dd = st[32 + (c0 >> 2) + 8 * h + e];  // D of columns 32h + 4e ..
+            const int c = 32 * h + 4 * e;
+            const float d0 = __uint_as_float(a[4 * e]) - dd.x;
+            const float d1 = __uint_as_float(a[4 * e + 1]) - dd.y;
+            const float d2 = __uint_as_float(a[4 * e + 2]) - dd.z;
+            const float d3 = __uint_as_float(a[4 * e + 3]) - dd.w;
+            pk[16 * h + 2 * e] = pack_bf16x2(pr[c] * d0, pr[c + 1] * d1);
+            pk[16 * h + 2 * e + 1] = pack_bf16x2(pr[c + 2] * d2, pr[c + 3] * d3);
+          }
         }
-        tmem_st32(t_dp, pk);  // dS^T into the first 32 columns of this warpgroup's run
+        // dS^T then P^T into this warpgroup's 64 dP^T columns (all read above)
+        tmem_st32(t_dp, pk);
+        tmem_st32(t_dp + 32, pk_p);
         tmem_st_wait();
         tc_fence_before_sync();
-        mbar_arrive(bar(C::KB_DSF));
+        mbar_arrive(bar(C::KB_PDS));
       }
       mbar_arrive(bar(C::KB_QE + s));  // this thread is done with stage s's statistics
     }
