@@ -256,6 +256,53 @@ def paged_inputs(seq_lens, Hq, Hkv, d, page_size, seed, max_pages_per_seq=None,
     return PagedInputs(q, k_cache, v_cache, table, lens, page_size)
 
 
+@dataclass
+class PagedFp8Inputs:
+    q: torch.Tensor            # [B, Hq, d] bf16
+    k_cache: torch.Tensor      # [num_pages, page_size, Hkv, d] uint8 (E4M3 codes)
+    v_cache: torch.Tensor      # [num_pages, page_size, Hkv, d] uint8 (E4M3 codes)
+    k_scale: torch.Tensor      # [num_pages, Hkv] float32
+    v_scale: torch.Tensor      # [num_pages, Hkv] float32
+    block_table: torch.Tensor  # [B, max_pages_per_seq] int32, -1 = unused
+    seq_lens: torch.Tensor     # [B] int32
+    page_size: int
+
+    @property
+    def num_pages(self) -> int:
+        return int(self.k_cache.shape[0])
+
+
+E4M3_MAX = 448.0
+
+
+def quantize_e4m3_per_page(cache: torch.Tensor):
+    """bf16 [num_pages, page_size, Hkv, d] -> (E4M3 codes uint8, scales float32
+    [num_pages, Hkv]) with scale = amax / 448 per (page, KV head) (1 where the
+    block is all zero), the codes being round-to-nearest of x / scale."""
+    x = cache.float()
+    amax = x.abs().amax(dim=(1, 3))
+    sc = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+    codes = (x / sc[:, None, :, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), sc.contiguous()
+
+
+def fp8_paged_inputs(seq_lens, Hq, Hkv, d, page_size, seed, **kw) -> PagedFp8Inputs:
+    """A paged cache as ``paged_inputs`` builds it, quantised to E4M3 with one
+    scale per (page, KV head) for K and for V."""
+    base = paged_inputs(seq_lens, Hq, Hkv, d, page_size, seed, **kw)
+    k8, ks = quantize_e4m3_per_page(base.k_cache)
+    v8, vs = quantize_e4m3_per_page(base.v_cache)
+    return PagedFp8Inputs(base.q, k8, v8, ks, vs, base.block_table, base.seq_lens, page_size)
+
+
+def fp8_kv_bytes(seq_lens, Hkv: int, d: int, page_size: int) -> int:
+    """Bytes of an FP8 cache the attended tokens occupy: one byte per K and V
+    element, plus the K and V scale of every (page, KV head) read."""
+    lens = torch.as_tensor(seq_lens, dtype=torch.int64)
+    pages = int(((lens + page_size - 1) // page_size).sum())
+    return int(lens.sum()) * Hkv * d * 2 + pages * Hkv * 4 * 2
+
+
 def decode_config_inputs(cfg: DecodeConfig) -> PagedInputs:
     lens = decode_lengths(cfg.B, cfg.len_lo, cfg.len_hi)
     return paged_inputs(lens, cfg.Hq, cfg.Hkv, cfg.d, cfg.page_size, cfg.seed,

@@ -1,0 +1,105 @@
+"""CPU oracle for decode over an FP8 (e4m3) paged KV cache -- TEST INFRASTRUCTURE ONLY.
+
+Plain float64 numpy.  The cache holds one byte per element in the OCP 8-bit
+floating-point format E4M3 (1 sign bit, 4 exponent bits with bias 7, 3
+mantissa bits; exponent field 0 encodes subnormals m * 2^-9; the all-ones
+exponent with all-ones mantissa is NaN; there is no infinity), plus one fp32
+scale per (physical page, KV head) for K and one for V.  The dequantised
+cache is
+    K[page, row, h, :] = k_scale[page, h] * e4m3(k_bytes[page, row, h, :])
+and likewise V; decode is then exact softmax attention of one query row per
+(sequence, query head) over the sequence's tokens, gathered through the block
+table exactly as for a bf16 cache.
+
+Sources (page title, section):
+  * "Attention Kernel" -- "Paged 与 ragged KV" (token t lives in block
+    t / page_size at offset t mod page_size; the block table maps it to a
+    physical page) and "正确性契约" (the cache quantisation schema is part of
+    the kernel's contract, next to page size and valid-token counts).
+  * "Attention 算子加速史" -- section 3 (FP8 operands with scale factors on
+    FlashAttention-3) and section 4 (paged decode).
+  * "Attention Kernel" -- "问题与成本" and "Online softmax" (the attention
+    itself, and the zero output / -inf LSE of a row with no key).
+
+Pinned in ``tests/test_oracle_fp8_pins.py``: the E4M3 decoding against torch's
+float8_e4m3fn for all 256 codes; with unit scales and codes whose values are
+exact in bf16, against the C bf16 decode oracle on the same values; scale
+laws (V scale scales O, K scale acts as the softmax scale); per-page scales
+applied to the right pages.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def e4m3_to_float(codes) -> np.ndarray:
+    """Values of E4M3 bytes (uint8 array) as float64: sign * 2^(e-7) * (1 + m/8)
+    for exponent field e > 0, sign * m * 2^-9 for e = 0, NaN for 0x7F / 0xFF."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    normal = sign * np.ldexp(1.0 + m / 8.0, e - 7)
+    sub = sign * m * 2.0 ** -9
+    out = np.where(e == 0, sub, normal)
+    return np.where((c & 0x7F) == 0x7F, np.nan, out)
+
+
+def dequantize(cache_bytes, scales) -> np.ndarray:
+    """[num_pages, page_size, Hkv, d] bytes and [num_pages, Hkv] scales -> float64 values."""
+    vals = e4m3_to_float(cache_bytes)
+    s = np.asarray(scales, dtype=np.float64)
+    return vals * s[:, None, :, None]
+
+
+def _f64(x) -> np.ndarray:
+    if isinstance(x, np.ndarray):
+        if x.dtype == np.uint16:  # bf16 bit patterns
+            return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        return x.astype(np.float64)
+    return x.detach().cpu().double().numpy()
+
+
+def decode_paged_fp8(q, k_bytes, v_bytes, k_scale, v_scale, block_table, seq_lens, scale):
+    """One query row per (sequence, query head) over an FP8 paged cache.
+
+    q [B, Hq, d] (bf16 tensor or floats); k_bytes, v_bytes uint8 [num_pages,
+    page_size, Hkv, d]; k_scale, v_scale [num_pages, Hkv]; block_table int
+    [B, max_pages]; seq_lens [B].  Returns (o [B, Hq, d], lse [B, Hq]) float64;
+    a sequence of length 0 gives o = 0 and lse = -inf.
+    """
+    Q = _f64(q)
+    kb = np.asarray(k_bytes.cpu().numpy() if hasattr(k_bytes, "cpu") else k_bytes, np.uint8)
+    vb = np.asarray(v_bytes.cpu().numpy() if hasattr(v_bytes, "cpu") else v_bytes, np.uint8)
+    ks = np.asarray(k_scale.cpu().numpy() if hasattr(k_scale, "cpu") else k_scale, np.float64)
+    vs = np.asarray(v_scale.cpu().numpy() if hasattr(v_scale, "cpu") else v_scale, np.float64)
+    tbl = np.asarray(block_table.cpu().numpy() if hasattr(block_table, "cpu") else block_table)
+    lens = np.asarray(seq_lens.cpu().numpy() if hasattr(seq_lens, "cpu") else seq_lens)
+    B, Hq, d = Q.shape
+    num_pages, page_size, Hkv, dk = kb.shape
+    if dk != d or vb.shape != kb.shape or ks.shape != (num_pages, Hkv) or vs.shape != ks.shape:
+        raise ValueError("cache / scale shapes disagree")
+    g = Hq // Hkv
+    K = dequantize(kb, ks)
+    V = dequantize(vb, vs)
+    o = np.zeros((B, Hq, d))
+    lse = np.full((B, Hq), -np.inf)
+    for b in range(B):
+        n = int(lens[b])
+        if n == 0:
+            continue
+        t = np.arange(n)
+        pages = tbl[b, t // page_size]
+        if (pages < 0).any() or (pages >= num_pages).any():
+            raise ValueError("block table entry out of range")
+        rows = t % page_size
+        for hq in range(Hq):
+            h = hq // g
+            kk = K[pages, rows, h, :]          # [n, d]
+            vv = V[pages, rows, h, :]
+            s = scale * (kk @ Q[b, hq])
+            mx = s.max()
+            w = np.exp(s - mx)
+            o[b, hq] = (w @ vv) / w.sum()
+            lse[b, hq] = mx + np.log(w.sum())
+    return o, lse

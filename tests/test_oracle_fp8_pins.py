@@ -1,0 +1,92 @@
+"""Pins for the FP8-cache decode oracle (``oracle/kv_fp8.py``), each against
+something other than itself:
+
+* E4M3 decoding against torch's float8_e4m3fn for all 256 codes (a library
+  routine), plus values fixed by the format's definition;
+* with per-(page, head) scales that are powers of two, every dequantised
+  value is exact in bf16, so the FP8 oracle must equal the C bf16 decode
+  oracle (an independent implementation) run on that bf16 cache;
+* scale laws: the V scale scales O and leaves the LSE alone; a uniform K
+  scale c is the softmax scale multiplied by c.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle.kv_fp8 import decode_paged_fp8, dequantize, e4m3_to_float
+from exact_softmax_attention_fwd_b200 import workloads as W
+
+
+def test_e4m3_all_codes_match_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    ours = e4m3_to_float(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert nan.sum() == 2  # 0x7F and 0xFF
+    np.testing.assert_array_equal(ours[~nan], ref[~nan])
+
+
+def test_e4m3_values_from_the_format():
+    v = e4m3_to_float(np.array([0x00, 0x80, 0x01, 0x07, 0x08, 0x38, 0xB8, 0x7E, 0xFE, 0x3C],
+                               dtype=np.uint8))
+    want = [0.0, -0.0, 2.0 ** -9, 7 * 2.0 ** -9, 2.0 ** -6, 1.0, -1.0, 448.0, -448.0, 1.5]
+    np.testing.assert_array_equal(v, want)
+
+
+def _random_codes(shape, gen):
+    c = torch.randint(0, 256, shape, generator=gen, dtype=torch.int64).to(torch.uint8)
+    c[(c & 0x7F) == 0x7F] = 0x3C  # no NaN codes
+    return c
+
+
+@pytest.mark.parametrize("page_size,d,Hq,Hkv", [(16, 64, 4, 2), (32, 128, 8, 2), (16, 128, 2, 2)])
+def test_fp8_decode_equals_bf16_oracle_on_exact_values(page_size, d, Hq, Hkv):
+    gen = torch.Generator().manual_seed(31)
+    lens = torch.tensor([1, 37, 0, 100], dtype=torch.int32)
+    base = W.paged_inputs(lens, Hq, Hkv, d, page_size, seed=31, extra_pages=2)
+    P = base.num_pages
+    k8 = _random_codes((P, page_size, Hkv, d), gen)
+    v8 = _random_codes((P, page_size, Hkv, d), gen)
+    # powers of two keep k_scale * e4m3 exact in bf16 (3 mantissa bits)
+    ks = torch.pow(2.0, torch.randint(-4, 3, (P, Hkv), generator=gen).double()).float()
+    vs = torch.pow(2.0, torch.randint(-4, 3, (P, Hkv), generator=gen).double()).float()
+    kd = torch.from_numpy(dequantize(k8.numpy(), ks.numpy())).to(torch.bfloat16)
+    vd = torch.from_numpy(dequantize(v8.numpy(), vs.numpy())).to(torch.bfloat16)
+    np.testing.assert_array_equal(kd.double().numpy(), dequantize(k8.numpy(), ks.numpy()))
+    scale = 0.03
+    o, lse = decode_paged_fp8(base.q, k8, v8, ks, vs, base.block_table, lens, scale)
+    o_ref, lse_ref = oracle.decode_paged(base.q, kd, vd, base.block_table, lens, scale)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-10)
+    fin = np.isfinite(lse_ref)
+    np.testing.assert_allclose(lse[fin], lse_ref[fin], rtol=0, atol=1e-10)
+    assert np.array_equal(np.isneginf(lse), np.isneginf(lse_ref))
+
+
+def test_fp8_scale_laws():
+    c = W.fp8_paged_inputs(torch.tensor([70, 5], dtype=torch.int32), 4, 2, 64, 16, seed=32)
+    o, lse = decode_paged_fp8(c.q, c.k_cache, c.v_cache, c.k_scale, c.v_scale, c.block_table,
+                              c.seq_lens, 0.1)
+    # a power-of-two factor keeps the float32 scales exact
+    o2, lse2 = decode_paged_fp8(c.q, c.k_cache, c.v_cache, c.k_scale, c.v_scale * 4.0,
+                                c.block_table, c.seq_lens, 0.1)
+    np.testing.assert_allclose(o2, 4.0 * o, rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(lse2, lse)
+    o3, lse3 = decode_paged_fp8(c.q, c.k_cache, c.v_cache, c.k_scale * 2.0, c.v_scale,
+                                c.block_table, c.seq_lens, 0.05)
+    np.testing.assert_allclose(o3, o, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse3, lse, rtol=1e-12, atol=1e-12)
+
+
+def test_fp8_generator_roundtrip_error_is_within_e4m3_rounding():
+    base = W.paged_inputs(torch.tensor([64], dtype=torch.int32), 2, 2, 64, 16, seed=33)
+    codes, sc = W.quantize_e4m3_per_page(base.k_cache)
+    back = dequantize(codes.numpy(), sc.numpy())
+    x = base.k_cache.double().numpy()
+    # E4M3 keeps 3 mantissa bits: relative error <= 2^-4 on normals; absolute
+    # error <= half the subnormal step (2^-10 * scale) below the normal range
+    err = np.abs(back - x)
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * sc.numpy()[:, None, :, None])
+    assert (err <= bound * (1 + 1e-12)).all()
+    assert np.abs(back).max() <= 448.0 * float(sc.double().max()) * (1 + 1e-12)
