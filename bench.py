@@ -55,6 +55,7 @@ def parse_args():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-ragged", action="store_true")
     ap.add_argument("--ragged-workload", default="ragged_gqa_causal")
+    ap.add_argument("--no-decode-fp8", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--backward-workload", default="mha_causal_2k")
     ap.add_argument("--no-paged-prefill", action="store_true")
@@ -75,15 +76,29 @@ def load_peaks():
     return d
 
 
-def kernel_source_sha() -> str:
-    """Hash of the CUDA sources: ncu traffic figures are valid only for this hash."""
+# Device-code sources of each kernel family: its ncu counters stay valid while
+# these files are unchanged (the other kernels' sources do not affect them).
+KERNEL_SOURCES = {
+    "attn_prefill_sm100_kernel": ("prefill_sm100.cuh", "varlen_schedule.cuh",
+                                  "sm100_primitives.cuh"),
+    "attn_decode_split_kernel": ("decode_sm100.cuh", "sm100_primitives.cuh"),
+    "attn_decode_split_fp8_kernel": ("decode_sm100.cuh", "sm100_primitives.cuh"),
+    "attn_bwd_dkdv_kernel": ("bwd_sm100.cuh", "sm100_primitives.cuh"),
+    "attn_bwd_dq_kernel": ("bwd_sm100.cuh", "sm100_primitives.cuh"),
+}
+
+
+def kernel_source_sha(kernel: str = None) -> str:
+    """Hash of a kernel family's CUDA sources (of every .cu/.cuh when kernel is
+    None): ncu traffic figures are valid only for this hash."""
     csrc = os.path.join(ROOT, "exact_softmax_attention_fwd_b200", "csrc")
+    names = (sorted(KERNEL_SOURCES[kernel]) if kernel is not None else
+             sorted(n for n in os.listdir(csrc) if n.endswith((".cu", ".cuh"))))
     h = hashlib.sha256()
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    for name in names:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -95,7 +110,7 @@ def ncu_traffic(kernel_key: str, config_name: str):
     with open(path) as f:
         t = json.load(f)
     e = t.get(kernel_key, {}).get(config_name)
-    if not e or e.get("source_sha") != kernel_source_sha():
+    if not e or e.get("source_sha") != kernel_source_sha(kernel_key):
         return None
     return float(e["dram_bytes_per_launch"])
 
@@ -414,6 +429,8 @@ def run_ours(args, world, rank, local):
         line["paged_prefill"] = paged_prefill_leg(args, dev, world, peaks)
     if not args.no_backward:
         line["backward"] = backward_leg(args, dev, world, peaks)
+    if not args.no_decode and not args.no_decode_fp8:
+        line["decode_fp8"] = decode_fp8_leg(args, dev, world, peaks)
     if not args.no_e2e:
         line["e2e"] = e2e_leg(args, cfg, q_h, k_h, v_h, kl_h, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -443,6 +460,53 @@ def _timed_calls(args, dev, world, one):
         e1.record(stream)
     torch.cuda.synchronize(dev)
     return [a.elapsed_time(b) for a, b in evs]
+
+
+def decode_fp8_leg(args, dev, world, peaks):
+    """Paged decode over the same workload with its cache quantised to E4M3
+    (one scale per page and KV head): the split kernel reads half the K/V bytes.
+    Algorithmic bytes: the FP8 K/V of the attended tokens and their pages'
+    scales, plus q, o, lse, the block-table entries and the lengths."""
+    import torch
+
+    from exact_softmax_attention_fwd_b200 import (attn_decode_paged_fp8,
+                                                  attn_decode_workspace_size,
+                                                  attn_get_device_error)
+    from exact_softmax_attention_fwd_b200 import workloads as W
+
+    dcfg = W.CONFIGS[args.decode_workload]
+    base = W.decode_config_inputs(dcfg)
+    k8, ks = W.quantize_e4m3_per_page(base.k_cache)
+    v8, vs = W.quantize_e4m3_per_page(base.v_cache)
+    q, tbl, lens = base.q.to(dev), base.block_table.to(dev), base.seq_lens.to(dev)
+    k8, v8, ks, vs = k8.to(dev), v8.to(dev), ks.to(dev), vs.to(dev)
+    ws = torch.empty(attn_decode_workspace_size(dcfg.B, dcfg.Hq, dcfg.max_pages_per_seq,
+                                                dcfg.page_size, dcfg.d),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty((dcfg.B, dcfg.Hq, dcfg.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((dcfg.B, dcfg.Hq), dtype=torch.float32, device=dev)
+
+    def one():
+        attn_decode_paged_fp8(q, k8, v8, ks, vs, tbl, lens, dcfg.scale, out=o, lse=lse,
+                              workspace=ws)
+
+    ms = _timed_calls(args, dev, world, one)
+    st, fl = attn_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word set in the FP8 decode leg: {fl:#x}")
+    pages = int(sum(-(-int(n) // dcfg.page_size) for n in base.seq_lens.tolist()))
+    nbytes = (W.fp8_kv_bytes(base.seq_lens, dcfg.Hkv, dcfg.d, dcfg.page_size) + 2 * q.numel() * 2
+              + pages * 4 + lens.numel() * 4 + lse.numel() * 4)
+    bytes_per_s, avg = weak_scaling_value(nbytes, sum(ms) / len(ms), world)
+    gbs = nbytes / (avg * 1e-3) / 1e9
+    tokens = int(base.seq_lens.sum())
+    return {"workload": dcfg.name + " (E4M3 cache, per-page scales)", "value": bytes_per_s / 1e9,
+            "unit": "GB/s", "ms": avg, "median_ms": statistics.median(ms), "calls": len(ms),
+            "gpu_launches_per_call": 2, "tokens_per_s": world * tokens / (avg * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes": nbytes,
+                         "kernel": "attn_decode_split_fp8_kernel + attn_decode_merge_kernel",
+                         "traffic": ncu_traffic("attn_decode_split_fp8_kernel", dcfg.name)}}
 
 
 def backward_leg(args, dev, world, peaks):
@@ -483,7 +547,10 @@ def backward_leg(args, dev, world, peaks):
             "flops_counted": "2.5x forward (dV, dP, dQ, dK and the recomputed S)",
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                         "per_call_flops": flops, "executed_flops_per_call": 3.5 * cfg.flops()}}
+                         "per_call_flops": flops, "executed_flops_per_call": 3.5 * cfg.flops(),
+                         "kernel": "attn_bwd_prep_kernel + attn_bwd_dkdv_kernel + attn_bwd_dq_kernel",
+                         "traffic": ncu_traffic("attn_bwd_dkdv_kernel", cfg.name),
+                         "traffic_kernel": "attn_bwd_dkdv_kernel"}}
 
 
 def paged_prefill_leg(args, dev, world, peaks):

@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     attn_bwd_workspace_size,
     attn_fwd_block_sparse,
     attn_decode_paged,
+    attn_decode_paged_fp8,
     attn_decode_workspace_size,
     attn_fwd,
     attn_fwd_masked,

@@ -47,6 +47,8 @@ SIGNATURES = {
     "attn_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P,
                                _SZ, _P]),
+    "attn_decode_paged_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P,
+                                   _P, _P, _SZ, _P]),
     "attn_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P,
                                        _P, _P]),
     "attn_bwd_workspace_size": (_SZ, [_I, _I, _I]),
@@ -358,6 +360,46 @@ def attn_decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float, 
                                           num_pages, float(scale), _ptr(out), _ptr(lse),
                                           _ptr(workspace), ws_bytes, _stream(stream))
     _check(st, "attn_decode_paged")
+    return out, lse
+
+
+def attn_decode_paged_fp8(q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
+                          scale: float, out=None, lse=None, workspace=None,
+                          return_lse: bool = True, stream=None):
+    """attn_decode_paged over an E4M3 cache: k_cache / v_cache uint8 [num_pages,
+    page_size, Hkv, d] codes, k_scale / v_scale float32 [num_pages, Hkv]."""
+    import torch
+    _require_cuda(q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens)
+    B, Hq, d = q.shape
+    num_pages, page_size, Hkv, dk = k_cache.shape
+    if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
+        raise ValueError("FP8 caches are uint8 E4M3 codes")
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or dk != d:
+        raise ValueError("cache shapes disagree")
+    for t in (k_scale, v_scale):
+        if t.dtype != torch.float32 or tuple(t.shape) != (num_pages, Hkv):
+            raise ValueError("scales must be float32 [num_pages, Hkv]")
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be int32 [B, max_pages_per_seq]")
+    if seq_lens.dtype != torch.int32 or tuple(seq_lens.shape) != (B,):
+        raise ValueError("seq_lens must be int32 [B]")
+    for t in (q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens):
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    max_pages = block_table.shape[1]
+    need = attn_decode_workspace_size(B, Hq, max_pages, page_size, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = load_library().attn_decode_paged_fp8(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_table),
+        _ptr(seq_lens), page_size, B, Hq, Hkv, d, max_pages, num_pages, float(scale), _ptr(out),
+        _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "attn_decode_paged_fp8")
     return out, lse
 
 

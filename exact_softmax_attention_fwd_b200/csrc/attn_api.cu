@@ -219,6 +219,83 @@ int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mdo, const CUtensorMap&
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Paged decode over a bf16 cache, or (fp8) an E4M3 cache with per-(page, KV
+// head) scales: validation, then the split kernel and the merge kernel.
+int decode_paged_common(bool fp8, const void* q, const void* k_cache, const void* v_cache,
+                        const float* k_scale, const float* v_scale, const int32_t* block_table,
+                        const int32_t* seq_lens, int page_size, int B, int Hq, int Hkv, int d,
+                        int max_pages_per_seq, int num_pages, float scale, void* o, float* lse,
+                        void* workspace, size_t workspace_bytes, attn_stream_t stream_) {
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr ||
+      seq_lens == nullptr || o == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || max_pages_per_seq < 1 || num_pages < 1 ||
+      page_size < 1)
+    return ATTN_ERR_INVALID_ARG;
+  if (B > 65535 || Hkv > 65535 || (long long)max_pages_per_seq * page_size > (1ll << 30))
+    return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (page_size % 16 != 0 || page_size > 256) return ATTN_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 8) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      !aligned4(block_table) || !aligned4(seq_lens) || (lse != nullptr && !aligned4(lse)))
+    return ATTN_ERR_ALIGNMENT;
+  if (fp8 && (!aligned4(k_scale) || !aligned4(v_scale))) return ATTN_ERR_ALIGNMENT;
+  const size_t need = attn_decode_workspace_size(B, Hq, max_pages_per_seq, page_size, d);
+  if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
+
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const long long tokens = (long long)max_pages_per_seq * page_size;
+  DecodeParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.q = static_cast<const uint16_t*>(q);
+  if (!fp8) {
+    prm.k_cache = static_cast<const uint16_t*>(k_cache);
+    prm.v_cache = static_cast<const uint16_t*>(v_cache);
+  }
+  prm.block_table = block_table;
+  prm.seq_lens = seq_lens;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.page_size = page_size;
+  prm.max_pages = max_pages_per_seq;
+  prm.num_pages = num_pages;
+  prm.n_split = (int)((tokens + kSplitTokens - 1) / kSplitTokens);
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  const size_t parts = (size_t)B * Hq * prm.n_split;
+  prm.o_part = static_cast<float*>(workspace);
+  prm.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + parts * d * sizeof(float));
+  prm.o = static_cast<uint16_t*>(o);
+  prm.lse = lse;
+
+  DecodeFp8Params pf;
+  pf.d = prm;
+  pf.k8 = static_cast<const uint8_t*>(k_cache);
+  pf.v8 = static_cast<const uint8_t*>(v_cache);
+  pf.k_scale = k_scale;
+  pf.v_scale = v_scale;
+  dim3 grid_split((prm.n_split + 3) / 4, Hkv, B);
+  dim3 grid_merge((unsigned)(((long long)B * Hq + 3) / 4));
+  if (d == 128) {
+    if (fp8)
+      attn_decode_split_fp8_kernel<128><<<grid_split, 128, 0, stream>>>(pf);
+    else
+      attn_decode_split_kernel<128><<<grid_split, 128, 0, stream>>>(prm);
+    attn_decode_merge_kernel<128><<<grid_merge, 128, 0, stream>>>(prm);
+  } else {
+    if (fp8)
+      attn_decode_split_fp8_kernel<64><<<grid_split, 128, 0, stream>>>(pf);
+    else
+      attn_decode_split_kernel<64><<<grid_split, 128, 0, stream>>>(prm);
+    attn_decode_merge_kernel<64><<<grid_merge, 128, 0, stream>>>(prm);
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 size_t bwd_workspace_bytes(int B, int Hq, int Sq) {
   const size_t pad = ((size_t)Sq + 127) / 128 * 128;
   return 2 * (size_t)B * Hq * pad * sizeof(float);
@@ -513,58 +590,20 @@ int attn_decode_paged(const void* q, const void* k_cache, const void* v_cache,
                       int Hq, int Hkv, int d, int max_pages_per_seq, int num_pages, float scale,
                       void* o, float* lse, void* workspace, size_t workspace_bytes,
                       attn_stream_t stream_) {
-  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr ||
-      seq_lens == nullptr || o == nullptr)
-    return ATTN_ERR_INVALID_ARG;
-  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || max_pages_per_seq < 1 || num_pages < 1 ||
-      page_size < 1)
-    return ATTN_ERR_INVALID_ARG;
-  if (B > 65535 || Hkv > 65535 || (long long)max_pages_per_seq * page_size > (1ll << 30))
-    return ATTN_ERR_INVALID_ARG;
-  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  if (page_size % 16 != 0 || page_size > 256) return ATTN_ERR_UNSUPPORTED;
-  if (Hq / Hkv > 8) return ATTN_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
-      !aligned4(block_table) || !aligned4(seq_lens) || (lse != nullptr && !aligned4(lse)))
-    return ATTN_ERR_ALIGNMENT;
-  const size_t need = attn_decode_workspace_size(B, Hq, max_pages_per_seq, page_size, d);
-  if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
+  return decode_paged_common(false, q, k_cache, v_cache, nullptr, nullptr, block_table, seq_lens,
+                             page_size, B, Hq, Hkv, d, max_pages_per_seq, num_pages, scale, o,
+                             lse, workspace, workspace_bytes, stream_);
+}
 
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  const long long tokens = (long long)max_pages_per_seq * page_size;
-  DecodeParams prm;
-  prm.q = static_cast<const uint16_t*>(q);
-  prm.k_cache = static_cast<const uint16_t*>(k_cache);
-  prm.v_cache = static_cast<const uint16_t*>(v_cache);
-  prm.block_table = block_table;
-  prm.seq_lens = seq_lens;
-  prm.B = B;
-  prm.Hq = Hq;
-  prm.Hkv = Hkv;
-  prm.group = Hq / Hkv;
-  prm.page_size = page_size;
-  prm.max_pages = max_pages_per_seq;
-  prm.num_pages = num_pages;
-  prm.n_split = (int)((tokens + kSplitTokens - 1) / kSplitTokens);
-  prm.scale_log2 = scale * 1.4426950408889634f;
-  const size_t parts = (size_t)B * Hq * prm.n_split;
-  prm.o_part = static_cast<float*>(workspace);
-  prm.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + parts * d * sizeof(float));
-  prm.o = static_cast<uint16_t*>(o);
-  prm.lse = lse;
-
-  dim3 grid_split((prm.n_split + 3) / 4, Hkv, B);
-  dim3 grid_merge((unsigned)(((long long)B * Hq + 3) / 4));
-  if (d == 128) {
-    attn_decode_split_kernel<128><<<grid_split, 128, 0, stream>>>(prm);
-    attn_decode_merge_kernel<128><<<grid_merge, 128, 0, stream>>>(prm);
-  } else {
-    attn_decode_split_kernel<64><<<grid_split, 128, 0, stream>>>(prm);
-    attn_decode_merge_kernel<64><<<grid_merge, 128, 0, stream>>>(prm);
-  }
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+int attn_decode_paged_fp8(const void* q, const void* k_cache, const void* v_cache,
+                          const float* k_scale, const float* v_scale, const int32_t* block_table,
+                          const int32_t* seq_lens, int page_size, int B, int Hq, int Hkv, int d,
+                          int max_pages_per_seq, int num_pages, float scale, void* o, float* lse,
+                          void* workspace, size_t workspace_bytes, attn_stream_t stream_) {
+  if (k_scale == nullptr || v_scale == nullptr) return ATTN_ERR_INVALID_ARG;
+  return decode_paged_common(true, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens,
+                             page_size, B, Hq, Hkv, d, max_pages_per_seq, num_pages, scale, o,
+                             lse, workspace, workspace_bytes, stream_);
 }
 
 int attn_get_device_error(attn_stream_t stream_, unsigned int* flags_out) {

@@ -311,6 +311,35 @@ int attn_decode_paged_noalloc(const void* q, const void* k_cache, const void* v_
                               float scale, void* o, float* lse, attn_stream_t stream);
 
 /*
+ * attn_decode_paged_fp8 -- attn_decode_paged over an FP8 (E4M3) KV cache
+ * with one scale per (physical page, KV head).
+ * Source: "Attention Kernel", sections "Paged 与 ragged KV" and "正确性契约"
+ * (the cache quantisation schema is part of the kernel contract, with the
+ * page size, block table and valid-token counts); "Attention 算子加速史",
+ * section 3 (FP8 operands with scale factors) and section 4 (paged decode).
+ *
+ *   k_cache, v_cache  [num_pages, page_size, Hkv, d] uint8: OCP E4M3 codes
+ *                     (bias 7, 3 mantissa bits, subnormals; 0x7F/0xFF are
+ *                     NaN and must not occur)
+ *   k_scale, v_scale  [num_pages, Hkv] fp32 device arrays: the cache element
+ *                     K[page, r, h, i] is k_scale[page, h] * e4m3(code), V
+ *                     likewise (finite scales; any sign)
+ *   The attention computed is attn_decode_paged's over those dequantised
+ *   values.  The kernel widens the codes exactly (to bf16 for q K^T, to f16
+ *   for P V with P rounded to f16), applies the K scale to the fp32 scores
+ *   and the V scale to each page's fp32 partial output.
+ * Other arguments, workspace (attn_decode_workspace_size), device-side
+ * checks and errors as attn_decode_paged; INVALID_ARG also for a NULL scale
+ * array, ALIGNMENT when a scale array is not 4-byte aligned (the caches need
+ * 16 bytes).
+ */
+int attn_decode_paged_fp8(const void* q, const void* k_cache, const void* v_cache,
+                          const float* k_scale, const float* v_scale, const int32_t* block_table,
+                          const int32_t* seq_lens, int page_size, int B, int Hq, int Hkv, int d,
+                          int max_pages_per_seq, int num_pages, float scale, void* o, float* lse,
+                          void* workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
  * attn_bwd_workspace_size -- bytes of device workspace attn_bwd needs:
  * 8 * B * Hq * ceil(Sq / 128) * 128 (two fp32 row statistics per query row,
  * padded to whole 128-row tiles).  0 for invalid arguments.

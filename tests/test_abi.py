@@ -31,7 +31,7 @@ def test_header_declares_expected_entry_points():
     for n in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_fwd_varlen_workspace_size",
               "attn_fwd_paged", "attn_fwd_window", "attn_fwd_block_sparse",
               "attn_decode_paged", "attn_decode_workspace_size", "attn_get_device_error",
-              "attn_bwd", "attn_bwd_workspace_size", "attn_strerror"):
+              "attn_bwd", "attn_bwd_workspace_size", "attn_decode_paged_fp8", "attn_strerror"):
         assert n in names
 
 
@@ -215,6 +215,32 @@ def test_workspace_size_formula(lib):
     assert got >= parts * d * 4 + parts * 4
     assert got <= parts * d * 4 + parts * 4 + 256
     assert lib.attn_decode_workspace_size(0, 1, 1, 16, 128) == 0
+
+
+def _dec8(lib, q=FAKE, kc=FAKE, vc=FAKE, ks=FAKE, vs=FAKE, tbl=FAKE, lens=FAKE, ps=16, B_=2, Hq=8,
+          Hkv=2, d=128, maxp=4, npages=8, scale=0.1, o=FAKE, lse=None, ws=FAKE, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = lib.attn_decode_workspace_size(B_, Hq, maxp, ps, d) if B_ > 0 else 0
+    return lib.attn_decode_paged_fp8(q, kc, vc, ks, vs, tbl, lens, ps, B_, Hq, Hkv, d, maxp,
+                                     npages, scale, o, lse, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(ks=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(vs=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(q=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(kc=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), B.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), B.ATTN_ERR_INVALID_ARG),
+    (dict(ps=8), B.ATTN_ERR_UNSUPPORTED),
+    (dict(d=96), B.ATTN_ERR_UNSUPPORTED),
+    (dict(kc=FAKE + 8), B.ATTN_ERR_ALIGNMENT),
+    (dict(vs=FAKE + 2), B.ATTN_ERR_ALIGNMENT),
+    (dict(ks=FAKE + 1), B.ATTN_ERR_ALIGNMENT),
+    (dict(ws_bytes=16), B.ATTN_ERR_WORKSPACE),
+])
+def test_decode_fp8_validation(lib, kw, status):
+    assert _dec8(lib, **kw) == status
 
 
 def _bwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, do=FAKE, dq=FAKE, dk=FAKE, dv=FAKE,
