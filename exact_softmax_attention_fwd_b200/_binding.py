@@ -112,6 +112,19 @@ def _check(status, what):
         raise AttnError(status, what)
 
 
+def _out(t, shape, dtype, device, name):
+    """A caller-supplied output buffer, checked against what the kernels write
+    (shape, dtype, contiguity, device), or a new one when ``t`` is None."""
+    import torch
+    if t is None:
+        return torch.empty(tuple(shape), dtype=dtype, device=device)
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}")
+    return t
+
+
 def _require_cuda(*tensors):
     for t in tensors:
         if t is not None and not t.is_cuda:
@@ -132,10 +145,9 @@ def attn_fwd_masked(q, k, v, causal: bool, scale: float, k_lens=None, out=None, 
         raise ValueError("q/k/v shapes disagree")
     if k_lens is not None and (k_lens.dtype != torch.int32 or tuple(k_lens.shape) != (B,)):
         raise ValueError("k_lens must be int32 [B]")
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None and return_lse:
-        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    out = _out(out, q.shape, torch.bfloat16, q.device, "out")
+    if lse is not None or return_lse:
+        lse = _out(lse, (B, Hq, Sq), torch.float32, q.device, "lse")
     st = load_library().attn_fwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq,
                                         Hkv, Sq, Sk, d, int(bool(causal)), float(scale),
                                         _ptr(k_lens), _stream(stream))
@@ -164,10 +176,9 @@ def attn_fwd_window(q, k, v, scale: float, window: int = 0, prefix: int = 0, k_l
         raise ValueError("q/k/v shapes disagree")
     if k_lens is not None and (k_lens.dtype != torch.int32 or tuple(k_lens.shape) != (B,)):
         raise ValueError("k_lens must be int32 [B]")
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None and return_lse:
-        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    out = _out(out, q.shape, torch.bfloat16, q.device, "out")
+    if lse is not None or return_lse:
+        lse = _out(lse, (B, Hq, Sq), torch.float32, q.device, "lse")
     st = load_library().attn_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq,
                                         Hkv, Sq, Sk, d, float(scale), _ptr(k_lens), int(window),
                                         int(prefix), _stream(stream))
@@ -194,10 +205,9 @@ def attn_fwd_block_sparse(q, k, v, block_mask, causal: bool, scale: float, k_len
         raise ValueError("block_mask must be contiguous uint8 [B, 1 or Hq, ceil(Sq/128), ceil(Sk/128)]")
     if k_lens is not None and (k_lens.dtype != torch.int32 or tuple(k_lens.shape) != (B,)):
         raise ValueError("k_lens must be int32 [B]")
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None and return_lse:
-        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    out = _out(out, q.shape, torch.bfloat16, q.device, "out")
+    if lse is not None or return_lse:
+        lse = _out(lse, (B, Hq, Sq), torch.float32, q.device, "lse")
     st = load_library().attn_fwd_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B,
                                               Hq, Hkv, Sq, Sk, d, int(bool(causal)), float(scale),
                                               _ptr(k_lens), _ptr(block_mask), block_mask.shape[1],
@@ -229,9 +239,9 @@ def attn_bwd(q, k, v, o, lse, d_o, causal: bool, scale: float, k_lens=None, dq=N
         raise ValueError("lse must be contiguous float32 [B, Hq, Sq]")
     if k_lens is not None and (k_lens.dtype != torch.int32 or tuple(k_lens.shape) != (B,)):
         raise ValueError("k_lens must be int32 [B]")
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
+    dq = _out(dq, q.shape, torch.bfloat16, q.device, "dq")
+    dk = _out(dk, k.shape, torch.bfloat16, q.device, "dk")
+    dv = _out(dv, v.shape, torch.bfloat16, q.device, "dv")
     need = attn_bwd_workspace_size(B, Hq, Sq)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
@@ -271,10 +281,9 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, caus
     need = attn_fwd_varlen_workspace_size(B, total_q, max_seqlen_q)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None and return_lse:
-        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    out = _out(out, q.shape, torch.bfloat16, q.device, "out")
+    if lse is not None or return_lse:
+        lse = _out(lse, (Hq, total_q), torch.float32, q.device, "lse")
     ws_bytes = workspace.numel() * workspace.element_size()
     st = load_library().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
                                         _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, Hq, Hkv,
@@ -311,10 +320,9 @@ def attn_fwd_paged(q, k_cache, v_cache, block_table, cu_seqlens_q, seq_lens_k, m
     need = attn_fwd_varlen_workspace_size(B, total_q, max_seqlen_q)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None and return_lse:
-        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    out = _out(out, q.shape, torch.bfloat16, q.device, "out")
+    if lse is not None or return_lse:
+        lse = _out(lse, (Hq, total_q), torch.float32, q.device, "lse")
     ws_bytes = workspace.numel() * workspace.element_size()
     st = load_library().attn_fwd_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
                                        _ptr(cu_seqlens_q), _ptr(seq_lens_k), page_size, B, Hq,
@@ -350,10 +358,9 @@ def attn_decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float, 
     need = attn_decode_workspace_size(B, Hq, max_pages, page_size, d)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    if out is None:
-        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
-    if lse is None and return_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    out = _out(out, (B, Hq, d), torch.bfloat16, q.device, "out")
+    if lse is not None or return_lse:
+        lse = _out(lse, (B, Hq), torch.float32, q.device, "lse")
     ws_bytes = workspace.numel() * workspace.element_size()
     st = load_library().attn_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
                                           _ptr(seq_lens), page_size, B, Hq, Hkv, d, max_pages,
@@ -390,10 +397,9 @@ def attn_decode_paged_fp8(q, k_cache, v_cache, k_scale, v_scale, block_table, se
     need = attn_decode_workspace_size(B, Hq, max_pages, page_size, d)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    if out is None:
-        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
-    if lse is None and return_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    out = _out(out, (B, Hq, d), torch.bfloat16, q.device, "out")
+    if lse is not None or return_lse:
+        lse = _out(lse, (B, Hq), torch.float32, q.device, "lse")
     ws_bytes = workspace.numel() * workspace.element_size()
     st = load_library().attn_decode_paged_fp8(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_table),
@@ -431,10 +437,9 @@ def attn_decode_paged_noalloc(q, k_cache, v_cache, block_table, seq_lens, scale,
     for t in (q, k_cache, v_cache, block_table, seq_lens):
         if not t.is_contiguous():
             raise ValueError("inputs must be contiguous")
-    if out is None:
-        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
-    if lse is None and return_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    out = _out(out, (B, Hq, d), torch.bfloat16, q.device, "out")
+    if lse is not None or return_lse:
+        lse = _out(lse, (B, Hq), torch.float32, q.device, "lse")
     st = load_library().attn_decode_paged_noalloc(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens), page_size, B,
         Hq, Hkv, d, block_table.shape[1], num_pages, float(scale), _ptr(out), _ptr(lse),

@@ -287,3 +287,17 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         B.attn_fwd(q, q, q, False, 0.1)
+
+
+def test_binding_checks_caller_output_buffers():
+    import torch
+    cpu = torch.device("cpu")
+    good = torch.empty((2, 3, 4), dtype=torch.bfloat16)
+    assert B._out(good, (2, 3, 4), torch.bfloat16, cpu, "out") is good
+    fresh = B._out(None, (2, 3), torch.float32, cpu, "lse")
+    assert tuple(fresh.shape) == (2, 3) and fresh.dtype == torch.float32
+    for bad in (torch.empty((2, 3, 5), dtype=torch.bfloat16),      # too small a row
+                torch.empty((2, 3, 4), dtype=torch.float16),       # wrong dtype
+                torch.empty((2, 4, 3), dtype=torch.bfloat16).transpose(1, 2)):  # not contiguous
+        with pytest.raises(ValueError):
+            B._out(bad, (2, 3, 4), torch.bfloat16, cpu, "out")
