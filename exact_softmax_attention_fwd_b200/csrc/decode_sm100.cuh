@@ -23,16 +23,17 @@
 // The next 16 tokens' K (V) are requested as soon as the current K (V)
 // registers are consumed, so loads overlap the softmax and the other MMA.
 //
-// FP8 cache (attn_decode_split_fp8_kernel; "Attention Kernel", section "正确性契约": the cache quantisation
-// schema is part of the contract; "Attention 算子加速史", section 3: FP8
-// operands with scale factors): K and V may be stored as E4M3 bytes with one
-// fp32 scale per (physical page, KV head).  The kernel then streams half the
-// bytes, keeps the raw bytes in the prefetch registers and widens them right
-// before use: K to bf16 (exact: E4M3 has 3 mantissa bits) for the q K^T MMA,
-// whose fp32 scores are multiplied by the page's K scale; V to f16 (exact)
-// for an f16 P^T V MMA (P <= 1 is rounded to f16), whose fp32 result for the
-// 16 tokens -- which always lie in one page -- is multiplied by the page's V
-// scale before it joins the accumulator.
+// FP8 cache (attn_decode_split_fp8_kernel; "Attention Kernel", section
+// "正确性契约": the cache quantisation schema is part of the contract;
+// "Attention 算子加速史", section 3: FP8 operands with scale factors): K and V
+// may be stored as E4M3 bytes with one fp32 scale per (physical page, KV
+// head).  The kernel then streams half the bytes, keeps the raw bytes in the
+// prefetch registers and widens them to f16 right before use (exact: E4M3 has
+// 3 mantissa bits and a narrower exponent range).  q K^T is an f16 MMA on q
+// scaled by a power of two into f16's range; its fp32 scores are multiplied
+// back and by the page's K scale.  P^T V is an f16 MMA (P <= 1 is rounded to
+// f16) whose fp32 result for the 16 tokens -- which always lie in one page --
+// is multiplied by the page's V scale before it joins the accumulator.
 //
 // Merge kernel: one warp per (b, query head) combines the splits in a fixed
 // order: LSE = M + log2 sum_s 2^(lse_s - M), O = sum_s 2^(lse_s - LSE) o_s,
