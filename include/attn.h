@@ -325,9 +325,11 @@ int attn_decode_paged_noalloc(const void* q, const void* k_cache, const void* v_
  *                     K[page, r, h, i] is k_scale[page, h] * e4m3(code), V
  *                     likewise (finite scales; any sign)
  *   The attention computed is attn_decode_paged's over those dequantised
- *   values.  The kernel widens the codes exactly (to bf16 for q K^T, to f16
- *   for P V with P rounded to f16), applies the K scale to the fp32 scores
- *   and the V scale to each page's fp32 partial output.
+ *   values.  The kernel widens the codes exactly to f16 for two f16 MMAs:
+ *   q K^T with q multiplied by a power of two into f16's range (exact for bf16
+ *   q down to f16's subnormals), and P V with P rounded to f16; the K scale
+ *   (and that power of two) multiply the fp32 scores, the V scale each page's
+ *   fp32 partial output.
  * Other arguments, workspace (attn_decode_workspace_size), device-side
  * checks and errors as attn_decode_paged; INVALID_ARG also for a NULL scale
  * array, ALIGNMENT when a scale array is not 4-byte aligned (the caches need
