@@ -21,11 +21,20 @@ Sources (page title, section):
   * "Attention Kernel" -- "问题与成本" and "Online softmax" (the attention
     itself, and the zero output / -inf LSE of a row with no key).
 
+``attn_fwd_fp8`` states prefill over E4M3 Q, K and V with block scaling
+("Attention 算子加速史", section 3: FlashAttention-3 pairs FP8 with block-level
+adaptive scaling; the pages give no block shape): one fp32 scale per (batch,
+head, block of 128 consecutive rows) of each tensor, value = scale * e4m3(code),
+then exact masked attention of the dequantised values (the masking rules of
+the bf16 prefill: key lengths, bottom-right causal alignment, zero output and
+-inf LSE for a row with no visible key).
+
 Pinned in ``tests/test_oracle_fp8_pins.py``: the E4M3 decoding against torch's
-float8_e4m3fn for all 256 codes; with unit scales and codes whose values are
-exact in bf16, against the C bf16 decode oracle on the same values; scale
-laws (V scale scales O, K scale acts as the softmax scale); per-page scales
-applied to the right pages.
+float8_e4m3fn for all 256 codes; with power-of-two scales, whose dequantised
+values are exact in bf16, against the C bf16 decode and prefill oracles on
+those values; scale laws (a V scale scales O, a K scale acts as the softmax
+scale); per-page scales applied to the right pages and a block scale confined
+to its 128 rows.
 """
 from __future__ import annotations
 
@@ -102,4 +111,54 @@ def decode_paged_fp8(q, k_bytes, v_bytes, k_scale, v_scale, block_table, seq_len
             w = np.exp(s - mx)
             o[b, hq] = (w @ vv) / w.sum()
             lse[b, hq] = mx + np.log(w.sum())
+    return o, lse
+
+
+def dequantize_blocks(codes, scales, block: int = 128) -> np.ndarray:
+    """[B, H, S, d] E4M3 bytes and [B, H, ceil(S/block)] scales -> float64 values."""
+    vals = e4m3_to_float(np.asarray(codes, dtype=np.uint8))
+    sc = np.asarray(scales, dtype=np.float64)
+    S = vals.shape[2]
+    if sc.shape != vals.shape[:2] + (-(-S // block),):
+        raise ValueError("scales must be [B, H, ceil(S / block)]")
+    return vals * np.repeat(sc, block, axis=2)[:, :, :S, None]
+
+
+def attn_fwd_fp8(q_codes, k_codes, v_codes, q_scale, k_scale, v_scale, causal, scale,
+                 k_lens=None):
+    """Prefill over block-scaled E4M3 inputs, float64.
+
+    q_codes [B, Hq, Sq, d], k_codes / v_codes [B, Hkv, Sk, d] uint8; scales
+    [B, H, ceil(S/128)] for each tensor.  Key j is visible to row i iff
+    j < k_len and (causal => j <= i + k_len - Sq).  Returns (o [B, Hq, Sq, d],
+    lse [B, Hq, Sq]).
+    """
+    def arr(x):
+        return np.asarray(x.cpu().numpy() if hasattr(x, "cpu") else x)
+    Q = dequantize_blocks(arr(q_codes), arr(q_scale))
+    K = dequantize_blocks(arr(k_codes), arr(k_scale))
+    V = dequantize_blocks(arr(v_codes), arr(v_scale))
+    B, Hq, Sq, d = Q.shape
+    _, Hkv, Sk, _ = K.shape
+    if K.shape != V.shape or K.shape[0] != B or K.shape[3] != d or Hq % Hkv:
+        raise ValueError("q/k/v shapes disagree")
+    g = Hq // Hkv
+    o = np.zeros((B, Hq, Sq, d))
+    lse = np.full((B, Hq, Sq), -np.inf)
+    i = np.arange(Sq)[:, None]
+    j = np.arange(Sk)[None, :]
+    for b in range(B):
+        kl = Sk if k_lens is None else int(arr(k_lens)[b])
+        vis = j < kl
+        if causal:
+            vis = vis & (j <= i + (kl - Sq))
+        live = vis.any(axis=1)
+        for hq in range(Hq):
+            s = np.where(vis, scale * (Q[b, hq] @ K[b, hq // g].T), -np.inf)
+            m = np.where(live, s.max(axis=1), 0.0)
+            w = np.where(vis, np.exp(s - m[:, None]), 0.0)
+            den = w.sum(axis=1)
+            den_safe = np.where(live, den, 1.0)
+            o[b, hq] = np.where(live[:, None], (w @ V[b, hq // g]) / den_safe[:, None], 0.0)
+            lse[b, hq] = np.where(live, m + np.log(den_safe), -np.inf)
     return o, lse

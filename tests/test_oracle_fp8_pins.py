@@ -52,8 +52,10 @@ def test_fp8_decode_equals_bf16_oracle_on_exact_values(page_size, d, Hq, Hkv):
     # powers of two keep k_scale * e4m3 exact in bf16 (3 mantissa bits)
     ks = torch.pow(2.0, torch.randint(-4, 3, (P, Hkv), generator=gen).double()).float()
     vs = torch.pow(2.0, torch.randint(-4, 3, (P, Hkv), generator=gen).double()).float()
-    kd = torch.from_numpy(dequantize(k8.numpy(), ks.numpy())).to(torch.bfloat16)
-    vd = torch.from_numpy(dequantize(v8.numpy(), vs.numpy())).to(torch.bfloat16)
+    # the bf16 reference cache, dequantised independently of the oracle (torch's
+    # float8 decode, scales broadcast per page and head)
+    kd = (k8.view(torch.float8_e4m3fn).double() * ks.double()[:, None, :, None]).to(torch.bfloat16)
+    vd = (v8.view(torch.float8_e4m3fn).double() * vs.double()[:, None, :, None]).to(torch.bfloat16)
     np.testing.assert_array_equal(kd.double().numpy(), dequantize(k8.numpy(), ks.numpy()))
     scale = 0.03
     o, lse = decode_paged_fp8(base.q, k8, v8, ks, vs, base.block_table, lens, scale)
@@ -90,3 +92,67 @@ def test_fp8_generator_roundtrip_error_is_within_e4m3_rounding():
     bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * sc.numpy()[:, None, :, None])
     assert (err <= bound * (1 + 1e-12)).all()
     assert np.abs(back).max() <= 448.0 * float(sc.double().max()) * (1 + 1e-12)
+
+
+# --------------------------------------------------------------------------- block-scaled prefill
+
+from oracle.kv_fp8 import attn_fwd_fp8, dequantize_blocks  # noqa: E402
+
+
+def _codes(shape, gen):
+    return _random_codes(shape, gen)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,d,causal,k_lens", [
+    (1, 2, 1, 200, 300, 64, True, None),
+    (2, 4, 2, 130, 130, 64, False, [130, 90]),
+    (1, 2, 2, 300, 150, 128, True, [150]),        # Sq > Sk: leading rows see no key
+])
+def test_fp8_prefill_equals_bf16_oracle_on_exact_values(B, Hq, Hkv, Sq, Sk, d, causal, k_lens):
+    gen = torch.Generator().manual_seed(51)
+    q8 = _codes((B, Hq, Sq, d), gen)
+    k8 = _codes((B, Hkv, Sk, d), gen)
+    v8 = _codes((B, Hkv, Sk, d), gen)
+
+    def p2(shape):  # power-of-two block scales: dequantised values exact in bf16
+        return torch.pow(2.0, torch.randint(-6, 1, shape, generator=gen).double()).float()
+
+    qs, ks, vs = p2((B, Hq, -(-Sq // 128))), p2((B, Hkv, -(-Sk // 128))), p2((B, Hkv, -(-Sk // 128)))
+    def deq(codes, sc):  # independent of the oracle: torch's float8 decode, rows of 128
+        rows = sc.double().repeat_interleave(128, dim=2)[:, :, :codes.shape[2], None]
+        return (codes.view(torch.float8_e4m3fn).double() * rows).to(torch.bfloat16)
+
+    Q, K, V = deq(q8, qs), deq(k8, ks), deq(v8, vs)
+    np.testing.assert_array_equal(Q.double().numpy(), dequantize_blocks(q8.numpy(), qs.numpy()))
+    scale = 0.02
+    o, lse = attn_fwd_fp8(q8, k8, v8, qs, ks, vs, causal, scale, k_lens=k_lens)
+    o_ref, lse_ref = oracle.attn_fwd(Q, K, V, causal, scale, k_lens=k_lens)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-10)
+    assert np.array_equal(np.isneginf(lse), np.isneginf(lse_ref))
+    fin = np.isfinite(lse_ref)
+    np.testing.assert_allclose(lse[fin], lse_ref[fin], rtol=0, atol=1e-10)
+
+
+def test_fp8_prefill_scale_laws_and_block_locality():
+    gen = torch.Generator().manual_seed(52)
+    B, H, S, d = 1, 2, 260, 64
+    q8, k8, v8 = _codes((B, H, S, d), gen), _codes((B, H, S, d), gen), _codes((B, H, S, d), gen)
+    nb = -(-S // 128)
+    one = torch.ones((B, H, nb))
+    o, lse = attn_fwd_fp8(q8, k8, v8, one * 0.01, one * 0.01, one, True, 0.5)
+    # V scale x 4 scales O; a uniform K scale x 2 is the softmax scale x 2
+    o2, lse2 = attn_fwd_fp8(q8, k8, v8, one * 0.01, one * 0.01, one * 4.0, True, 0.5)
+    np.testing.assert_allclose(o2, 4.0 * o, rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(lse2, lse)
+    o3, lse3 = attn_fwd_fp8(q8, k8, v8, one * 0.01, one * 0.02, one, True, 0.25)
+    np.testing.assert_allclose(o3, o, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse3, lse, rtol=1e-12, atol=1e-12)
+    # a Q scale change in one block of head 0 moves only that block's rows
+    for blk, lo, hi in ((0, 0, 128), (2, 256, S)):
+        qs = (one * 0.01).clone()
+        qs[0, 0, blk] *= 2.0
+        o4, _ = attn_fwd_fp8(q8, k8, v8, qs, one * 0.01, one, True, 0.5)
+        changed = np.abs(o4 - o).max(axis=-1) > 0
+        assert changed[0, 0, max(lo, 1):hi].all()  # causal row 0 sees only key 0: O = v0
+        assert not changed[0, 0, :lo].any() and not changed[0, 0, hi:].any()
+        assert not changed[0, 1].any()
