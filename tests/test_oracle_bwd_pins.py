@@ -9,7 +9,10 @@ other than itself:
   dQ = 0; the key-sum of dK is 0 (softmax is blind to a shift shared by every
   key); the column sums of dV equal the sums of dO over rows that see a key;
   the causal first row has dQ = 0; scale 0 gives dQ = dK = 0 and dV as the
-  visible-count-weighted sum of dO; padded keys get no gradient.
+  visible-count-weighted sum of dO; padded keys get no gradient;
+* sliding-window, prefix-LM and per-head block masks, and a ragged batch as
+  one packed sequence under its document (block-diagonal) mask, against float64
+  autograd through SDPA with masks written element by element in the test.
 """
 import numpy as np
 import pytest
@@ -179,3 +182,103 @@ def test_bwd_accepts_bf16_bits():
     b = attn_bwd(*bits, True, 0.5)
     for x, y in zip(a, b):
         np.testing.assert_array_equal(x, y)
+
+
+# --------------------------------------------------------------------------- masks and ragged batches
+
+from oracle.attn_bwd import attn_bwd_varlen  # noqa: E402
+
+
+def _sdpa_masked(q, k, v, scale, mask):
+    """float64 SDPA with an explicit boolean mask [B or 1, Hq or 1, Sq, Sk] (GQA by
+    repeating K/V); every row must see a key."""
+    g = q.shape[1] // k.shape[1]
+    return F.scaled_dot_product_attention(q, k.repeat_interleave(g, 1), v.repeat_interleave(g, 1),
+                                          attn_mask=mask, scale=scale)
+
+
+def _rule_mask(Sq, Sk, window=0, prefix=0, block=None):
+    """The causal visibility rule written element by element (independently of
+    the oracle's vectorised form): row i sits at key position p = i + Sk - Sq
+    and sees key j iff j <= p and, with a window w, p - j < w; with a prefix P,
+    also every j < P; a block mask entry 0 hides (i // 128, j // 128)."""
+    m = torch.zeros((Sq, Sk), dtype=torch.bool)
+    for i in range(Sq):
+        p = i + Sk - Sq
+        for j in range(Sk):
+            ok = j <= p and (window == 0 or p - j < window)
+            if prefix > 0 and j < prefix:
+                ok = True
+            if block is not None and not block[i // 128][j // 128]:
+                ok = False
+            m[i, j] = ok
+    return m
+
+
+def _grads_autograd(q, k, v, do, scale, mask):
+    q, k, v = (x.clone().requires_grad_() for x in (q, k, v))
+    (_sdpa_masked(q, k, v, scale, mask) * do).sum().backward()
+    return q.grad.numpy(), k.grad.numpy(), v.grad.numpy()
+
+
+@pytest.mark.parametrize("Sq,Sk,window,prefix", [(9, 9, 3, 0), (6, 11, 4, 0), (10, 10, 0, 3),
+                                                   (7, 12, 0, 8)])
+def test_bwd_window_and_prefix_match_autograd(Sq, Sk, window, prefix):
+    gen = torch.Generator().manual_seed(19)
+    B, Hq, Hkv, d = 1, 4, 2, 3
+    q, k, v = _rand((B, Hq, Sq, d), gen), _rand((B, Hkv, Sk, d), gen), _rand((B, Hkv, Sk, d), gen)
+    do = _rand((B, Hq, Sq, d), gen)
+    mask = _rule_mask(Sq, Sk, window, prefix)[None, None]
+    ref = _grads_autograd(q, k, v, do, 0.6, mask)
+    got = attn_bwd(q, k, v, do, True, 0.6, window=window, prefix=prefix)
+    for x, y in zip(got, ref):
+        np.testing.assert_allclose(x, y, rtol=0, atol=1e-10)
+
+
+def test_bwd_block_mask_matches_autograd():
+    """A per-head 128 x 128 block mask on 300 x 300 causal problems (every row
+    keeps its diagonal block, so each row sees a key)."""
+    gen = torch.Generator().manual_seed(20)
+    B, Hq, Hkv, S, d = 1, 2, 1, 300, 4
+    q, k, v = _rand((B, Hq, S, d), gen), _rand((B, Hkv, S, d), gen), _rand((B, Hkv, S, d), gen)
+    do = _rand((B, Hq, S, d), gen)
+    bm = np.ones((B, Hq, 3, 3), np.uint8)
+    bm[0, 0, 2, 0] = 0
+    bm[0, 1, 1, 0] = 0
+    bm[0, 1, 2, 1] = 0
+    mask = torch.stack([_rule_mask(S, S, block=bm[0, h]) for h in range(Hq)])
+    ref = _grads_autograd(q, k, v, do, 0.5, mask[None])
+    got = attn_bwd(q, k, v, do, True, 0.5, block_mask=bm)
+    for x, y in zip(got, ref):
+        np.testing.assert_allclose(x, y, rtol=0, atol=1e-10)
+    # an all-ones mask is no mask
+    ones = attn_bwd(q, k, v, do, True, 0.5, block_mask=np.ones_like(bm))
+    plain = attn_bwd(q, k, v, do, True, 0.5)
+    for x, y in zip(ones, plain):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_bwd_ragged_batch_is_the_document_masked_packed_sequence():
+    """A ragged batch differentiated per sequence equals autograd of one packed
+    sequence under the block-diagonal (document) mask with bottom-right causal
+    alignment inside each document."""
+    gen = torch.Generator().manual_seed(21)
+    lq, lk = [3, 5, 2], [3, 7, 4]
+    Hq, Hkv, d = 2, 1, 3
+    cq = np.concatenate([[0], np.cumsum(lq)])
+    ck = np.concatenate([[0], np.cumsum(lk)])
+    q, do = _rand((cq[-1], Hq, d), gen), _rand((cq[-1], Hq, d), gen)
+    k, v = _rand((ck[-1], Hkv, d), gen), _rand((ck[-1], Hkv, d), gen)
+    got = attn_bwd_varlen(q, k, v, do, cq, ck, True, 0.7)
+    mask = np.zeros((cq[-1], ck[-1]), bool)
+    for b in range(len(lq)):
+        mask[cq[b]:cq[b + 1], ck[b]:ck[b + 1]] = _rule_mask(lq[b], lk[b]).numpy()
+    pk = lambda x: x.permute(1, 0, 2)[None]  # packed [T, H, d] -> [1, H, T, d]
+    ref = _grads_autograd(pk(q), pk(k), pk(v), pk(do), 0.7, torch.from_numpy(mask)[None, None])
+    for x, y in zip(got, ref):
+        np.testing.assert_allclose(x, y[0].transpose(1, 0, 2), rtol=0, atol=1e-10)
+    # a sequence with no keys contributes nothing and receives nothing
+    ck2 = ck.copy()
+    ck2[1:] = ck[1:] - ck[1]  # sequence 0 keeps 0 keys; the others shift down
+    g0 = attn_bwd_varlen(q, k[:ck2[-1]], v[:ck2[-1]], do, cq, ck2, True, 0.7)
+    assert not g0[0][:cq[1]].any()
