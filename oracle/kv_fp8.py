@@ -34,7 +34,9 @@ float8_e4m3fn for all 256 codes; with power-of-two scales, whose dequantised
 values are exact in bf16, against the C bf16 decode and prefill oracles on
 those values; scale laws (a V scale scales O, a K scale acts as the softmax
 scale); per-page scales applied to the right pages and a block scale confined
-to its 128 rows.
+to its 128 rows.  ``attn_fwd_paged_fp8`` (queries appended to an E4M3 paged
+cache) is pinned against the C paged-prefill oracle the same way and, with one
+query per sequence, against ``decode_paged_fp8``.
 """
 from __future__ import annotations
 
@@ -161,4 +163,50 @@ def attn_fwd_fp8(q_codes, k_codes, v_codes, q_scale, k_scale, v_scale, causal, s
             den_safe = np.where(live, den, 1.0)
             o[b, hq] = np.where(live[:, None], (w @ V[b, hq // g]) / den_safe[:, None], 0.0)
             lse[b, hq] = np.where(live, m + np.log(den_safe), -np.inf)
+    return o, lse
+
+
+def attn_fwd_paged_fp8(q, k_bytes, v_bytes, k_scale, v_scale, block_table, cu_seqlens_q,
+                       seq_lens_k, causal, scale):
+    """Packed queries appended to an E4M3 paged cache (per-(page, KV head) scales).
+
+    q [total_q, Hq, d] (bf16 tensor or floats); caches and scales as in
+    ``decode_paged_fp8``; cu_seqlens_q [B + 1]; seq_lens_k [B].  Key token t of
+    sequence b is the dequantised row (block_table[b][t // page_size],
+    t % page_size); the sequence's len_q queries are its last len_q positions
+    (bottom-right causal rule).  Returns (o [total_q, Hq, d], lse [Hq, total_q])
+    float64; a sequence with no key gives o = 0, lse = -inf.
+    """
+    def arr(x):
+        return np.asarray(x.cpu().numpy() if hasattr(x, "cpu") else x)
+    Q = _f64(q)
+    K = dequantize(arr(k_bytes), arr(k_scale))
+    V = dequantize(arr(v_bytes), arr(v_scale))
+    tbl, cq, lens = arr(block_table), arr(cu_seqlens_q), arr(seq_lens_k)
+    num_pages, page_size, Hkv, d = K.shape
+    total_q, Hq, _ = Q.shape
+    g = Hq // Hkv
+    o = np.zeros((total_q, Hq, d))
+    lse = np.full((Hq, total_q), -np.inf)
+    for b in range(len(lens)):
+        qa, qe, n = int(cq[b]), int(cq[b + 1]), int(lens[b])
+        lq = qe - qa
+        if lq == 0 or n == 0:
+            continue
+        t = np.arange(n)
+        pages = tbl[b, t // page_size]
+        if (pages < 0).any() or (pages >= num_pages).any():
+            raise ValueError("block table entry out of range")
+        kk, vv = K[pages, t % page_size], V[pages, t % page_size]  # [n, Hkv, d]
+        i = np.arange(lq)[:, None]
+        j = np.arange(n)[None, :]
+        vis = (j <= i + (n - lq)) if causal else np.ones((lq, n), bool)
+        live = vis.any(axis=1)
+        for hq in range(Hq):
+            s_ = np.where(vis, scale * (Q[qa:qe, hq] @ kk[:, hq // g].T), -np.inf)
+            m = np.where(live, s_.max(axis=1), 0.0)
+            w = np.where(vis, np.exp(s_ - m[:, None]), 0.0)
+            den = np.where(live, w.sum(axis=1), 1.0)
+            o[qa:qe, hq] = np.where(live[:, None], (w @ vv[:, hq // g]) / den[:, None], 0.0)
+            lse[hq, qa:qe] = np.where(live, m + np.log(den), -np.inf)
     return o, lse

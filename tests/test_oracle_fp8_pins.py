@@ -156,3 +156,41 @@ def test_fp8_prefill_scale_laws_and_block_locality():
         assert changed[0, 0, max(lo, 1):hi].all()  # causal row 0 sees only key 0: O = v0
         assert not changed[0, 0, :lo].any() and not changed[0, 0, hi:].any()
         assert not changed[0, 1].any()
+
+
+# --------------------------------------------------------------------------- paged prefill over an E4M3 cache
+
+from oracle.kv_fp8 import attn_fwd_paged_fp8  # noqa: E402
+
+
+def test_fp8_paged_prefill_equals_bf16_paged_oracle_on_exact_values():
+    gen = torch.Generator().manual_seed(61)
+    lq, lk = [5, 0, 40, 1], [37, 3, 100, 16]
+    Hq, Hkv, d, ps = 4, 2, 64, 16
+    q, cu_q, c = W.paged_prefill_inputs(lq, lk, Hq, Hkv, d, ps, seed=61)
+    P = c.k_cache.shape[0]
+    k8 = _random_codes((P, ps, Hkv, d), gen)
+    v8 = _random_codes((P, ps, Hkv, d), gen)
+    ks = torch.pow(2.0, torch.randint(-4, 3, (P, Hkv), generator=gen).double()).float()
+    vs = torch.pow(2.0, torch.randint(-4, 3, (P, Hkv), generator=gen).double()).float()
+    kd = (k8.view(torch.float8_e4m3fn).double() * ks.double()[:, None, :, None]).to(torch.bfloat16)
+    vd = (v8.view(torch.float8_e4m3fn).double() * vs.double()[:, None, :, None]).to(torch.bfloat16)
+    lens = torch.tensor(lk, dtype=torch.int32)
+    for causal in (True, False):
+        o, lse = attn_fwd_paged_fp8(q, k8, v8, ks, vs, c.block_table, cu_q, lens, causal, 0.05)
+        o_ref, lse_ref = oracle.attn_fwd_paged(q, kd, vd, c.block_table, cu_q, lens, causal, 0.05)
+        np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-10)
+        fin = np.isfinite(lse_ref)
+        np.testing.assert_allclose(lse[fin], lse_ref[fin], rtol=0, atol=1e-10)
+
+
+def test_fp8_paged_prefill_one_query_per_sequence_is_decode():
+    c = W.fp8_paged_inputs(torch.tensor([70, 1, 33], dtype=torch.int32), 8, 2, 64, 16, seed=62)
+    q = c.q  # [B, Hq, d]: one new token per sequence
+    cu_q = torch.arange(q.shape[0] + 1, dtype=torch.int32)
+    o, lse = attn_fwd_paged_fp8(q, c.k_cache, c.v_cache, c.k_scale, c.v_scale, c.block_table,
+                                cu_q, c.seq_lens, True, 0.1)
+    o_d, lse_d = decode_paged_fp8(q, c.k_cache, c.v_cache, c.k_scale, c.v_scale, c.block_table,
+                                  c.seq_lens, 0.1)
+    np.testing.assert_allclose(o, o_d, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse.T, lse_d, rtol=0, atol=1e-12)
