@@ -13,8 +13,10 @@
  *
  * Conventions shared by every entry point:
  *   - Tensors are dense and contiguous (row-major in the order given).  q, k,
- *     v, o, k_cache and v_cache hold bfloat16; lse holds float32; index
- *     arrays hold int32.  Accumulation is float32.
+ *     v, o, k_cache and v_cache hold bfloat16 (attn_decode_paged_fp8's caches
+ *     hold E4M3 bytes with float32 scales); the backward's d_o, dq, dk and dv
+ *     hold bfloat16; lse holds float32; index arrays hold int32.
+ *     Accumulation is float32.
  *   - Every pointer argument except `workspace` sizes is a DEVICE pointer on
  *     the current CUDA device.  The caller owns all memory; the library
  *     allocates nothing per call and never synchronises the stream in a
