@@ -48,7 +48,10 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mha_causal_2k")
+    ap.add_argument("--workload", default="gqa_causal_32k")
+    ap.add_argument("--prefill-legs",
+                    default="mha_causal_2k,gqa_causal_8k,gqa_causal_8k_padded,tiny_mha",
+                    help="prefill configurations timed on their own after the headline")
     ap.add_argument("--decode-workload", default="paged_decode")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -57,7 +60,7 @@ def parse_args():
     ap.add_argument("--ragged-workload", default="ragged_gqa_causal")
     ap.add_argument("--no-decode-fp8", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
-    ap.add_argument("--backward-workload", default="mha_causal_2k")
+    ap.add_argument("--backward-workloads", default="mha_causal_2k,gqa_causal_8k")
     ap.add_argument("--no-paged-prefill", action="store_true")
     ap.add_argument("--paged-prefill-workload", default="paged_prefill_gqa")
     return ap.parse_args()
@@ -118,7 +121,7 @@ def ncu_traffic(kernel_key: str, config_name: str):
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML while the timed region runs."""
 
-    def __init__(self, device, period_s: float = 0.02):
+    def __init__(self, device, period_s: float = 0.005):
         self.samples = []
         self.reasons = set()
         self.max_mhz = None
@@ -236,36 +239,48 @@ def run_reference(args, world, rank):
     import oracle
     from exact_softmax_attention_fwd_b200 import workloads as W
     cfg = W.CONFIGS[args.workload]
+    dcfg = None if args.no_decode else W.CONFIGS[args.decode_workload]
     q, k, v, k_lens = W.config_inputs(cfg)
-    n_rows = 4096  # rows per step: a few seconds of the host's cores
+    dinp = None if dcfg is None else W.decode_config_inputs(dcfg)
+    n_rows = 2048  # prefill rows per step: well under a second of the host's cores
     threads = os.cpu_count() or 1
     oracle.build()
-    times, flops = [], []
+    times, flops, dtimes = [], [], []
     for step in range(args.warmup + args.steps):
         rows = W.sample_rows(cfg.B, cfg.Hq, cfg.S, n_rows, seed=5000 + step)
-        i = (rows % cfg.S).double()
-        vis = (i + 1) if cfg.causal else torch.full_like(i, float(cfg.S))
-        f = float(4.0 * cfg.d * vis.sum())
+        f = _visible_pair_flops(cfg, rows, k_lens)
         t0 = time.perf_counter()
         oracle.attn_fwd(q, k, v, cfg.causal, cfg.scale, k_lens=k_lens, rows=rows, n_threads=threads)
         dt = time.perf_counter() - t0
+        if dinp is not None:  # the whole decode batch
+            t1 = time.perf_counter()
+            oracle.decode_paged(dinp.q, dinp.k_cache, dinp.v_cache, dinp.block_table,
+                                dinp.seq_lens, dcfg.scale, n_threads=threads)
+            ddt = time.perf_counter() - t1
         if step >= args.warmup:
             times.append(dt)
             flops.append(f)
+            if dinp is not None:
+                dtimes.append(ddt)
     value = sum(flops) / sum(times) / 1e12
-    ms = 1e3 * sum(times) / len(times)
-    sample = f"{n_rows} seeded rows of {cfg.name} per step (of {cfg.B * cfg.Hq * cfg.S})"
+    ms = 1e3 * (sum(times) + sum(dtimes)) / len(times)
+    sample = (f"{n_rows} seeded query rows of {cfg.name} per step (of {cfg.B * cfg.Hq * cfg.S})"
+              + ("" if dinp is None else f" and the whole {dcfg.name} batch"))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_dict(cfg, None),
+        "data": "synthetic", "config": config_dict(cfg, dcfg),
         "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
+    if dinp is not None:
+        nbytes = decode_algorithmic_bytes(dcfg, dinp)
+        line["decode"] = {"value": nbytes * len(dtimes) / sum(dtimes) / 1e9, "unit": "GB/s",
+                          "ms": 1e3 * sum(dtimes) / len(dtimes)}
     return line
 
 
@@ -274,7 +289,9 @@ def run_reference(args, world, rank):
 
 def config_dict(cfg, dcfg):
     d = {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "Sq": cfg.S, "Sk": cfg.S,
-         "d": cfg.d, "causal": cfg.causal, "inputs": "bf16 N(0,1) seeded",
+         "d": cfg.d, "causal": cfg.causal,
+         "inputs": f"bf16 N(0,1){' x ' + str(cfg.value_scale) if cfg.value_scale != 1.0 else ''} "
+                   f"seeded{', key padding 0-25%' if cfg.padded else ''}",
          "l2": "flushed before every timed kernel (256 MiB write)"}
     if dcfg is not None:
         d["decode_workload"] = dcfg.name
@@ -283,28 +300,178 @@ def config_dict(cfg, dcfg):
     return d
 
 
-def cpu_baseline_leg(cfg, q, k, v, k_lens):
-    """The oracle on a bounded sample of the prefill workload (about 10-30 s of CPU)."""
-    import torch
+# The oracle's sample per prefill configuration for the CPU baseline: None =
+# every row; an int = that many seeded rows (the 32k configuration: the 512
+# (head, row) pairs its parity test checks, timed and extrapolated).
+CPU_SAMPLE_ROWS = {"tiny_mha": None, "mha_causal_2k": None, "gqa_causal_8k": None,
+                   "gqa_causal_8k_padded": None, "gqa_causal_32k": 512}
+CPU_SAMPLE_SEED = {"gqa_causal_32k": 41}
 
+
+def _visible_pair_flops(cfg, rows, k_lens):
+    """4*d per visible (row, key) pair over the given flat rows (None = all)."""
+    import torch
+    S = cfg.S
+    if rows is None:
+        i = torch.arange(S, dtype=torch.float64).repeat(cfg.B * cfg.Hq)
+        b = torch.arange(cfg.B).repeat_interleave(cfg.Hq * S)
+    else:
+        i = (rows % S).double()
+        b = rows // (cfg.Hq * S)
+    kl = (torch.full((cfg.B,), float(S), dtype=torch.float64) if k_lens is None
+          else k_lens.double())[b]
+    if cfg.causal:  # bottom-right: row i sees keys j <= i + kl - S, j < kl
+        vis = torch.clamp(torch.minimum(i + kl - S + 1, kl), min=0)
+    else:
+        vis = kl
+    return float(4.0 * cfg.d * vis.sum())
+
+
+def cpu_baseline_prefill(cfg, q, k, v, k_lens):
+    """The oracle as it stands on this host's cores, on the configuration's
+    sample: every row, or the seeded sample of CPU_SAMPLE_ROWS (then the full
+    problem's time is extrapolated from the sample's share of visible pairs
+    and labelled as such).  `value` counts the metric's FLOPs (the nominal
+    causal formula for full runs, visible-pair FLOPs for a sample)."""
     import oracle
     from exact_softmax_attention_fwd_b200 import workloads as W
     threads = os.cpu_count() or 1
-    # size the sample from a short calibration run
-    rows = W.sample_rows(cfg.B, cfg.Hq, cfg.S, 512, seed=77)
-    t0 = time.perf_counter()
-    oracle.attn_fwd(q, k, v, cfg.causal, cfg.scale, k_lens=k_lens, rows=rows, n_threads=threads)
-    t_cal = time.perf_counter() - t0
-    n = int(max(512, min(cfg.B * cfg.Hq * cfg.S, 512 * 12.0 / max(t_cal, 1e-3))))
-    rows = W.sample_rows(cfg.B, cfg.Hq, cfg.S, n, seed=78)
-    i = (rows % cfg.S).double()
-    vis = (i + 1) if cfg.causal else torch.full_like(i, float(cfg.S))
-    flops = float(4.0 * cfg.d * vis.sum())
+    n = CPU_SAMPLE_ROWS.get(cfg.name)
+    rows = None if n is None else W.sample_rows(cfg.B, cfg.Hq, cfg.S, n,
+                                                seed=CPU_SAMPLE_SEED.get(cfg.name, 78))
     t0 = time.perf_counter()
     oracle.attn_fwd(q, k, v, cfg.causal, cfg.scale, k_lens=k_lens, rows=rows, n_threads=threads)
     dt = time.perf_counter() - t0
-    return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
-            "sample": f"{rows.numel()} seeded query rows of {cfg.name} ({dt:.1f} s)"}
+    out = {"unit": "TFLOPS", "cores": threads, "kind": "oracle", "seconds": dt}
+    if rows is None:
+        out["value"] = cfg.flops() / dt / 1e12
+        out["sample"] = f"all {cfg.B * cfg.Hq * cfg.S} query rows of {cfg.name} ({dt:.1f} s)"
+    else:
+        f_sample = _visible_pair_flops(cfg, rows, k_lens)
+        f_all = _visible_pair_flops(cfg, None, k_lens)
+        out["value"] = f_sample / dt / 1e12
+        out["sample"] = (f"{rows.numel()} seeded (head, query row) pairs of {cfg.name} "
+                         f"({dt:.2f} s)")
+        out["extrapolated_full_problem_s"] = dt * f_all / f_sample
+        out["extrapolation"] = ("EXTRAPOLATED, not measured: the sample's time scaled by "
+                                "the full problem's visible pairs over the sample's")
+    return out
+
+
+def cpu_baseline_decode(dcfg, dinp):
+    """The decode oracle on the whole paged_decode batch (GB/s of the same
+    algorithmic bytes the GPU figure counts)."""
+    import oracle
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    oracle.decode_paged(dinp.q, dinp.k_cache, dinp.v_cache, dinp.block_table, dinp.seq_lens,
+                        dcfg.scale, n_threads=threads)
+    dt = time.perf_counter() - t0
+    nbytes = decode_algorithmic_bytes(dcfg, dinp)
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "seconds": dt, "sample": f"the whole {dcfg.name} batch ({dcfg.B} sequences, {dt:.2f} s)"}
+
+
+def decode_algorithmic_bytes(dcfg, dinp) -> int:
+    """K+V of the attended tokens, q, o, the block-table entries used, lengths, LSE."""
+    from exact_softmax_attention_fwd_b200 import workloads as W
+    kv = W.decode_kv_bytes(dinp.seq_lens, dcfg.Hkv, dcfg.d)
+    table = int(sum(-(-int(n) // dcfg.page_size) for n in dinp.seq_lens.tolist())) * 4
+    return kv + 2 * dinp.q.numel() * 2 + table + dinp.seq_lens.numel() * 4 + dcfg.B * dcfg.Hq * 4
+
+
+def leg_calls(args, est_ms: float, world: int, floor_ms: float = 200.0, cap: int = 4000) -> int:
+    """Calls to time in a leg: at least --steps, and enough for the region to
+    last about floor_ms so that the clock sampler sees it (the estimate is
+    the slowest rank's, so every rank makes the same number of calls)."""
+    est = max_over_ranks(max(est_ms, 1e-3), world)
+    return int(max(args.steps, min(cap, math.ceil(floor_ms / est))))
+
+
+def timed_calls(args, dev, world, one, est_calls: int = 3):
+    """Warm up, estimate the call time, then time n calls of `one` (L2 flushed
+    before each, CUDA events on the launch stream around each) with NVML clock
+    samples over the region.  Returns (per-call ms, clocks summary)."""
+    import torch
+
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, args.warmup)):
+        flush.fill_(1.0)
+        one()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(est_calls):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    n = leg_calls(args, e0.elapsed_time(e1) / est_calls + 0.05, world)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    sampler = ClockSampler(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with sampler:
+        for a, b in evs:
+            flush.fill_(1.0)
+            a.record(stream)
+            one()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    return [a.elapsed_time(b) for a, b in evs], sampler.summary()
+
+
+def tensor_roofline(flops, ms, peaks, kernel, config_name, world):
+    """Roofline object of a tensor-bound launch from its per-call times."""
+    mean = sum(ms) / len(ms)
+    med = statistics.median(ms)
+    mean_all = max_over_ranks(mean, world)
+    achieved = flops / (mean_all * 1e-3) / 1e12
+    achieved_med = flops / (med * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+            "achieved_median": achieved_med, "frac_median": achieved_med / peaks["bf16_tflops"],
+            "traffic": ncu_traffic(kernel, config_name), "kernel": kernel,
+            "peak_source": f"{peaks['source']} bf16 burst (kernel timed alone)",
+            "per_launch_flops": flops, "mean_ms": mean_all, "median_ms": med, "calls": len(ms)}
+
+
+def prefill_leg(args, cfg, dev, world, peaks, cpu: bool):
+    """One prefill configuration timed on its own (attn_fwd_masked; inputs
+    resident; L2 flushed before each call), with its own clock record and, on
+    rank 0 of a 1-GPU run, the oracle's time on the same inputs."""
+    import torch
+
+    from exact_softmax_attention_fwd_b200 import attn_fwd_masked, attn_get_device_error
+    from exact_softmax_attention_fwd_b200 import workloads as W
+
+    q_h, k_h, v_h, kl_h = W.config_inputs(cfg)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    kl = None if kl_h is None else kl_h.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((cfg.B, cfg.Hq, cfg.S), dtype=torch.float32, device=dev)
+
+    def one():
+        attn_fwd_masked(q, k, v, cfg.causal, cfg.scale, k_lens=kl, out=o, lse=lse)
+
+    ms, clocks = timed_calls(args, dev, world, one)
+    st, fl = attn_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word set in the {cfg.name} leg: {fl:#x}")
+    flops = cfg.flops()
+    rl = tensor_roofline(flops, ms, peaks, "attn_prefill_sm100_kernel", cfg.name, world)
+    leg = {"workload": cfg.name, "value": world * rl["achieved"], "unit": "TFLOPS",
+           "ms": rl["mean_ms"], "median_ms": rl["median_ms"], "calls": len(ms),
+           "gpu_launches_per_call": 1, "config": config_dict(cfg, None), "roofline": rl,
+           "clocks": clocks}
+    if cfg.padded:
+        leg["flops_counted"] = "nominal 4*B*Hq*S*S*d/2 (padded keys included), as the metric states"
+    del q, k, v, o, lse
+    if cpu:
+        leg["cpu_baseline"] = cpu_baseline_prefill(cfg, q_h, k_h, v_h, kl_h)
+    return leg
 
 
 def run_ours(args, world, rank, local):
@@ -318,6 +485,7 @@ def run_ours(args, world, rank, local):
     peaks = load_peaks()
     cfg = W.CONFIGS[args.workload]
     dcfg = None if args.no_decode else W.CONFIGS[args.decode_workload]
+    cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
 
     # ---- inputs resident in HBM before the timed region
     q_h, k_h, v_h, kl_h = W.config_inputs(cfg)
@@ -335,10 +503,7 @@ def run_ours(args, world, rank, local):
                          dtype=torch.uint8, device=dev)
         do = torch.empty((dcfg.B, dcfg.Hq, dcfg.d), dtype=torch.bfloat16, device=dev)
         dlse = torch.empty((dcfg.B, dcfg.Hq), dtype=torch.float32, device=dev)
-        kv_bytes = W.decode_kv_bytes(dinp.seq_lens, dcfg.Hkv, dcfg.d)
-        table_bytes = int(sum(-(-int(n) // dcfg.page_size) for n in dinp.seq_lens.tolist())) * 4
-        decode_bytes = (kv_bytes + 2 * dq.numel() * 2 + table_bytes + dlens.numel() * 4
-                        + dlse.numel() * 4)
+        decode_bytes = decode_algorithmic_bytes(dcfg, dinp)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -388,78 +553,60 @@ def run_ours(args, world, rank, local):
         raise RuntimeError(f"device error word set in the timed region: {fl:#x}")
 
     pre_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    flops_per_s, pre_avg = weak_scaling_value(flops, sum(pre_ms) / len(pre_ms), world)
     step_ms = max_over_ranks(t_all0.elapsed_time(t_all1) / args.steps, world)
-    value = flops_per_s / 1e12
-    achieved = flops / (pre_avg * 1e-3) / 1e12
-    traffic = ncu_traffic("attn_prefill_sm100_kernel", cfg.name)
+    rl = tensor_roofline(flops, pre_ms, peaks, "attn_prefill_sm100_kernel", cfg.name, world)
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
+        "metric": METRIC, "value": world * rl["achieved"], "unit": "TFLOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": config_dict(cfg, dcfg),
-        "roofline": {"bound": "tensor", "achieved": achieved,
-                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
-                     "kernel": "attn_prefill_sm100_kernel",
-                     "peak_source": f"{peaks['source']} bf16 burst (kernel timed alone)",
-                     "per_launch_flops": flops, "median_ms": statistics.median(pre_ms)},
+        "data": "synthetic", "config": config_dict(cfg, dcfg), "roofline": rl,
     }
     launches_per_step = 1
     if dcfg is not None:
         dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
         bytes_per_s, dec_avg = weak_scaling_value(decode_bytes, sum(dec_ms) / len(dec_ms), world)
         gbs = decode_bytes / (dec_avg * 1e-3) / 1e9
-        dtraffic = ncu_traffic("attn_decode_split_kernel", dcfg.name)
+        dmed = statistics.median(dec_ms)
         line["decode"] = {
-            "value": bytes_per_s / 1e9, "unit": "GB/s", "ms": dec_avg,
+            "value": bytes_per_s / 1e9, "unit": "GB/s", "ms": dec_avg, "median_ms": dmed,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": dtraffic,
+                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                         "achieved_median": decode_bytes / (dmed * 1e-3) / 1e9,
+                         "traffic": ncu_traffic("attn_decode_split_kernel", dcfg.name),
                          "kernel": "attn_decode_split_kernel + attn_decode_merge_kernel",
                          "peak_source": f"{peaks['source']} copy bandwidth",
-                         "algorithmic_bytes": decode_bytes, "median_ms": statistics.median(dec_ms)},
+                         "algorithmic_bytes": decode_bytes},
         }
         launches_per_step += 2
     line["gpu_launches"] = launches_per_step * args.steps
     line["clocks"] = sampler.summary()
+    del q, k, v, o, lse
 
+    # ---- the other prefill configurations, each timed on its own
+    legs = {}
+    for name in args.prefill_legs.split(","):
+        name = name.strip()
+        if name and name != cfg.name:
+            legs[name] = prefill_leg(args, W.CONFIGS[name], dev, world, peaks, cpu)
+    if legs:
+        line["prefill_legs"] = legs
     if not args.no_ragged:
         line["ragged"] = ragged_leg(args, dev, world, peaks)
     if not args.no_paged_prefill:
         line["paged_prefill"] = paged_prefill_leg(args, dev, world, peaks)
     if not args.no_backward:
-        line["backward"] = backward_leg(args, dev, world, peaks)
+        line["backward"] = {name.strip(): backward_leg(args, W.CONFIGS[name.strip()], dev, world,
+                                                       peaks)
+                            for name in args.backward_workloads.split(",") if name.strip()}
     if not args.no_decode and not args.no_decode_fp8:
         line["decode_fp8"] = decode_fp8_leg(args, dev, world, peaks)
     if not args.no_e2e:
         line["e2e"] = e2e_leg(args, cfg, q_h, k_h, v_h, kl_h, dev, world)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_leg(cfg, q_h, k_h, v_h, kl_h)
+    if cpu:
+        line["cpu_baseline"] = cpu_baseline_prefill(cfg, q_h, k_h, v_h, kl_h)
+        if dcfg is not None:
+            line["decode"]["cpu_baseline"] = cpu_baseline_decode(dcfg, dinp)
     return line if rank == 0 else None
-
-
-def _timed_calls(args, dev, world, one):
-    """Warm up, then time n calls of `one` (L2 flushed before each, CUDA events on the
-    launch stream around each); returns the per-call milliseconds."""
-    import torch
-
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    for _ in range(3):
-        flush.fill_(1.0)
-        one()
-    torch.cuda.synchronize(dev)
-    n = max(5, min(args.steps, 50))
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(n)]
-    barrier(world)
-    for e0, e1 in evs:
-        flush.fill_(1.0)
-        e0.record(stream)
-        one()
-        e1.record(stream)
-    torch.cuda.synchronize(dev)
-    return [a.elapsed_time(b) for a, b in evs]
 
 
 def decode_fp8_leg(args, dev, world, peaks):
@@ -490,7 +637,7 @@ def decode_fp8_leg(args, dev, world, peaks):
         attn_decode_paged_fp8(q, k8, v8, ks, vs, tbl, lens, dcfg.scale, out=o, lse=lse,
                               workspace=ws)
 
-    ms = _timed_calls(args, dev, world, one)
+    ms, clocks = timed_calls(args, dev, world, one)
     st, fl = attn_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error word set in the FP8 decode leg: {fl:#x}")
@@ -503,13 +650,15 @@ def decode_fp8_leg(args, dev, world, peaks):
     return {"workload": dcfg.name + " (E4M3 cache, per-page scales)", "value": bytes_per_s / 1e9,
             "unit": "GB/s", "ms": avg, "median_ms": statistics.median(ms), "calls": len(ms),
             "gpu_launches_per_call": 2, "tokens_per_s": world * tokens / (avg * 1e-3),
+            "clocks": clocks,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes": nbytes,
+                         "achieved_median": nbytes / (statistics.median(ms) * 1e-3) / 1e9,
                          "kernel": "attn_decode_split_fp8_kernel + attn_decode_merge_kernel",
                          "traffic": ncu_traffic("attn_decode_split_fp8_kernel", dcfg.name)}}
 
 
-def backward_leg(args, dev, world, peaks):
+def backward_leg(args, cfg, dev, world, peaks):
     """The backward pass from the saved LSE (attn_bwd: the row-statistics kernel, the
     dK/dV kernel and the dQ kernel) on a prefill workload, timed on its own: the
     forward outputs are computed once before timing, inputs resident, L2 flushed
@@ -521,7 +670,6 @@ def backward_leg(args, dev, world, peaks):
                                                   attn_fwd_masked, attn_get_device_error)
     from exact_softmax_attention_fwd_b200 import workloads as W
 
-    cfg = W.CONFIGS[args.backward_workload]
     q_h, k_h, v_h, kl_h = W.config_inputs(cfg)
     do_h = W.grad_output(cfg.B, cfg.Hq, cfg.S, cfg.d, seed=cfg.seed)
     q, k, v, do = q_h.to(dev), k_h.to(dev), v_h.to(dev), do_h.to(dev)
@@ -535,22 +683,20 @@ def backward_leg(args, dev, world, peaks):
         attn_bwd(q, k, v, o, lse, do, cfg.causal, cfg.scale, k_lens=kl, dq=dq, dk=dk, dv=dv,
                  workspace=ws)
 
-    ms = _timed_calls(args, dev, world, one)
+    ms, clocks = timed_calls(args, dev, world, one)
     st, fl = attn_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error word set in the backward leg: {fl:#x}")
     flops = 2.5 * cfg.flops()
-    flops_per_s, avg = weak_scaling_value(flops, sum(ms) / len(ms), world)
-    achieved = flops / (avg * 1e-3) / 1e12
-    return {"workload": cfg.name, "value": flops_per_s / 1e12, "unit": "TFLOPS", "ms": avg,
-            "median_ms": statistics.median(ms), "calls": len(ms), "gpu_launches_per_call": 3,
+    rl = tensor_roofline(flops, ms, peaks, "attn_bwd_dkdv_kernel", cfg.name, world)
+    rl["kernel"] = "attn_bwd_prep_kernel + attn_bwd_dkdv_kernel + attn_bwd_dq_kernel"
+    rl["traffic_kernel"] = "attn_bwd_dkdv_kernel"
+    rl["executed_flops_per_call"] = 3.5 * cfg.flops()
+    return {"workload": cfg.name, "value": world * rl["achieved"], "unit": "TFLOPS",
+            "ms": rl["mean_ms"], "median_ms": rl["median_ms"], "calls": len(ms),
+            "gpu_launches_per_call": 3,
             "flops_counted": "2.5x forward (dV, dP, dQ, dK and the recomputed S)",
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                         "per_call_flops": flops, "executed_flops_per_call": 3.5 * cfg.flops(),
-                         "kernel": "attn_bwd_prep_kernel + attn_bwd_dkdv_kernel + attn_bwd_dq_kernel",
-                         "traffic": ncu_traffic("attn_bwd_dkdv_kernel", cfg.name),
-                         "traffic_kernel": "attn_bwd_dkdv_kernel"}}
+            "clocks": clocks, "roofline": rl}
 
 
 def paged_prefill_leg(args, dev, world, peaks):
@@ -577,20 +723,17 @@ def paged_prefill_leg(args, dev, world, peaks):
         attn_fwd_paged(q, kc, vc, tbl, cu_q, lens, max_q, True, pc.scale, out=o, lse=lse,
                        workspace=ws)
 
-    ms = _timed_calls(args, dev, world, one)
+    ms, clocks = timed_calls(args, dev, world, one)
     st, fl = attn_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error word set in the paged-prefill leg: {fl:#x}")
-    flops = pc.flops()
-    flops_per_s, avg = weak_scaling_value(flops, sum(ms) / len(ms), world)
-    achieved = flops / (avg * 1e-3) / 1e12
-    return {"workload": pc.name, "value": flops_per_s / 1e12, "unit": "TFLOPS", "ms": avg,
-            "median_ms": statistics.median(ms), "calls": len(ms), "gpu_launches_per_call": 2,
+    rl = tensor_roofline(pc.flops(), ms, peaks, "attn_prefill_sm100_kernel", pc.name, world)
+    return {"workload": pc.name, "value": world * rl["achieved"], "unit": "TFLOPS",
+            "ms": rl["mean_ms"], "median_ms": rl["median_ms"], "calls": len(ms),
+            "gpu_launches_per_call": 2,
             "sequences": pc.B, "new_tokens": int(q.shape[0]), "page_size": pc.page_size,
             "keys": f"cached uniform {pc.cached_lo}..{pc.cached_hi} + {pc.new_tokens} new (seed {pc.seed})",
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                         "per_call_flops": flops}}
+            "clocks": clocks, "roofline": rl}
 
 
 def ragged_leg(args, dev, world, peaks):
@@ -613,41 +756,20 @@ def ragged_leg(args, dev, world, peaks):
                      device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((rc.Hq, q.shape[0]), dtype=torch.float32, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
     def one():
         attn_fwd_varlen(q, k, v, cu_q, cu_k, max_q, rc.causal, rc.scale, out=o, lse=lse,
                         workspace=ws)
 
-    for _ in range(3):
-        flush.fill_(1.0)
-        one()
-    torch.cuda.synchronize(dev)
-    n = max(5, min(args.steps, 50))
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(n)]
-    barrier(world)
-    for e0, e1 in evs:
-        flush.fill_(1.0)
-        e0.record(stream)
-        one()
-        e1.record(stream)
-    torch.cuda.synchronize(dev)
+    ms, clocks = timed_calls(args, dev, world, one)
     st, fl = attn_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error word set in the ragged leg: {fl:#x}")
-    ms = [a.elapsed_time(b) for a, b in evs]
-    flops = rc.flops(lens)
-    flops_per_s, avg = weak_scaling_value(flops, sum(ms) / len(ms), world)
-    achieved = flops / (avg * 1e-3) / 1e12
-    return {"workload": rc.name, "value": flops_per_s / 1e12, "unit": "TFLOPS", "ms": avg,
-            "median_ms": statistics.median(ms), "calls": n, "gpu_launches_per_call": 2,
-            "sequences": rc.B, "total_tokens": int(q.shape[0]),
+    rl = tensor_roofline(rc.flops(lens), ms, peaks, "attn_prefill_sm100_kernel", rc.name, world)
+    return {"workload": rc.name, "value": world * rl["achieved"], "unit": "TFLOPS",
+            "ms": rl["mean_ms"], "median_ms": rl["median_ms"], "calls": len(ms),
+            "gpu_launches_per_call": 2, "sequences": rc.B, "total_tokens": int(q.shape[0]),
             "lengths": f"uniform {rc.len_lo}..{rc.len_hi} (seed {rc.seed})",
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                         "per_call_flops": flops}}
+            "clocks": clocks, "roofline": rl}
 
 
 def e2e_leg(args, cfg, q_h, k_h, v_h, kl_h, dev, world):

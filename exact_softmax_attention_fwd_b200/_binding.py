@@ -125,6 +125,15 @@ def _out(t, shape, dtype, device, name):
     return t
 
 
+def _require_bf16(**tensors):
+    """Raise unless every named tensor is bfloat16 (the kernels read these bytes
+    as bf16: any other dtype would be misread, or read past its allocation)."""
+    import torch
+    for name, t in tensors.items():
+        if t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be torch.bfloat16, got {t.dtype}")
+
+
 def _require_cuda(*tensors):
     for t in tensors:
         if t is not None and not t.is_cuda:
@@ -342,6 +351,7 @@ def attn_decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float, 
                       lse=None, workspace=None, return_lse: bool = True, stream=None):
     """Single-query attention over a paged cache (see include/attn.h for layouts)."""
     import torch
+    _require_bf16(q=q, k_cache=k_cache, v_cache=v_cache)
     _require_cuda(q, k_cache, v_cache, block_table, seq_lens)
     B, Hq, d = q.shape
     num_pages, page_size, Hkv, dk = k_cache.shape
@@ -376,6 +386,7 @@ def attn_decode_paged_fp8(q, k_cache, v_cache, k_scale, v_scale, block_table, se
     """attn_decode_paged over an E4M3 cache: k_cache / v_cache uint8 [num_pages,
     page_size, Hkv, d] codes, k_scale / v_scale float32 [num_pages, Hkv]."""
     import torch
+    _require_bf16(q=q)
     _require_cuda(q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens)
     B, Hq, d = q.shape
     num_pages, page_size, Hkv, dk = k_cache.shape
@@ -425,6 +436,7 @@ def attn_decode_paged_noalloc(q, k_cache, v_cache, block_table, seq_lens, scale,
     device caches the area's address: make it before any stream capture.
     """
     import torch
+    _require_bf16(q=q, k_cache=k_cache, v_cache=v_cache)
     _require_cuda(q, k_cache, v_cache, block_table, seq_lens)
     B, Hq, d = q.shape
     num_pages, page_size, Hkv, dk = k_cache.shape

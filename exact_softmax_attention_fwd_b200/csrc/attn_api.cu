@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -32,34 +33,92 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// cuTensorMapEncodeTiled, looked up once (thread-safe static initialisation).
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
                                          &q) != cudaSuccess ||
         q != cudaDriverEntryPointSuccess)
       return nullptr;
-    fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
   return fn;
+}
+
+// A tensor map is a pure function of (address, sizes, strides, box, layout),
+// so encoded maps are kept in a small cache keyed by exactly those: repeated
+// calls on the same buffers (a serving loop, a benchmark) skip the encode.
+struct MapKey {
+  const void* ptr;
+  int kind;  // 0: [planes, rows, D] tiles; 1: token-major [tokens, heads, D]
+  int D;
+  long long a, b;  // rows, planes  |  heads, tokens
+  unsigned box_rows;
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && kind == o.kind && D == o.D && a == o.a && b == o.b &&
+           box_rows == o.box_rows;
+  }
+};
+
+class MapCache {
+ public:
+  bool find(const MapKey& k, CUtensorMap* out) {
+    std::lock_guard<std::mutex> g(mu_);
+    for (int i = 0; i < kSize; ++i)
+      if (used_[i] && keys_[i] == k) {
+        *out = maps_[i];
+        return true;
+      }
+    return false;
+  }
+  void put(const MapKey& k, const CUtensorMap& m) {
+    std::lock_guard<std::mutex> g(mu_);
+    const int i = next_;
+    next_ = (next_ + 1) % kSize;
+    keys_[i] = k;
+    maps_[i] = m;
+    used_[i] = true;
+  }
+
+ private:
+  static constexpr int kSize = 64;
+  std::mutex mu_;
+  MapKey keys_[kSize] = {};
+  CUtensorMap maps_[kSize] = {};
+  bool used_[kSize] = {};
+  int next_ = 0;
+};
+
+MapCache& map_cache() {
+  static MapCache c;
+  return c;
+}
+
+bool encode_3d(CUtensorMap* map, const void* ptr, const cuuint64_t dims[3],
+               const cuuint64_t strides[2], const cuuint32_t box[3]) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 3-D bf16 map over a contiguous [planes, rows, D] tensor, box = box_rows rows
 // x 64 columns, 128-byte swizzle (the layout the tcgen05 descriptors expect).
 bool make_tile_map(CUtensorMap* map, const void* ptr, int D, long long rows, long long planes,
                    unsigned box_rows = 128) {
-  EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr) return false;
+  const MapKey key{ptr, 0, D, rows, planes, box_rows};
+  if (map_cache().find(key, map)) return true;
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
   const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
   const cuuint32_t box[3] = {64, box_rows, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (!encode_3d(map, ptr, dims, strides, box)) return false;
+  map_cache().put(key, *map);
+  return true;
 }
 
 // 3-D bf16 map over a packed token-major [tokens, heads, D] tensor, box =
@@ -69,32 +128,53 @@ bool make_tile_map(CUtensorMap* map, const void* ptr, int D, long long rows, lon
 // num_pages * page_size tokens, read one page (box_rows = page_size) at a time.
 bool make_token_map(CUtensorMap* map, const void* ptr, int D, long long heads, long long tokens,
                     unsigned box_rows = 128) {
-  EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr) return false;
+  const MapKey key{ptr, 1, D, heads, tokens, box_rows};
+  if (map_cache().find(key, map)) return true;
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)tokens};
   const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
   const cuuint32_t box[3] = {64, 1, box_rows};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (!encode_3d(map, ptr, dims, strides, box)) return false;
+  map_cache().put(key, *map);
+  return true;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
-// Streaming multiprocessors of the current device (cached per device).
+// Streaming multiprocessors of the current device (cached per device; the
+// slots are atomics, so concurrent first calls at worst query twice).
 int sm_count() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (cached[dev] == 0) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    cached[dev] = n;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
+}
+
+// cudaFuncSetAttribute(kernel, max dynamic shared memory) once per kernel and
+// device: `done` holds one bit per device for which it has been set.
+template <typename Kernel>
+bool set_smem_once(Kernel kern, int bytes, std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit)) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  done.fetch_or(bit, std::memory_order_release);
+  return true;
+}
+
+// The unit-list kernel's shared memory grows with the level count; the limit
+// is raised once per device to what the largest level count needs.
+bool schedule_smem_ready() {
+  static std::atomic<unsigned long long> done{0};
+  return set_smem_once(attn_varlen_schedule_kernel, (2 * kVarlenMaxLevels + 32) * (int)sizeof(int),
+                       done);
 }
 
 template <int D, bool CAUSAL, int LAYOUT = kLayoutDense, bool MASKS = false>
@@ -104,9 +184,8 @@ int launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
   using C = PrefillCfg<D>;
   constexpr bool VARLEN = LAYOUT != kLayoutDense;
   auto kern = attn_prefill_sm100_kernel<D, CAUSAL, LAYOUT, MASKS>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-      cudaSuccess)
-    return ATTN_ERR_CUDA;
+  static std::atomic<unsigned long long> smem_set{0};
+  if (!set_smem_once(kern, C::SMEM_BYTES, smem_set)) return ATTN_ERR_CUDA;
   // persistent: one CTA per SM (or fewer when there are fewer work units)
   const long long units =
       VARLEN ? max_units * prm.Hq : (long long)prm.n_qblocks * prm.Hq * prm.B;
@@ -206,15 +285,13 @@ int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mdo, const CUtensorMap&
   attn_bwd_prep_kernel<D><<<(unsigned)prep_blocks, 256, 0, stream>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   auto kv = attn_bwd_dkdv_kernel<D, CAUSAL>;
-  if (cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, C::KV_SMEM) !=
-      cudaSuccess)
-    return ATTN_ERR_CUDA;
+  static std::atomic<unsigned long long> kv_smem_set{0};
+  if (!set_smem_once(kv, C::KV_SMEM, kv_smem_set)) return ATTN_ERR_CUDA;
   kv<<<(unsigned)kv_units, C::NUM_THREADS, C::KV_SMEM, stream>>>(mq, mdo, mk, mv, prm);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   auto dq = attn_bwd_dq_kernel<D, CAUSAL>;
-  if (cudaFuncSetAttribute(dq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::Q_SMEM) !=
-      cudaSuccess)
-    return ATTN_ERR_CUDA;
+  static std::atomic<unsigned long long> q_smem_set{0};
+  if (!set_smem_once(dq, C::Q_SMEM, q_smem_set)) return ATTN_ERR_CUDA;
   dq<<<(unsigned)q_units, C::NUM_THREADS, C::Q_SMEM, stream>>>(mq, mdo, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -458,10 +535,7 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   int shift, n_levels;
   varlen_levels(total_k, shift, n_levels);  // total_k bounds every key range
   const size_t sched_smem = (size_t)(2 * n_levels + 32) * sizeof(int);
-  if (cudaFuncSetAttribute(attn_varlen_schedule_kernel,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sched_smem) !=
-      cudaSuccess)
-    return ATTN_ERR_CUDA;
+  if (!schedule_smem_ready()) return ATTN_ERR_CUDA;
   attn_varlen_schedule_kernel<<<1, 1024, sched_smem, stream>>>(
       cu_seqlens_q, cu_seqlens_k, nullptr, B, (int)total_q, (int)total_k, max_seqlen_q, 0, causal,
       0, 0, shift, n_levels, units, unit_count, (int)max_units);
@@ -532,10 +606,7 @@ int attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache,
   int shift, n_levels;
   varlen_levels(max_keys, shift, n_levels);
   const size_t sched_smem = (size_t)(2 * n_levels + 32) * sizeof(int);
-  if (cudaFuncSetAttribute(attn_varlen_schedule_kernel,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sched_smem) !=
-      cudaSuccess)
-    return ATTN_ERR_CUDA;
+  if (!schedule_smem_ready()) return ATTN_ERR_CUDA;
   attn_varlen_schedule_kernel<<<1, 1024, sched_smem, stream>>>(
       cu_seqlens_q, nullptr, seq_lens_k, B, (int)total_q, 0, max_seqlen_q, max_keys, causal,
       0, 0, shift, n_levels, units, unit_count, (int)max_units);

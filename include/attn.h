@@ -297,7 +297,9 @@ int attn_get_device_error(attn_stream_t stream, unsigned int* flags_out);
  *     anything is launched.
  *   - The first call on a device looks up the scratch area's device address
  *     (with that device current) and caches it; make that first call before
- *     any stream capture on that device.
+ *     any stream capture on that device.  The cached address belongs to the
+ *     device's primary context: after cudaDeviceReset on that device it is
+ *     stale, and this call must not be used again in the same process.
  *   - Every call on a device shares the same scratch area.  Calls whose
  *     kernels overlap on the GPU (different streams, or different host
  *     threads) race on it and produce garbage; serialise them.  Each call

@@ -301,3 +301,39 @@ def test_binding_checks_caller_output_buffers():
                 torch.empty((2, 4, 3), dtype=torch.bfloat16).transpose(1, 2)):  # not contiguous
         with pytest.raises(ValueError):
             B._out(bad, (2, 3, 4), torch.bfloat16, cpu, "out")
+
+
+@pytest.mark.parametrize("entry", ["attn_decode_paged", "attn_decode_paged_noalloc"])
+def test_decode_binding_refuses_non_bf16_q_and_caches(entry):
+    # an E4M3 cache (uint8, the FP8 decode's layout) or an fp16 q would be read
+    # as bf16 bytes; the binding rejects them before any CUDA call
+    import torch
+    fn = getattr(B, entry)
+    q = torch.zeros(2, 4, 128, dtype=torch.bfloat16)
+    cache = torch.zeros(3, 16, 2, 128, dtype=torch.bfloat16)
+    cache8 = torch.zeros(3, 16, 2, 128, dtype=torch.uint8)
+    tbl = torch.zeros(2, 2, dtype=torch.int32)
+    lens = torch.ones(2, dtype=torch.int32)
+    for args in ((q, cache8, cache8), (q, cache, cache8), (q.half(), cache, cache),
+                 (q.float(), cache, cache)):
+        with pytest.raises(ValueError, match="bfloat16"):
+            fn(*args, tbl, lens, 0.1)
+
+
+def test_fp8_decode_binding_refuses_non_bf16_q():
+    import torch
+    q = torch.zeros(2, 4, 128, dtype=torch.float16)
+    c8 = torch.zeros(3, 16, 2, 128, dtype=torch.uint8)
+    sc = torch.ones(3, 2, dtype=torch.float32)
+    with pytest.raises(ValueError, match="bfloat16"):
+        B.attn_decode_paged_fp8(q, c8, c8, sc, sc, torch.zeros(2, 2, dtype=torch.int32),
+                                torch.ones(2, dtype=torch.int32), 0.1)
+
+
+def test_noalloc_scratch_size_matches_the_header():
+    text = open(HEADER).read()
+    m = re.search(r"#define\s+ATTN_NOALLOC_SCRATCH_BYTES\s+\(?([^\n/]+?)\)?\s*(?://.*)?$", text,
+                  flags=re.M)
+    assert m, "ATTN_NOALLOC_SCRATCH_BYTES not found in attn.h"
+    expr = m.group(1).replace("u", "").replace("U", "").replace("ll", "").replace("LL", "")
+    assert eval(expr, {}, {}) == B.NOALLOC_SCRATCH_BYTES

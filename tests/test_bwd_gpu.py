@@ -99,6 +99,30 @@ def test_bwd_chained_with_cuda_forward_mha_causal_2k():
     _check_all(got, ref, "mha_causal_2k")
 
 
+def test_bwd_chained_with_cuda_forward_gqa_causal_8k_two_groups():
+    """The gqa_causal_8k workload (B=2, Hq=32, Hkv=8, S=8192, d=128, causal, 4
+    query heads per KV head), forward and backward on the GPU for the whole
+    problem; every gradient element of two KV-head groups checked against the
+    oracle: batch 0 with KV head 0 (query heads 0-3) and batch 1 with KV head 7
+    (query heads 28-31).  Heads of different groups never interact, so the
+    oracle on a group's slice gives that group's exact gradients, dK and dV
+    summed over its four query heads."""
+    cfg = W.CONFIGS["gqa_causal_8k"]
+    q, k, v, _ = W.config_inputs(cfg)
+    do = W.grad_output(cfg.B, cfg.Hq, cfg.S, cfg.d, seed=cfg.seed)
+    scale = 1 / math.sqrt(cfg.d)
+    o, lse = attn_fwd_masked(q.to(DEV), k.to(DEV), v.to(DEV), True, scale)
+    dq, dk, dv = _gpu_bwd(q, k, v, o.cpu(), lse.cpu(), do, True, scale)
+    g = cfg.Hq // cfg.Hkv
+    for b, kvh in ((0, 0), (1, 7)):
+        hs = slice(kvh * g, (kvh + 1) * g)
+        sl = lambda x, h: x[b:b + 1, h].contiguous()
+        ref = oracle_bwd(sl(q, hs), sl(k, slice(kvh, kvh + 1)), sl(v, slice(kvh, kvh + 1)),
+                         sl(do, hs), True, scale)
+        got = (sl(dq, hs), sl(dk, slice(kvh, kvh + 1)), sl(dv, slice(kvh, kvh + 1)))
+        _check_all(got, ref, f"gqa_causal_8k batch {b} KV head {kvh}")
+
+
 def test_bwd_is_deterministic():
     B, Hq, Hkv, S, d = 2, 8, 2, 700, 128
     q, k, v = [x.to(DEV) for x in W.prefill_inputs(B, Hq, Hkv, S, S, d, seed=173)]
