@@ -8,12 +8,15 @@ first call does, and raises if the library is missing or no GPU is present.
 from ._binding import (  # noqa: F401
     AttnError,
     attn_bwd,
+    attn_bwd_varlen,
+    attn_bwd_varlen_workspace_size,
     attn_bwd_workspace_size,
     attn_fwd_block_sparse,
     attn_decode_paged,
     attn_decode_paged_fp8,
     attn_decode_workspace_size,
     attn_fwd,
+    attn_fwd_fp8,
     attn_fwd_masked,
     attn_fwd_paged,
     attn_fwd_varlen,

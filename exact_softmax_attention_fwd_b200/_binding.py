@@ -37,6 +37,8 @@ SIGNATURES = {
     "attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "attn_fwd_masked": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P]),
     "attn_fwd_window": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _I, _I, _P]),
+    "attn_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P,
+                          _P]),
     "attn_fwd_block_sparse": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _I,
                                    _P]),
     "attn_fwd_varlen_workspace_size": (_SZ, [_I, ctypes.c_longlong, _I]),
@@ -54,6 +56,10 @@ SIGNATURES = {
     "attn_bwd_workspace_size": (_SZ, [_I, _I, _I]),
     "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P,
                       _SZ, _P]),
+    "attn_bwd_varlen_workspace_size": (_SZ, [_I, _I, _I]),
+    "attn_bwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I,
+                             ctypes.c_longlong, ctypes.c_longlong, _I, _I, _I, _I, _F, _P, _SZ,
+                             _P]),
     "attn_get_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
     "attn_strerror": (ctypes.c_char_p, [_I]),
     "attn_split_tokens": (_I, []),
@@ -225,6 +231,37 @@ def attn_fwd_block_sparse(q, k, v, block_mask, causal: bool, scale: float, k_len
     return out, lse
 
 
+def attn_fwd_fp8(q, k, v, q_scale, k_scale, v_scale, causal: bool, scale: float, k_lens=None,
+                 out=None, lse=None, return_lse: bool = True, stream=None):
+    """Prefill over block-scaled E4M3 inputs: q [B,Hq,Sq,128], k/v [B,Hkv,Sk,128] uint8
+    codes; q_scale [B,Hq,ceil(Sq/128)], k_scale/v_scale [B,Hkv,ceil(Sk/128)] float32.
+    Returns O [B,Hq,Sq,128] bf16 and LSE [B,Hq,Sq] fp32."""
+    import torch
+    for t in (q, k, v):
+        if t.dtype != torch.uint8 or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous uint8 E4M3 codes")
+    B, Hq, Sq, d = q.shape
+    Bk, Hkv, Sk, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or dk != d:
+        raise ValueError("q/k/v shapes disagree")
+    for t, shape in ((q_scale, (B, Hq, -(-Sq // 128))), (k_scale, (B, Hkv, -(-Sk // 128))),
+                     (v_scale, (B, Hkv, -(-Sk // 128)))):
+        if t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError(f"block scales must be contiguous float32 {shape}")
+    _require_cuda(q, k, v, q_scale, k_scale, v_scale, k_lens)
+    if k_lens is not None and (k_lens.dtype != torch.int32 or tuple(k_lens.shape) != (B,)):
+        raise ValueError("k_lens must be int32 [B]")
+    out = _out(out, q.shape, torch.bfloat16, q.device, "out")
+    if lse is not None or return_lse:
+        lse = _out(lse, (B, Hq, Sq), torch.float32, q.device, "lse")
+    st = load_library().attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(q_scale), _ptr(k_scale),
+                                     _ptr(v_scale), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, d,
+                                     int(bool(causal)), float(scale), _ptr(k_lens),
+                                     _stream(stream))
+    _check(st, "attn_fwd_fp8")
+    return out, lse
+
+
 def attn_bwd_workspace_size(B: int, Hq: int, Sq: int) -> int:
     return int(load_library().attn_bwd_workspace_size(B, Hq, Sq))
 
@@ -260,6 +297,50 @@ def attn_bwd(q, k, v, o, lse, d_o, causal: bool, scale: float, k_lens=None, dq=N
                                  int(bool(causal)), float(scale), _ptr(k_lens), _ptr(workspace),
                                  ws_bytes, _stream(stream))
     _check(st, "attn_bwd")
+    return dq, dk, dv
+
+
+def attn_bwd_varlen_workspace_size(B: int, Hq: int, max_seqlen_q: int) -> int:
+    return int(load_library().attn_bwd_varlen_workspace_size(B, Hq, max_seqlen_q))
+
+
+def attn_bwd_varlen(q, k, v, o, lse, d_o, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                    max_seqlen_k: int, causal: bool, scale: float, dq=None, dk=None, dv=None,
+                    workspace=None, stream=None):
+    """dQ, dK, dV of attn_fwd_varlen.  q, o, d_o [total_q, Hq, d], k/v [total_k, Hkv, d]
+    bf16 packed; lse [Hq, total_q] fp32 as the forward returned it; cu_seqlens_q/k int32
+    [B+1] on the device; max_seqlen_q/k bound the sequences' lengths."""
+    import torch
+    _require_bf16(q=q, k=k, v=v, o=o, d_o=d_o)
+    _require_cuda(q, k, v, o, lse, d_o, cu_seqlens_q, cu_seqlens_k, dq, dk, dv, workspace)
+    for t in (q, k, v, o, d_o):
+        if not t.is_contiguous():
+            raise ValueError("q, k, v, o, d_o must be contiguous")
+    if q.dim() != 3 or k.dim() != 3 or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("q [total_q, Hq, d]; k, v [total_k, Hkv, d]")
+    total_q, Hq, d = q.shape
+    total_k, Hkv, dk_ = k.shape
+    if dk_ != d or tuple(o.shape) != tuple(q.shape) or tuple(d_o.shape) != tuple(q.shape):
+        raise ValueError("o and d_o must have q's shape and the head dims must agree")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (Hq, total_q) or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous float32 [Hq, total_q]")
+    B = cu_seqlens_q.shape[0] - 1
+    for t in (cu_seqlens_q, cu_seqlens_k):
+        if t.dtype != torch.int32 or tuple(t.shape) != (B + 1,) or not t.is_contiguous():
+            raise ValueError("cu_seqlens_q / cu_seqlens_k must be contiguous int32 [B+1]")
+    dq = _out(dq, q.shape, torch.bfloat16, q.device, "dq")
+    dk = _out(dk, k.shape, torch.bfloat16, q.device, "dk")
+    dv = _out(dv, v.shape, torch.bfloat16, q.device, "dv")
+    need = attn_bwd_varlen_workspace_size(B, Hq, max_seqlen_q)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = load_library().attn_bwd_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(d_o), _ptr(dq), _ptr(dk), _ptr(dv),
+        _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, Hq, Hkv, total_q, total_k, int(max_seqlen_q),
+        int(max_seqlen_k), d, int(bool(causal)), float(scale), _ptr(workspace), ws_bytes,
+        _stream(stream))
+    _check(st, "attn_bwd_varlen")
     return dq, dk, dv
 
 

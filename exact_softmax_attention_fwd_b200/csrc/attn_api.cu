@@ -12,6 +12,7 @@
 #include "attn.h"
 #include "bwd_sm100.cuh"
 #include "decode_sm100.cuh"
+#include "prefill_fp8_sm100.cuh"
 #include "prefill_sm100.cuh"
 #include "sm100_primitives.cuh"
 #include "varlen_schedule.cuh"
@@ -52,7 +53,7 @@ EncodeTiledFn encode_fn() {
 // calls on the same buffers (a serving loop, a benchmark) skip the encode.
 struct MapKey {
   const void* ptr;
-  int kind;  // 0: [planes, rows, D] tiles; 1: token-major [tokens, heads, D]
+  int kind;  // 0: [planes, rows, D] tiles; 1: token-major [tokens, heads, D]; 2, 3: E4M3 forms
   int D;
   long long a, b;  // rows, planes  |  heads, tokens
   unsigned box_rows;
@@ -97,13 +98,14 @@ MapCache& map_cache() {
 }
 
 bool encode_3d(CUtensorMap* map, const void* ptr, const cuuint64_t dims[3],
-               const cuuint64_t strides[2], const cuuint32_t box[3]) {
+               const cuuint64_t strides[2], const cuuint32_t box[3],
+               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return enc(map, dtype, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -134,6 +136,39 @@ bool make_token_map(CUtensorMap* map, const void* ptr, int D, long long heads, l
   const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
   const cuuint32_t box[3] = {64, 1, box_rows};
   if (!encode_3d(map, ptr, dims, strides, box)) return false;
+  map_cache().put(key, *map);
+  return true;
+}
+
+// 3-D map over a paged E4M3 pool read as the token-major byte tensor
+// [tokens, heads, D]: box = 16 tokens of one head x all D bytes of the row,
+// 128-byte swizzle for 128-byte rows, 64-byte swizzle for 64-byte rows.
+bool make_token_map_u8(CUtensorMap* map, const void* ptr, int D, long long heads,
+                       long long tokens) {
+  const MapKey key{ptr, 2, D, heads, tokens, 16u};
+  if (map_cache().find(key, map)) return true;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)tokens};
+  const cuuint64_t strides[2] = {(cuuint64_t)D, (cuuint64_t)heads * D};
+  const cuuint32_t box[3] = {(cuuint32_t)D, 1, 16};
+  if (!encode_3d(map, ptr, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                 D >= 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+    return false;
+  map_cache().put(key, *map);
+  return true;
+}
+
+// 3-D map over a contiguous E4M3 [planes, rows, D] tensor (one byte per
+// element): box = 128 rows x all D bytes (D = 128: one 128-byte swizzle span).
+bool make_tile_map_u8(CUtensorMap* map, const void* ptr, int D, long long rows,
+                      long long planes) {
+  const MapKey key{ptr, 3, D, rows, planes, 128u};
+  if (map_cache().find(key, map)) return true;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
+  const cuuint64_t strides[2] = {(cuuint64_t)D, (cuuint64_t)rows * D};
+  const cuuint32_t box[3] = {(cuuint32_t)D, 128, 1};
+  if (!encode_3d(map, ptr, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return false;
   map_cache().put(key, *map);
   return true;
 }
@@ -273,7 +308,7 @@ int prefill_dense(const void* q, const void* k, const void* v, void* o, float* l
 }
 // Backward: the row-statistics pass, then dK/dV (one CTA per key tile and KV
 // head) and dQ (one CTA per query tile and query head), in stream order.
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool VARLEN = false>
 int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mdo, const CUtensorMap& mk,
                const CUtensorMap& mv, const BwdParams& prm, cudaStream_t stream) {
   using C = BwdCfg<D>;
@@ -282,17 +317,28 @@ int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mdo, const CUtensorMap&
   const long long kv_units = (long long)prm.n_kt * prm.B * prm.Hkv;
   const long long q_units = (long long)prm.n_qt * prm.B * prm.Hq;
   if (prep_blocks > INT_MAX || kv_units > INT_MAX || q_units > INT_MAX) return ATTN_ERR_INVALID_ARG;
-  attn_bwd_prep_kernel<D><<<(unsigned)prep_blocks, 256, 0, stream>>>(prm);
+  attn_bwd_prep_kernel<D, VARLEN><<<(unsigned)prep_blocks, 256, 0, stream>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  auto kv = attn_bwd_dkdv_kernel<D, CAUSAL>;
+  auto kv = attn_bwd_dkdv_kernel<D, CAUSAL, VARLEN>;
   static std::atomic<unsigned long long> kv_smem_set{0};
   if (!set_smem_once(kv, C::KV_SMEM, kv_smem_set)) return ATTN_ERR_CUDA;
   kv<<<(unsigned)kv_units, C::NUM_THREADS, C::KV_SMEM, stream>>>(mq, mdo, mk, mv, prm);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  auto dq = attn_bwd_dq_kernel<D, CAUSAL>;
+  auto dq = attn_bwd_dq_kernel<D, CAUSAL, VARLEN>;
   static std::atomic<unsigned long long> q_smem_set{0};
   if (!set_smem_once(dq, C::Q_SMEM, q_smem_set)) return ATTN_ERR_CUDA;
   dq<<<(unsigned)q_units, C::NUM_THREADS, C::Q_SMEM, stream>>>(mq, mdo, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, bool FP8>
+int launch_decode_split(const CUtensorMap& mk, const CUtensorMap& mv, const DecodeFp8Params& pf,
+                        dim3 grid, cudaStream_t stream) {
+  using C = DecodeTmaCfg<D, FP8>;
+  auto kern = attn_decode_split_tma_kernel<D, FP8>;
+  static std::atomic<unsigned long long> smem_set{0};
+  if (!set_smem_once(kern, C::SMEM, smem_set)) return ATTN_ERR_CUDA;
+  kern<<<grid, 32, C::SMEM, stream>>>(mk, mv, pf);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -309,7 +355,8 @@ int decode_paged_common(bool fp8, const void* q, const void* k_cache, const void
   if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || max_pages_per_seq < 1 || num_pages < 1 ||
       page_size < 1)
     return ATTN_ERR_INVALID_ARG;
-  if (B > 65535 || Hkv > 65535 || (long long)max_pages_per_seq * page_size > (1ll << 30))
+  if (B > 65535 || Hkv > 65535 || (long long)max_pages_per_seq * page_size > (1ll << 30) ||
+      (long long)num_pages * page_size > 0x7fffffffLL)
     return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
@@ -355,21 +402,30 @@ int decode_paged_common(bool fp8, const void* q, const void* k_cache, const void
   pf.v8 = static_cast<const uint8_t*>(v_cache);
   pf.k_scale = k_scale;
   pf.v_scale = v_scale;
-  dim3 grid_split((prm.n_split + 3) / 4, Hkv, B);
+  // K/V reach the split kernel through tensor maps over the pool, read as the
+  // token-major tensor [num_pages * page_size, Hkv, d]
+  CUtensorMap mk, mv;
+  const long long pool_tokens = (long long)num_pages * page_size;
+  const bool maps_ok =
+      fp8 ? make_token_map_u8(&mk, k_cache, d, Hkv, pool_tokens) &&
+                make_token_map_u8(&mv, v_cache, d, Hkv, pool_tokens)
+          : make_token_map(&mk, k_cache, d, Hkv, pool_tokens, 16) &&
+                make_token_map(&mv, v_cache, d, Hkv, pool_tokens, 16);
+  if (!maps_ok) return ATTN_ERR_CUDA;
+  dim3 grid_split(prm.n_split, Hkv, B);
   dim3 grid_merge((unsigned)(((long long)B * Hq + 3) / 4));
-  if (d == 128) {
-    if (fp8)
-      attn_decode_split_fp8_kernel<128><<<grid_split, 128, 0, stream>>>(pf);
-    else
-      attn_decode_split_kernel<128><<<grid_split, 128, 0, stream>>>(prm);
+  int st = ATTN_OK;
+  if (d == 128)
+    st = fp8 ? launch_decode_split<128, true>(mk, mv, pf, grid_split, stream)
+             : launch_decode_split<128, false>(mk, mv, pf, grid_split, stream);
+  else
+    st = fp8 ? launch_decode_split<64, true>(mk, mv, pf, grid_split, stream)
+             : launch_decode_split<64, false>(mk, mv, pf, grid_split, stream);
+  if (st != ATTN_OK) return st;
+  if (d == 128)
     attn_decode_merge_kernel<128><<<grid_merge, 128, 0, stream>>>(prm);
-  } else {
-    if (fp8)
-      attn_decode_split_fp8_kernel<64><<<grid_split, 128, 0, stream>>>(pf);
-    else
-      attn_decode_split_kernel<64><<<grid_split, 128, 0, stream>>>(prm);
+  else
     attn_decode_merge_kernel<64><<<grid_merge, 128, 0, stream>>>(prm);
-  }
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -442,6 +498,79 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
                 : launch_bwd<64, false>(mq, mdo, mk, mv, prm, stream);
 }
 
+
+size_t attn_bwd_varlen_workspace_size(int B, int Hq, int max_seqlen_q) {
+  if (B < 1 || Hq < 1 || max_seqlen_q < 1) return 0;
+  return bwd_workspace_bytes(B, Hq, max_seqlen_q);
+}
+
+int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* d_o, void* dq, void* dk, void* dv, const int32_t* cu_seqlens_q,
+                    const int32_t* cu_seqlens_k, int B, int Hq, int Hkv, long long total_q,
+                    long long total_k, int max_seqlen_q, int max_seqlen_k, int d, int causal,
+                    float scale, void* workspace, size_t workspace_bytes,
+                    attn_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (q == nullptr || o == nullptr || lse == nullptr || d_o == nullptr || dq == nullptr ||
+      workspace == nullptr || cu_seqlens_q == nullptr || cu_seqlens_k == nullptr ||
+      (total_k > 0 && (k == nullptr || v == nullptr || dk == nullptr || dv == nullptr)))
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq > 65535) return ATTN_ERR_INVALID_ARG;
+  if (total_q < 0 || total_k < 0 || total_q > 0x7fffffffLL || total_k > 0x7fffffffLL)
+    return ATTN_ERR_INVALID_ARG;
+  if (max_seqlen_q < 1 || max_seqlen_k < 1 || max_seqlen_q > (1 << 30) || max_seqlen_k > (1 << 30))
+    return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(d_o) || !aligned16(dq) ||
+      !aligned16(workspace) || !aligned4(lse) || !aligned4(cu_seqlens_q) ||
+      !aligned4(cu_seqlens_k) ||
+      (total_k > 0 && (!aligned16(k) || !aligned16(v) || !aligned16(dk) || !aligned16(dv))))
+    return ATTN_ERR_ALIGNMENT;
+  if (workspace_bytes < bwd_workspace_bytes(B, Hq, max_seqlen_q)) return ATTN_ERR_WORKSPACE;
+  const long long n_qt = (max_seqlen_q + 127) / 128, n_kt = (max_seqlen_k + 127) / 128;
+  if (n_qt * B * Hq > INT_MAX || n_kt * B * Hkv > INT_MAX) return ATTN_ERR_INVALID_ARG;
+  if (total_q == 0) return ATTN_OK;  // no query row: no gradient to form
+  if (total_k == 0)  // no key anywhere: every output row is constant zero, so dQ = 0
+    return cudaMemsetAsync(dq, 0, (size_t)total_q * Hq * d * 2, stream) == cudaSuccess
+               ? ATTN_OK
+               : ATTN_ERR_CUDA;
+  CUtensorMap mq, mdo, mk, mv;
+  if (!make_token_map(&mq, q, d, Hq, total_q) || !make_token_map(&mdo, d_o, d, Hq, total_q) ||
+      !make_token_map(&mk, k, d, Hkv, total_k) || !make_token_map(&mv, v, d, Hkv, total_k))
+    return ATTN_ERR_CUDA;
+  BwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.o = static_cast<const uint16_t*>(o);
+  prm.d_o = static_cast<const uint16_t*>(d_o);
+  prm.lse = lse;
+  prm.Sq_pad = (int)(n_qt * 128);
+  prm.nlse2 = static_cast<float*>(workspace);
+  prm.dsum = prm.nlse2 + (size_t)B * Hq * prm.Sq_pad;
+  prm.dq = static_cast<uint16_t*>(dq);
+  prm.dk = static_cast<uint16_t*>(dk);
+  prm.dv = static_cast<uint16_t*>(dv);
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.Sq = max_seqlen_q;
+  prm.Sk = max_seqlen_k;
+  prm.group = Hq / Hkv;
+  prm.n_qt = (int)n_qt;
+  prm.n_kt = (int)n_kt;
+  prm.scale = scale;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.cu_q = cu_seqlens_q;
+  prm.cu_k = cu_seqlens_k;
+  prm.total_q = (int)total_q;
+  prm.total_k = (int)total_k;
+  if (d == 128)
+    return causal ? launch_bwd<128, true, true>(mq, mdo, mk, mv, prm, stream)
+                  : launch_bwd<128, false, true>(mq, mdo, mk, mv, prm, stream);
+  return causal ? launch_bwd<64, true, true>(mq, mdo, mk, mv, prm, stream)
+                : launch_bwd<64, false, true>(mq, mdo, mk, mv, prm, stream);
+}
 
 const char* attn_strerror(int status) {
   switch (status) {
@@ -639,6 +768,63 @@ int attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache,
                   : launch_prefill<128, false, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units);
   return causal ? launch_prefill<64, true, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units)
                 : launch_prefill<64, false, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units);
+}
+
+int attn_fwd_fp8(const void* q, const void* k, const void* v, const float* q_scale,
+                 const float* k_scale, const float* v_scale, void* o, float* lse, int B, int Hq,
+                 int Hkv, int Sq, int Sk, int d, int causal, float scale, const int32_t* k_lens,
+                 attn_stream_t stream_) {
+  if (q_scale == nullptr || (Sk > 0 && (k_scale == nullptr || v_scale == nullptr)))
+    return ATTN_ERR_INVALID_ARG;
+  const int st = check_prefill_args(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens);
+  if (st != ATTN_OK) return st;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned4(q_scale) || (Sk > 0 && (!aligned4(k_scale) || !aligned4(v_scale))))
+    return ATTN_ERR_ALIGNMENT;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (Sk == 0)  // no key: every row empty
+    return prefill_dense(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens, 0, 0,
+                         nullptr, 1, stream);
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_tile_map_u8(&mq, q, d, Sq, (long long)B * Hq) ||
+      !make_tile_map_u8(&mk, k, d, Sk, (long long)B * Hkv) ||
+      !make_tile_map_u8(&mv, v, d, Sk, (long long)B * Hkv) ||
+      !make_tile_map(&mo, o, d, Sq, (long long)B * Hq, 32))
+    return ATTN_ERR_CUDA;
+  PrefillFp8Params f;
+  std::memset(&f, 0, sizeof(f));
+  PrefillParams& prm = f.p;
+  prm.lse = lse;
+  prm.k_lens = k_lens;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.Sq = Sq;
+  prm.Sk = Sk;
+  prm.group = Hq / Hkv;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.n_qblocks = (Sq + 255) / 256;
+  prm.mask_heads = 1;
+  prm.n_qt = (Sq + 127) / 128;
+  prm.n_kt = (Sk + 127) / 128;
+  f.q_scale = q_scale;
+  f.k_scale = k_scale;
+  f.v_scale = v_scale;
+  using C = PrefillFp8Cfg;
+  const long long units = (long long)prm.n_qblocks * Hq * B;
+  const int sms = sm_count();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  dim3 grid((unsigned)(units < sms ? units : sms));
+  if (causal) {
+    static std::atomic<unsigned long long> done{0};
+    if (!set_smem_once(attn_prefill_fp8_kernel<true>, C::SMEM_BYTES, done)) return ATTN_ERR_CUDA;
+    attn_prefill_fp8_kernel<true><<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, f);
+  } else {
+    static std::atomic<unsigned long long> done{0};
+    if (!set_smem_once(attn_prefill_fp8_kernel<false>, C::SMEM_BYTES, done)) return ATTN_ERR_CUDA;
+    attn_prefill_fp8_kernel<false><<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, f);
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,

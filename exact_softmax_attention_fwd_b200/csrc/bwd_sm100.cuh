@@ -66,7 +66,50 @@ struct BwdParams {
   uint16_t* dv;         // [B, Hkv, Sk, d]
   int B, Hq, Hkv, Sq, Sk, group, Sq_pad, n_qt, n_kt;
   float scale, scale_log2;
+  // ragged batches (VARLEN instantiations): q, o, dO, dQ packed [total_q, Hq, d],
+  // k, v, dK, dV packed [total_k, Hkv, d], LSE [Hq, total_q]; Sq / Sk are the
+  // largest query / key lengths the call allows (max_seqlen_q / _k)
+  const int* cu_q;      // [B + 1]
+  const int* cu_k;      // [B + 1]
+  int total_q, total_k;
 };
+
+// One sequence of a backward call: query rows [q0, q0 + lq) and keys
+// [k0, k0 + lk) of the packed tensors (fixed-length batches: q0 = k0 = 0,
+// lq = Sq, lk = the clamped key length).  False when a ragged sequence's
+// offsets are not valid (decreasing, outside the tensors, or longer than the
+// call's maxima): nothing of it is computed or written, and it is flagged.
+struct BwdSeq {
+  int q0, lq, k0, lk;
+};
+
+template <bool VARLEN>
+__device__ __forceinline__ bool bwd_sequence(const BwdParams& p, int b, bool report, BwdSeq& s) {
+  if (!VARLEN) {
+    s.q0 = s.k0 = 0;
+    s.lq = p.Sq;
+    int kl = p.k_lens == nullptr ? p.Sk : __ldg(p.k_lens + b);
+    if (kl < 0 || kl > p.Sk) {
+      if (report) flag_device_error(kDevErrBadLength);
+      kl = kl < 0 ? 0 : p.Sk;
+    }
+    s.lk = kl;
+    return true;
+  }
+  const int qa = __ldg(p.cu_q + b), qb = __ldg(p.cu_q + b + 1);
+  const int ka = __ldg(p.cu_k + b), kb = __ldg(p.cu_k + b + 1);
+  if (qa < 0 || qb < qa || qb > p.total_q || ka < 0 || kb < ka || kb > p.total_k ||
+      qb - qa > p.Sq || kb - ka > p.Sk) {
+    if (report) flag_device_error(kDevErrBadLength);
+    s.q0 = s.lq = s.k0 = s.lk = 0;
+    return false;
+  }
+  s.q0 = qa;
+  s.lq = qb - qa;
+  s.k0 = ka;
+  s.lk = kb - ka;
+  return true;
+}
 
 template <int D>
 struct BwdCfg {
@@ -134,7 +177,7 @@ __device__ __forceinline__ float bwd_keep(bool visible, float x) {
 
 // D = rowsum(dO * O) and -LSE*log2(e) for every padded query row.  D/8
 // threads per row, 8 elements each, reduced by shuffles.
-template <int D>
+template <int D, bool VARLEN>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const BwdParams p) {
   constexpr int TPR = D / 8;
   const long long n_rows = (long long)p.B * p.Hq * p.Sq_pad;
@@ -144,10 +187,16 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const BwdParams p) {
   const bool valid = row < n_rows;
   const long long bh = valid ? row / p.Sq_pad : 0;
   const int i = valid ? (int)(row % p.Sq_pad) : 0;
-  const bool live = valid && i < p.Sq;
+  BwdSeq sq;
+  const int b = (int)(bh / p.Hq), h = (int)(bh % p.Hq);
+  const bool seq_ok = valid && bwd_sequence<VARLEN>(p, b, false, sq);
+  const bool live = seq_ok && i < sq.lq;
+  // dense: [B*Hq, Sq] rows; ragged: token q0 + i of head h in [total_q, Hq]
+  const size_t row_el = VARLEN ? ((size_t)(sq.q0 + i) * p.Hq + h) : ((size_t)bh * p.Sq + i);
+  const size_t lse_at = VARLEN ? ((size_t)h * p.total_q + sq.q0 + i) : ((size_t)bh * p.Sq + i);
   float acc = 0.f;
   if (live) {
-    const size_t off = ((size_t)bh * p.Sq + i) * D + part * 8;
+    const size_t off = row_el * D + part * 8;
     const uint4 a = ld_stream_v4(p.d_o + off);
     const uint4 b = ld_stream_v4(p.o + off);
     const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
@@ -163,23 +212,12 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const BwdParams p) {
   if (valid && part == 0) {
     float nl = -INFINITY;
     if (live) {
-      const float l = p.lse[(size_t)bh * p.Sq + i];
+      const float l = p.lse[lse_at];
       nl = (l == -INFINITY) ? -INFINITY : -l * 1.4426950408889634f;
     }
     p.nlse2[row] = nl;
     p.dsum[row] = live ? acc : 0.f;
   }
-}
-
-// The valid key count of batch b (clamped and flagged when out of range).
-__device__ __forceinline__ int bwd_klen(const BwdParams& p, int b, bool report) {
-  if (p.k_lens == nullptr) return p.Sk;
-  int kl = __ldg(p.k_lens + b);
-  if (kl < 0 || kl > p.Sk) {
-    if (report) flag_device_error(kDevErrBadLength);
-    kl = kl < 0 ? 0 : p.Sk;
-  }
-  return kl;
 }
 
 // SS MMA over the head dimension: D[tm] = A B^T, A and B 128-row K-major tiles.
@@ -229,7 +267,7 @@ __device__ __forceinline__ void bwd_store32(uint16_t* dst, const uint32_t (&v)[3
 // tile major, so under a causal mask the heaviest key tiles (the first ones,
 // seen by the most query tiles) start first.
 // ===========================================================================
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_do,
@@ -250,16 +288,23 @@ __global__ void __launch_bounds__(384, 1)
   const int bh_kv = blockIdx.x % (p.B * p.Hkv);
   const int kb = blockIdx.x / (p.B * p.Hkv);
   const int b = bh_kv / p.Hkv, kvh = bh_kv % p.Hkv;
-  const int klen = bwd_klen(p, b, threadIdx.x == 0);
-  const long long koff = (long long)klen - p.Sq;  // key j is visible to row i iff j <= i + koff
+  BwdSeq sq;
+  const bool seq_ok = bwd_sequence<VARLEN>(p, b, threadIdx.x == 0 && kb == 0 && kvh == 0, sq);
+  const int klen = seq_ok ? sq.lk : 0;
+  const long long koff = (long long)klen - sq.lq;  // key j is visible to row i iff j <= i + koff
   const int key0 = kb * 128;
+  const int n_qt = VARLEN ? (sq.lq + 127) / 128 : p.n_qt;  // this sequence's query tiles
   int qt_lo = 0;
   if (CAUSAL) {
     const long long first_row = (long long)key0 - koff;  // the first row that sees key0
-    qt_lo = first_row <= 0 ? 0 : (int)min(first_row / 128, (long long)p.n_qt);
+    qt_lo = first_row <= 0 ? 0 : (int)min(first_row / 128, (long long)n_qt);
   }
-  const int nq = (key0 >= klen) ? 0 : p.n_qt - qt_lo;
+  const int nq = (!seq_ok || key0 >= klen) ? 0 : n_qt - qt_lo;
   const int N = p.group * nq;  // (query head, query tile) iterations
+  // dK/dV rows this CTA writes: a ragged sequence's own keys only (rows past
+  // them belong to the next sequence); fixed-length batches write every key
+  // row of the tile (padded keys get zeros)
+  const int key_rows = VARLEN ? (seq_ok ? sq.lk : 0) : p.Sk;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::KB_KV), 1);
@@ -298,9 +343,12 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_v);
       mbar_arrive_expect_tx(bar(C::KB_KV), 2 * C::TILE_BYTES);
+      // fixed-length maps are (d, S, B*H); ragged ones (d, H, tokens)
       for (int cb = 0; cb < C::NCB; ++cb) {
-        tma_load_3d(sK + cb * C::CB_BYTES, &tm_k, bar(C::KB_KV), 64 * cb, key0, bh_kv);
-        tma_load_3d(sV + cb * C::CB_BYTES, &tm_v, bar(C::KB_KV), 64 * cb, key0, bh_kv);
+        tma_load_3d(sK + cb * C::CB_BYTES, &tm_k, bar(C::KB_KV), 64 * cb, VARLEN ? kvh : key0,
+                    VARLEN ? sq.k0 + key0 : bh_kv);
+        tma_load_3d(sV + cb * C::CB_BYTES, &tm_v, bar(C::KB_KV), 64 * cb, VARLEN ? kvh : key0,
+                    VARLEN ? sq.k0 + key0 : bh_kv);
       }
       int issued = 0;
       bool ok = true;
@@ -313,10 +361,10 @@ __global__ void __launch_bounds__(384, 1)
         const int qt = qt_lo + n % nq;
         const int bh_q = b * p.Hq + hq;
         mbar_arrive_expect_tx(bar(C::KB_QF + s), 2 * C::TILE_BYTES + C::STAT_BYTES);
+        const int qy = VARLEN ? hq : qt * 128, qz = VARLEN ? sq.q0 + qt * 128 : bh_q;
         for (int cb = 0; cb < C::NCB; ++cb) {
-          tma_load_3d(sQ(s) + cb * C::CB_BYTES, &tm_q, bar(C::KB_QF + s), 64 * cb, qt * 128, bh_q);
-          tma_load_3d(sDO(s) + cb * C::CB_BYTES, &tm_do, bar(C::KB_QF + s), 64 * cb, qt * 128,
-                      bh_q);
+          tma_load_3d(sQ(s) + cb * C::CB_BYTES, &tm_q, bar(C::KB_QF + s), 64 * cb, qy, qz);
+          tma_load_3d(sDO(s) + cb * C::CB_BYTES, &tm_do, bar(C::KB_QF + s), 64 * cb, qy, qz);
         }
         const size_t srow = (size_t)bh_q * p.Sq_pad + (size_t)qt * 128;
         bulk_load(sST(s), p.nlse2 + srow, 512, bar(C::KB_QF + s));
@@ -471,9 +519,11 @@ __global__ void __launch_bounds__(384, 1)
       ok = mbar_wait_warp(bar(C::KB_ACC), 0, abort_flag);
       tc_fence_after_sync();
     }
-    if (!have || ok) {
+    if ((!have || ok) && key0 < key_rows) {
       const uint32_t t_acc = tmem + lane_off + (wg ? C::KV_TM_DK : C::KV_TM_DV);
-      uint16_t* out = (wg ? p.dk : p.dv) + ((size_t)bh_kv * p.Sk + (j < p.Sk ? j : 0)) * D;
+      const int jj = j < key_rows ? j : 0;
+      uint16_t* out = (wg ? p.dk : p.dv) +
+                      (VARLEN ? ((size_t)(sq.k0 + jj) * p.Hkv + kvh) : ((size_t)bh_kv * p.Sk + jj)) * D;
       const float mul = wg ? p.scale : 1.f;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
@@ -484,7 +534,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] = 0u;
         }
-        if (j < p.Sk) bwd_store32(out + c, v, mul);
+        if (j < key_rows) bwd_store32(out + c, v, mul);
       }
     }
   }
@@ -500,7 +550,7 @@ __global__ void __launch_bounds__(384, 1)
 // tile major from the last tile down, so under a causal mask the heaviest
 // tiles start first.
 // ===========================================================================
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_do,
@@ -520,14 +570,19 @@ __global__ void __launch_bounds__(384, 1)
   const int bh_q = blockIdx.x % (p.B * p.Hq);
   const int qt = p.n_qt - 1 - (int)(blockIdx.x / (p.B * p.Hq));
   const int b = bh_q / p.Hq, hq = bh_q % p.Hq;
-  const int bh_kv = b * p.Hkv + hq / p.group;
-  const int klen = bwd_klen(p, b, threadIdx.x == 0);
-  const long long koff = (long long)klen - p.Sq;
+  const int kvh = hq / p.group;
+  const int bh_kv = b * p.Hkv + kvh;
+  BwdSeq sq;
+  const bool seq_ok = bwd_sequence<VARLEN>(p, b, threadIdx.x == 0, sq);
+  const int klen = seq_ok ? sq.lk : 0;
+  const int n_rows = seq_ok ? sq.lq : 0;  // dQ rows of this sequence
+  const long long koff = (long long)klen - sq.lq;
   const int row0 = qt * 128;
-  const int last_row = min(row0 + 127, p.Sq - 1);
+  const int last_row = min(row0 + 127, n_rows - 1);
   long long max_key = (long long)klen - 1;  // the last key any row of the tile sees
   if (CAUSAL) max_key = min(max_key, (long long)last_row + koff);
-  const int N = max_key < 0 ? 0 : (int)(max_key / 128) + 1;  // key tiles [0, N)
+  // key tiles [0, N); none for a tile past the sequence's rows
+  const int N = (max_key < 0 || row0 >= n_rows) ? 0 : (int)(max_key / 128) + 1;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::QB_QF), 1);
@@ -565,9 +620,10 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_v);
       mbar_arrive_expect_tx(bar(C::QB_QF), 2 * C::TILE_BYTES);
+      const int qy = VARLEN ? hq : row0, qz = VARLEN ? sq.q0 + row0 : bh_q;
       for (int cb = 0; cb < C::NCB; ++cb) {
-        tma_load_3d(sQ + cb * C::CB_BYTES, &tm_q, bar(C::QB_QF), 64 * cb, row0, bh_q);
-        tma_load_3d(sDO + cb * C::CB_BYTES, &tm_do, bar(C::QB_QF), 64 * cb, row0, bh_q);
+        tma_load_3d(sQ + cb * C::CB_BYTES, &tm_q, bar(C::QB_QF), 64 * cb, qy, qz);
+        tma_load_3d(sDO + cb * C::CB_BYTES, &tm_do, bar(C::QB_QF), 64 * cb, qy, qz);
       }
       int issued = 0;
       bool ok = true;
@@ -577,9 +633,10 @@ __global__ void __launch_bounds__(384, 1)
             !(ok = mbar_wait(bar(C::QB_KVE + s), ((n / C::STAGES) - 1) & 1u, abort_flag)))
           break;
         mbar_arrive_expect_tx(bar(C::QB_KVF + s), 2 * C::TILE_BYTES);
+        const int ky = VARLEN ? kvh : n * 128, kz = VARLEN ? sq.k0 + n * 128 : bh_kv;
         for (int cb = 0; cb < C::NCB; ++cb) {
-          tma_load_3d(sK(s) + cb * C::CB_BYTES, &tm_k, bar(C::QB_KVF + s), 64 * cb, n * 128, bh_kv);
-          tma_load_3d(sV(s) + cb * C::CB_BYTES, &tm_v, bar(C::QB_KVF + s), 64 * cb, n * 128, bh_kv);
+          tma_load_3d(sK(s) + cb * C::CB_BYTES, &tm_k, bar(C::QB_KVF + s), 64 * cb, ky, kz);
+          tma_load_3d(sV(s) + cb * C::CB_BYTES, &tm_v, bar(C::QB_KVF + s), 64 * cb, ky, kz);
         }
         ++issued;
       }
@@ -698,10 +755,13 @@ __global__ void __launch_bounds__(384, 1)
       ok = mbar_wait_warp(bar(C::QB_ACC), 0, abort_flag);
       tc_fence_after_sync();
     }
-    if (!have || ok) {
+    if ((!have || ok) && row0 < n_rows) {
       constexpr int HALF = D / 2;
       const uint32_t t_acc = tmem + lane_off + C::Q_TM_DQ + wg * HALF;
-      uint16_t* out = p.dq + ((size_t)bh_q * p.Sq + row) * D + wg * HALF;
+      const int rr = row < n_rows ? row : 0;
+      uint16_t* out = p.dq +
+                      (VARLEN ? ((size_t)(sq.q0 + rr) * p.Hq + hq) : ((size_t)bh_q * p.Sq + rr)) * D +
+                      wg * HALF;
 #pragma unroll
       for (int c = 0; c < HALF; c += 32) {
         uint32_t v[32];
@@ -711,7 +771,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] = 0u;
         }
-        if (row < p.Sq) bwd_store32(out + c, v, p.scale);
+        if (row < n_rows) bwd_store32(out + c, v, p.scale);
       }
     }
   }

@@ -606,6 +606,365 @@ __global__ void __launch_bounds__(128) attn_decode_split_fp8_kernel(const Decode
   }
 }
 
+// ---------------------------------------------------------------------------
+// Split kernel with the K/V stream staged in shared memory by TMA.
+//
+// One warp (and CTA) per (sequence b, KV head, split of kSplitTokens tokens),
+// the MMA fragments and the online softmax of the register kernels above, but
+// the 16-token K and V tiles of each step arrive by tensor-memory-access copies
+// (cp.async.bulk.tensor, no multicast) into a DEC_STAGES-deep ring of shared
+// memory, so the bytes in flight no longer cost registers: lane 0 keeps the
+// next DEC_STAGES - 1 steps' copies outstanding while the warp computes.  The
+// cache is read by the copies as the token-major tensor [num_pages *
+// page_size, Hkv, D] (page p starts at token p * page_size); a 16-token step
+// never crosses a page (page sizes are multiples of 16), so a step is one box
+// of 16 rows x (up to) 128 bytes per 128-byte column block, for K and for V.
+// The boxes land 128-byte swizzled (64-byte for 64-byte rows), which keeps the
+// fragment loads from shared memory free of bank conflicts for K.
+//
+// Each lane reads one block-table entry (and, for E4M3 caches, one pair of
+// scales) up front: the split's steps are at most 32, one per lane, and a
+// step's page is fetched from its lane by a shuffle.  Tokens past the length
+// and steps on a page id outside the pool contribute exact zeros (their
+// fragments are zeroed after the shared-memory load, so stale or non-finite
+// slot contents never reach the MMAs); bad ids are flagged.
+// ---------------------------------------------------------------------------
+constexpr int kDecodeStages = 4;
+
+template <int D, bool FP8>
+struct DecodeTmaCfg {
+  static constexpr int E = FP8 ? 1 : 2;            // bytes per element
+  static constexpr int ROW = D * E;                // bytes per token row of one head
+  static constexpr int BOX_BYTES = ROW < 128 ? ROW : 128;  // inner box extent in bytes
+  static constexpr int NBOX = ROW / BOX_BYTES;     // column boxes per row
+  static constexpr int TILE = 16 * ROW;            // 16 tokens of K (or V)
+  static constexpr int STAGE = 2 * TILE;           // K then V
+  static constexpr int SMEM = kDecodeStages * STAGE + 64 + 1024;  // ring, barriers, alignment
+  static_assert(kSplitTokens / 16 <= 32, "one block-table entry per lane");
+};
+
+// Byte offset inside a K or V tile of byte `byte` of token row `tok`, with the
+// swizzle the copies apply (the 16-byte chunk index XOR the row within its
+// 1024-byte (128-byte rows) or 512-byte (64-byte rows) atom).
+template <int D, bool FP8>
+__device__ __forceinline__ uint32_t dec_tile_off(int tok, int byte) {
+  using C = DecodeTmaCfg<D, FP8>;
+  const uint32_t box = (uint32_t)(byte / C::BOX_BYTES);
+  const uint32_t a = (uint32_t)(tok * C::BOX_BYTES + byte % C::BOX_BYTES);
+  const uint32_t sw = C::BOX_BYTES == 128 ? (a ^ ((a >> 3) & 0x70u)) : (a ^ ((a >> 3) & 0x30u));
+  return box * (16u * C::BOX_BYTES) + sw;
+}
+
+__device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(addr));
+  return r;
+}
+
+__device__ __forceinline__ uint2 lds_u2(uint32_t addr) {
+  uint2 r;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
+  return r;
+}
+
+template <int D, bool FP8>
+__global__ void __launch_bounds__(32) attn_decode_split_tma_kernel(
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    const DecodeFp8Params f) {
+  using C = DecodeTmaCfg<D, FP8>;
+  constexpr int KW = D * C::E / 16;   // 32-bit words of a thread's K quarter row
+  constexpr int VW = D * C::E / 32;   // 32-bit words of a thread's V eighth row
+  const DecodeParams& p = f.d;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  const uint32_t bars = sbase + kDecodeStages * C::STAGE;
+  const int lane = threadIdx.x;
+  const int split = blockIdx.x;
+  const int kvh = blockIdx.y;
+  const int b = blockIdx.z;
+  const int len = decode_clamped_len(p, b, lane == 0 && split == 0 && kvh == 0);
+  const int t_begin = split * kSplitTokens;
+  if (t_begin >= len) return;  // the merge kernel never reads splits past the end
+  const int t_end = min(t_begin + kSplitTokens, len);
+  const int n_steps = (t_end - t_begin + 15) / 16;
+
+  // this lane's step: its page (or -1 when the id is outside the pool) and scales
+  int my_page = -1;
+  float my_ks = 0.f, my_vs = 0.f;
+  if (lane < n_steps) {
+    const int t = t_begin + 16 * lane;
+    const int pg = p.block_table[(size_t)b * p.max_pages + t / p.page_size];
+    if (pg >= 0 && pg < p.num_pages) {
+      my_page = pg;
+      if (FP8) {
+        my_ks = __ldg(f.k_scale + (size_t)pg * p.Hkv + kvh);
+        my_vs = __ldg(f.v_scale + (size_t)pg * p.Hkv + kvh);
+      }
+    } else {
+      flag_device_error(kDevErrBadPage);
+    }
+  }
+  if (lane == 0) {
+    for (int s = 0; s < kDecodeStages; ++s) mbar_init(bars + 8u * s, 1);
+    mbar_init_fence();
+    tma_prefetch_map(&tm_k);
+    tma_prefetch_map(&tm_v);
+  }
+  __syncwarp();
+  // Step i's copies into slot i % kDecodeStages (lane 0; every lane calls it for
+  // the shuffle).  A step on a bad page arms its barrier with no bytes.
+  auto issue = [&](int i) {
+    const int pg = __shfl_sync(0xffffffffu, my_page, i);
+    if (lane == 0) {
+      const int slot = i % kDecodeStages;
+      const uint32_t bar = bars + 8u * slot;
+      const uint32_t dst = sbase + slot * C::STAGE;
+      fence_proxy_async_smem();  // the warp's reads of this slot precede the refill
+      mbar_arrive_expect_tx(bar, pg >= 0 ? (uint32_t)C::STAGE : 0u);
+      if (pg >= 0) {
+        const int tok = pg * p.page_size + (t_begin + 16 * i) % p.page_size;
+#pragma unroll
+        for (int bx = 0; bx < C::NBOX; ++bx) {
+          const int col = bx * (C::BOX_BYTES / C::E);
+          tma_load_3d(dst + bx * 16 * C::BOX_BYTES, &tm_k, bar, col, kvh, tok);
+          tma_load_3d(dst + C::TILE + bx * 16 * C::BOX_BYTES, &tm_v, bar, col, kvh, tok);
+        }
+      }
+    }
+  };
+  int n_issued = 0;
+  for (; n_issued < kDecodeStages - 1 && n_issued < n_steps; ++n_issued) issue(n_issued);
+
+  const int g = lane >> 2;   // MMA group id: head row of S / P, d-row block of V^T
+  const int tq = lane & 3;   // thread within the group
+  const int hq0 = kvh * p.group;
+
+  // q as the A operand (rows = heads, padded to 16; layout as the register
+  // kernels).  E4M3 caches: f16 q scaled by 2^-qe into f16's range.
+  uint32_t qa[D / 16][2];
+  float qscale = 1.f;
+  {
+    uint32_t raw[D / 8];
+    if (g < p.group) {
+      const uint16_t* src = p.q + ((size_t)b * p.Hq + hq0 + g) * D + (D / 4) * tq;
+#pragma unroll
+      for (int w = 0; w < D / 32; ++w) {
+        const uint4 x = *reinterpret_cast<const uint4*>(src + 8 * w);
+        raw[4 * w + 0] = x.x;
+        raw[4 * w + 1] = x.y;
+        raw[4 * w + 2] = x.z;
+        raw[4 * w + 3] = x.w;
+      }
+    } else {
+#pragma unroll
+      for (int w = 0; w < D / 8; ++w) raw[w] = 0u;
+    }
+    if (!FP8) {
+#pragma unroll
+      for (int w = 0; w < D / 8; ++w) qa[w >> 1][w & 1] = raw[w];
+    } else {
+      float mxq = 0.f;
+#pragma unroll
+      for (int w = 0; w < D / 8; ++w)
+        mxq = fmaxf(mxq, fmaxf(fabsf(__uint_as_float(raw[w] << 16)),
+                               fabsf(__uint_as_float(raw[w] & 0xFFFF0000u))));
+      mxq = fmaxf(mxq, __shfl_xor_sync(0xffffffffu, mxq, 1));
+      mxq = fmaxf(mxq, __shfl_xor_sync(0xffffffffu, mxq, 2));
+      int qe = 0;
+      if (mxq >= 16384.f) qe = ilogbf(mxq) - 13;
+      qscale = ldexpf(1.f, qe);
+      const float qinv = ldexpf(1.f, -qe);
+#pragma unroll
+      for (int w = 0; w < D / 8; ++w)
+        qa[w >> 1][w & 1] = pack_f16x2(__uint_as_float(raw[w] << 16) * qinv,
+                                       __uint_as_float(raw[w] & 0xFFFF0000u) * qinv);
+    }
+  }
+
+  float c2 = p.scale_log2;
+  const bool scale_pos = c2 > 0.f;
+  if (!scale_pos) c2 = 1.f;
+  float m_run = -INFINITY;  // per head row g, log2 units
+  float l_run = 0.f;        // sum of P (f32): the LSE
+  float lr_run = 0.f;       // sum of the rounded P the MMA consumes: normalises O
+  float acc[D / 16][4];
+#pragma unroll
+  for (int mc = 0; mc < D / 16; ++mc) acc[mc][0] = acc[mc][1] = acc[mc][2] = acc[mc][3] = 0.f;
+
+  int i = 0;
+#pragma unroll 1
+  for (; i < n_steps; ++i) {
+    if (n_issued < n_steps) issue(n_issued++);  // step i + kDecodeStages - 1
+    const int slot = i % kDecodeStages;
+    const int pg = __shfl_sync(0xffffffffu, my_page, i);
+    const int n_here = pg >= 0 ? min(16, t_end - (t_begin + 16 * i)) : 0;
+    const float ksc = FP8 ? __shfl_sync(0xffffffffu, my_ks, i) : 1.f;
+    const float vsc = FP8 ? __shfl_sync(0xffffffffu, my_vs, i) : 1.f;
+    const uint32_t kt = sbase + slot * C::STAGE;
+    const uint32_t vt = kt + C::TILE;
+    const bool landed = mbar_wait(bars + 8u * slot, (uint32_t)(i / kDecodeStages) & 1u, nullptr);
+    if (!__all_sync(0xffffffffu, landed)) break;  // timed out: flagged, wind down
+
+    // ---- S = q K^T (16 padded head rows x 16 tokens)
+    float sc[2][4];
+#pragma unroll
+    for (int nc = 0; nc < 2; ++nc) {
+      const int tok = nc * 8 + g;
+      uint32_t kw[KW];
+#pragma unroll
+      for (int w = 0; w < KW / 4; ++w) {
+        const uint4 x = lds_u4(kt + dec_tile_off<D, FP8>(tok, (D * C::E / 4) * tq + 16 * w));
+        kw[4 * w + 0] = x.x;
+        kw[4 * w + 1] = x.y;
+        kw[4 * w + 2] = x.z;
+        kw[4 * w + 3] = x.w;
+      }
+      if (tok >= n_here) {
+#pragma unroll
+        for (int w = 0; w < KW; ++w) kw[w] = 0u;
+      }
+      sc[nc][0] = sc[nc][1] = sc[nc][2] = sc[nc][3] = 0.f;
+      if (!FP8) {
+#pragma unroll
+        for (int kc = 0; kc < D / 16; ++kc)
+          mma_m16n8k16_bf16(sc[nc], qa[kc][0], 0u, qa[kc][1], 0u, kw[2 * kc], kw[2 * kc + 1]);
+      } else {
+#pragma unroll
+        for (int kc = 0; kc < D / 16; ++kc) {
+          const uint32_t w = kw[kc];
+          mma_m16n8k16_f16(sc[nc], qa[kc][0], 0u, qa[kc][1], 0u, e4m3x2_to_f16x2(w),
+                           e4m3x2_to_f16x2(w >> 16));
+        }
+      }
+    }
+
+    // ---- online softmax for head row g over this thread's 4 tokens
+    const float kq = FP8 ? ksc * qscale : 1.f;
+    float s4[4] = {sc[0][0] * kq, sc[0][1] * kq, sc[1][0] * kq, sc[1][1] * kq};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int tok = (e >> 1) * 8 + 2 * tq + (e & 1);
+      if (tok >= n_here) s4[e] = -INFINITY;
+      else if (!scale_pos) s4[e] *= p.scale_log2;
+    }
+    float mx = fmaxf(fmaxf(s4[0], s4[1]), fmaxf(s4[2], s4[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx * c2);
+    // nothing accumulated while m_run = -inf (also avoids -inf - -inf = NaN)
+    const float alpha = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_new);
+    const float base = (m_new == -INFINITY) ? 0.f : m_new;
+    float pr[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) pr[e] = ex2(fmaf(s4[e], c2, -base));
+    // P^T rows (tokens) 2tq, 2tq+1 and 2tq+8, 2tq+9, column g (head): bf16 for a
+    // bf16 cache, f16 (P <= 1) for the f16 MMA of an E4M3 cache
+    const uint32_t pb0 = FP8 ? pack_f16x2(pr[0], pr[1]) : pack_bf16x2(pr[0], pr[1]);
+    const uint32_t pb1 = FP8 ? pack_f16x2(pr[2], pr[3]) : pack_bf16x2(pr[2], pr[3]);
+    float rs = (pr[0] + pr[1]) + (pr[2] + pr[3]);
+    float rr = FP8 ? (f16_to_f32(pb0) + f16_to_f32(pb0 >> 16)) +
+                         (f16_to_f32(pb1) + f16_to_f32(pb1 >> 16))
+                   : sum_f32x2(add_f32x2(bf16x2_to_f32x2(pb0), bf16x2_to_f32x2(pb1)));
+    rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+    rr += __shfl_xor_sync(0xffffffffu, rr, 1);
+    rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+    rr += __shfl_xor_sync(0xffffffffu, rr, 2);
+    l_run = l_run * alpha + rs;
+    lr_run = lr_run * alpha + rr;
+    m_run = m_new;
+
+    // ---- O^T += V^T P^T; accumulator columns are heads 2tq and 2tq+1.  V^T
+    // rows d = (D/8)*g + 2*mc (+1), columns = tokens 2tq, 2tq+1, 2tq+8, 2tq+9.
+    uint32_t vw[4][VW > 0 ? VW : 1];
+#pragma unroll
+    for (int ti = 0; ti < 4; ++ti) {
+      const int tok = 2 * tq + (ti & 1) + 8 * (ti >> 1);
+      const int byte0 = (D * C::E / 8) * g;
+      if constexpr (VW >= 4) {
+#pragma unroll
+        for (int w = 0; w < VW / 4; ++w) {
+          const uint4 x = lds_u4(vt + dec_tile_off<D, FP8>(tok, byte0 + 16 * w));
+          vw[ti][4 * w + 0] = x.x;
+          vw[ti][4 * w + 1] = x.y;
+          vw[ti][4 * w + 2] = x.z;
+          vw[ti][4 * w + 3] = x.w;
+        }
+      } else {
+        const uint2 x = lds_u2(vt + dec_tile_off<D, FP8>(tok, byte0));
+        vw[ti][0] = x.x;
+        vw[ti][1] = x.y;
+      }
+      if (tok >= n_here) {  // masked tokens must not inject NaN
+#pragma unroll
+        for (int w = 0; w < VW; ++w) vw[ti][w] = 0u;
+      }
+    }
+    __syncwarp();  // every lane has read the slot; it may be refilled
+    const float a_h0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
+    const float a_h1 = __shfl_sync(0xffffffffu, alpha, (2 * tq + 1) * 4);
+#pragma unroll
+    for (int mc = 0; mc < D / 16; ++mc) {
+      if (!FP8) {
+        acc[mc][0] *= a_h0;
+        acc[mc][1] *= a_h1;
+        acc[mc][2] *= a_h0;
+        acc[mc][3] *= a_h1;
+        mma_m16n8k16_bf16(acc[mc], prmt(vw[0][mc], vw[1][mc], 0x5410u),
+                          prmt(vw[0][mc], vw[1][mc], 0x7632u), prmt(vw[2][mc], vw[3][mc], 0x5410u),
+                          prmt(vw[2][mc], vw[3][mc], 0x7632u), pb0, pb1);
+      } else {
+        uint32_t vh[4];
+#pragma unroll
+        for (int ti = 0; ti < 4; ++ti) vh[ti] = e4m3x2_to_f16x2(vw[ti][mc >> 1] >> (16 * (mc & 1)));
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_m16n8k16_f16(part, prmt(vh[0], vh[1], 0x5410u), prmt(vh[0], vh[1], 0x7632u),
+                         prmt(vh[2], vh[3], 0x5410u), prmt(vh[2], vh[3], 0x7632u), pb0, pb1);
+        acc[mc][0] = fmaf(vsc, part[0], acc[mc][0] * a_h0);
+        acc[mc][1] = fmaf(vsc, part[1], acc[mc][1] * a_h1);
+        acc[mc][2] = fmaf(vsc, part[2], acc[mc][2] * a_h0);
+        acc[mc][3] = fmaf(vsc, part[3], acc[mc][3] * a_h1);
+      }
+    }
+  }
+  // after a timed-out wait: no copy may still be landing when the CTA exits
+  // (steps [i, n_issued) were issued but not consumed; bounded waits)
+  if (lane == 0)
+    for (int j = i; j < n_issued; ++j)
+      mbar_wait(bars + 8u * (j % kDecodeStages), (uint32_t)(j / kDecodeStages) & 1u, nullptr);
+  __syncwarp();
+
+  // ---- this split's normalised partial output and its log2-sum-exp
+  const int h0 = 2 * tq, h1 = 2 * tq + 1;
+  const float l_h0 = __shfl_sync(0xffffffffu, lr_run, h0 * 4);
+  const float l_h1 = __shfl_sync(0xffffffffu, lr_run, h1 * 4);
+  const float inv0 = l_h0 > 0.f ? 1.f / l_h0 : 0.f;
+  const float inv1 = l_h1 > 0.f ? 1.f / l_h1 : 0.f;
+  const int dbase = (D / 8) * g;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int h = hh ? h1 : h0;
+    if (h >= p.group) continue;
+    const float inv = hh ? inv1 : inv0;
+    float* dst = p.o_part + (((size_t)b * p.Hq + hq0 + h) * p.n_split + split) * D + dbase;
+#pragma unroll
+    for (int mc = 0; mc < D / 16; mc += 2) {
+      float4 w;
+      w.x = acc[mc][hh] * inv;          // d = dbase + 2mc
+      w.y = acc[mc][2 + hh] * inv;      // d = dbase + 2mc + 1
+      w.z = acc[mc + 1][hh] * inv;      // d = dbase + 2mc + 2
+      w.w = acc[mc + 1][2 + hh] * inv;  // d = dbase + 2mc + 3
+      *reinterpret_cast<float4*>(dst + 2 * mc) = w;
+    }
+  }
+  if (tq == 0 && g < p.group) {
+    const float lse2 = l_run > 0.f ? m_run + lg2(l_run) : -INFINITY;
+    p.lse_part[((size_t)b * p.Hq + hq0 + g) * p.n_split + split] = lse2;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(128) attn_decode_merge_kernel(const DecodeParams p) {
   const int warp = threadIdx.x >> 5;

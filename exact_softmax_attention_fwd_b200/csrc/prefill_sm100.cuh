@@ -21,10 +21,14 @@
 //     next unit is loaded as soon as the last MMA reading the current one
 //     retires, and K/V of the next unit stream in while the current unit
 //     finishes.  No multicast.
-//   * warp 1, lane 0  -- tcgen05 MMA issuer: S_i = Q_i K_j^T (SS form, both
+//   * warp 1           -- tcgen05 MMA issuer: S_i = Q_i K_j^T (SS form, both
 //     operands in shared memory) and O_i += P_i V_j (TS form, P read from
 //     tensor memory), ping-ponging between the two query tiles so that the
-//     tensor core works on one tile while the other tile's softmax runs.
+//     tensor core works on one tile while the other tile's softmax runs.  The
+//     whole warp runs the schedule and the waits in uniform control flow and
+//     one lane, picked by elect.sync, issues each group of MMAs: the
+//     descriptors then stay in uniform registers, and a tile's MMAs go out
+//     several times faster than from a lane-0-only branch.
 //   * warps 2-3       -- idle (they complete the first warpgroup).
 //   * warps 4-7 and 8-11 -- one softmax warpgroup per query tile; thread r of
 //     a warpgroup owns row r (= TMEM lane r).  Per KV tile: load the S row
@@ -451,32 +455,35 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ======================= tcgen05 MMA issuer =======================
-    if (lane == 0) {
+    // The whole warp walks the schedule and waits; one elected lane issues
+    // each group of MMAs and their commits (warp-uniform control flow keeps
+    // the descriptors in uniform registers).
+    {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-      // S_i = Q_i K^T over d in steps of 16 (32 bytes inside a 128-byte swizzled row,
-      // 64-column blocks 16 KB apart).
+      auto wait = [&](uint32_t b, uint32_t ph) -> bool {
+        if (__all_sync(0xffffffffu, mbar_test(b, ph))) return true;
+        const bool r = mbar_wait_slow(b, ph, abort_flag);
+        return __all_sync(0xffffffffu, r);
+      };
       auto issue_qk = [&](int i, int stage) {
-        const uint32_t qa = opaque_u32(sbase + C::OFF_Q + i * C::TILE_BYTES);
-        const uint32_t ka = opaque_u32(sbase + C::OFF_K + stage * C::TILE_BYTES);
+        const uint64_t qd = smem_desc_sw128(opaque_u32(sbase + C::OFF_Q + i * C::TILE_BYTES), 16, 1024);
+        const uint64_t kd = smem_desc_sw128(opaque_u32(sbase + C::OFF_K + stage * C::TILE_BYTES), 16, 1024);
+        const uint32_t dt = tmem + C::tmem_s(i);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * C::CB_BYTES + (ks & 3) * 32;
-          umma_ss(tmem + C::tmem_s(i), smem_desc_sw128(qa + off, 16, 1024),
-                  smem_desc_sw128(ka + off, 16, 1024), idesc_qk, ks > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((ks >> 2) * C::CB_BYTES + (ks & 3) * 32) >> 4);
+          umma_ss(dt, qd + off, kd + off, idesc_qk, ks > 0 ? 1u : 0u);
         }
       };
-      // O_i (+)= P_i V over the 128 keys in steps of 16: P from TMEM (8 columns
-      // per step), V as an MN-major operand (16 keys = 2048 bytes per step).
       auto issue_pv = [&](int i, int stage, bool accumulate) {
-        const uint32_t va = opaque_u32(sbase + C::OFF_V + stage * C::TILE_BYTES);
+        const uint64_t vd = smem_desc_sw128(opaque_u32(sbase + C::OFF_V + stage * C::TILE_BYTES), C::CB_BYTES, 1024);
         const uint32_t ts = opaque_u32(tmem + C::tmem_s(i));
+        const uint32_t dt = tmem + C::tmem_o(i);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          umma_ts(tmem + C::tmem_o(i), ts + ks * 8,
-                  smem_desc_sw128(va + ks * 2048, C::CB_BYTES, 1024), idesc_pv,
+        for (int ks = 0; ks < 8; ++ks)
+          umma_ts(dt, ts + ks * 8, vd + (uint64_t)((ks * 2048) >> 4), idesc_pv,
                   (accumulate || ks > 0) ? 1u : 0u);
-        }
       };
       uint32_t kv = 0;                  // ring position
       uint32_t q_waits0 = 0, q_waits1 = 0;  // Q_FULL phases consumed per tile slot
@@ -486,29 +493,29 @@ __global__ void __launch_bounds__(384, 1)
       for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT, MASKS>(p, k, u); ++k) {
         const int jb = u.kv_first, je = u.kv_last;  // the unit's K/V stream
         if (je <= jb) continue;
-        // prologue: S_i(jb) for each tile whose range starts at the stream's start
         {
           const int s = kv % C::STAGES;
-          if (!(ok = mbar_wait(bar(C::B_KFULL + s), (kv / C::STAGES) & 1u, abort_flag))) break;
+          if (!(ok = wait(bar(C::B_KFULL + s), (kv / C::STAGES) & 1u))) break;
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (!ok) break;
             if (u.kv_begin[i] != jb || u.kv_end[i] <= jb) continue;
             uint32_t& qw = i ? q_waits1 : q_waits0;
-            if (!(ok = mbar_wait(bar(C::B_QFULL + i), qw & 1u, abort_flag))) break;
+            if (!(ok = wait(bar(C::B_QFULL + i), qw & 1u))) break;
             ++qw;
             tc_fence_after_sync();
-            issue_qk(i, s);
-            umma_commit(bar(C::B_SFULL + i));
-            if (u.kv_end[i] == jb + 1) umma_commit(bar(C::B_QFREE + i));  // Q_i read for the last time
+            if (elect_one()) {
+              issue_qk(i, s);
+              umma_commit(bar(C::B_SFULL + i));
+              if (u.kv_end[i] == jb + 1) umma_commit(bar(C::B_QFREE + i));
+            }
+            __syncwarp();
           }
           if (!ok) break;
-          umma_commit(bar(C::B_KEMPTY + s));
+          if (elect_one()) umma_commit(bar(C::B_KEMPTY + s));
+          __syncwarp();
         }
         if (MASKS && p.block_mask != nullptr) {
-          // Block-sparse stream: the key tiles some query tile computes, in
-          // order.  Per stream tile kb: PV for each tile computing kb, then the
-          // QK of each tile that computes the next stream tile.
           auto on = [&](int i, int kb) {
             return prefill_block_on(p, u.b, u.hq, u.row0[i], u.kv_begin[i], u.kv_end[i], kb);
           };
@@ -523,39 +530,46 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t idx = kv + pos;
             const int s = idx % C::STAGES;
             const int s1 = (idx + 1) % C::STAGES;
-            if (!(ok = mbar_wait(bar(C::B_VFULL + s), (idx / C::STAGES) & 1u, abort_flag))) break;
+            if (!(ok = wait(bar(C::B_VFULL + s), (idx / C::STAGES) & 1u))) break;
             bool k_next = false;
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
               if (!ok) break;
               if (on(i, kb)) {
                 uint32_t& pw = i ? p_waits1 : p_waits0;
-                if (!(ok = mbar_wait(bar(C::B_PFULL + i), pw & 1u, abort_flag))) break;
+                if (!(ok = wait(bar(C::B_PFULL + i), pw & 1u))) break;
                 ++pw;
                 tc_fence_after_sync();
-                issue_pv(i, s, kb > u.kv_begin[i]);
-                if (kb == u.kv_end[i] - 1) umma_commit(bar(C::B_OFULL + i));
+                if (elect_one()) {
+                  issue_pv(i, s, kb > u.kv_begin[i]);
+                  if (kb == u.kv_end[i] - 1) umma_commit(bar(C::B_OFULL + i));
+                }
+                __syncwarp();
               }
               if (kbn >= 0 && on(i, kbn)) {
                 if (!k_next) {
-                  if (!(ok = mbar_wait(bar(C::B_KFULL + s1), ((idx + 1) / C::STAGES) & 1u,
-                                       abort_flag)))
-                    break;
+                  if (!(ok = wait(bar(C::B_KFULL + s1), ((idx + 1) / C::STAGES) & 1u))) break;
                   k_next = true;
                 }
-                if (kbn == u.kv_begin[i]) {  // this tile's first S: its Q must have landed
+                if (kbn == u.kv_begin[i]) {
                   uint32_t& qw = i ? q_waits1 : q_waits0;
-                  if (!(ok = mbar_wait(bar(C::B_QFULL + i), qw & 1u, abort_flag))) break;
+                  if (!(ok = wait(bar(C::B_QFULL + i), qw & 1u))) break;
                   ++qw;
                 }
                 tc_fence_after_sync();
-                issue_qk(i, s1);
-                umma_commit(bar(C::B_SFULL + i));
-                if (kbn == u.kv_end[i] - 1) umma_commit(bar(C::B_QFREE + i));
+                if (elect_one()) {
+                  issue_qk(i, s1);
+                  umma_commit(bar(C::B_SFULL + i));
+                  if (kbn == u.kv_end[i] - 1) umma_commit(bar(C::B_QFREE + i));
+                }
+                __syncwarp();
               }
             }
-            umma_commit(bar(C::B_VEMPTY + s));
-            if (k_next) umma_commit(bar(C::B_KEMPTY + s1));
+            if (elect_one()) {
+              umma_commit(bar(C::B_VEMPTY + s));
+              if (k_next) umma_commit(bar(C::B_KEMPTY + s1));
+            }
+            __syncwarp();
             kb = kbn;
           }
           kv += pos;
@@ -565,58 +579,66 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t idx = kv + (uint32_t)(j - jb);
           const int s = idx % C::STAGES;
           const int s1 = (idx + 1) % C::STAGES;
-          if (!(ok = mbar_wait(bar(C::B_VFULL + s), (idx / C::STAGES) & 1u, abort_flag))) break;
+          if (!(ok = wait(bar(C::B_VFULL + s), (idx / C::STAGES) & 1u))) break;
           bool k_next = false;  // K_(j+1) seen to have landed
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (!ok) break;
             const int b0 = u.kv_begin[i], e0 = u.kv_end[i];
             if (j < b0 || j >= e0) {
-              // a tile whose range starts one K/V tile later gets its first S now
               if (MASKS && j + 1 == b0 && b0 < e0) {
                 if (!k_next) {
-                  if (!(ok = mbar_wait(bar(C::B_KFULL + s1), ((idx + 1) / C::STAGES) & 1u,
-                                       abort_flag)))
-                    break;
+                  if (!(ok = wait(bar(C::B_KFULL + s1), ((idx + 1) / C::STAGES) & 1u))) break;
                   k_next = true;
                 }
                 uint32_t& qw = i ? q_waits1 : q_waits0;
-                if (!(ok = mbar_wait(bar(C::B_QFULL + i), qw & 1u, abort_flag))) break;
+                if (!(ok = wait(bar(C::B_QFULL + i), qw & 1u))) break;
                 ++qw;
                 tc_fence_after_sync();
-                issue_qk(i, s1);
-                umma_commit(bar(C::B_SFULL + i));
-                if (e0 == b0 + 1) umma_commit(bar(C::B_QFREE + i));
+                if (elect_one()) {
+                  issue_qk(i, s1);
+                  umma_commit(bar(C::B_SFULL + i));
+                  if (e0 == b0 + 1) umma_commit(bar(C::B_QFREE + i));
+                }
+                __syncwarp();
               }
               continue;
             }
             uint32_t& pw = i ? p_waits1 : p_waits0;
-            if (!(ok = mbar_wait(bar(C::B_PFULL + i), pw & 1u, abort_flag))) break;
+            if (!(ok = wait(bar(C::B_PFULL + i), pw & 1u))) break;
             ++pw;
             tc_fence_after_sync();
-            issue_pv(i, s, j > b0);
-            if (j + 1 < e0) {
-              if (!k_next) {
-                if (!(ok = mbar_wait(bar(C::B_KFULL + s1), ((idx + 1) / C::STAGES) & 1u,
-                                     abort_flag)))
-                  break;
-                tc_fence_after_sync();
-                k_next = true;
-              }
-              issue_qk(i, s1);
-              umma_commit(bar(C::B_SFULL + i));
-              if (j + 2 == e0) umma_commit(bar(C::B_QFREE + i));
-            } else {
-              umma_commit(bar(C::B_OFULL + i));
+            const bool more = j + 1 < e0;
+            if (more && !k_next) {
+              // K_(j+1) is normally in long before P_i(j); wait for it first so
+              // that PV and the next QK go out back to back
+              if (!(ok = wait(bar(C::B_KFULL + s1), ((idx + 1) / C::STAGES) & 1u))) break;
+              tc_fence_after_sync();
+              k_next = true;
             }
+            if (elect_one()) {
+              issue_pv(i, s, j > b0);
+              if (more) {
+                issue_qk(i, s1);
+                umma_commit(bar(C::B_SFULL + i));
+                if (j + 2 == e0) umma_commit(bar(C::B_QFREE + i));
+              } else {
+                umma_commit(bar(C::B_OFULL + i));
+              }
+            }
+            __syncwarp();
           }
-          umma_commit(bar(C::B_VEMPTY + s));
-          if (k_next) umma_commit(bar(C::B_KEMPTY + s1));
+          if (elect_one()) {
+            umma_commit(bar(C::B_VEMPTY + s));
+            if (k_next) umma_commit(bar(C::B_KEMPTY + s1));
+          }
+          __syncwarp();
         }
         kv += (uint32_t)(je - jb);
       }
       // Drain: every MMA issued above has completed before TMEM is released.
-      umma_commit(bar(C::B_DRAIN));
+      if (elect_one()) umma_commit(bar(C::B_DRAIN));
+      __syncwarp();
       mbar_wait(bar(C::B_DRAIN), 0, nullptr);
     }
     __syncwarp();

@@ -206,6 +206,17 @@ __device__ __forceinline__ uint32_t opaque_u32(uint32_t x) {
   return x;
 }
 
+// One lane of the (converged) warp gets true: the issuing lane of a
+// warp-uniform loop (the other lanes keep the loop's values in uniform
+// registers and run its waits, but issue nothing).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // Register reallocation between warpgroups (all four warps of a warpgroup
 // execute the same instruction).  The counts must add up to what the CTA was
 // launched with, or an increase waits forever: see the prefill kernel.

@@ -286,6 +286,33 @@ def quantize_e4m3_per_page(cache: torch.Tensor):
     return codes.contiguous(), sc.contiguous()
 
 
+def quantize_e4m3_blocks(x: torch.Tensor, block: int = 128):
+    """bf16 [B, H, S, d] -> (E4M3 codes uint8 [B, H, S, d], scales float32
+    [B, H, ceil(S / block)]) with scale = amax / 448 per block of `block`
+    consecutive rows of one (batch, head) (1 where the block is all zero), the
+    codes being round-to-nearest of x / scale (torch's float8_e4m3fn cast)."""
+    B, H, S, d = x.shape
+    nb = -(-S // block)
+    xf = x.float()
+    pad = nb * block - S
+    if pad:
+        xf = torch.cat([xf, torch.zeros(B, H, pad, d)], dim=2)
+    blocks = xf.view(B, H, nb, block, d)
+    amax = blocks.abs().amax(dim=(3, 4))
+    sc = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+    codes = (blocks / sc[:, :, :, None, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    codes = codes.view(B, H, nb * block, d)[:, :, :S].contiguous()
+    return codes, sc.contiguous()
+
+
+def fp8_prefill_inputs(B, Hq, Hkv, Sq, Sk, d, seed, value_scale=1.0):
+    """Block-scaled E4M3 prefill inputs drawn as ``prefill_inputs`` draws bf16
+    ones: (q8, k8, v8, q_scale, k_scale, v_scale)."""
+    q, k, v = prefill_inputs(B, Hq, Hkv, Sq, Sk, d, seed, value_scale)
+    (q8, qs), (k8, ks), (v8, vs) = (quantize_e4m3_blocks(t) for t in (q, k, v))
+    return q8, k8, v8, qs, ks, vs
+
+
 def fp8_paged_inputs(seq_lens, Hq, Hkv, d, page_size, seed, **kw) -> PagedFp8Inputs:
     """A paged cache as ``paged_inputs`` builds it, quantised to E4M3 with one
     scale per (page, KV head) for K and for V."""

@@ -96,6 +96,27 @@ int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float*
                     const int32_t* k_lens, attn_stream_t stream);
 
 /*
+ * attn_fwd_fp8 -- attn_fwd_masked over block-scaled E4M3 Q, K and V.
+ * Source: "Attention 算子加速史", section 3.3 (FP8 operands with block-level
+ * scaling); the operation is attn_fwd_masked's on the dequantised values.
+ *   q [B, Hq, Sq, d], k, v [B, Hkv, Sk, d]: uint8 E4M3 codes (OCP E4M3: bias
+ *   7, 3 mantissa bits, no infinity; 0x7F / 0xFF are NaN and must not occur)
+ *   q_scale [B, Hq, ceil(Sq/128)], k_scale, v_scale [B, Hkv, ceil(Sk/128)]
+ *   fp32 device arrays: element (b, h, i, :) of a tensor is
+ *   scale[b, h, i / 128] * e4m3(code).  Scales must be positive and finite.
+ *   o [B, Hq, Sq, d] bf16 and lse [B, Hq, Sq] fp32 (nullable) are written as
+ *   by attn_fwd_masked; causal, scale, k_lens likewise.
+ *   d must be 128.  S = Q K^T runs on E4M3 tensor-core MMAs (the two block
+ *   scales enter the fp32 scores); P V runs in bf16 on V widened exactly.
+ * Errors: as attn_fwd_masked, plus INVALID_ARG for a NULL scale array,
+ * UNSUPPORTED for d != 128, ALIGNMENT for scales not 4-byte aligned.
+ */
+int attn_fwd_fp8(const void* q, const void* k, const void* v, const float* q_scale,
+                 const float* k_scale, const float* v_scale, void* o, float* lse, int B, int Hq,
+                 int Hkv, int Sq, int Sk, int d, int causal, float scale, const int32_t* k_lens,
+                 attn_stream_t stream);
+
+/*
  * attn_fwd_window -- causal prefill with a sliding window or a prefix-LM mask.
  * Source: "Attention Kernel", section "可编程 mask" (masks such as a sliding
  * window or a prefix-LM rule: block-level sparsity decides which tiles are
@@ -385,6 +406,46 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
              const void* d_o, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk,
              int d, int causal, float scale, const int32_t* k_lens, void* workspace,
              size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * attn_bwd_varlen_workspace_size -- bytes of device workspace attn_bwd_varlen
+ * needs: 8 * B * Hq * ceil(max_seqlen_q / 128) * 128 (two fp32 row statistics
+ * per query row, each sequence padded to max_seqlen_q in whole 128-row tiles).
+ * 0 for invalid arguments.
+ */
+size_t attn_bwd_varlen_workspace_size(int B, int Hq, int max_seqlen_q);
+
+/*
+ * attn_bwd_varlen -- backward pass of attn_fwd_varlen (a ragged, packed batch).
+ * Source: "Attention Kernel", section "Backward 与重计算" (the backward uses
+ * the forward's scale, mask and head mapping, packed-sequence boundaries must
+ * agree with the forward's, and accumulation must be free of races), and
+ * section "Paged 与 ragged KV" (a ragged batch is a list of sequences given by
+ * cumulative lengths, each attended on its own).
+ *   Sequence b owns query tokens [cu_seqlens_q[b], cu_seqlens_q[b+1]) and keys
+ *   [cu_seqlens_k[b], cu_seqlens_k[b+1]); its gradients are those attn_bwd
+ *   gives for that sequence alone (bottom-right causal alignment when causal).
+ *   q, o, d_o, dq [total_q, Hq, d] bf16   k, v, dk, dv [total_k, Hkv, d] bf16
+ *   lse [Hq, total_q] fp32 (attn_fwd_varlen's layout)
+ *   cu_seqlens_q / cu_seqlens_k: device int32 [B + 1], non-decreasing from 0.
+ *   max_seqlen_q / max_seqlen_k bound every sequence's query / key length.
+ *   dq rows and dk, dv rows of every valid sequence are written (keys no query
+ *   sees get zero); tokens outside every sequence are not touched.
+ *   workspace: at least attn_bwd_varlen_workspace_size(B, Hq, max_seqlen_q)
+ *   bytes, 16-byte aligned, caller-owned, not shared with a concurrent call.
+ *   Deterministic (no atomics), as attn_bwd.
+ * Errors: INVALID_ARG (NULL pointers, B/Hq/Hkv < 1, Hq % Hkv != 0, totals or
+ * maxima out of range), UNSUPPORTED (d not 64 or 128), ALIGNMENT (tensors 16
+ * bytes, lse and offsets 4), WORKSPACE.  A sequence whose offsets are not
+ * valid (decreasing, outside [0, total], or longer than the maxima) is skipped
+ * -- none of its rows is written -- and sets ATTN_DEVERR_BAD_LENGTH.
+ * total_q = 0 does nothing; total_k = 0 only zero-fills dq.
+ */
+int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* d_o, void* dq, void* dk, void* dv, const int32_t* cu_seqlens_q,
+                    const int32_t* cu_seqlens_k, int B, int Hq, int Hkv, long long total_q,
+                    long long total_k, int max_seqlen_q, int max_seqlen_k, int d, int causal,
+                    float scale, void* workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /* attn_strerror -- static description of an attn_status value. */
 const char* attn_strerror(int status);

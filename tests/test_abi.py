@@ -337,3 +337,70 @@ def test_noalloc_scratch_size_matches_the_header():
     assert m, "ATTN_NOALLOC_SCRATCH_BYTES not found in attn.h"
     expr = m.group(1).replace("u", "").replace("U", "").replace("ll", "").replace("LL", "")
     assert eval(expr, {}, {}) == B.NOALLOC_SCRATCH_BYTES
+
+
+def _bwd_varlen(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, do=FAKE, dq=FAKE, dk=FAKE, dv=FAKE,
+                cu_q=FAKE, cu_k=FAKE, B_=2, Hq=2, Hkv=1, total_q=300, total_k=400, max_q=200,
+                max_k=250, d=128, causal=1, scale=0.1, ws=FAKE, ws_bytes=1 << 20):
+    return lib.attn_bwd_varlen(q, k, v, o, lse, do, dq, dk, dv, cu_q, cu_k, B_, Hq, Hkv, total_q,
+                               total_k, max_q, max_k, d, causal, scale, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(cu_q=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(cu_k=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(dk=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(B_=0), B.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), B.ATTN_ERR_INVALID_ARG),
+    (dict(total_q=-1), B.ATTN_ERR_INVALID_ARG),
+    (dict(max_q=0), B.ATTN_ERR_INVALID_ARG),
+    (dict(max_k=0), B.ATTN_ERR_INVALID_ARG),
+    (dict(causal=2), B.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), B.ATTN_ERR_INVALID_ARG),
+    (dict(d=96), B.ATTN_ERR_UNSUPPORTED),
+    (dict(q=FAKE + 8), B.ATTN_ERR_ALIGNMENT),
+    (dict(cu_q=FAKE + 2), B.ATTN_ERR_ALIGNMENT),
+    (dict(lse=FAKE + 1), B.ATTN_ERR_ALIGNMENT),
+    (dict(ws=FAKE + 4), B.ATTN_ERR_ALIGNMENT),
+    (dict(ws_bytes=2 * 2 * 2 * 256 * 4 - 1), B.ATTN_ERR_WORKSPACE),
+])
+def test_bwd_varlen_validation(lib, kw, status):
+    assert _bwd_varlen(lib, **kw) == status
+
+
+def test_bwd_varlen_workspace_size_formula(lib):
+    # two fp32 statistics per query row; every sequence padded to max_seqlen_q in 128-row tiles
+    assert lib.attn_bwd_varlen_workspace_size(2, 2, 200) == 2 * 2 * 2 * 256 * 4
+    assert lib.attn_bwd_varlen_workspace_size(16, 32, 8192) == 2 * 16 * 32 * 8192 * 4
+    assert lib.attn_bwd_varlen_workspace_size(0, 1, 1) == 0
+
+
+def _fwd_fp8(lib, q=FAKE, k=FAKE, v=FAKE, qs=FAKE, ks=FAKE, vs=FAKE, o=FAKE, lse=None, B_=1,
+             Hq=2, Hkv=2, Sq=128, Sk=128, d=128, causal=0, scale=0.1, k_lens=None):
+    return lib.attn_fwd_fp8(q, k, v, qs, ks, vs, o, lse, B_, Hq, Hkv, Sq, Sk, d, causal, scale,
+                            k_lens, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(qs=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(vs=None), B.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), B.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), B.ATTN_ERR_INVALID_ARG),
+    (dict(d=64), B.ATTN_ERR_UNSUPPORTED),
+    (dict(k=FAKE + 8), B.ATTN_ERR_ALIGNMENT),
+    (dict(ks=FAKE + 2), B.ATTN_ERR_ALIGNMENT),
+])
+def test_fwd_fp8_validation(lib, kw, status):
+    assert _fwd_fp8(lib, **kw) == status
+
+
+def test_fp8_prefill_binding_checks_codes_and_scales():
+    import torch
+    q8 = torch.zeros(1, 2, 130, 128, dtype=torch.uint8)
+    qs = torch.ones(1, 2, 2, dtype=torch.float32)
+    with pytest.raises(ValueError, match="uint8"):
+        B.attn_fwd_fp8(q8.float(), q8, q8, qs, qs, qs, True, 0.1)
+    with pytest.raises(ValueError, match="block scales"):  # one per 128-row block: [1, 2, 2]
+        B.attn_fwd_fp8(q8, q8, q8, qs[:, :, :1].contiguous(), qs, qs, True, 0.1)

@@ -99,3 +99,19 @@ def test_fp8_decode_deterministic_and_bad_page_flagged():
                           c.v_scale.to(DEV), c.block_table.to(DEV), c.seq_lens.to(DEV), 0.1)
     st, flags = attn_get_device_error()
     assert st != 0 and flags & 0x2
+
+
+def test_fp8_slots_past_the_length_never_reach_the_result():
+    """As for the bf16 cache: unused slots of the last page may hold the E4M3
+    NaN code (0x7F) without changing a bit of the result."""
+    c = W.fp8_paged_inputs(torch.tensor([37, 500, 16], dtype=torch.int32), 8, 2, 128, 16,
+                           seed=44)
+    o1, l1 = _run(c, 0.088)
+    kc, vc = c.k_cache.clone(), c.v_cache.clone()
+    for b, n in enumerate(c.seq_lens.tolist()):
+        last = int(c.block_table[b, (n - 1) // 16])
+        kc[last, n % 16 or 16:] = 0x7F
+        vc[last, n % 16 or 16:] = 0x7F
+    c2 = W.PagedFp8Inputs(c.q, kc, vc, c.k_scale, c.v_scale, c.block_table, c.seq_lens, 16)
+    o2, l2 = _run(c2, 0.088)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)

@@ -144,3 +144,20 @@ def test_bad_page_id_flagged_not_faulting():
     check(o[0], o_ref[0], lse[0], lse_ref[0], what="unaffected sequence")
     st, flags = attn_get_device_error()
     assert st == 0
+
+
+def test_slots_past_the_length_never_reach_the_result():
+    """The last page of a sequence is partial; its unused slots (and a whole
+    unused page) may hold anything, NaN included, without changing a bit."""
+    inp = W.paged_inputs(torch.tensor([37, 500, 16], dtype=torch.int32), 8, 2, 128, 16, seed=19,
+                         extra_pages=1)
+    o1, l1 = _run(inp, 0.088)
+    kc, vc = inp.k_cache.clone(), inp.v_cache.clone()
+    for b, n in enumerate(inp.seq_lens.tolist()):
+        last = int(inp.block_table[b, (n - 1) // 16])
+        kc[last, n % 16 or 16:] = float("nan")
+        vc[last, n % 16 or 16:] = float("nan")
+    kc[-1] = float("nan")  # the unused page
+    vc[-1] = float("nan")
+    o2, l2 = _run(W.PagedInputs(inp.q, kc, vc, inp.block_table, inp.seq_lens, 16), 0.088)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)

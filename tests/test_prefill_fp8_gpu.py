@@ -1,0 +1,90 @@
+"""GPU parity of attn_fwd_fp8 (prefill over block-scaled E4M3 Q, K, V) against
+the FP8 prefill oracle.
+
+"Attention 算子加速史", section 3.3: FP8 operands with block-level scaling.
+Inputs are the seeded bf16 workloads quantised per (batch, head, 128-row block)
+with scale = amax / 448 (``workloads.quantize_e4m3_blocks``); the CUDA path
+gets the codes and scales, the float64 oracle (``oracle/kv_fp8.py``,
+``attn_fwd_fp8``) the same bytes, dequantised from the format's definition.
+The comparison uses the forward's bar (``tests/parity.py``): the kernel's
+score products of E4M3 codes are exact, V is widened exactly, and the
+weights are rounded to bf16 as in the bf16 kernel.
+"""
+import math
+
+import pytest
+import torch
+
+from oracle.kv_fp8 import attn_fwd_fp8 as oracle_fp8
+from exact_softmax_attention_fwd_b200 import attn_fwd_fp8, attn_get_device_error
+from exact_softmax_attention_fwd_b200 import workloads as W
+
+from parity import check
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _run(q8, k8, v8, qs, ks, vs, causal, scale, k_lens=None):
+    dv = [t.to(DEV) for t in (q8, k8, v8, qs, ks, vs)]
+    kl = None if k_lens is None else k_lens.to(DEV)
+    o, lse = attn_fwd_fp8(*dv, causal, scale, k_lens=kl)
+    torch.cuda.synchronize()
+    st, flags = attn_get_device_error()
+    assert st == 0, f"device error flags {flags:#x}"
+    return o.cpu(), lse.cpu()
+
+
+CASES = [
+    # B, Hq, Hkv, Sq, Sk, causal
+    (1, 2, 2, 256, 256, False),
+    (1, 4, 2, 300, 300, True),     # ragged tail
+    (2, 4, 1, 129, 517, True),     # Sq < Sk: bottom-right diagonal
+    (2, 2, 2, 300, 100, True),     # Sq > Sk: leading rows see no key
+    (1, 8, 2, 640, 640, False),    # GQA, several key tiles
+    (1, 2, 2, 1024, 1024, True),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[str(c) for c in CASES])
+def test_fp8_prefill_cases(case):
+    B, Hq, Hkv, Sq, Sk, causal = case
+    x = W.fp8_prefill_inputs(B, Hq, Hkv, Sq, Sk, 128, seed=301 + Sq + Sk)
+    scale = 1 / math.sqrt(128)
+    o, lse = _run(*x, causal, scale)
+    o_ref, lse_ref = oracle_fp8(*x, causal, scale)
+    check(o, o_ref, lse, lse_ref, what=f"fp8 prefill {case}")
+
+
+def test_fp8_prefill_mha_causal_2k_full():
+    """The 2k causal workload's shapes (B=4, H=16, S=2048), quantised, every element."""
+    c = W.CONFIGS["mha_causal_2k"]
+    x = W.fp8_prefill_inputs(c.B, c.Hq, c.Hkv, c.S, c.S, c.d, seed=c.seed)
+    o, lse = _run(*x, True, c.scale)
+    o_ref, lse_ref = oracle_fp8(*x, True, c.scale)
+    check(o, o_ref, lse, lse_ref, what="fp8 mha_causal_2k")
+
+
+def test_fp8_prefill_key_padding_and_empty_rows():
+    x = W.fp8_prefill_inputs(3, 4, 2, 256, 256, 128, seed=303)
+    k_lens = torch.tensor([0, 77, 256], dtype=torch.int32)
+    o, lse = _run(*x, True, 0.088, k_lens=k_lens)
+    o_ref, lse_ref = oracle_fp8(*x, True, 0.088, k_lens=k_lens)
+    stats = check(o, o_ref, lse, lse_ref, what="fp8 padding")
+    assert stats["empty_rows"] > 0
+    assert torch.all(o[0] == 0) and torch.all(torch.isneginf(lse[0]))
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.2])
+def test_fp8_prefill_unusual_scales(scale):
+    x = W.fp8_prefill_inputs(1, 2, 1, 300, 300, 128, seed=305)
+    o, lse = _run(*x, True, scale)
+    o_ref, lse_ref = oracle_fp8(*x, True, scale)
+    check(o, o_ref, lse, lse_ref, what=f"fp8 scale {scale}")
+
+
+def test_fp8_prefill_deterministic():
+    x = W.fp8_prefill_inputs(2, 4, 2, 700, 700, 128, seed=307)
+    a = _run(*x, True, 0.088)
+    b = _run(*x, True, 0.088)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
