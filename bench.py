@@ -51,7 +51,8 @@ def parse_args():
     ap.add_argument("--workload", default="gqa_causal_32k")
     ap.add_argument("--prefill-legs",
                     default="mha_causal_2k,gqa_causal_8k,gqa_causal_8k_padded,tiny_mha",
-                    help="prefill configurations timed on their own after the headline")
+                    help="prefill configurations timed on their own after the headline "
+                         "('none' for no leg)")
     ap.add_argument("--decode-workload", default="paged_decode")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -61,6 +62,8 @@ def parse_args():
     ap.add_argument("--no-decode-fp8", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--backward-workloads", default="mha_causal_2k,gqa_causal_8k")
+    ap.add_argument("--no-prefill-fp8", action="store_true")
+    ap.add_argument("--prefill-fp8-workload", default="gqa_causal_8k")
     ap.add_argument("--no-paged-prefill", action="store_true")
     ap.add_argument("--paged-prefill-workload", default="paged_prefill_gqa")
     return ap.parse_args()
@@ -84,8 +87,10 @@ def load_peaks():
 KERNEL_SOURCES = {
     "attn_prefill_sm100_kernel": ("prefill_sm100.cuh", "varlen_schedule.cuh",
                                   "sm100_primitives.cuh"),
-    "attn_decode_split_kernel": ("decode_sm100.cuh", "sm100_primitives.cuh"),
-    "attn_decode_split_fp8_kernel": ("decode_sm100.cuh", "sm100_primitives.cuh"),
+    "attn_prefill_fp8_kernel": ("prefill_fp8_sm100.cuh", "prefill_sm100.cuh",
+                                "sm100_primitives.cuh"),
+    "attn_decode_split_tma_kernel": ("decode_sm100.cuh", "sm100_primitives.cuh"),
+    "attn_decode_split_tma_kernel_e4m3": ("decode_sm100.cuh", "sm100_primitives.cuh"),
     "attn_bwd_dkdv_kernel": ("bwd_sm100.cuh", "sm100_primitives.cuh"),
     "attn_bwd_dq_kernel": ("bwd_sm100.cuh", "sm100_primitives.cuh"),
 }
@@ -572,8 +577,8 @@ def run_ours(args, world, rank, local):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                          "achieved_median": decode_bytes / (dmed * 1e-3) / 1e9,
-                         "traffic": ncu_traffic("attn_decode_split_kernel", dcfg.name),
-                         "kernel": "attn_decode_split_kernel + attn_decode_merge_kernel",
+                         "traffic": ncu_traffic("attn_decode_split_tma_kernel", dcfg.name),
+                         "kernel": "attn_decode_split_tma_kernel + attn_decode_merge_kernel",
                          "peak_source": f"{peaks['source']} copy bandwidth",
                          "algorithmic_bytes": decode_bytes},
         }
@@ -586,10 +591,13 @@ def run_ours(args, world, rank, local):
     legs = {}
     for name in args.prefill_legs.split(","):
         name = name.strip()
-        if name and name != cfg.name:
+        if name and name != "none" and name != cfg.name:
             legs[name] = prefill_leg(args, W.CONFIGS[name], dev, world, peaks, cpu)
     if legs:
         line["prefill_legs"] = legs
+    if not args.no_prefill_fp8:
+        line["prefill_fp8"] = prefill_fp8_leg(args, W.CONFIGS[args.prefill_fp8_workload], dev,
+                                              world, peaks)
     if not args.no_ragged:
         line["ragged"] = ragged_leg(args, dev, world, peaks)
     if not args.no_paged_prefill:
@@ -607,6 +615,43 @@ def run_ours(args, world, rank, local):
         if dcfg is not None:
             line["decode"]["cpu_baseline"] = cpu_baseline_decode(dcfg, dinp)
     return line if rank == 0 else None
+
+
+def prefill_fp8_leg(args, cfg, dev, world, peaks):
+    """attn_fwd_fp8 on a prefill configuration's inputs quantised to E4M3 with one
+    scale per (batch, head, 128-row block), timed like the other legs.  FLOPs as
+    the bf16 prefill.  Roofline: Q K^T runs on E4M3 MMAs, P V on bf16 ones, so at
+    the tensor peaks the launch would take (F/2)/(2 P) + (F/2)/P = 0.75 F / P
+    with P the measured bf16 peak and 2 P the E4M3 rate (the nominal 2:1
+    ratio): the peak reported is P / 0.75."""
+    import torch
+
+    from exact_softmax_attention_fwd_b200 import attn_fwd_fp8, attn_get_device_error
+    from exact_softmax_attention_fwd_b200 import workloads as W
+
+    q8, k8, v8, qs, ks, vs = (t.to(dev) for t in W.fp8_prefill_inputs(
+        cfg.B, cfg.Hq, cfg.Hkv, cfg.S, cfg.S, cfg.d, cfg.seed, cfg.value_scale))
+    kl = None if not cfg.padded else W.key_padding(cfg.B, cfg.S).to(dev)
+    o = torch.empty(q8.shape, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((cfg.B, cfg.Hq, cfg.S), dtype=torch.float32, device=dev)
+
+    def one():
+        attn_fwd_fp8(q8, k8, v8, qs, ks, vs, cfg.causal, cfg.scale, k_lens=kl, out=o, lse=lse)
+
+    ms, clocks = timed_calls(args, dev, world, one)
+    st, fl = attn_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word set in the FP8 prefill leg: {fl:#x}")
+    peaks_mixed = dict(peaks)
+    peaks_mixed["bf16_tflops"] = peaks["bf16_tflops"] / 0.75
+    rl = tensor_roofline(cfg.flops(), ms, peaks_mixed, "attn_prefill_fp8_kernel", cfg.name, world)
+    rl["peak_source"] = (f"{peaks['source']} bf16 burst / 0.75 (Q K^T at twice the bf16 rate, "
+                         "P V at the bf16 rate)")
+    rl["frac_of_bf16_peak"] = rl["achieved"] / peaks["bf16_tflops"]
+    return {"workload": cfg.name + " (E4M3 Q, K, V; one scale per 128-row block)",
+            "value": world * rl["achieved"], "unit": "TFLOPS", "ms": rl["mean_ms"],
+            "median_ms": rl["median_ms"], "calls": len(ms), "gpu_launches_per_call": 1,
+            "clocks": clocks, "roofline": rl}
 
 
 def decode_fp8_leg(args, dev, world, peaks):
@@ -654,8 +699,8 @@ def decode_fp8_leg(args, dev, world, peaks):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes": nbytes,
                          "achieved_median": nbytes / (statistics.median(ms) * 1e-3) / 1e9,
-                         "kernel": "attn_decode_split_fp8_kernel + attn_decode_merge_kernel",
-                         "traffic": ncu_traffic("attn_decode_split_fp8_kernel", dcfg.name)}}
+                         "kernel": "attn_decode_split_tma_kernel (E4M3) + attn_decode_merge_kernel",
+                         "traffic": ncu_traffic("attn_decode_split_tma_kernel_e4m3", dcfg.name)}}
 
 
 def backward_leg(args, cfg, dev, world, peaks):

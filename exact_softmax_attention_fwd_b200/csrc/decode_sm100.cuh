@@ -629,17 +629,18 @@ __global__ void __launch_bounds__(128) attn_decode_split_fp8_kernel(const Decode
 // fragments are zeroed after the shared-memory load, so stale or non-finite
 // slot contents never reach the MMAs); bad ids are flagged.
 // ---------------------------------------------------------------------------
-constexpr int kDecodeStages = 4;
-
 template <int D, bool FP8>
 struct DecodeTmaCfg {
+  // ring depth: the bytes in flight per warp against the warps an SM holds
+  // (shared memory per warp grows with the depth)
+  static constexpr int STAGES = FP8 ? 4 : 4;
   static constexpr int E = FP8 ? 1 : 2;            // bytes per element
   static constexpr int ROW = D * E;                // bytes per token row of one head
   static constexpr int BOX_BYTES = ROW < 128 ? ROW : 128;  // inner box extent in bytes
   static constexpr int NBOX = ROW / BOX_BYTES;     // column boxes per row
   static constexpr int TILE = 16 * ROW;            // 16 tokens of K (or V)
   static constexpr int STAGE = 2 * TILE;           // K then V
-  static constexpr int SMEM = kDecodeStages * STAGE + 64 + 1024;  // ring, barriers, alignment
+  static constexpr int SMEM = STAGES * STAGE + 64 + 1024;  // ring, barriers, alignment
   static_assert(kSplitTokens / 16 <= 32, "one block-table entry per lane");
 };
 
@@ -680,7 +681,7 @@ __global__ void __launch_bounds__(32) attn_decode_split_tma_kernel(
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
-  const uint32_t bars = sbase + kDecodeStages * C::STAGE;
+  const uint32_t bars = sbase + C::STAGES * C::STAGE;
   const int lane = threadIdx.x;
   const int split = blockIdx.x;
   const int kvh = blockIdx.y;
@@ -708,18 +709,18 @@ __global__ void __launch_bounds__(32) attn_decode_split_tma_kernel(
     }
   }
   if (lane == 0) {
-    for (int s = 0; s < kDecodeStages; ++s) mbar_init(bars + 8u * s, 1);
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(bars + 8u * s, 1);
     mbar_init_fence();
     tma_prefetch_map(&tm_k);
     tma_prefetch_map(&tm_v);
   }
   __syncwarp();
-  // Step i's copies into slot i % kDecodeStages (lane 0; every lane calls it for
+  // Step i's copies into slot i % C::STAGES (lane 0; every lane calls it for
   // the shuffle).  A step on a bad page arms its barrier with no bytes.
   auto issue = [&](int i) {
     const int pg = __shfl_sync(0xffffffffu, my_page, i);
     if (lane == 0) {
-      const int slot = i % kDecodeStages;
+      const int slot = i % C::STAGES;
       const uint32_t bar = bars + 8u * slot;
       const uint32_t dst = sbase + slot * C::STAGE;
       fence_proxy_async_smem();  // the warp's reads of this slot precede the refill
@@ -736,7 +737,7 @@ __global__ void __launch_bounds__(32) attn_decode_split_tma_kernel(
     }
   };
   int n_issued = 0;
-  for (; n_issued < kDecodeStages - 1 && n_issued < n_steps; ++n_issued) issue(n_issued);
+  for (; n_issued < C::STAGES - 1 && n_issued < n_steps; ++n_issued) issue(n_issued);
 
   const int g = lane >> 2;   // MMA group id: head row of S / P, d-row block of V^T
   const int tq = lane & 3;   // thread within the group
@@ -797,15 +798,15 @@ __global__ void __launch_bounds__(32) attn_decode_split_tma_kernel(
   int i = 0;
 #pragma unroll 1
   for (; i < n_steps; ++i) {
-    if (n_issued < n_steps) issue(n_issued++);  // step i + kDecodeStages - 1
-    const int slot = i % kDecodeStages;
+    if (n_issued < n_steps) issue(n_issued++);  // step i + C::STAGES - 1
+    const int slot = i % C::STAGES;
     const int pg = __shfl_sync(0xffffffffu, my_page, i);
     const int n_here = pg >= 0 ? min(16, t_end - (t_begin + 16 * i)) : 0;
     const float ksc = FP8 ? __shfl_sync(0xffffffffu, my_ks, i) : 1.f;
     const float vsc = FP8 ? __shfl_sync(0xffffffffu, my_vs, i) : 1.f;
     const uint32_t kt = sbase + slot * C::STAGE;
     const uint32_t vt = kt + C::TILE;
-    const bool landed = mbar_wait(bars + 8u * slot, (uint32_t)(i / kDecodeStages) & 1u, nullptr);
+    const bool landed = mbar_wait(bars + 8u * slot, (uint32_t)(i / C::STAGES) & 1u, nullptr);
     if (!__all_sync(0xffffffffu, landed)) break;  // timed out: flagged, wind down
 
     // ---- S = q K^T (16 padded head rows x 16 tokens)
@@ -933,7 +934,7 @@ __global__ void __launch_bounds__(32) attn_decode_split_tma_kernel(
   // (steps [i, n_issued) were issued but not consumed; bounded waits)
   if (lane == 0)
     for (int j = i; j < n_issued; ++j)
-      mbar_wait(bars + 8u * (j % kDecodeStages), (uint32_t)(j / kDecodeStages) & 1u, nullptr);
+      mbar_wait(bars + 8u * (j % C::STAGES), (uint32_t)(j / C::STAGES) & 1u, nullptr);
   __syncwarp();
 
   // ---- this split's normalised partial output and its log2-sum-exp

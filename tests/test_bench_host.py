@@ -47,8 +47,8 @@ def test_source_hash_is_per_kernel_family(fake_root):
     after = {k: bench.kernel_source_sha(k) for k in bench.KERNEL_SOURCES}
     assert after["attn_bwd_dkdv_kernel"] != before["attn_bwd_dkdv_kernel"]
     assert after["attn_bwd_dq_kernel"] != before["attn_bwd_dq_kernel"]
-    for k in ("attn_prefill_sm100_kernel", "attn_decode_split_kernel",
-              "attn_decode_split_fp8_kernel"):
+    for k in ("attn_prefill_sm100_kernel", "attn_prefill_fp8_kernel",
+              "attn_decode_split_tma_kernel", "attn_decode_split_tma_kernel_e4m3"):
         assert after[k] == before[k], k
     _touch(fake_root, "sm100_primitives.cuh")  # shared by every family
     again = {k: bench.kernel_source_sha(k) for k in bench.KERNEL_SOURCES}

@@ -157,7 +157,10 @@ def test_slots_past_the_length_never_reach_the_result():
         last = int(inp.block_table[b, (n - 1) // 16])
         kc[last, n % 16 or 16:] = float("nan")
         vc[last, n % 16 or 16:] = float("nan")
-    kc[-1] = float("nan")  # the unused page
-    vc[-1] = float("nan")
+    used = set(int(x) for x in inp.block_table.flatten().tolist() if x >= 0)
+    unused = [pg for pg in range(inp.num_pages) if pg not in used]
+    assert len(unused) == 1
+    kc[unused[0]] = float("nan")  # the page no sequence references
+    vc[unused[0]] = float("nan")
     o2, l2 = _run(W.PagedInputs(inp.q, kc, vc, inp.block_table, inp.seq_lens, 16), 0.088)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
