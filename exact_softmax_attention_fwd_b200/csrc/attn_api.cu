@@ -375,10 +375,6 @@ int decode_paged_common(bool fp8, const void* q, const void* k_cache, const void
   DecodeParams prm;
   std::memset(&prm, 0, sizeof(prm));
   prm.q = static_cast<const uint16_t*>(q);
-  if (!fp8) {
-    prm.k_cache = static_cast<const uint16_t*>(k_cache);
-    prm.v_cache = static_cast<const uint16_t*>(v_cache);
-  }
   prm.block_table = block_table;
   prm.seq_lens = seq_lens;
   prm.B = B;
@@ -398,8 +394,6 @@ int decode_paged_common(bool fp8, const void* q, const void* k_cache, const void
 
   DecodeFp8Params pf;
   pf.d = prm;
-  pf.k8 = static_cast<const uint8_t*>(k_cache);
-  pf.v8 = static_cast<const uint8_t*>(v_cache);
   pf.k_scale = k_scale;
   pf.v_scale = v_scale;
   // K/V reach the split kernel through tensor maps over the pool, read as the

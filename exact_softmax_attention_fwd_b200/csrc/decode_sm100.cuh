@@ -9,31 +9,30 @@
 // log-sum-exp, a light kernel merges them) and "Attention Kernel", section
 // "Online softmax" (the merge rule).
 //
-// Split kernel: one warp per (sequence b, KV head, split of kSplitTokens
-// tokens).  The warp serves all Hq/Hkv query heads that share the KV head
-// (GQA), 16 tokens at a time, with warp-level bf16 MMAs whose operands come
-// straight from global memory into registers -- no shared memory:
+// Split kernel: one warp (and CTA) per (sequence b, KV head, split of
+// kSplitTokens tokens).  The warp serves all Hq/Hkv query heads that share the
+// KV head (GQA), 16 tokens at a time, with warp-level MMAs:
 //   S (heads x 16 tokens)  = q (16 padded heads x d) . K^T
 //   O^T (d x heads)       += V^T (d x 16 tokens) . P^T (16 tokens x heads)
 // The contraction index of each MMA may be permuted freely as long as both
 // operands use the same permutation, and an output index may be relabelled
 // if the write-back uses the same labels.  Both are chosen so that every
-// thread loads 16-byte contiguous pieces of K and V rows: for K a thread owns
+// thread reads 16-byte contiguous pieces of K and V rows: for K a thread owns
 // a contiguous quarter of a row, for V a contiguous eighth of four rows.
-// The next 16 tokens' K (V) are requested as soon as the current K (V)
-// registers are consumed, so loads overlap the softmax and the other MMA.
+// K and V reach the warp through a ring of shared-memory slots filled by
+// tensor-memory-access copies (see attn_decode_split_tma_kernel), so that the
+// bytes in flight cost no registers.
 //
-// FP8 cache (attn_decode_split_fp8_kernel; "Attention Kernel", section
-// "正确性契约": the cache quantisation schema is part of the contract;
-// "Attention 算子加速史", section 3: FP8 operands with scale factors): K and V
-// may be stored as E4M3 bytes with one fp32 scale per (physical page, KV
-// head).  The kernel then streams half the bytes, keeps the raw bytes in the
-// prefetch registers and widens them to f16 right before use (exact: E4M3 has
-// 3 mantissa bits and a narrower exponent range).  q K^T is an f16 MMA on q
-// scaled by a power of two into f16's range; its fp32 scores are multiplied
-// back and by the page's K scale.  P^T V is an f16 MMA (P <= 1 is rounded to
-// f16) whose fp32 result for the 16 tokens -- which always lie in one page --
-// is multiplied by the page's V scale before it joins the accumulator.
+// FP8 cache ("Attention Kernel", section "正确性契约": the cache quantisation
+// schema is part of the contract; "Attention 算子加速史", section 3: FP8
+// operands with scale factors): K and V may be stored as E4M3 bytes with one
+// fp32 scale per (physical page, KV head).  The kernel then streams half the
+// bytes and widens them to f16 right before use (exact: E4M3 has 3 mantissa
+// bits and a narrower exponent range).  q K^T is an f16 MMA on q scaled by a
+// power of two into f16's range; its fp32 scores are multiplied back and by
+// the page's K scale.  P^T V is an f16 MMA (P <= 1 is rounded to f16) whose
+// fp32 result for the 16 tokens -- which always lie in one page -- is
+// multiplied by the page's V scale before it joins the accumulator.
 //
 // Merge kernel: one warp per (b, query head) combines the splits in a fixed
 // order: LSE = M + log2 sum_s 2^(lse_s - M), O = sum_s 2^(lse_s - LSE) o_s,
@@ -50,8 +49,6 @@ constexpr int kSplitTokens = 512;
 
 struct DecodeParams {
   const uint16_t* q;        // [B, Hq, D]
-  const uint16_t* k_cache;  // [num_pages, page_size, Hkv, D]
-  const uint16_t* v_cache;
   const int* block_table;   // [B, max_pages]
   const int* seq_lens;      // [B]
   float* o_part;            // [B, Hq, n_split, D]
@@ -62,15 +59,11 @@ struct DecodeParams {
   float scale_log2;
 };
 
-// Parameters of the FP8 split kernel: the decode parameters (k_cache and
-// v_cache unused) plus the E4M3 caches and their scales.  (A separate struct:
-// growing DecodeParams itself raised the bf16 split kernel's register count
-// past the 168 that keeps three blocks resident.)
+// Parameters of the split kernel: the decode parameters plus, for E4M3
+// caches, the K and V scales (the cache pointers live in the tensor maps).
 struct DecodeFp8Params {
   DecodeParams d;
-  const uint8_t* k8;     // [num_pages, page_size, Hkv, D] E4M3 codes
-  const uint8_t* v8;
-  const float* k_scale;  // [num_pages, Hkv]
+  const float* k_scale;  // [num_pages, Hkv] (E4M3 caches only)
   const float* v_scale;
 };
 
@@ -84,18 +77,6 @@ __device__ __forceinline__ int decode_clamped_len(const DecodeParams& p, int b, 
   return len;
 }
 
-template <int D>
-struct DecodeGroupRegs {
-  uint32_t k[2][D / 8];   // tokens nc*8 + g (nc = 0, 1): D/4 bf16 each
-  uint32_t v[4][D / 16];  // tokens 2tq, 2tq+1, 2tq+8, 2tq+9: D/8 bf16 each
-};
-
-template <int D>
-struct DecodeGroupRegs8 {  // the elements of DecodeGroupRegs as raw E4M3 bytes
-  uint32_t k[2][D / 16];
-  uint32_t v[4][D / 32];
-};
-
 // Two E4M3 bytes (bits 0-7 and 8-15) -> f16x2 (exact), element order kept.
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
   uint32_t r;
@@ -107,11 +88,6 @@ __device__ __forceinline__ float f16_to_f32(uint32_t h16) {
   float f;
   asm("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"((unsigned short)(h16 & 0xFFFFu)));
   return f;
-}
-
-// f16x2 holding E4M3 values -> bf16x2 (exact for those values).
-__device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
-  return pack_bf16x2(f16_to_f32(h), f16_to_f32(h >> 16));
 }
 
 // Two floats -> packed f16x2 (round to nearest even); `lo` lands in bits 0-15.
@@ -129,481 +105,6 @@ __device__ __forceinline__ void mma_m16n8k16_f16(float (&c)[4], uint32_t a0, uin
       "{%8, %9}, {%0, %1, %2, %3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-template <int D>
-__device__ __forceinline__ bool decode_page_row(const DecodeParams& p, int b, int t0, int& page,
-                                                int& row) {
-  page = p.block_table[(size_t)b * p.max_pages + t0 / p.page_size];
-  row = t0 % p.page_size;
-  return page >= 0 && page < p.num_pages;
-}
-
-// K rows for 16 tokens starting at logical token t0 (page-relative row `row`).
-template <int D>
-__device__ __forceinline__ void decode_load_k(const DecodeParams& p, int page, int row, int kvh,
-                                              int g, int tq, int n_valid, uint32_t (&k)[2][D / 8]) {
-#pragma unroll
-  for (int nc = 0; nc < 2; ++nc) {
-    const int tok = nc * 8 + g;
-    if (tok < n_valid) {
-      const uint16_t* src = p.k_cache +
-                            (((size_t)page * p.page_size + row + tok) * p.Hkv + kvh) * D +
-                            (D / 4) * tq;
-#pragma unroll
-      for (int w = 0; w < D / 32; ++w) {
-        const uint4 x = ld_stream_v4(src + 8 * w);
-        k[nc][4 * w + 0] = x.x;
-        k[nc][4 * w + 1] = x.y;
-        k[nc][4 * w + 2] = x.z;
-        k[nc][4 * w + 3] = x.w;
-      }
-    } else {
-#pragma unroll
-      for (int w = 0; w < D / 8; ++w) k[nc][w] = 0u;
-    }
-  }
-}
-
-template <int D>
-__device__ __forceinline__ void decode_load_v(const DecodeParams& p, int page, int row, int kvh,
-                                              int g, int tq, int n_valid, uint32_t (&v)[4][D / 16]) {
-#pragma unroll
-  for (int ti = 0; ti < 4; ++ti) {
-    const int tok = 2 * tq + (ti & 1) + 8 * (ti >> 1);
-    if (tok < n_valid) {
-      const uint16_t* src = p.v_cache +
-                            (((size_t)page * p.page_size + row + tok) * p.Hkv + kvh) * D +
-                            (D / 8) * g;
-#pragma unroll
-      for (int w = 0; w < D / 64; ++w) {
-        const uint4 x = ld_stream_v4(src + 8 * w);
-        v[ti][4 * w + 0] = x.x;
-        v[ti][4 * w + 1] = x.y;
-        v[ti][4 * w + 2] = x.z;
-        v[ti][4 * w + 3] = x.w;
-      }
-    } else {
-#pragma unroll
-      for (int w = 0; w < D / 16; ++w) v[ti][w] = 0u;  // masked tokens must not inject NaN
-    }
-  }
-}
-
-// As decode_load_k / decode_load_v, for E4M3 caches: the same elements, one
-// byte each (a K quarter row is D/4 bytes, a V eighth row D/8 bytes).
-template <int D>
-__device__ __forceinline__ void decode_load_k8(const DecodeFp8Params& f, int page, int row, int kvh,
-                                               int g, int tq, int n_valid,
-                                               uint32_t (&k)[2][D / 16]) {
-#pragma unroll
-  for (int nc = 0; nc < 2; ++nc) {
-    const int tok = nc * 8 + g;
-    if (tok < n_valid) {
-      const uint8_t* src =
-          f.k8 + (((size_t)page * f.d.page_size + row + tok) * f.d.Hkv + kvh) * D + (D / 4) * tq;
-#pragma unroll
-      for (int w = 0; w < D / 64; ++w) {
-        const uint4 x = ld_stream_v4(src + 16 * w);
-        k[nc][4 * w + 0] = x.x;
-        k[nc][4 * w + 1] = x.y;
-        k[nc][4 * w + 2] = x.z;
-        k[nc][4 * w + 3] = x.w;
-      }
-    } else {
-#pragma unroll
-      for (int w = 0; w < D / 16; ++w) k[nc][w] = 0u;
-    }
-  }
-}
-
-template <int D>
-__device__ __forceinline__ void decode_load_v8(const DecodeFp8Params& f, int page, int row, int kvh,
-                                               int g, int tq, int n_valid,
-                                               uint32_t (&v)[4][D / 32]) {
-#pragma unroll
-  for (int ti = 0; ti < 4; ++ti) {
-    const int tok = 2 * tq + (ti & 1) + 8 * (ti >> 1);
-    if (tok < n_valid) {
-      const uint8_t* src =
-          f.v8 + (((size_t)page * f.d.page_size + row + tok) * f.d.Hkv + kvh) * D + (D / 8) * g;
-      if constexpr (D == 128) {
-        const uint4 x = ld_stream_v4(src);
-        v[ti][0] = x.x;
-        v[ti][1] = x.y;
-        v[ti][2] = x.z;
-        v[ti][3] = x.w;
-      } else {
-        const uint2 x = __ldg(reinterpret_cast<const uint2*>(src));
-        v[ti][0] = x.x;
-        v[ti][1] = x.y;
-      }
-    } else {
-#pragma unroll
-      for (int w = 0; w < D / 32; ++w) v[ti][w] = 0u;  // zero bytes are +0.0
-    }
-  }
-}
-
-template <int D>
-__global__ void __launch_bounds__(128) attn_decode_split_kernel(const DecodeParams p) {
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int split = blockIdx.x * 4 + warp;
-  const int kvh = blockIdx.y;
-  const int b = blockIdx.z;
-  if (split >= p.n_split) return;
-  const int len = decode_clamped_len(p, b, lane == 0 && split == 0 && kvh == 0);
-  const int t_begin = split * kSplitTokens;
-  if (t_begin >= len) return;  // the merge kernel never reads splits past the end
-  const int t_end = min(t_begin + kSplitTokens, len);
-
-  const int g = lane >> 2;   // MMA group id: head row of S / P, d-row block of V^T
-  const int tq = lane & 3;   // thread within the group
-  const int hq0 = kvh * p.group;
-
-  // q as the A operand of S = q K^T: row g = query head hq0 + g (rows g + 8 and
-  // heads beyond the group are zero padding); k-chunk kc holds
-  // d = (D/4)*tq + 4*kc + {0,1} (a0a1) and + {2,3} (a4a5).
-  uint32_t qa[D / 16][2];
-  if (g < p.group) {
-    const uint16_t* src = p.q + ((size_t)b * p.Hq + hq0 + g) * D + (D / 4) * tq;
-#pragma unroll
-    for (int w = 0; w < D / 32; ++w) {
-      const uint4 x = *reinterpret_cast<const uint4*>(src + 8 * w);
-      qa[2 * w][0] = x.x;
-      qa[2 * w][1] = x.y;
-      qa[2 * w + 1][0] = x.z;
-      qa[2 * w + 1][1] = x.w;
-    }
-  } else {
-#pragma unroll
-    for (int kc = 0; kc < D / 16; ++kc) qa[kc][0] = qa[kc][1] = 0u;
-  }
-
-  float c2 = p.scale_log2;
-  const bool scale_pos = c2 > 0.f;
-  if (!scale_pos) c2 = 1.f;
-  float m_run = -INFINITY;  // per head row g, log2 units
-  float l_run = 0.f;   // sum of P (f32): the LSE
-  float lr_run = 0.f;  // sum of bf16(P): normalises O
-  float acc[D / 16][4];
-#pragma unroll
-  for (int mc = 0; mc < D / 16; ++mc) acc[mc][0] = acc[mc][1] = acc[mc][2] = acc[mc][3] = 0.f;
-
-  DecodeGroupRegs<D> cur;
-  int page, row;
-  bool page_ok = decode_page_row<D>(p, b, t_begin, page, row);
-  int n_valid = page_ok ? min(16, t_end - t_begin) : 0;
-  if (!page_ok && lane == 0) flag_device_error(kDevErrBadPage);
-  decode_load_k<D>(p, page, row, kvh, g, tq, n_valid, cur.k);
-  decode_load_v<D>(p, page, row, kvh, g, tq, n_valid, cur.v);
-
-#pragma unroll 1
-  for (int t0 = t_begin; t0 < t_end; t0 += 16) {
-    const int n_here = n_valid;
-    const int t1 = t0 + 16;
-    int page_n = 0, row_n = 0, n_next = 0;
-    if (t1 < t_end) {
-      const bool ok_n = decode_page_row<D>(p, b, t1, page_n, row_n);
-      if (!ok_n && lane == 0) flag_device_error(kDevErrBadPage);
-      n_next = ok_n ? min(16, t_end - t1) : 0;
-    }
-
-    // ---- S = q K^T (16 padded head rows x 16 tokens)
-    float sc[2][4];
-#pragma unroll
-    for (int nc = 0; nc < 2; ++nc) {
-      sc[nc][0] = sc[nc][1] = sc[nc][2] = sc[nc][3] = 0.f;
-#pragma unroll
-      for (int kc = 0; kc < D / 16; ++kc)
-        mma_m16n8k16_bf16(sc[nc], qa[kc][0], 0u, qa[kc][1], 0u, cur.k[nc][2 * kc],
-                          cur.k[nc][2 * kc + 1]);
-    }
-    if (t1 < t_end) decode_load_k<D>(p, page_n, row_n, kvh, g, tq, n_next, cur.k);
-
-    // ---- online softmax for head row g over this thread's 4 tokens
-    float s4[4] = {sc[0][0], sc[0][1], sc[1][0], sc[1][1]};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int tok = (e >> 1) * 8 + 2 * tq + (e & 1);
-      if (tok >= n_here) s4[e] = -INFINITY;
-      else if (!scale_pos) s4[e] *= p.scale_log2;
-    }
-    float mx = fmaxf(fmaxf(s4[0], s4[1]), fmaxf(s4[2], s4[3]));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float m_new = fmaxf(m_run, mx * c2);
-    // nothing accumulated while m_run = -inf (also avoids -inf - -inf = NaN)
-    const float alpha = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_new);
-    const float base = (m_new == -INFINITY) ? 0.f : m_new;
-    float pr[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) pr[e] = ex2(fmaf(s4[e], c2, -base));
-    const uint32_t pb0 = pack_bf16x2(pr[0], pr[1]);  // P^T rows 2tq, 2tq+1 (tokens), column g (head)
-    const uint32_t pb1 = pack_bf16x2(pr[2], pr[3]);  // tokens 2tq+8, 2tq+9
-    // row sums over the f32 P (for the LSE) and over the bf16-rounded P that
-    // the MMA consumes (normalises O)
-    float rs = (pr[0] + pr[1]) + (pr[2] + pr[3]);
-    float rr = sum_f32x2(add_f32x2(bf16x2_to_f32x2(pb0), bf16x2_to_f32x2(pb1)));
-    rs += __shfl_xor_sync(0xffffffffu, rs, 1);
-    rr += __shfl_xor_sync(0xffffffffu, rr, 1);
-    rs += __shfl_xor_sync(0xffffffffu, rs, 2);
-    rr += __shfl_xor_sync(0xffffffffu, rr, 2);
-    l_run = l_run * alpha + rs;
-    lr_run = lr_run * alpha + rr;
-    m_run = m_new;
-
-    // ---- O^T += V^T P^T; accumulator columns are heads 2tq and 2tq+1
-    const float a_h0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
-    const float a_h1 = __shfl_sync(0xffffffffu, alpha, (2 * tq + 1) * 4);
-#pragma unroll
-    for (int mc = 0; mc < D / 16; ++mc) {
-      acc[mc][0] *= a_h0;
-      acc[mc][1] *= a_h1;
-      acc[mc][2] *= a_h0;
-      acc[mc][3] *= a_h1;
-      // A = V^T block: row g <-> d = (D/8)*g + 2*mc, row g+8 <-> d + 1;
-      // columns = tokens 2tq, 2tq+1 (a0a1, a2a3) and 2tq+8, 2tq+9 (a4a5, a6a7).
-      const uint32_t a01 = prmt(cur.v[0][mc], cur.v[1][mc], 0x5410u);
-      const uint32_t a23 = prmt(cur.v[0][mc], cur.v[1][mc], 0x7632u);
-      const uint32_t a45 = prmt(cur.v[2][mc], cur.v[3][mc], 0x5410u);
-      const uint32_t a67 = prmt(cur.v[2][mc], cur.v[3][mc], 0x7632u);
-      mma_m16n8k16_bf16(acc[mc], a01, a23, a45, a67, pb0, pb1);
-    }
-    if (t1 < t_end) decode_load_v<D>(p, page_n, row_n, kvh, g, tq, n_next, cur.v);
-    n_valid = n_next;
-  }
-
-  // ---- write this split's normalised partial output and its log2-sum-exp
-  const int h0 = 2 * tq, h1 = 2 * tq + 1;
-  const float l_h0 = __shfl_sync(0xffffffffu, lr_run, h0 * 4);
-  const float l_h1 = __shfl_sync(0xffffffffu, lr_run, h1 * 4);
-  const float inv0 = l_h0 > 0.f ? 1.f / l_h0 : 0.f;
-  const float inv1 = l_h1 > 0.f ? 1.f / l_h1 : 0.f;
-  const int dbase = (D / 8) * g;
-#pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const int h = hh ? h1 : h0;
-    if (h >= p.group) continue;
-    const float inv = hh ? inv1 : inv0;
-    float* dst = p.o_part + (((size_t)b * p.Hq + hq0 + h) * p.n_split + split) * D + dbase;
-#pragma unroll
-    for (int mc = 0; mc < D / 16; mc += 2) {
-      float4 w;
-      w.x = acc[mc][hh] * inv;          // d = dbase + 2mc
-      w.y = acc[mc][2 + hh] * inv;      // d = dbase + 2mc + 1
-      w.z = acc[mc + 1][hh] * inv;      // d = dbase + 2mc + 2
-      w.w = acc[mc + 1][2 + hh] * inv;  // d = dbase + 2mc + 3
-      *reinterpret_cast<float4*>(dst + 2 * mc) = w;
-    }
-  }
-  if (tq == 0 && g < p.group) {
-    const float lse2 = l_run > 0.f ? m_run + lg2(l_run) : -INFINITY;
-    p.lse_part[((size_t)b * p.Hq + hq0 + g) * p.n_split + split] = lse2;
-  }
-}
-
-// attn_decode_split_kernel over E4M3 caches (the FP8 notes at the top): the
-// same warp decomposition, loads of half the bytes, widening to f16 right
-// before each (f16) MMA, the K scale on the fp32 scores and the V scale on
-// each page's fp32 partial P V.
-template <int D>
-__global__ void __launch_bounds__(128) attn_decode_split_fp8_kernel(const DecodeFp8Params f) {
-  const DecodeParams& p = f.d;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int split = blockIdx.x * 4 + warp;
-  const int kvh = blockIdx.y;
-  const int b = blockIdx.z;
-  if (split >= p.n_split) return;
-  const int len = decode_clamped_len(p, b, lane == 0 && split == 0 && kvh == 0);
-  const int t_begin = split * kSplitTokens;
-  if (t_begin >= len) return;
-  const int t_end = min(t_begin + kSplitTokens, len);
-
-  const int g = lane >> 2;
-  const int tq = lane & 3;
-  const int hq0 = kvh * p.group;
-
-  // q as the f16 A operand of S = q K^T (fragment layout as in
-  // attn_decode_split_kernel), so that K needs a single E4M3 -> f16 widening.
-  // The row is multiplied by 2^-qe first, qe >= 0 the smallest exponent that
-  // keeps every |q| below 2^14 (f16's range ends at 65504), and the scores by
-  // 2^qe after the MMA: bf16's 8 significant bits fit f16's 11, so q is carried
-  // exactly except for elements below 2^-14 * 2^qe (f16 subnormals), which
-  // lose bits at 2^-25 * 2^qe -- far below the scores' own fp32 rounding.
-  uint32_t qa[D / 16][2];
-  float qscale = 1.f;  // 2^qe
-  {
-    uint32_t raw[D / 8];
-    float mxq = 0.f;
-    if (g < p.group) {
-      const uint16_t* src = p.q + ((size_t)b * p.Hq + hq0 + g) * D + (D / 4) * tq;
-#pragma unroll
-      for (int w = 0; w < D / 32; ++w) {
-        const uint4 x = *reinterpret_cast<const uint4*>(src + 8 * w);
-        raw[4 * w + 0] = x.x;
-        raw[4 * w + 1] = x.y;
-        raw[4 * w + 2] = x.z;
-        raw[4 * w + 3] = x.w;
-      }
-#pragma unroll
-      for (int w = 0; w < D / 8; ++w)
-        mxq = fmaxf(mxq, fmaxf(fabsf(__uint_as_float(raw[w] << 16)),
-                               fabsf(__uint_as_float(raw[w] & 0xFFFF0000u))));
-    } else {
-#pragma unroll
-      for (int w = 0; w < D / 8; ++w) raw[w] = 0u;
-    }
-    mxq = fmaxf(mxq, __shfl_xor_sync(0xffffffffu, mxq, 1));  // the row's 4 threads
-    mxq = fmaxf(mxq, __shfl_xor_sync(0xffffffffu, mxq, 2));
-    int qe = 0;
-    if (mxq >= 16384.f) qe = ilogbf(mxq) - 13;  // mxq < 2^(qe + 14): |q| * 2^-qe < 2^14
-    qscale = ldexpf(1.f, qe);
-    const float qinv = ldexpf(1.f, -qe);
-#pragma unroll
-    for (int w = 0; w < D / 8; ++w) {
-      const uint32_t h = pack_f16x2(__uint_as_float(raw[w] << 16) * qinv,
-                                    __uint_as_float(raw[w] & 0xFFFF0000u) * qinv);
-      qa[w >> 1][w & 1] = h;  // word w: d = (D/4)*tq + 2*w, +1 (a0a1 / a4a5 of chunk w/2)
-    }
-  }
-
-  float c2 = p.scale_log2;
-  const bool scale_pos = c2 > 0.f;
-  if (!scale_pos) c2 = 1.f;
-  float m_run = -INFINITY;
-  float l_run = 0.f;   // sum of P (f32): the LSE
-  float lr_run = 0.f;  // sum of f16(P): normalises O
-  float acc[D / 16][4];
-#pragma unroll
-  for (int mc = 0; mc < D / 16; ++mc) acc[mc][0] = acc[mc][1] = acc[mc][2] = acc[mc][3] = 0.f;
-
-  DecodeGroupRegs8<D> cur;
-  int page, row;
-  bool page_ok = decode_page_row<D>(p, b, t_begin, page, row);
-  int n_valid = page_ok ? min(16, t_end - t_begin) : 0;
-  if (!page_ok && lane == 0) flag_device_error(kDevErrBadPage);
-  float ksc = 0.f, vsc = 0.f;  // scales of the page holding the current 16 tokens
-  if (n_valid > 0) {
-    ksc = __ldg(f.k_scale + (size_t)page * p.Hkv + kvh);
-    vsc = __ldg(f.v_scale + (size_t)page * p.Hkv + kvh);
-  }
-  decode_load_k8<D>(f, page, row, kvh, g, tq, n_valid, cur.k);
-  decode_load_v8<D>(f, page, row, kvh, g, tq, n_valid, cur.v);
-
-#pragma unroll 1
-  for (int t0 = t_begin; t0 < t_end; t0 += 16) {
-    const int n_here = n_valid;
-    const int t1 = t0 + 16;
-    int page_n = 0, row_n = 0, n_next = 0;
-    float ksc_n = 0.f, vsc_n = 0.f;
-    if (t1 < t_end) {
-      const bool ok_n = decode_page_row<D>(p, b, t1, page_n, row_n);
-      if (!ok_n && lane == 0) flag_device_error(kDevErrBadPage);
-      n_next = ok_n ? min(16, t_end - t1) : 0;
-      if (n_next > 0) {
-        ksc_n = __ldg(f.k_scale + (size_t)page_n * p.Hkv + kvh);
-        vsc_n = __ldg(f.v_scale + (size_t)page_n * p.Hkv + kvh);
-      }
-    }
-
-    // ---- S = q K^T; raw word kc holds d = (D/4)*tq + 4*kc + {0, 1, 2, 3}
-    float sc[2][4];
-#pragma unroll
-    for (int nc = 0; nc < 2; ++nc) {
-      sc[nc][0] = sc[nc][1] = sc[nc][2] = sc[nc][3] = 0.f;
-#pragma unroll
-      for (int kc = 0; kc < D / 16; ++kc) {
-        const uint32_t w = cur.k[nc][kc];
-        mma_m16n8k16_f16(sc[nc], qa[kc][0], 0u, qa[kc][1], 0u, e4m3x2_to_f16x2(w),
-                         e4m3x2_to_f16x2(w >> 16));
-      }
-    }
-    if (t1 < t_end) decode_load_k8<D>(f, page_n, row_n, kvh, g, tq, n_next, cur.k);
-
-    // ---- online softmax for head row g over this thread's 4 tokens
-    const float kq = ksc * qscale;  // K scale and q's power-of-two scale
-    float s4[4] = {sc[0][0] * kq, sc[0][1] * kq, sc[1][0] * kq, sc[1][1] * kq};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int tok = (e >> 1) * 8 + 2 * tq + (e & 1);
-      if (tok >= n_here) s4[e] = -INFINITY;
-      else if (!scale_pos) s4[e] *= p.scale_log2;
-    }
-    float mx = fmaxf(fmaxf(s4[0], s4[1]), fmaxf(s4[2], s4[3]));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float m_new = fmaxf(m_run, mx * c2);
-    const float alpha = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_new);
-    const float base = (m_new == -INFINITY) ? 0.f : m_new;
-    float pr[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) pr[e] = ex2(fmaf(s4[e], c2, -base));
-    // P^T as f16 (P <= 1) for the f16 MMA: tokens 2tq, 2tq+1 and 2tq+8, 2tq+9
-    const uint32_t pb0 = pack_f16x2(pr[0], pr[1]);
-    const uint32_t pb1 = pack_f16x2(pr[2], pr[3]);
-    float rs = (pr[0] + pr[1]) + (pr[2] + pr[3]);
-    float rr = (f16_to_f32(pb0) + f16_to_f32(pb0 >> 16)) + (f16_to_f32(pb1) + f16_to_f32(pb1 >> 16));
-    rs += __shfl_xor_sync(0xffffffffu, rs, 1);
-    rr += __shfl_xor_sync(0xffffffffu, rr, 1);
-    rs += __shfl_xor_sync(0xffffffffu, rs, 2);
-    rr += __shfl_xor_sync(0xffffffffu, rr, 2);
-    l_run = l_run * alpha + rs;
-    lr_run = lr_run * alpha + rr;
-    m_run = m_new;
-
-    // ---- O^T += vsc * (V^T P^T); V^T rows d = (D/8)*g + 2*mc (+1), columns =
-    // tokens 2tq, 2tq+1, 2tq+8, 2tq+9 from the f16x2 of each token's raw word mc/2
-    const float a_h0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
-    const float a_h1 = __shfl_sync(0xffffffffu, alpha, (2 * tq + 1) * 4);
-#pragma unroll
-    for (int mc = 0; mc < D / 16; ++mc) {
-      uint32_t vh[4];
-#pragma unroll
-      for (int ti = 0; ti < 4; ++ti) vh[ti] = e4m3x2_to_f16x2(cur.v[ti][mc >> 1] >> (16 * (mc & 1)));
-      float part[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_m16n8k16_f16(part, prmt(vh[0], vh[1], 0x5410u), prmt(vh[0], vh[1], 0x7632u),
-                       prmt(vh[2], vh[3], 0x5410u), prmt(vh[2], vh[3], 0x7632u), pb0, pb1);
-      acc[mc][0] = fmaf(vsc, part[0], acc[mc][0] * a_h0);
-      acc[mc][1] = fmaf(vsc, part[1], acc[mc][1] * a_h1);
-      acc[mc][2] = fmaf(vsc, part[2], acc[mc][2] * a_h0);
-      acc[mc][3] = fmaf(vsc, part[3], acc[mc][3] * a_h1);
-    }
-    if (t1 < t_end) decode_load_v8<D>(f, page_n, row_n, kvh, g, tq, n_next, cur.v);
-    n_valid = n_next;
-    ksc = ksc_n;
-    vsc = vsc_n;
-  }
-
-  // ---- this split's normalised partial output and its log2-sum-exp
-  const int h0 = 2 * tq, h1 = 2 * tq + 1;
-  const float l_h0 = __shfl_sync(0xffffffffu, lr_run, h0 * 4);
-  const float l_h1 = __shfl_sync(0xffffffffu, lr_run, h1 * 4);
-  const float inv0 = l_h0 > 0.f ? 1.f / l_h0 : 0.f;
-  const float inv1 = l_h1 > 0.f ? 1.f / l_h1 : 0.f;
-  const int dbase = (D / 8) * g;
-#pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const int h = hh ? h1 : h0;
-    if (h >= p.group) continue;
-    const float inv = hh ? inv1 : inv0;
-    float* dst = p.o_part + (((size_t)b * p.Hq + hq0 + h) * p.n_split + split) * D + dbase;
-#pragma unroll
-    for (int mc = 0; mc < D / 16; mc += 2) {
-      float4 w;
-      w.x = acc[mc][hh] * inv;
-      w.y = acc[mc][2 + hh] * inv;
-      w.z = acc[mc + 1][hh] * inv;
-      w.w = acc[mc + 1][2 + hh] * inv;
-      *reinterpret_cast<float4*>(dst + 2 * mc) = w;
-    }
-  }
-  if (tq == 0 && g < p.group) {
-    const float lse2 = l_run > 0.f ? m_run + lg2(l_run) : -INFINITY;
-    p.lse_part[((size_t)b * p.Hq + hq0 + g) * p.n_split + split] = lse2;
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -633,7 +134,7 @@ template <int D, bool FP8>
 struct DecodeTmaCfg {
   // ring depth: the bytes in flight per warp against the warps an SM holds
   // (shared memory per warp grows with the depth)
-  static constexpr int STAGES = FP8 ? 4 : 4;
+  static constexpr int STAGES = FP8 ? 4 : 3;
   static constexpr int E = FP8 ? 1 : 2;            // bytes per element
   static constexpr int ROW = D * E;                // bytes per token row of one head
   static constexpr int BOX_BYTES = ROW < 128 ? ROW : 128;  // inner box extent in bytes
