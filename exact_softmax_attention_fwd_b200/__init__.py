@@ -8,8 +8,10 @@ first call does, and raises if the library is missing or no GPU is present.
 from ._binding import (  # noqa: F401
     AttnError,
     attn_bwd,
+    attn_bwd_block_sparse,
     attn_bwd_varlen,
     attn_bwd_varlen_workspace_size,
+    attn_bwd_window,
     attn_bwd_workspace_size,
     attn_fwd_block_sparse,
     attn_decode_paged,

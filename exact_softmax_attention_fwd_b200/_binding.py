@@ -56,6 +56,8 @@ SIGNATURES = {
     "attn_bwd_workspace_size": (_SZ, [_I, _I, _I]),
     "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P,
                       _SZ, _P]),
+    "attn_bwd_window": (_I, [_P] * 9 + [_I] * 6 + [_F, _P, _I, _I, _P, _SZ, _P]),
+    "attn_bwd_block_sparse": (_I, [_P] * 9 + [_I] * 7 + [_F, _P, _P, _I, _P, _SZ, _P]),
     "attn_bwd_varlen_workspace_size": (_SZ, [_I, _I, _I]),
     "attn_bwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I,
                              ctypes.c_longlong, ctypes.c_longlong, _I, _I, _I, _I, _F, _P, _SZ,
@@ -297,6 +299,72 @@ def attn_bwd(q, k, v, o, lse, d_o, causal: bool, scale: float, k_lens=None, dq=N
                                  int(bool(causal)), float(scale), _ptr(k_lens), _ptr(workspace),
                                  ws_bytes, _stream(stream))
     _check(st, "attn_bwd")
+    return dq, dk, dv
+
+
+def _bwd_fixed_checks(q, k, v, o, lse, d_o, k_lens):
+    import torch
+    _require_bf16(q=q, k=k, v=v, o=o, d_o=d_o)
+    _require_cuda(q, k, v, o, lse, d_o, k_lens)
+    for t in (q, k, v, o, d_o):
+        if not t.is_contiguous():
+            raise ValueError("q, k, v, o, d_o must be contiguous")
+    B, Hq, Sq, d = q.shape
+    Bk, Hkv, Sk, dk_ = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or dk_ != d:
+        raise ValueError("q/k/v shapes disagree")
+    if tuple(o.shape) != tuple(q.shape) or tuple(d_o.shape) != tuple(q.shape):
+        raise ValueError("o and d_o must have q's shape")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, Sq) or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous float32 [B, Hq, Sq]")
+    if k_lens is not None and (k_lens.dtype != torch.int32 or tuple(k_lens.shape) != (B,)):
+        raise ValueError("k_lens must be int32 [B]")
+    return B, Hq, Hkv, Sq, Sk, d
+
+
+def attn_bwd_window(q, k, v, o, lse, d_o, scale: float, window: int = 0, prefix: int = 0,
+                    k_lens=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of attn_fwd_window (causal, sliding window or prefix-LM)."""
+    import torch
+    B, Hq, Hkv, Sq, Sk, d = _bwd_fixed_checks(q, k, v, o, lse, d_o, k_lens)
+    dq = _out(dq, q.shape, torch.bfloat16, q.device, "dq")
+    dk = _out(dk, k.shape, torch.bfloat16, q.device, "dk")
+    dv = _out(dv, v.shape, torch.bfloat16, q.device, "dv")
+    if workspace is None:
+        workspace = torch.empty(max(attn_bwd_workspace_size(B, Hq, Sq), 16), dtype=torch.uint8,
+                                device=q.device)
+    st = load_library().attn_bwd_window(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(d_o), _ptr(dq), _ptr(dk), _ptr(dv), B,
+        Hq, Hkv, Sq, Sk, d, float(scale), _ptr(k_lens), int(window), int(prefix), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "attn_bwd_window")
+    return dq, dk, dv
+
+
+def attn_bwd_block_sparse(q, k, v, o, lse, d_o, block_mask, causal: bool, scale: float,
+                          k_lens=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of attn_fwd_block_sparse; block_mask uint8 [B, 1 or Hq, ceil(Sq/128),
+    ceil(Sk/128)] on the device, as given to the forward."""
+    import torch
+    B, Hq, Hkv, Sq, Sk, d = _bwd_fixed_checks(q, k, v, o, lse, d_o, k_lens)
+    _require_cuda(block_mask)
+    nq, nk = -(-Sq // 128), -(-Sk // 128)
+    if (block_mask.dtype != torch.uint8 or block_mask.dim() != 4 or
+            tuple(block_mask.shape) not in ((B, 1, nq, nk), (B, Hq, nq, nk)) or
+            not block_mask.is_contiguous()):
+        raise ValueError(f"block_mask must be contiguous uint8 [B, 1 or Hq, {nq}, {nk}]")
+    dq = _out(dq, q.shape, torch.bfloat16, q.device, "dq")
+    dk = _out(dk, k.shape, torch.bfloat16, q.device, "dk")
+    dv = _out(dv, v.shape, torch.bfloat16, q.device, "dv")
+    if workspace is None:
+        workspace = torch.empty(max(attn_bwd_workspace_size(B, Hq, Sq), 16), dtype=torch.uint8,
+                                device=q.device)
+    st = load_library().attn_bwd_block_sparse(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(d_o), _ptr(dq), _ptr(dk), _ptr(dv), B,
+        Hq, Hkv, Sq, Sk, d, int(bool(causal)), float(scale), _ptr(k_lens), _ptr(block_mask),
+        block_mask.shape[1], _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _check(st, "attn_bwd_block_sparse")
     return dq, dk, dv
 
 

@@ -308,7 +308,7 @@ int prefill_dense(const void* q, const void* k, const void* v, void* o, float* l
 }
 // Backward: the row-statistics pass, then dK/dV (one CTA per key tile and KV
 // head) and dQ (one CTA per query tile and query head), in stream order.
-template <int D, bool CAUSAL, bool VARLEN = false>
+template <int D, bool CAUSAL, bool VARLEN = false, bool MASKS = false>
 int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mdo, const CUtensorMap& mk,
                const CUtensorMap& mv, const BwdParams& prm, cudaStream_t stream) {
   using C = BwdCfg<D>;
@@ -319,12 +319,12 @@ int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mdo, const CUtensorMap&
   if (prep_blocks > INT_MAX || kv_units > INT_MAX || q_units > INT_MAX) return ATTN_ERR_INVALID_ARG;
   attn_bwd_prep_kernel<D, VARLEN><<<(unsigned)prep_blocks, 256, 0, stream>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  auto kv = attn_bwd_dkdv_kernel<D, CAUSAL, VARLEN>;
+  auto kv = attn_bwd_dkdv_kernel<D, CAUSAL, VARLEN, MASKS>;
   static std::atomic<unsigned long long> kv_smem_set{0};
   if (!set_smem_once(kv, C::KV_SMEM, kv_smem_set)) return ATTN_ERR_CUDA;
   kv<<<(unsigned)kv_units, C::NUM_THREADS, C::KV_SMEM, stream>>>(mq, mdo, mk, mv, prm);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  auto dq = attn_bwd_dq_kernel<D, CAUSAL, VARLEN>;
+  auto dq = attn_bwd_dq_kernel<D, CAUSAL, VARLEN, MASKS>;
   static std::atomic<unsigned long long> q_smem_set{0};
   if (!set_smem_once(dq, C::Q_SMEM, q_smem_set)) return ATTN_ERR_CUDA;
   dq<<<(unsigned)q_units, C::NUM_THREADS, C::Q_SMEM, stream>>>(mq, mdo, mk, mv, prm);
@@ -439,10 +439,17 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Sq) {
   return bwd_workspace_bytes(B, Hq, Sq);
 }
 
-int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-             const void* d_o, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk,
-             int d, int causal, float scale, const int32_t* k_lens, void* workspace,
-             size_t workspace_bytes, attn_stream_t stream_) {
+}  // extern "C"
+
+namespace attn_b200 {
+namespace {
+// The fixed-length backward, with the programmable masks of the forward
+// (window / prefix: causal only; block mask: nullable).
+int bwd_dense(const void* q, const void* k, const void* v, const void* o, const float* lse,
+              const void* d_o, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk,
+              int d, int causal, float scale, const int32_t* k_lens, int window, int prefix,
+              const uint8_t* block_mask, int mask_heads, void* workspace, size_t workspace_bytes,
+              attn_stream_t stream_) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (o == nullptr || lse == nullptr || d_o == nullptr || dq == nullptr || workspace == nullptr ||
       (Sk > 0 && (dk == nullptr || dv == nullptr)))
@@ -485,11 +492,53 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   prm.n_kt = (Sk + 127) / 128;
   prm.scale = scale;
   prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.window = window;
+  prm.prefix = prefix;
+  prm.block_mask = block_mask;
+  prm.mask_heads = mask_heads;
+  if (window > 0 || prefix > 0 || block_mask != nullptr) {
+    if (d == 128)
+      return causal ? launch_bwd<128, true, false, true>(mq, mdo, mk, mv, prm, stream)
+                    : launch_bwd<128, false, false, true>(mq, mdo, mk, mv, prm, stream);
+    return causal ? launch_bwd<64, true, false, true>(mq, mdo, mk, mv, prm, stream)
+                  : launch_bwd<64, false, false, true>(mq, mdo, mk, mv, prm, stream);
+  }
   if (d == 128)
     return causal ? launch_bwd<128, true>(mq, mdo, mk, mv, prm, stream)
                   : launch_bwd<128, false>(mq, mdo, mk, mv, prm, stream);
   return causal ? launch_bwd<64, true>(mq, mdo, mk, mv, prm, stream)
                 : launch_bwd<64, false>(mq, mdo, mk, mv, prm, stream);
+}
+}  // namespace
+}  // namespace attn_b200
+
+extern "C" {
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* d_o, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk,
+             int d, int causal, float scale, const int32_t* k_lens, void* workspace,
+             size_t workspace_bytes, attn_stream_t stream) {
+  return bwd_dense(q, k, v, o, lse, d_o, dq, dk, dv, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens,
+                   0, 0, nullptr, 1, workspace, workspace_bytes, stream);
+}
+
+int attn_bwd_window(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* d_o, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq,
+                    int Sk, int d, float scale, const int32_t* k_lens, int window, int prefix,
+                    void* workspace, size_t workspace_bytes, attn_stream_t stream) {
+  if (window < 0 || prefix < 0 || (window > 0 && prefix > 0)) return ATTN_ERR_INVALID_ARG;
+  return bwd_dense(q, k, v, o, lse, d_o, dq, dk, dv, B, Hq, Hkv, Sq, Sk, d, 1, scale, k_lens,
+                   window, prefix, nullptr, 1, workspace, workspace_bytes, stream);
+}
+
+int attn_bwd_block_sparse(const void* q, const void* k, const void* v, const void* o,
+                          const float* lse, const void* d_o, void* dq, void* dk, void* dv, int B,
+                          int Hq, int Hkv, int Sq, int Sk, int d, int causal, float scale,
+                          const int32_t* k_lens, const uint8_t* block_mask, int mask_heads,
+                          void* workspace, size_t workspace_bytes, attn_stream_t stream) {
+  if (block_mask == nullptr || (mask_heads != 1 && mask_heads != Hq)) return ATTN_ERR_INVALID_ARG;
+  return bwd_dense(q, k, v, o, lse, d_o, dq, dk, dv, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens,
+                   0, 0, block_mask, mask_heads, workspace, workspace_bytes, stream);
 }
 
 

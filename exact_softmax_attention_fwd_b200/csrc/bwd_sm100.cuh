@@ -72,7 +72,21 @@ struct BwdParams {
   const int* cu_q;      // [B + 1]
   const int* cu_k;      // [B + 1]
   int total_q, total_k;
+  // programmable masks (MASKS instantiations, fixed-length batches): sliding
+  // window / prefix-LM (causal only, 0 = off) and a uint8 block mask
+  // [B, mask_heads, n_qt, n_kt] over 128 x 128 blocks (nullable), as the forward's
+  int window, prefix;
+  const uint8_t* block_mask;
+  int mask_heads;
 };
+
+// Whether the 128 x 128 block (query tile qt, key tile kt) of query head hq is
+// switched on by the block mask (always, without one).
+__device__ __forceinline__ bool bwd_block_on(const BwdParams& p, int b, int hq, int qt, int kt) {
+  if (p.block_mask == nullptr) return true;
+  const size_t h = p.mask_heads == 1 ? 0 : (size_t)hq;
+  return __ldg(p.block_mask + (((size_t)b * p.mask_heads + h) * p.n_qt + qt) * p.n_kt + kt) != 0;
+}
 
 // One sequence of a backward call: query rows [q0, q0 + lq) and keys
 // [k0, k0 + lk) of the packed tensors (fixed-length batches: q0 = k0 = 0,
@@ -267,7 +281,7 @@ __device__ __forceinline__ void bwd_store32(uint16_t* dst, const uint32_t (&v)[3
 // tile major, so under a causal mask the heaviest key tiles (the first ones,
 // seen by the most query tiles) start first.
 // ===========================================================================
-template <int D, bool CAUSAL, bool VARLEN>
+template <int D, bool CAUSAL, bool VARLEN, bool MASKS>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_do,
@@ -294,12 +308,22 @@ __global__ void __launch_bounds__(384, 1)
   const long long koff = (long long)klen - sq.lq;  // key j is visible to row i iff j <= i + koff
   const int key0 = kb * 128;
   const int n_qt = VARLEN ? (sq.lq + 127) / 128 : p.n_qt;  // this sequence's query tiles
-  int qt_lo = 0;
+  int qt_lo = 0, qt_hi = n_qt;
   if (CAUSAL) {
     const long long first_row = (long long)key0 - koff;  // the first row that sees key0
     qt_lo = first_row <= 0 ? 0 : (int)min(first_row / 128, (long long)n_qt);
   }
-  const int nq = (!seq_ok || key0 >= klen) ? 0 : n_qt - qt_lo;
+  if (MASKS) {
+    const long long key1 = min((long long)key0 + 127, (long long)klen - 1);
+    // prefix keys are seen by every row; a window hides the tile from rows
+    // at or past key1 + window - koff
+    if (p.prefix > 0 && key0 < min(p.prefix, klen)) qt_lo = 0;
+    if (p.window > 0) {
+      const long long row_end = key1 + p.window - koff;
+      qt_hi = row_end <= 0 ? 0 : (int)min((row_end + 127) / 128, (long long)n_qt);
+    }
+  }
+  const int nq = (!seq_ok || key0 >= klen || qt_hi <= qt_lo) ? 0 : qt_hi - qt_lo;
   const int N = p.group * nq;  // (query head, query tile) iterations
   // dK/dV rows this CTA writes: a ragged sequence's own keys only (rows past
   // them belong to the next sequence); fixed-length batches write every key
@@ -433,8 +457,18 @@ __global__ void __launch_bounds__(384, 1)
       const int qt = qt_lo + n % nq;
       // columns c >= cmin are visible to this key (c relative to this warpgroup's run)
       long long cm = (j >= klen) ? 64 : (CAUSAL ? (long long)j - koff - qt * 128 - c0 : 0);
+      long long cx = 64;  // columns [cmin, cmax) are visible to this key
+      if (MASKS) {
+        if (p.window > 0 && j < klen) cx = (long long)j + p.window - koff - qt * 128 - c0;
+        if (p.prefix > 0 && j < p.prefix && j < klen) {
+          cm = 0;
+          cx = 64;
+        }
+        if (!bwd_block_on(p, b, kvh * p.group + n / nq, qt, kb)) cm = 64;
+      }
       const int cmin = (int)(cm < 0 ? 0 : (cm > 64 ? 64 : cm));
-      const bool edge = __any_sync(0xffffffffu, cmin > 0);
+      const int cmax = MASKS ? (int)(cx < 0 ? 0 : (cx > 64 ? 64 : cx)) : 64;
+      const bool edge = __any_sync(0xffffffffu, cmin > 0 || cmax < 64);
       if (!(ok = mbar_wait_warp(bar(C::KB_SF), n & 1u, abort_flag))) break;
       tc_fence_after_sync();
       float pr[64];
@@ -467,10 +501,10 @@ __global__ void __launch_bounds__(384, 1)
           split_f32x2(fma_f32x2(f32x2(__uint_as_float(s2), __uint_as_float(s3)), c2x2,
                                 f32x2(nl.z, nl.w)), x2, x3);
           if (edge) {
-            x0 = bwd_keep(c >= cmin, x0);
-            x1 = bwd_keep(c + 1 >= cmin, x1);
-            x2 = bwd_keep(c + 2 >= cmin, x2);
-            x3 = bwd_keep(c + 3 >= cmin, x3);
+            x0 = bwd_keep(c >= cmin && c < cmax, x0);
+            x1 = bwd_keep(c + 1 >= cmin && c + 1 < cmax, x1);
+            x2 = bwd_keep(c + 2 >= cmin && c + 2 < cmax, x2);
+            x3 = bwd_keep(c + 3 >= cmin && c + 3 < cmax, x3);
           }
           pr[c] = ex2(x0);
           pr[c + 1] = ex2(x1);
@@ -550,7 +584,7 @@ __global__ void __launch_bounds__(384, 1)
 // tile major from the last tile down, so under a causal mask the heaviest
 // tiles start first.
 // ===========================================================================
-template <int D, bool CAUSAL, bool VARLEN>
+template <int D, bool CAUSAL, bool VARLEN, bool MASKS>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_do,
@@ -580,9 +614,17 @@ __global__ void __launch_bounds__(384, 1)
   const int row0 = qt * 128;
   const int last_row = min(row0 + 127, n_rows - 1);
   long long max_key = (long long)klen - 1;  // the last key any row of the tile sees
-  if (CAUSAL) max_key = min(max_key, (long long)last_row + koff);
-  // key tiles [0, N); none for a tile past the sequence's rows
-  const int N = (max_key < 0 || row0 >= n_rows) ? 0 : (int)(max_key / 128) + 1;
+  if (CAUSAL)
+    max_key = min(max_key, max((long long)last_row + koff, MASKS ? (long long)p.prefix - 1 : -1LL));
+  // the first key tile any row sees (a sliding window starts it past 0)
+  int kt_lo = 0;
+  if (MASKS && p.window > 0) {
+    const long long min_key = (long long)row0 + koff - p.window + 1;
+    kt_lo = min_key <= 0 ? 0 : (int)(min_key / 128);
+  }
+  // key tiles [kt_lo, kt_lo + N); none for a tile past the sequence's rows
+  const int kt_end = max_key < 0 ? 0 : (int)(max_key / 128) + 1;
+  const int N = (row0 >= n_rows || kt_end <= kt_lo) ? 0 : kt_end - kt_lo;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::QB_QF), 1);
@@ -633,7 +675,8 @@ __global__ void __launch_bounds__(384, 1)
             !(ok = mbar_wait(bar(C::QB_KVE + s), ((n / C::STAGES) - 1) & 1u, abort_flag)))
           break;
         mbar_arrive_expect_tx(bar(C::QB_KVF + s), 2 * C::TILE_BYTES);
-        const int ky = VARLEN ? kvh : n * 128, kz = VARLEN ? sq.k0 + n * 128 : bh_kv;
+        const int kt = kt_lo + n;
+        const int ky = VARLEN ? kvh : kt * 128, kz = VARLEN ? sq.k0 + kt * 128 : bh_kv;
         for (int cb = 0; cb < C::NCB; ++cb) {
           tma_load_3d(sK(s) + cb * C::CB_BYTES, &tm_k, bar(C::QB_KVF + s), 64 * cb, ky, kz);
           tma_load_3d(sV(s) + cb * C::CB_BYTES, &tm_v, bar(C::QB_KVF + s), 64 * cb, ky, kz);
@@ -692,14 +735,20 @@ __global__ void __launch_bounds__(384, 1)
     const float dd = p.dsum[srow];
     const uint64_t c2x2 = f32x2(p.scale_log2, p.scale_log2);
     const uint64_t nlx2 = f32x2(nl, nl);
-    // keys j < kend are visible to this row
-    long long kend = klen;
-    if (CAUSAL) kend = min(kend, (long long)row + koff + 1);
+    // keys klo <= j < kend are visible to this row
+    long long kend = klen, klo = 0;
+    if (CAUSAL)
+      kend = min(kend, max((long long)row + koff, MASKS ? (long long)p.prefix - 1 : -1LL) + 1);
+    if (MASKS && p.window > 0) klo = max(0LL, (long long)row + koff - p.window + 1);
     bool ok = true;
     for (int n = 0; ok && n < N; ++n) {
-      const long long cm = kend - (long long)n * 128 - c0;  // visible iff c < cmax
+      const long long t0 = (long long)(kt_lo + n) * 128 + c0;  // this run's first key
+      long long cm = kend - t0;  // visible iff cmin <= c < cmax
+      if (MASKS && !bwd_block_on(p, b, hq, qt, kt_lo + n)) cm = 0;
+      const long long cn = MASKS ? klo - t0 : 0;
+      const int cmin = (int)(cn < 0 ? 0 : (cn > 64 ? 64 : cn));
       const int cmax = (int)(cm < 0 ? 0 : (cm > 64 ? 64 : cm));
-      const bool edge = __any_sync(0xffffffffu, cmax < 64);
+      const bool edge = __any_sync(0xffffffffu, cmax < 64 || cmin > 0);
       if (!(ok = mbar_wait_warp(bar(C::QB_SF + (n & 1)), (n >> 1) & 1u, abort_flag))) break;
       tc_fence_after_sync();
       const uint32_t t_s = tmem + lane_off + ((n & 1) ? C::Q_TM_S1 : C::Q_TM_S0) + c0;
@@ -719,8 +768,8 @@ __global__ void __launch_bounds__(384, 1)
           split_f32x2(fma_f32x2(f32x2(__uint_as_float(s0), __uint_as_float(s1)), c2x2, nlx2), x0,
                       x1);
           if (edge) {
-            x0 = bwd_keep(c < cmax, x0);
-            x1 = bwd_keep(c + 1 < cmax, x1);
+            x0 = bwd_keep(c < cmax && c >= cmin, x0);
+            x1 = bwd_keep(c + 1 < cmax && c + 1 >= cmin, x1);
           }
           pr[c] = ex2(x0);
           pr[c + 1] = ex2(x1);

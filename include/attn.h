@@ -408,6 +408,37 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
              size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * attn_bwd_window -- backward pass of attn_fwd_window (causal, with a sliding
+ * window or a prefix-LM mask).
+ * Source: "Attention Kernel", section "Backward 与重计算" (the forward's mask
+ * applies unchanged) and section "可编程 mask" (window and prefix rules).
+ *   Arguments and layouts as attn_bwd (causal implied); window, prefix
+ *   exactly as given to attn_fwd_window (>= 0, not both > 0); the workspace is
+ *   attn_bwd_workspace_size(B, Hq, Sq) bytes.  Keys no visible pair reaches
+ *   get zero dK, dV; rows with no visible key get zero dQ.
+ * Errors: as attn_bwd, plus INVALID_ARG for a negative window or prefix, or both.
+ */
+int attn_bwd_window(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* d_o, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq,
+                    int Sk, int d, float scale, const int32_t* k_lens, int window, int prefix,
+                    void* workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * attn_bwd_block_sparse -- backward pass of attn_fwd_block_sparse.
+ * Source: as attn_bwd_window; "可编程 mask" (block-level sparsity).
+ *   block_mask, mask_heads exactly as given to attn_fwd_block_sparse: uint8
+ *   [B, mask_heads, ceil(Sq/128), ceil(Sk/128)] device array, mask_heads 1 or
+ *   Hq; 0 hides the 128 x 128 block.  Other arguments as attn_bwd.
+ * Errors: as attn_bwd, plus INVALID_ARG for a NULL block_mask or another
+ * mask_heads.
+ */
+int attn_bwd_block_sparse(const void* q, const void* k, const void* v, const void* o,
+                          const float* lse, const void* d_o, void* dq, void* dk, void* dv, int B,
+                          int Hq, int Hkv, int Sq, int Sk, int d, int causal, float scale,
+                          const int32_t* k_lens, const uint8_t* block_mask, int mask_heads,
+                          void* workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
  * attn_bwd_varlen_workspace_size -- bytes of device workspace attn_bwd_varlen
  * needs: 8 * B * Hq * ceil(max_seqlen_q / 128) * 128 (two fp32 row statistics
  * per query row, each sequence padded to max_seqlen_q in whole 128-row tiles).

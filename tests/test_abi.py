@@ -404,3 +404,17 @@ def test_fp8_prefill_binding_checks_codes_and_scales():
         B.attn_fwd_fp8(q8.float(), q8, q8, qs, qs, qs, True, 0.1)
     with pytest.raises(ValueError, match="block scales"):  # one per 128-row block: [1, 2, 2]
         B.attn_fwd_fp8(q8, q8, q8, qs[:, :, :1].contiguous(), qs, qs, True, 0.1)
+
+
+def test_bwd_masked_entry_validation(lib):
+    F_ = FAKE
+    # window and prefix together, or negative: rejected before any CUDA call
+    args = [F_] * 9 + [1, 2, 1, 200, 200, 128, 0.1, None]
+    assert lib.attn_bwd_window(*args, 16, 16, F_, 1 << 20, None) == B.ATTN_ERR_INVALID_ARG
+    assert lib.attn_bwd_window(*args, -1, 0, F_, 1 << 20, None) == B.ATTN_ERR_INVALID_ARG
+    assert lib.attn_bwd_window(*args[:14], 80, 0.1, None, 16, 0, F_, 1 << 20,
+                               None) == B.ATTN_ERR_UNSUPPORTED
+    bargs = [F_] * 9 + [1, 2, 1, 200, 200, 128, 1, 0.1, None]
+    assert lib.attn_bwd_block_sparse(*bargs, None, 1, F_, 1 << 20, None) == B.ATTN_ERR_INVALID_ARG
+    assert lib.attn_bwd_block_sparse(*bargs, F_, 3, F_, 1 << 20, None) == B.ATTN_ERR_INVALID_ARG
+    assert lib.attn_bwd_block_sparse(*bargs, F_, 1, F_, 16, None) == B.ATTN_ERR_WORKSPACE
