@@ -26,6 +26,13 @@ DEV = "cuda:0"
 
 def _check(got, ref, what):
     for name, g, r in zip(("dq", "dk", "dv"), got, ref):
+        if not np.any(r):
+            # A gradient that vanishes by cancellation, not for want of a visible
+            # pair (a window of 1: each row's weight is 1, so dS = dP - D = 0 in
+            # exact arithmetic): the kernel forms D from the bf16-rounded O, so
+            # it is zero only to rounding.
+            assert float(g.float().abs().max()) <= 1e-3, f"{what} {name}"
+            continue
         check_grad(g.cpu(), r, what=f"{what} {name}")
 
 
