@@ -65,6 +65,7 @@ def parse_args():
     ap.add_argument("--no-prefill-fp8", action="store_true")
     ap.add_argument("--prefill-fp8-workload", default="gqa_causal_8k")
     ap.add_argument("--no-paged-prefill", action="store_true")
+    ap.add_argument("--no-paged-prefill-fp8", action="store_true")
     ap.add_argument("--paged-prefill-workload", default="paged_prefill_gqa")
     return ap.parse_args()
 
@@ -602,6 +603,8 @@ def run_ours(args, world, rank, local):
         line["ragged"] = ragged_leg(args, dev, world, peaks)
     if not args.no_paged_prefill:
         line["paged_prefill"] = paged_prefill_leg(args, dev, world, peaks)
+    if not args.no_paged_prefill_fp8:
+        line["paged_prefill_fp8"] = paged_prefill_leg(args, dev, world, peaks, fp8=True)
     if not args.no_backward:
         line["backward"] = {name.strip(): backward_leg(args, W.CONFIGS[name.strip()], dev, world,
                                                        peaks)
@@ -744,38 +747,56 @@ def backward_leg(args, cfg, dev, world, peaks):
             "clocks": clocks, "roofline": rl}
 
 
-def paged_prefill_leg(args, dev, world, peaks):
+def paged_prefill_leg(args, dev, world, peaks, fp8: bool = False):
     """Chunked prefill over a paged cache (attn_fwd_paged: the unit-list kernel and the
-    prefill kernel reading K/V page by page), timed on its own like the ragged leg."""
+    prefill kernel reading K/V page by page), timed on its own like the ragged leg.
+    fp8: the same over the cache quantised to E4M3 with one scale per (page, KV head)
+    (attn_fwd_paged_fp8: the referenced pages dequantised, then the bf16 kernels)."""
     import torch
 
-    from exact_softmax_attention_fwd_b200 import (attn_fwd_paged, attn_fwd_varlen_workspace_size,
+    from exact_softmax_attention_fwd_b200 import (attn_fwd_paged, attn_fwd_paged_fp8,
+                                                  attn_fwd_paged_fp8_workspace_size,
+                                                  attn_fwd_varlen_workspace_size,
                                                   attn_get_device_error)
     from exact_softmax_attention_fwd_b200 import workloads as W
 
     pc = W.CONFIGS[args.paged_prefill_workload]
     q_h, cu_q_h, cache, lq, lk = W.paged_prefill_config_inputs(pc)
     q, cu_q = q_h.to(dev), cu_q_h.to(dev)
-    kc, vc = cache.k_cache.to(dev), cache.v_cache.to(dev)
     tbl, lens = cache.block_table.to(dev), cache.seq_lens.to(dev)
     max_q = int(lq.max())
-    ws = torch.empty(attn_fwd_varlen_workspace_size(pc.B, q.shape[0], max_q), dtype=torch.uint8,
-                     device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((pc.Hq, q.shape[0]), dtype=torch.float32, device=dev)
+    if fp8:
+        k8, ks = W.quantize_e4m3_per_page(cache.k_cache)
+        v8, vs = W.quantize_e4m3_per_page(cache.v_cache)
+        k8, v8, ks, vs = k8.to(dev), v8.to(dev), ks.to(dev), vs.to(dev)
+        ws = torch.empty(attn_fwd_paged_fp8_workspace_size(pc.B, q.shape[0], max_q, tbl.shape[1],
+                                                           pc.page_size, pc.Hkv, pc.d),
+                         dtype=torch.uint8, device=dev)
 
-    def one():
-        attn_fwd_paged(q, kc, vc, tbl, cu_q, lens, max_q, True, pc.scale, out=o, lse=lse,
-                       workspace=ws)
+        def one():
+            attn_fwd_paged_fp8(q, k8, v8, ks, vs, tbl, cu_q, lens, max_q, True, pc.scale, out=o,
+                               lse=lse, workspace=ws)
+    else:
+        kc, vc = cache.k_cache.to(dev), cache.v_cache.to(dev)
+        ws = torch.empty(attn_fwd_varlen_workspace_size(pc.B, q.shape[0], max_q),
+                         dtype=torch.uint8, device=dev)
+
+        def one():
+            attn_fwd_paged(q, kc, vc, tbl, cu_q, lens, max_q, True, pc.scale, out=o, lse=lse,
+                           workspace=ws)
 
     ms, clocks = timed_calls(args, dev, world, one)
     st, fl = attn_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error word set in the paged-prefill leg: {fl:#x}")
-    rl = tensor_roofline(pc.flops(), ms, peaks, "attn_prefill_sm100_kernel", pc.name, world)
-    return {"workload": pc.name, "value": world * rl["achieved"], "unit": "TFLOPS",
+    rl = tensor_roofline(pc.flops(), ms, peaks, "attn_prefill_sm100_kernel",
+                         pc.name + ("_e4m3" if fp8 else ""), world)
+    return {"workload": pc.name + (" (E4M3 cache, one scale per page and KV head)" if fp8 else ""),
+            "value": world * rl["achieved"], "unit": "TFLOPS",
             "ms": rl["mean_ms"], "median_ms": rl["median_ms"], "calls": len(ms),
-            "gpu_launches_per_call": 2,
+            "gpu_launches_per_call": 3 if fp8 else 2,
             "sequences": pc.B, "new_tokens": int(q.shape[0]), "page_size": pc.page_size,
             "keys": f"cached uniform {pc.cached_lo}..{pc.cached_hi} + {pc.new_tokens} new (seed {pc.seed})",
             "clocks": clocks, "roofline": rl}

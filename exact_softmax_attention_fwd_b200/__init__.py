@@ -21,6 +21,8 @@ from ._binding import (  # noqa: F401
     attn_fwd_fp8,
     attn_fwd_masked,
     attn_fwd_paged,
+    attn_fwd_paged_fp8,
+    attn_fwd_paged_fp8_workspace_size,
     attn_fwd_varlen,
     attn_fwd_varlen_workspace_size,
     attn_fwd_window,

@@ -46,6 +46,9 @@ SIGNATURES = {
                              ctypes.c_longlong, _I, _I, _I, _F, _P, _SZ, _P]),
     "attn_fwd_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_longlong, _I, _I,
                             _I, _I, _I, _F, _P, _P, _P, _SZ, _P]),
+    "attn_fwd_paged_fp8_workspace_size": (_SZ, [_I, ctypes.c_longlong, _I, _I, _I, _I, _I]),
+    "attn_fwd_paged_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I,
+                                ctypes.c_longlong, _I, _I, _I, _I, _I, _F, _P, _P, _P, _SZ, _P]),
     "attn_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P,
                                _SZ, _P]),
@@ -488,6 +491,59 @@ def attn_fwd_paged(q, k_cache, v_cache, block_table, cu_seqlens_q, seq_lens_k, m
                                        num_pages, d, int(bool(causal)), float(scale), _ptr(out),
                                        _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream))
     _check(st, "attn_fwd_paged")
+    return out, lse
+
+
+def attn_fwd_paged_fp8_workspace_size(B: int, total_q: int, max_seqlen_q: int,
+                                      max_pages_per_seq: int, page_size: int, Hkv: int,
+                                      d: int) -> int:
+    return int(load_library().attn_fwd_paged_fp8_workspace_size(
+        B, total_q, max_seqlen_q, max_pages_per_seq, page_size, Hkv, d))
+
+
+def attn_fwd_paged_fp8(q, k_cache, v_cache, k_scale, v_scale, block_table, cu_seqlens_q,
+                       seq_lens_k, max_seqlen_q: int, causal: bool, scale: float, out=None,
+                       lse=None, workspace=None, return_lse: bool = True, stream=None):
+    """attn_fwd_paged over an E4M3 cache: k_cache / v_cache uint8 [num_pages, page_size,
+    Hkv, d] codes, k_scale / v_scale float32 [num_pages, Hkv]; q [total_q, Hq, d] bf16."""
+    import torch
+    _require_bf16(q=q)
+    if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
+        raise ValueError("FP8 caches are uint8 E4M3 codes")
+    _require_cuda(q, k_cache, v_cache, k_scale, v_scale, block_table, cu_seqlens_q, seq_lens_k)
+    if q.dim() != 3 or k_cache.dim() != 4 or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("q [total_q, Hq, d]; caches [num_pages, page_size, Hkv, d]")
+    total_q, Hq, d = q.shape
+    num_pages, page_size, Hkv, dk = k_cache.shape
+    if dk != d:
+        raise ValueError("head dims disagree")
+    for t in (k_scale, v_scale):
+        if t.dtype != torch.float32 or tuple(t.shape) != (num_pages, Hkv) or not t.is_contiguous():
+            raise ValueError("scales must be contiguous float32 [num_pages, Hkv]")
+    B = cu_seqlens_q.shape[0] - 1
+    for t, shape in ((cu_seqlens_q, (B + 1,)), (seq_lens_k, (B,))):
+        if t.dtype != torch.int32 or tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError("cu_seqlens_q int32 [B+1], seq_lens_k int32 [B]")
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != B \
+            or not block_table.is_contiguous():
+        raise ValueError("block_table must be contiguous int32 [B, max_pages_per_seq]")
+    for t in (q, k_cache, v_cache):
+        if not t.is_contiguous():
+            raise ValueError("q and the caches must be contiguous")
+    max_pages = block_table.shape[1]
+    need = attn_fwd_paged_fp8_workspace_size(B, total_q, max_seqlen_q, max_pages, page_size, Hkv,
+                                             d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    out = _out(out, q.shape, torch.bfloat16, q.device, "out")
+    if lse is not None or return_lse:
+        lse = _out(lse, (Hq, total_q), torch.float32, q.device, "lse")
+    st = load_library().attn_fwd_paged_fp8(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_table),
+        _ptr(cu_seqlens_q), _ptr(seq_lens_k), page_size, B, Hq, Hkv, total_q, int(max_seqlen_q),
+        max_pages, num_pages, d, int(bool(causal)), float(scale), _ptr(out), _ptr(lse),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "attn_fwd_paged_fp8")
     return out, lse
 
 

@@ -12,6 +12,7 @@
 #include "attn.h"
 #include "bwd_sm100.cuh"
 #include "decode_sm100.cuh"
+#include "paged_fp8_sm100.cuh"
 #include "prefill_fp8_sm100.cuh"
 #include "prefill_sm100.cuh"
 #include "sm100_primitives.cuh"
@@ -423,6 +424,104 @@ int decode_paged_common(bool fp8, const void* q, const void* k_cache, const void
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+int check_paged_prefill_args(const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_table, const int32_t* cu_seqlens_q,
+                             const int32_t* seq_lens_k, int page_size, int B, int Hq, int Hkv,
+                             long long total_q, int max_seqlen_q, int max_pages_per_seq,
+                             int num_pages, int d, int causal, float scale, void* o, float* lse) {
+  if (q == nullptr || o == nullptr || k_cache == nullptr || v_cache == nullptr ||
+      block_table == nullptr || cu_seqlens_q == nullptr || seq_lens_k == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq > 65535) return ATTN_ERR_INVALID_ARG;
+  if (total_q < 0 || total_q > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  if (max_seqlen_q < 1 || max_seqlen_q > kVarlenMaxLevels * 256) return ATTN_ERR_INVALID_ARG;
+  if (max_pages_per_seq < 1 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
+  if ((long long)max_pages_per_seq * page_size > 0x7fffffffLL ||
+      (long long)num_pages * page_size > 0x7fffffffLL)
+    return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128)
+    return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(k_cache) || !aligned16(v_cache))
+    return ATTN_ERR_ALIGNMENT;
+  if ((lse != nullptr && !aligned4(lse)) || !aligned4(cu_seqlens_q) || !aligned4(seq_lens_k) ||
+      !aligned4(block_table))
+    return ATTN_ERR_ALIGNMENT;
+  return ATTN_OK;
+}
+
+// The paged prefill proper: the unit list in `workspace`, then the prefill
+// kernel over a bf16 pool (arguments already checked).
+int paged_prefill_run(const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_table, const int32_t* cu_seqlens_q,
+                      const int32_t* seq_lens_k, int page_size, int B, int Hq, int Hkv,
+                      long long total_q, int max_seqlen_q, int max_pages_per_seq, int num_pages,
+                      int d, int causal, float scale, void* o, float* lse, void* workspace,
+                      cudaStream_t stream) {
+  int* unit_count = static_cast<int*>(workspace);
+  int2* units = reinterpret_cast<int2*>(static_cast<char*>(workspace) + 16);
+  const long long max_units = varlen_max_units(B, total_q);
+  const int max_keys = max_pages_per_seq * page_size;
+  int shift, n_levels;
+  varlen_levels(max_keys, shift, n_levels);
+  const size_t sched_smem = (size_t)(2 * n_levels + 32) * sizeof(int);
+  if (!schedule_smem_ready()) return ATTN_ERR_CUDA;
+  attn_varlen_schedule_kernel<<<1, 1024, sched_smem, stream>>>(
+      cu_seqlens_q, nullptr, seq_lens_k, B, (int)total_q, 0, max_seqlen_q, max_keys, causal,
+      0, 0, shift, n_levels, units, unit_count, (int)max_units);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  CUtensorMap mq, mk, mv;
+  if (!make_token_map(&mq, q, d, Hq, total_q) ||
+      !make_token_map(&mk, k_cache, d, Hkv, (long long)num_pages * page_size, page_size) ||
+      !make_token_map(&mv, v_cache, d, Hkv, (long long)num_pages * page_size, page_size))
+    return ATTN_ERR_CUDA;
+  PrefillParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.lse = lse;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.o = static_cast<uint16_t*>(o);
+  prm.cu_q = cu_seqlens_q;
+  prm.seq_lens_k = seq_lens_k;
+  prm.block_table = block_table;
+  prm.max_pages = max_pages_per_seq;
+  prm.page_size = page_size;
+  prm.num_pages = num_pages;
+  prm.units = units;
+  prm.unit_count = unit_count;
+  prm.total_q = (int)total_q;
+  if (d == 128)
+    return causal ? launch_prefill<128, true, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units)
+                  : launch_prefill<128, false, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units);
+  return causal ? launch_prefill<64, true, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units)
+                : launch_prefill<64, false, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units);
+}
+
+// Workspace of the E4M3 paged prefill: the unit list, the remapped block
+// table [B, max_pages], and bf16 K and V pools of one page slot per
+// (sequence, logical page), each part 256-byte aligned.
+struct PagedFp8Layout {
+  size_t table_off, k_off, v_off, total;
+};
+
+PagedFp8Layout paged_fp8_layout(int B, size_t units_bytes, int max_pages, int page_size, int Hkv,
+                                int d) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  PagedFp8Layout L;
+  L.table_off = up(units_bytes);
+  const size_t slots = (size_t)B * max_pages;
+  L.k_off = L.table_off + up(slots * sizeof(int32_t));
+  const size_t pool = slots * page_size * Hkv * d * 2;
+  L.v_off = L.k_off + up(pool);
+  L.total = L.v_off + up(pool);
+  return L;
+}
+
 size_t bwd_workspace_bytes(int B, int Hq, int Sq) {
   const size_t pad = ((size_t)Sq + 127) / 128 * 128;
   return 2 * (size_t)B * Hq * pad * sizeof(float);
@@ -746,71 +845,63 @@ int attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache,
                    long long total_q, int max_seqlen_q, int max_pages_per_seq, int num_pages, int d,
                    int causal, float scale, void* o, float* lse, void* workspace,
                    size_t workspace_bytes, attn_stream_t stream_) {
-  if (q == nullptr || o == nullptr || k_cache == nullptr || v_cache == nullptr ||
-      block_table == nullptr || cu_seqlens_q == nullptr || seq_lens_k == nullptr)
-    return ATTN_ERR_INVALID_ARG;
-  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq > 65535) return ATTN_ERR_INVALID_ARG;
-  if (total_q < 0 || total_q > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
-  if (max_seqlen_q < 1 || max_seqlen_q > kVarlenMaxLevels * 256) return ATTN_ERR_INVALID_ARG;
-  if (max_pages_per_seq < 1 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
-  if ((long long)max_pages_per_seq * page_size > 0x7fffffffLL ||
-      (long long)num_pages * page_size > 0x7fffffffLL)
-    return ATTN_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
-  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128)
-    return ATTN_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(o) || !aligned16(k_cache) || !aligned16(v_cache))
-    return ATTN_ERR_ALIGNMENT;
-  if ((lse != nullptr && !aligned4(lse)) || !aligned4(cu_seqlens_q) || !aligned4(seq_lens_k) ||
-      !aligned4(block_table))
-    return ATTN_ERR_ALIGNMENT;
+  int st = check_paged_prefill_args(q, k_cache, v_cache, block_table, cu_seqlens_q, seq_lens_k,
+                                    page_size, B, Hq, Hkv, total_q, max_seqlen_q,
+                                    max_pages_per_seq, num_pages, d, causal, scale, o, lse);
+  if (st != ATTN_OK) return st;
   const size_t need = attn_fwd_varlen_workspace_size(B, total_q, max_seqlen_q);
   if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
   if (!aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (total_q == 0) return ATTN_OK;
-  int* unit_count = static_cast<int*>(workspace);
-  int2* units = reinterpret_cast<int2*>(static_cast<char*>(workspace) + 16);
-  const long long max_units = varlen_max_units(B, total_q);
-  const int max_keys = max_pages_per_seq * page_size;
-  int shift, n_levels;
-  varlen_levels(max_keys, shift, n_levels);
-  const size_t sched_smem = (size_t)(2 * n_levels + 32) * sizeof(int);
-  if (!schedule_smem_ready()) return ATTN_ERR_CUDA;
-  attn_varlen_schedule_kernel<<<1, 1024, sched_smem, stream>>>(
-      cu_seqlens_q, nullptr, seq_lens_k, B, (int)total_q, 0, max_seqlen_q, max_keys, causal,
-      0, 0, shift, n_levels, units, unit_count, (int)max_units);
+  return paged_prefill_run(q, k_cache, v_cache, block_table, cu_seqlens_q, seq_lens_k, page_size,
+                           B, Hq, Hkv, total_q, max_seqlen_q, max_pages_per_seq, num_pages, d,
+                           causal, scale, o, lse, workspace,
+                           reinterpret_cast<cudaStream_t>(stream_));
+}
+
+size_t attn_fwd_paged_fp8_workspace_size(int B, long long total_q, int max_seqlen_q,
+                                         int max_pages_per_seq, int page_size, int Hkv, int d) {
+  const size_t units = attn_fwd_varlen_workspace_size(B, total_q, max_seqlen_q);
+  if (units == 0 || max_pages_per_seq < 1 || page_size < 1 || Hkv < 1 || d < 1) return 0;
+  return paged_fp8_layout(B, units, max_pages_per_seq, page_size, Hkv, d).total;
+}
+
+int attn_fwd_paged_fp8(const void* q, const void* k_cache, const void* v_cache,
+                       const float* k_scale, const float* v_scale, const int32_t* block_table,
+                       const int32_t* cu_seqlens_q, const int32_t* seq_lens_k, int page_size,
+                       int B, int Hq, int Hkv, long long total_q, int max_seqlen_q,
+                       int max_pages_per_seq, int num_pages, int d, int causal, float scale,
+                       void* o, float* lse, void* workspace, size_t workspace_bytes,
+                       attn_stream_t stream_) {
+  if (k_scale == nullptr || v_scale == nullptr) return ATTN_ERR_INVALID_ARG;
+  int st = check_paged_prefill_args(q, k_cache, v_cache, block_table, cu_seqlens_q, seq_lens_k,
+                                    page_size, B, Hq, Hkv, total_q, max_seqlen_q,
+                                    max_pages_per_seq, num_pages, d, causal, scale, o, lse);
+  if (st != ATTN_OK) return st;
+  if (!aligned4(k_scale) || !aligned4(v_scale)) return ATTN_ERR_ALIGNMENT;
+  const size_t units = attn_fwd_varlen_workspace_size(B, total_q, max_seqlen_q);
+  const PagedFp8Layout L = paged_fp8_layout(B, units, max_pages_per_seq, page_size, Hkv, d);
+  if (workspace == nullptr || workspace_bytes < L.total) return ATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
+  if ((long long)B * max_pages_per_seq * page_size > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  if (total_q == 0) return ATTN_OK;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  char* ws = static_cast<char*>(workspace);
+  int32_t* table2 = reinterpret_cast<int32_t*>(ws + L.table_off);
+  uint16_t* k2 = reinterpret_cast<uint16_t*>(ws + L.k_off);
+  uint16_t* v2 = reinterpret_cast<uint16_t*>(ws + L.v_off);
+  // 1. the pages the batch references, dequantised into a bf16 pool of one
+  //    slot per (sequence, logical page), with the table that maps onto it
+  const int threads = 256;
+  attn_dequant_pages_kernel<<<dim3((unsigned)max_pages_per_seq, (unsigned)B), threads, 0, stream>>>(
+      static_cast<const uint8_t*>(k_cache), static_cast<const uint8_t*>(v_cache), k_scale,
+      v_scale, block_table, seq_lens_k, page_size, Hkv, d, max_pages_per_seq, num_pages, k2, v2,
+      table2);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  CUtensorMap mq, mk, mv;
-  if (!make_token_map(&mq, q, d, Hq, total_q) ||
-      !make_token_map(&mk, k_cache, d, Hkv, (long long)num_pages * page_size, page_size) ||
-      !make_token_map(&mv, v_cache, d, Hkv, (long long)num_pages * page_size, page_size))
-    return ATTN_ERR_CUDA;
-  PrefillParams prm;
-  std::memset(&prm, 0, sizeof(prm));
-  prm.lse = lse;
-  prm.B = B;
-  prm.Hq = Hq;
-  prm.Hkv = Hkv;
-  prm.group = Hq / Hkv;
-  prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.o = static_cast<uint16_t*>(o);
-  prm.cu_q = cu_seqlens_q;
-  prm.seq_lens_k = seq_lens_k;
-  prm.block_table = block_table;
-  prm.max_pages = max_pages_per_seq;
-  prm.page_size = page_size;
-  prm.num_pages = num_pages;
-  prm.units = units;
-  prm.unit_count = unit_count;
-  prm.total_q = (int)total_q;
-  if (d == 128)
-    return causal ? launch_prefill<128, true, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units)
-                  : launch_prefill<128, false, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units);
-  return causal ? launch_prefill<64, true, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units)
-                : launch_prefill<64, false, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units);
+  // 2. the bf16 paged prefill over that pool
+  return paged_prefill_run(q, k2, v2, table2, cu_seqlens_q, seq_lens_k, page_size, B, Hq, Hkv,
+                           total_q, max_seqlen_q, max_pages_per_seq, B * max_pages_per_seq, d,
+                           causal, scale, o, lse, workspace, stream);
 }
 
 int attn_fwd_fp8(const void* q, const void* k, const void* v, const float* q_scale,

@@ -117,6 +117,40 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, const float* q_sca
                  attn_stream_t stream);
 
 /*
+ * attn_fwd_paged_fp8_workspace_size -- bytes of device workspace
+ * attn_fwd_paged_fp8 needs: the unit list of attn_fwd_paged, a block table
+ * [B, max_pages_per_seq] and bf16 K and V pools of B * max_pages_per_seq
+ * pages (the batch's pages, dequantised).  0 for invalid arguments.
+ */
+size_t attn_fwd_paged_fp8_workspace_size(int B, long long total_q, int max_seqlen_q,
+                                         int max_pages_per_seq, int page_size, int Hkv, int d);
+
+/*
+ * attn_fwd_paged_fp8 -- attn_fwd_paged over an E4M3 paged cache.
+ * Source: "Attention Kernel", sections "Paged 与 ragged KV" (the paged
+ * layout) and "正确性契约" (the cache quantisation schema is part of the
+ * contract): element (page, r, h, i) of the K cache is
+ * k_scale[page, h] * e4m3(k_cache[page, r, h, i]) (V likewise).
+ *   q [total_q, Hq, d] bf16; k_cache, v_cache [num_pages, page_size, Hkv, d]
+ *   uint8 E4M3 codes (0x7F / 0xFF must not occur); k_scale, v_scale
+ *   [num_pages, Hkv] fp32 device arrays; the rest as attn_fwd_paged.
+ *   The call first writes the pages its sequences reach, dequantised to bf16
+ *   (round to nearest of scale * value), into the workspace, then runs the
+ *   bf16 paged prefill over them; no element of the cache is changed.
+ *   workspace: attn_fwd_paged_fp8_workspace_size(...) bytes, 16-byte aligned,
+ *   caller-owned, not shared with a concurrent call.
+ * Errors: as attn_fwd_paged, plus INVALID_ARG for a NULL scale array and
+ * ALIGNMENT for scales not 4-byte aligned.
+ */
+int attn_fwd_paged_fp8(const void* q, const void* k_cache, const void* v_cache,
+                       const float* k_scale, const float* v_scale, const int32_t* block_table,
+                       const int32_t* cu_seqlens_q, const int32_t* seq_lens_k, int page_size,
+                       int B, int Hq, int Hkv, long long total_q, int max_seqlen_q,
+                       int max_pages_per_seq, int num_pages, int d, int causal, float scale,
+                       void* o, float* lse, void* workspace, size_t workspace_bytes,
+                       attn_stream_t stream);
+
+/*
  * attn_fwd_window -- causal prefill with a sliding window or a prefix-LM mask.
  * Source: "Attention Kernel", section "可编程 mask" (masks such as a sliding
  * window or a prefix-LM rule: block-level sparsity decides which tiles are

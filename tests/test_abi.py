@@ -418,3 +418,27 @@ def test_bwd_masked_entry_validation(lib):
     assert lib.attn_bwd_block_sparse(*bargs, None, 1, F_, 1 << 20, None) == B.ATTN_ERR_INVALID_ARG
     assert lib.attn_bwd_block_sparse(*bargs, F_, 3, F_, 1 << 20, None) == B.ATTN_ERR_INVALID_ARG
     assert lib.attn_bwd_block_sparse(*bargs, F_, 1, F_, 16, None) == B.ATTN_ERR_WORKSPACE
+
+
+def test_paged_fp8_validation(lib):
+    F_ = FAKE
+    base = dict(q=F_, k=F_, v=F_, ks=F_, vs=F_, tbl=F_, cuq=F_, lens=F_, ps=16, B_=2, Hq=4, Hkv=2,
+                tq=100, mq=64, mp=8, np_=16, d=128, causal=1, scale=0.1, o=F_, lse=None, ws=F_,
+                wsb=1 << 30)
+
+    def call(**kw):
+        a = dict(base, **kw)
+        return lib.attn_fwd_paged_fp8(a["q"], a["k"], a["v"], a["ks"], a["vs"], a["tbl"], a["cuq"],
+                                      a["lens"], a["ps"], a["B_"], a["Hq"], a["Hkv"], a["tq"],
+                                      a["mq"], a["mp"], a["np_"], a["d"], a["causal"], a["scale"],
+                                      a["o"], a["lse"], a["ws"], a["wsb"], None)
+    assert call(ks=None) == B.ATTN_ERR_INVALID_ARG
+    assert call(vs=None) == B.ATTN_ERR_INVALID_ARG
+    assert call(ps=24) == B.ATTN_ERR_UNSUPPORTED
+    assert call(d=96) == B.ATTN_ERR_UNSUPPORTED
+    assert call(ks=F_ + 2) == B.ATTN_ERR_ALIGNMENT
+    assert call(wsb=1024) == B.ATTN_ERR_WORKSPACE
+    need = lib.attn_fwd_paged_fp8_workspace_size(2, 100, 64, 8, 16, 2, 128)
+    # unit list + table + two bf16 pools of B * max_pages pages
+    assert need >= 2 * 2 * 8 * 16 * 2 * 128 * 2
+    assert lib.attn_fwd_paged_fp8_workspace_size(0, 100, 64, 8, 16, 2, 128) == 0
