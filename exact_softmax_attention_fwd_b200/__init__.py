@@ -20,6 +20,8 @@ from ._binding import (  # noqa: F401
     attn_fwd,
     attn_fwd_fp8,
     attn_fwd_masked,
+    attn_fwd_host,
+    attn_fwd_host_workspace_size,
     attn_fwd_paged,
     attn_fwd_paged_fp8,
     attn_fwd_paged_fp8_workspace_size,

@@ -36,6 +36,8 @@ _SZ = ctypes.c_size_t
 SIGNATURES = {
     "attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "attn_fwd_masked": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P]),
+    "attn_fwd_host_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "attn_fwd_host": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _SZ, _P]),
     "attn_fwd_window": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _I, _I, _P]),
     "attn_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P,
                           _P]),
@@ -172,6 +174,61 @@ def attn_fwd_masked(q, k, v, causal: bool, scale: float, k_lens=None, out=None, 
                                         Hkv, Sq, Sk, d, int(bool(causal)), float(scale),
                                         _ptr(k_lens), _stream(stream))
     _check(st, "attn_fwd_masked")
+    return out, lse
+
+
+def attn_fwd_host_workspace_size(B: int, Hq: int, Hkv: int, Sq: int, Sk: int, d: int) -> int:
+    return int(load_library().attn_fwd_host_workspace_size(B, Hq, Hkv, Sq, Sk, d))
+
+
+def attn_fwd_host(q, k, v, causal: bool, scale: float, k_lens=None, out=None, lse=None,
+                  workspace=None, return_lse: bool = True, device=None, stream=None):
+    """attn_fwd_masked on HOST tensors (pinned for copy/compute overlap): q [B,Hq,Sq,d],
+    k/v [B,Hkv,Sk,d] bf16 CPU tensors, k_lens int32 [B] CPU tensor or None.  O and LSE
+    are host tensors, complete once ``stream`` (default: the current stream of
+    ``device``) reaches this call's end; synchronise it before reading them."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v), ("k_lens", k_lens)):
+        if t is not None and t.device.type != "cpu":
+            raise ValueError(f"{name} must be a host (CPU) tensor")
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bfloat16")
+    B, Hq, Sq, d = q.shape
+    Bk, Hkv, Sk, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or dk != d:
+        raise ValueError("q/k/v shapes disagree")
+    if k_lens is not None and (k_lens.dtype != torch.int32 or tuple(k_lens.shape) != (B,)
+                               or not k_lens.is_contiguous()):
+        raise ValueError("k_lens must be contiguous int32 [B]")
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    device = torch.device(device)
+    cpu = torch.device("cpu")
+    pin = q.is_pinned()
+    if out is None:
+        out = torch.empty(tuple(q.shape), dtype=torch.bfloat16, pin_memory=pin)
+    out = _out(out, q.shape, torch.bfloat16, cpu, "out")
+    if lse is not None or return_lse:
+        if lse is None:
+            lse = torch.empty((B, Hq, Sq), dtype=torch.float32, pin_memory=pin)
+        lse = _out(lse, (B, Hq, Sq), torch.float32, cpu, "lse")
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    need = attn_fwd_host_workspace_size(B, Hq, Hkv, Sq, Sk, d)
+    if workspace is None:
+        # allocated on ``stream``: the allocator reuses it only after the call's last copy
+        with torch.cuda.stream(stream):
+            workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+    if not workspace.is_cuda or workspace.device != device:
+        raise ValueError(f"workspace must be on {device}")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(device):
+        st = load_library().attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B,
+                                          Hq, Hkv, Sq, Sk, d, int(bool(causal)), float(scale),
+                                          _ptr(k_lens), _ptr(workspace), ws_bytes,
+                                          _stream(stream))
+    _check(st, "attn_fwd_host")
     return out, lse
 
 

@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "attn.h"
 #include "bwd_sm100.cuh"
@@ -502,6 +503,177 @@ int paged_prefill_run(const void* q, const void* k_cache, const void* v_cache,
                 : launch_prefill<64, false, kLayoutPaged>(mq, mk, mv, mq, prm, stream, max_units);
 }
 
+// ---------------------------------------------------------------------------
+// Prefill from and to host memory: the batch is cut into chunks of whole
+// (batch, KV head) pairs -- contiguous in every tensor -- and each chunk's
+// host-to-device copies, prefill launch and device-to-host copies run on
+// three streams (two copy streams owned by the library, the caller's stream
+// for the kernels) through two device buffer sets, so that copies of one
+// chunk overlap the kernels of another.
+// ---------------------------------------------------------------------------
+struct HostPipelineLayout {
+  int pairs_per_chunk, n_chunks;
+  size_t q_bytes, kv_bytes, lse_bytes;  // per chunk
+  size_t q_off[2], k_off[2], v_off[2], o_off[2], lse_off[2], klen_off, total;
+};
+
+HostPipelineLayout host_pipeline_layout(int B, int Hq, int Hkv, int Sq, int Sk, int d) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  HostPipelineLayout L;
+  const long long pairs = (long long)B * Hkv;
+  const int G = Hq / Hkv;
+  // about eight chunks: enough to overlap, few enough that each launch is large
+  L.pairs_per_chunk = (int)((pairs + 7) / 8);
+  L.n_chunks = (int)((pairs + L.pairs_per_chunk - 1) / L.pairs_per_chunk);
+  L.q_bytes = (size_t)L.pairs_per_chunk * G * Sq * d * 2;
+  L.kv_bytes = (size_t)L.pairs_per_chunk * Sk * d * 2;
+  L.lse_bytes = (size_t)L.pairs_per_chunk * G * Sq * 4;
+  size_t off = 0;
+  for (int sl = 0; sl < 2; ++sl) {
+    L.q_off[sl] = off;
+    off += up(L.q_bytes);
+    L.k_off[sl] = off;
+    off += up(L.kv_bytes);
+    L.v_off[sl] = off;
+    off += up(L.kv_bytes);
+    L.o_off[sl] = off;
+    off += up(L.q_bytes);
+    L.lse_off[sl] = off;
+    off += up(L.lse_bytes);
+  }
+  L.klen_off = off;  // key length of every (batch, KV head) pair
+  off += up((size_t)pairs * 4);
+  L.total = off;
+  return L;
+}
+
+// Two copy streams and the events of the two buffer sets, created once per
+// device and kept for the life of the process.  A call holds its device's
+// mutex while it enqueues, so that calls from several host threads do not
+// interleave their event records.
+struct HostPipelineRes {
+  std::mutex mu;
+  cudaStream_t h2d, d2h;
+  cudaEvent_t start, h2d_done[2], comp_done[2], d2h_done[2];
+  bool ready;
+};
+
+constexpr int kMaxPipelineDevices = 64;
+
+// On success the device's mutex is held; the caller releases it.
+int host_pipeline_res(HostPipelineRes** out) {
+  static HostPipelineRes res[kMaxPipelineDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxPipelineDevices) return ATTN_ERR_CUDA;
+  HostPipelineRes& r = res[dev];
+  r.mu.lock();
+  if (!r.ready) {
+    const unsigned fl = cudaEventDisableTiming;
+    if (cudaStreamCreateWithFlags(&r.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&r.d2h, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&r.start, fl) != cudaSuccess) {
+      r.mu.unlock();
+      return ATTN_ERR_CUDA;
+    }
+    for (int i = 0; i < 2; ++i)
+      if (cudaEventCreateWithFlags(&r.h2d_done[i], fl) != cudaSuccess ||
+          cudaEventCreateWithFlags(&r.comp_done[i], fl) != cudaSuccess ||
+          cudaEventCreateWithFlags(&r.d2h_done[i], fl) != cudaSuccess) {
+        r.mu.unlock();
+        return ATTN_ERR_CUDA;
+      }
+    r.ready = true;
+  }
+  *out = &r;
+  return ATTN_OK;
+}
+
+int host_pipeline_enqueue(HostPipelineRes* R, const HostPipelineLayout& L, const void* q,
+                          const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                          int Hkv, int Sq, int Sk, int d, int causal, float scale,
+                          const int32_t* k_lens, char* ws, cudaStream_t stream) {
+  int st = ATTN_OK;
+  const int G = Hq / Hkv;
+  const long long pairs = (long long)B * Hkv;
+  int32_t* klen_dev = reinterpret_cast<int32_t*>(ws + L.klen_off);
+  // the copy streams start after the caller's earlier work
+  if (cudaEventRecord(R->start, stream) != cudaSuccess ||
+      cudaStreamWaitEvent(R->h2d, R->start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(R->d2h, R->start, 0) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (k_lens != nullptr) {
+    // one key length per (batch, KV head) pair: the chunks are batches of pairs
+    std::vector<int32_t> per_pair((size_t)pairs);
+    for (long long pr = 0; pr < pairs; ++pr) per_pair[(size_t)pr] = k_lens[pr / Hkv];
+    if (cudaMemcpyAsync(klen_dev, per_pair.data(), (size_t)pairs * 4, cudaMemcpyHostToDevice,
+                        stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)  // per_pair is freed on return
+      return ATTN_ERR_CUDA;
+  }
+  const char* qh = static_cast<const char*>(q);
+  const char* kh = static_cast<const char*>(k);
+  const char* vh = static_cast<const char*>(v);
+  char* oh = static_cast<char*>(o);
+  char* lh = reinterpret_cast<char*>(lse);
+  const size_t q_pair = (size_t)G * Sq * d * 2, kv_pair = (size_t)Sk * d * 2,
+               l_pair = (size_t)G * Sq * 4;
+  for (int c = 0; c < L.n_chunks; ++c) {
+    const int sl = c & 1;
+    const long long p0 = (long long)c * L.pairs_per_chunk;
+    const int np = (int)(p0 + L.pairs_per_chunk <= pairs ? L.pairs_per_chunk : pairs - p0);
+    char* qd = ws + L.q_off[sl];
+    char* kd = ws + L.k_off[sl];
+    char* vd = ws + L.v_off[sl];
+    char* od = ws + L.o_off[sl];
+    float* ld = reinterpret_cast<float*>(ws + L.lse_off[sl]);
+    // inputs into buffer set sl once the kernels of chunk c - 2 are done with it
+    if (c >= 2 && cudaStreamWaitEvent(R->h2d, R->comp_done[sl], 0) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    if (cudaMemcpyAsync(qd, qh + p0 * q_pair, np * q_pair, cudaMemcpyHostToDevice, R->h2d) !=
+            cudaSuccess ||
+        (Sk > 0 && (cudaMemcpyAsync(kd, kh + p0 * kv_pair, np * kv_pair, cudaMemcpyHostToDevice,
+                                    R->h2d) != cudaSuccess ||
+                    cudaMemcpyAsync(vd, vh + p0 * kv_pair, np * kv_pair, cudaMemcpyHostToDevice,
+                                    R->h2d) != cudaSuccess)) ||
+        cudaEventRecord(R->h2d_done[sl], R->h2d) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    // the kernels, once the inputs landed and chunk c - 2's outputs left buffer set sl
+    if (cudaStreamWaitEvent(stream, R->h2d_done[sl], 0) != cudaSuccess ||
+        (c >= 2 && cudaStreamWaitEvent(stream, R->d2h_done[sl], 0) != cudaSuccess))
+      return ATTN_ERR_CUDA;
+    st = prefill_dense(qd, kd, vd, od, lse != nullptr ? ld : nullptr, np, G, 1, Sq, Sk, d, causal,
+                       scale, k_lens != nullptr ? klen_dev + p0 : nullptr, 0, 0, nullptr, 1,
+                       stream);
+    if (st != ATTN_OK) return st;
+    if (cudaEventRecord(R->comp_done[sl], stream) != cudaSuccess) return ATTN_ERR_CUDA;
+    // outputs back to the host
+    if (cudaStreamWaitEvent(R->d2h, R->comp_done[sl], 0) != cudaSuccess ||
+        cudaMemcpyAsync(oh + p0 * q_pair, od, np * q_pair, cudaMemcpyDeviceToHost, R->d2h) !=
+            cudaSuccess ||
+        (lse != nullptr && cudaMemcpyAsync(lh + p0 * l_pair, ld, np * l_pair,
+                                           cudaMemcpyDeviceToHost, R->d2h) != cudaSuccess) ||
+        cudaEventRecord(R->d2h_done[sl], R->d2h) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+  }
+  // the call is complete on the caller's stream once the last copies are
+  for (int sl = 0; sl < 2 && sl < L.n_chunks; ++sl)
+    if (cudaStreamWaitEvent(stream, R->d2h_done[(L.n_chunks - 1 - sl) & 1], 0) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+int host_pipeline_run(const HostPipelineLayout& L, const void* q, const void* k, const void* v,
+                      void* o, float* lse, int B, int Hq, int Hkv, int Sq, int Sk, int d,
+                      int causal, float scale, const int32_t* k_lens, char* ws,
+                      cudaStream_t stream) {
+  HostPipelineRes* R = nullptr;
+  const int st = host_pipeline_res(&R);
+  if (st != ATTN_OK) return st;
+  std::lock_guard<std::mutex> g(R->mu, std::adopt_lock);
+  return host_pipeline_enqueue(R, L, q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens,
+                               ws, stream);
+}
+
 // Workspace of the E4M3 paged prefill: the unit list, the remapped block
 // table [B, max_pages], and bf16 K and V pools of one page slot per
 // (sequence, logical page), each part 256-byte aligned.
@@ -736,6 +908,27 @@ int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float*
   if (st != ATTN_OK) return st;
   return prefill_dense(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens, 0, 0,
                        nullptr, 1, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t attn_fwd_host_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int d) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Sq < 1 || Sk < 0 || (d != 64 && d != 128))
+    return 0;
+  return host_pipeline_layout(B, Hq, Hkv, Sq, Sk, d).total;
+}
+
+int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                  int Hkv, int Sq, int Sk, int d, int causal, float scale, const int32_t* k_lens,
+                  void* workspace, size_t workspace_bytes, attn_stream_t stream_) {
+  int st = check_prefill_args(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, causal, scale, nullptr);
+  if (st != ATTN_OK) return st;
+  const HostPipelineLayout L = host_pipeline_layout(B, Hq, Hkv, Sq, Sk, d);
+  if (workspace == nullptr || workspace_bytes < L.total) return ATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
+  if (k_lens != nullptr)
+    for (int b = 0; b < B; ++b)  // host array: checked here, as the device path clamps
+      if (k_lens[b] < 0 || k_lens[b] > Sk) return ATTN_ERR_INVALID_ARG;
+  return host_pipeline_run(L, q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, d, causal, scale, k_lens,
+                           static_cast<char*>(workspace), reinterpret_cast<cudaStream_t>(stream_));
 }
 
 int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,

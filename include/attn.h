@@ -96,6 +96,39 @@ int attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float*
                     const int32_t* k_lens, attn_stream_t stream);
 
 /*
+ * attn_fwd_host_workspace_size -- bytes of device workspace attn_fwd_host
+ * needs for these extents: two buffer sets of one chunk's Q, K, V, O and LSE
+ * plus B * Hkv key lengths (a chunk is about an eighth of the B * Hkv
+ * (sequence, KV head) pairs).  0 for invalid arguments.
+ */
+size_t attn_fwd_host_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int d);
+
+/*
+ * attn_fwd_host -- attn_fwd_masked on tensors in HOST memory.
+ * Source: as attn_fwd_masked; the result is bit-identical to it.  The batch is
+ * cut into chunks of whole (sequence, KV head) pairs; each chunk's Q, K, V are
+ * copied in, computed and its O, LSE copied out through two device buffer
+ * sets, with the copies of one chunk overlapping the kernels of another.
+ *   q, k, v, o, lse: host pointers, same shapes and layouts as attn_fwd
+ *   (lse nullable).  Page-locked (pinned) memory gives the overlap; pageable
+ *   memory is correct but the copies then serialise with the host.
+ *   k_lens [B] int32 HOST array, nullable; values must lie in [0, Sk].
+ *   workspace: device buffer of attn_fwd_host_workspace_size() bytes,
+ *   16-byte aligned, caller-owned, not shared with a concurrent call.
+ *   stream: the kernels run on it; the copies run on two streams the library
+ *   creates once per device and keeps, ordered after the work already on
+ *   `stream`.  O and LSE are complete, and q, k, v may be reused, once
+ *   `stream` reaches the point where the call returned.
+ *   Unlike every other entry point this one may block: when k_lens is given
+ *   it synchronises `stream` once, and copies from pageable memory block.
+ * Errors: as attn_fwd_masked, plus INVALID_ARG for a k_lens value outside
+ * [0, Sk] and WORKSPACE for a missing or short workspace.
+ */
+int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                  int Hkv, int Sq, int Sk, int d, int causal, float scale, const int32_t* k_lens,
+                  void* workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
  * attn_fwd_fp8 -- attn_fwd_masked over block-scaled E4M3 Q, K and V.
  * Source: "Attention 算子加速史", section 3.3 (FP8 operands with block-level
  * scaling); the operation is attn_fwd_masked's on the dequantised values.

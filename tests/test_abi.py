@@ -442,3 +442,42 @@ def test_paged_fp8_validation(lib):
     # unit list + table + two bf16 pools of B * max_pages pages
     assert need >= 2 * 2 * 8 * 16 * 2 * 128 * 2
     assert lib.attn_fwd_paged_fp8_workspace_size(0, 100, 64, 8, 16, 2, 128) == 0
+
+
+def test_fwd_host_validation(lib):
+    F_ = FAKE
+
+    def call(q=F_, lens=None, ws=F_, wsb=1 << 40, d=128, Hq=4, Hkv=2, Sk=300):
+        return lib.attn_fwd_host(q, F_, F_, F_, None, 2, Hq, Hkv, 200, Sk, d, 1, 0.1, lens, ws, wsb,
+                                 None)
+    assert call(q=None) == B.ATTN_ERR_INVALID_ARG
+    assert call(Hq=3) == B.ATTN_ERR_INVALID_ARG
+    assert call(d=96) == B.ATTN_ERR_UNSUPPORTED
+    assert call(ws=None) == B.ATTN_ERR_WORKSPACE
+    assert call(wsb=1024) == B.ATTN_ERR_WORKSPACE
+    assert call(ws=F_ + 4) == B.ATTN_ERR_ALIGNMENT
+    # host key lengths are checked on the host, before any copy
+    for bad in ((300, 301), (-1, 5)):
+        lens = (ctypes.c_int32 * 2)(*bad)
+        assert call(lens=ctypes.cast(lens, ctypes.c_void_p)) == B.ATTN_ERR_INVALID_ARG
+
+
+def test_fwd_host_workspace_size_formula(lib):
+    def up(x):
+        return (x + 255) // 256 * 256
+    for (B_, Hq, Hkv, Sq, Sk, d) in ((1, 32, 8, 32768, 32768, 128), (3, 6, 3, 200, 333, 64),
+                                     (2, 4, 4, 1, 0, 128)):
+        pairs, G = B_ * Hkv, Hq // Hkv
+        ppc = (pairs + 7) // 8  # about eight chunks of whole (sequence, KV head) pairs
+        qb, kvb, lb = ppc * G * Sq * d * 2, ppc * Sk * d * 2, ppc * G * Sq * 4
+        want = 2 * (2 * up(qb) + 2 * up(kvb) + up(lb)) + up(pairs * 4)
+        assert lib.attn_fwd_host_workspace_size(B_, Hq, Hkv, Sq, Sk, d) == want
+    assert lib.attn_fwd_host_workspace_size(1, 3, 2, 128, 128, 128) == 0
+    assert lib.attn_fwd_host_workspace_size(1, 4, 2, 128, 128, 96) == 0
+
+
+def test_fwd_host_binding_refuses_device_tensors():
+    import torch
+    q = torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16, device="meta")
+    with pytest.raises(ValueError, match="host"):
+        B.attn_fwd_host(q, q, q, True, 0.1)
