@@ -368,6 +368,9 @@ int decode_paged_common(bool fp8, const void* q, const void* k_cache, const void
       !aligned4(block_table) || !aligned4(seq_lens) || (lse != nullptr && !aligned4(lse)))
     return ATTN_ERR_ALIGNMENT;
   if (fp8 && (!aligned4(k_scale) || !aligned4(v_scale))) return ATTN_ERR_ALIGNMENT;
+  // the split kernel's grid x runs over (split, KV head) pairs
+  const long long n_split_ll = ((long long)max_pages_per_seq * page_size + kSplitTokens - 1) / kSplitTokens;
+  if (n_split_ll * Hkv > INT_MAX) return ATTN_ERR_INVALID_ARG;
   const size_t need = attn_decode_workspace_size(B, Hq, max_pages_per_seq, page_size, d);
   if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
   if (!aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
@@ -408,7 +411,7 @@ int decode_paged_common(bool fp8, const void* q, const void* k_cache, const void
           : make_token_map(&mk, k_cache, d, Hkv, pool_tokens, 16) &&
                 make_token_map(&mv, v_cache, d, Hkv, pool_tokens, 16);
   if (!maps_ok) return ATTN_ERR_CUDA;
-  dim3 grid_split(prm.n_split, Hkv, B);
+  dim3 grid_split((unsigned)((long long)prm.n_split * Hkv), 1, B);
   dim3 grid_merge((unsigned)(((long long)B * Hq + 3) / 4));
   int st = ATTN_OK;
   if (d == 128)

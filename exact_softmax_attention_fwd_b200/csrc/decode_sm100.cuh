@@ -30,9 +30,18 @@
 // bytes and widens them to f16 right before use (exact: E4M3 has 3 mantissa
 // bits and a narrower exponent range).  q K^T is an f16 MMA on q scaled by a
 // power of two into f16's range; its fp32 scores are multiplied back and by
-// the page's K scale.  P^T V is an f16 MMA (P <= 1 is rounded to f16) whose
-// fp32 result for the 16 tokens -- which always lie in one page -- is
-// multiplied by the page's V scale before it joins the accumulator.
+// the page's K scale.  P^T V is an f16 MMA that accumulates straight into the
+// fp32 accumulator: the 16 tokens of a step always lie in one page, so the
+// page's V scale enters as a factor vs / vmax <= 1 on P before P is rounded
+// to f16 (vmax = the largest V scale of the split's pages), and the
+// accumulator, in units of vmax, is multiplied by vmax once at the end.  The
+// normaliser sums the weights as applied to the dequantised V: f16(P') * vmax
+// / vs per token.
+//
+// Rescaling is lazy, as in the prefill kernel: the exponent base of a head
+// row moves only when the row max exceeds it by more than 8 (log2 units), so
+// P <= 2^8 and the accumulator is rescaled only on the steps where some row
+// of the warp moved its base.
 //
 // Merge kernel: one warp per (b, query head) combines the splits in a fixed
 // order: LSE = M + log2 sum_s 2^(lse_s - M), O = sum_s 2^(lse_s - LSE) o_s,
@@ -110,37 +119,44 @@ __device__ __forceinline__ void mma_m16n8k16_f16(float (&c)[4], uint32_t a0, uin
 // ---------------------------------------------------------------------------
 // Split kernel with the K/V stream staged in shared memory by TMA.
 //
-// One warp (and CTA) per (sequence b, KV head, split of kSplitTokens tokens),
-// the MMA fragments and the online softmax of the register kernels above, but
-// the 16-token K and V tiles of each step arrive by tensor-memory-access copies
-// (cp.async.bulk.tensor, no multicast) into a DEC_STAGES-deep ring of shared
-// memory, so the bytes in flight no longer cost registers: lane 0 keeps the
-// next DEC_STAGES - 1 steps' copies outstanding while the warp computes.  The
-// cache is read by the copies as the token-major tensor [num_pages *
-// page_size, Hkv, D] (page p starts at token p * page_size); a 16-token step
-// never crosses a page (page sizes are multiples of 16), so a step is one box
-// of 16 rows x (up to) 128 bytes per 128-byte column block, for K and for V.
-// The boxes land 128-byte swizzled (64-byte for 64-byte rows), which keeps the
-// fragment loads from shared memory free of bank conflicts for K.
+// One warp (and CTA) per (sequence b, KV head, split of kSplitTokens tokens);
+// the grid's x index runs over the KV heads of a split first, so that the
+// warps reading the same pages run together.  The K and V rows of each step
+// arrive by tensor-memory-access copies (cp.async.bulk.tensor, no multicast)
+// into a STAGES-deep ring of shared memory, so the bytes in flight cost no
+// registers: lane 0 keeps the next STAGES - 1 steps' copies outstanding while
+// the warp computes.  The cache is read by the copies as the token-major
+// tensor [num_pages * page_size, Hkv, D] (page p starts at token p *
+// page_size).  A step is NH chunks of 16 tokens (one for bf16 caches, two for
+// E4M3 caches, whose rows are half as long, so that both move about the same
+// bytes per step); a chunk never crosses a page (page sizes are multiples of
+// 16), so it is one box of 16 rows x (up to) 128 bytes per 128-byte column
+// block, for K and for V.  The boxes land 128-byte swizzled (64-byte for
+// 64-byte rows), which keeps the fragment loads from shared memory free of
+// bank conflicts for K.
 //
 // Each lane reads one block-table entry (and, for E4M3 caches, one pair of
-// scales) up front: the split's steps are at most 32, one per lane, and a
-// step's page is fetched from its lane by a shuffle.  Tokens past the length
-// and steps on a page id outside the pool contribute exact zeros (their
+// scales) up front: the split has at most 32 chunks, one per lane, and a
+// chunk's page is fetched from its lane by a shuffle.  Tokens past the length
+// and chunks on a page id outside the pool contribute exact zeros (their
 // fragments are zeroed after the shared-memory load, so stale or non-finite
 // slot contents never reach the MMAs); bad ids are flagged.
 // ---------------------------------------------------------------------------
 template <int D, bool FP8>
 struct DecodeTmaCfg {
+  static constexpr int NH = FP8 ? 2 : 1;           // 16-token chunks per step
   // ring depth: the bytes in flight per warp against the warps an SM holds
-  // (shared memory per warp grows with the depth)
-  static constexpr int STAGES = FP8 ? 4 : 3;
+  // (shared memory per warp grows with the depth).  Measured on paged_decode:
+  // 3 slots of 8 KB for bf16 (2 slots: -2%); 2 slots of 8 KB for E4M3, which
+  // fits 13 warps per SM (3 slots: -4%, 4 slots: -15%)
+  static constexpr int STAGES = FP8 ? 2 : 3;
   static constexpr int E = FP8 ? 1 : 2;            // bytes per element
   static constexpr int ROW = D * E;                // bytes per token row of one head
   static constexpr int BOX_BYTES = ROW < 128 ? ROW : 128;  // inner box extent in bytes
   static constexpr int NBOX = ROW / BOX_BYTES;     // column boxes per row
   static constexpr int TILE = 16 * ROW;            // 16 tokens of K (or V)
-  static constexpr int STAGE = 2 * TILE;           // K then V
+  static constexpr int CHUNK = 2 * TILE;           // K then V of one chunk
+  static constexpr int STAGE = NH * CHUNK;
   static constexpr int SMEM = STAGES * STAGE + 64 + 1024;  // ring, barriers, alignment
   static_assert(kSplitTokens / 16 <= 32, "one block-table entry per lane");
 };
@@ -172,10 +188,11 @@ __device__ __forceinline__ uint2 lds_u2(uint32_t addr) {
 }
 
 template <int D, bool FP8>
-__global__ void __launch_bounds__(32) attn_decode_split_tma_kernel(
+__global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const DecodeFp8Params f) {
   using C = DecodeTmaCfg<D, FP8>;
+  constexpr int NH = C::NH;
   constexpr int KW = D * C::E / 16;   // 32-bit words of a thread's K quarter row
   constexpr int VW = D * C::E / 32;   // 32-bit words of a thread's V eighth row
   const DecodeParams& p = f.d;
@@ -184,19 +201,21 @@ __global__ void __launch_bounds__(32) attn_decode_split_tma_kernel(
   const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
   const uint32_t bars = sbase + C::STAGES * C::STAGE;
   const int lane = threadIdx.x;
-  const int split = blockIdx.x;
-  const int kvh = blockIdx.y;
+  const int kvh = (int)(blockIdx.x % (unsigned)p.Hkv);
+  const int split = (int)(blockIdx.x / (unsigned)p.Hkv);
   const int b = blockIdx.z;
   const int len = decode_clamped_len(p, b, lane == 0 && split == 0 && kvh == 0);
   const int t_begin = split * kSplitTokens;
   if (t_begin >= len) return;  // the merge kernel never reads splits past the end
   const int t_end = min(t_begin + kSplitTokens, len);
-  const int n_steps = (t_end - t_begin + 15) / 16;
+  const int n_chunks = (t_end - t_begin + 15) / 16;
+  const int n_steps = (n_chunks + NH - 1) / NH;
 
-  // this lane's step: its page (or -1 when the id is outside the pool) and scales
+  // this lane's chunk: its page (or -1 when the id is outside the pool, or
+  // past the split) and scales
   int my_page = -1;
   float my_ks = 0.f, my_vs = 0.f;
-  if (lane < n_steps) {
+  if (lane < n_chunks) {
     const int t = t_begin + 16 * lane;
     const int pg = p.block_table[(size_t)b * p.max_pages + t / p.page_size];
     if (pg >= 0 && pg < p.num_pages) {
@@ -216,18 +235,25 @@ __global__ void __launch_bounds__(32) attn_decode_split_tma_kernel(
     tma_prefetch_map(&tm_v);
   }
   __syncwarp();
-  // Step i's copies into slot i % C::STAGES (lane 0; every lane calls it for
-  // the shuffle).  A step on a bad page arms its barrier with no bytes.
+  // Step i's copies into slot i % C::STAGES (lane 0; every lane takes part in
+  // the shuffles).  Chunks on a bad page, or past the split, add no bytes.
   auto issue = [&](int i) {
-    const int pg = __shfl_sync(0xffffffffu, my_page, i);
+    int pg[NH];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) pg[h] = __shfl_sync(0xffffffffu, my_page, NH * i + h);
     if (lane == 0) {
       const int slot = i % C::STAGES;
       const uint32_t bar = bars + 8u * slot;
-      const uint32_t dst = sbase + slot * C::STAGE;
+      uint32_t bytes = 0;
+#pragma unroll
+      for (int h = 0; h < NH; ++h) bytes += pg[h] >= 0 ? (uint32_t)C::CHUNK : 0u;
       fence_proxy_async_smem();  // the warp's reads of this slot precede the refill
-      mbar_arrive_expect_tx(bar, pg >= 0 ? (uint32_t)C::STAGE : 0u);
-      if (pg >= 0) {
-        const int tok = pg * p.page_size + (t_begin + 16 * i) % p.page_size;
+      mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        if (pg[h] < 0) continue;
+        const uint32_t dst = sbase + slot * C::STAGE + h * C::CHUNK;
+        const int tok = pg[h] * p.page_size + (t_begin + 16 * (NH * i + h)) % p.page_size;
 #pragma unroll
         for (int bx = 0; bx < C::NBOX; ++bx) {
           const int col = bx * (C::BOX_BYTES / C::E);
@@ -239,6 +265,14 @@ __global__ void __launch_bounds__(32) attn_decode_split_tma_kernel(
   };
   int n_issued = 0;
   for (; n_issued < C::STAGES - 1 && n_issued < n_steps; ++n_issued) issue(n_issued);
+  // E4M3: the largest V scale of the split's pages (bad pages hold 0)
+  float vmax = FP8 ? my_vs : 1.f;
+  if (FP8) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    if (!(vmax > 0.f)) vmax = 1.f;
+  }
+  const float inv_vmax = FP8 ? 1.f / vmax : 1.f;
 
   const int g = lane >> 2;   // MMA group id: head row of S / P, d-row block of V^T
   const int tq = lane & 3;   // thread within the group
@@ -289,9 +323,9 @@ __global__ void __launch_bounds__(32) attn_decode_split_tma_kernel(
   float c2 = p.scale_log2;
   const bool scale_pos = c2 > 0.f;
   if (!scale_pos) c2 = 1.f;
-  float m_run = -INFINITY;  // per head row g, log2 units
+  float m_run = -INFINITY;  // exponent base of head row g (log2 units)
   float l_run = 0.f;        // sum of P (f32): the LSE
-  float lr_run = 0.f;       // sum of the rounded P the MMA consumes: normalises O
+  float lr_run = 0.f;       // sum of the weights the MMA applies: normalises O
   float acc[D / 16][4];
 #pragma unroll
   for (int mc = 0; mc < D / 16; ++mc) acc[mc][0] = acc[mc][1] = acc[mc][2] = acc[mc][3] = 0.f;
@@ -301,133 +335,179 @@ __global__ void __launch_bounds__(32) attn_decode_split_tma_kernel(
   for (; i < n_steps; ++i) {
     if (n_issued < n_steps) issue(n_issued++);  // step i + C::STAGES - 1
     const int slot = i % C::STAGES;
-    const int pg = __shfl_sync(0xffffffffu, my_page, i);
-    const int n_here = pg >= 0 ? min(16, t_end - (t_begin + 16 * i)) : 0;
-    const float ksc = FP8 ? __shfl_sync(0xffffffffu, my_ks, i) : 1.f;
-    const float vsc = FP8 ? __shfl_sync(0xffffffffu, my_vs, i) : 1.f;
-    const uint32_t kt = sbase + slot * C::STAGE;
-    const uint32_t vt = kt + C::TILE;
+    int n_here[NH];
+    float ksc[NH], vsc[NH];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      const int c = NH * i + h;
+      const int pg = __shfl_sync(0xffffffffu, my_page, c);
+      n_here[h] = pg >= 0 ? min(16, t_end - (t_begin + 16 * c)) : 0;  // <= 0 past the end
+      ksc[h] = FP8 ? __shfl_sync(0xffffffffu, my_ks, c) : 1.f;
+      vsc[h] = FP8 ? __shfl_sync(0xffffffffu, my_vs, c) : 1.f;
+    }
+    const uint32_t st = sbase + slot * C::STAGE;
     const bool landed = mbar_wait(bars + 8u * slot, (uint32_t)(i / C::STAGES) & 1u, nullptr);
     if (!__all_sync(0xffffffffu, landed)) break;  // timed out: flagged, wind down
 
-    // ---- S = q K^T (16 padded head rows x 16 tokens)
-    float sc[2][4];
+    // ---- S = q K^T (16 padded head rows x 16 tokens per chunk); two
+    // independent accumulation chains (even and odd d-chunks), summed
+    float s4[NH][4];
 #pragma unroll
-    for (int nc = 0; nc < 2; ++nc) {
-      const int tok = nc * 8 + g;
-      uint32_t kw[KW];
+    for (int h = 0; h < NH; ++h) {
+      const uint32_t kt = st + h * C::CHUNK;
 #pragma unroll
-      for (int w = 0; w < KW / 4; ++w) {
-        const uint4 x = lds_u4(kt + dec_tile_off<D, FP8>(tok, (D * C::E / 4) * tq + 16 * w));
-        kw[4 * w + 0] = x.x;
-        kw[4 * w + 1] = x.y;
-        kw[4 * w + 2] = x.z;
-        kw[4 * w + 3] = x.w;
-      }
-      if (tok >= n_here) {
+      for (int nc = 0; nc < 2; ++nc) {
+        const int tok = nc * 8 + g;
+        uint32_t kw[KW];
 #pragma unroll
-        for (int w = 0; w < KW; ++w) kw[w] = 0u;
-      }
-      sc[nc][0] = sc[nc][1] = sc[nc][2] = sc[nc][3] = 0.f;
-      if (!FP8) {
-#pragma unroll
-        for (int kc = 0; kc < D / 16; ++kc)
-          mma_m16n8k16_bf16(sc[nc], qa[kc][0], 0u, qa[kc][1], 0u, kw[2 * kc], kw[2 * kc + 1]);
-      } else {
-#pragma unroll
-        for (int kc = 0; kc < D / 16; ++kc) {
-          const uint32_t w = kw[kc];
-          mma_m16n8k16_f16(sc[nc], qa[kc][0], 0u, qa[kc][1], 0u, e4m3x2_to_f16x2(w),
-                           e4m3x2_to_f16x2(w >> 16));
+        for (int w = 0; w < KW / 4; ++w) {
+          const uint4 x = lds_u4(kt + dec_tile_off<D, FP8>(tok, (D * C::E / 4) * tq + 16 * w));
+          kw[4 * w + 0] = x.x;
+          kw[4 * w + 1] = x.y;
+          kw[4 * w + 2] = x.z;
+          kw[4 * w + 3] = x.w;
         }
+        if (tok >= n_here[h]) {
+#pragma unroll
+          for (int w = 0; w < KW; ++w) kw[w] = 0u;
+        }
+        float sx[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        if (!FP8) {
+#pragma unroll
+          for (int kc = 0; kc < D / 16; ++kc)
+            mma_m16n8k16_bf16(sx[kc & 1], qa[kc][0], 0u, qa[kc][1], 0u, kw[2 * kc], kw[2 * kc + 1]);
+        } else {
+#pragma unroll
+          for (int kc = 0; kc < D / 16; ++kc) {
+            const uint32_t w = kw[kc];
+            mma_m16n8k16_f16(sx[kc & 1], qa[kc][0], 0u, qa[kc][1], 0u, e4m3x2_to_f16x2(w),
+                             e4m3x2_to_f16x2(w >> 16));
+          }
+        }
+        // this thread's scores of head row g: tokens 8nc + 2tq and 8nc + 2tq + 1
+        const float kq = FP8 ? ksc[h] * qscale : 1.f;
+        s4[h][2 * nc + 0] = (sx[0][0] + sx[1][0]) * kq;
+        s4[h][2 * nc + 1] = (sx[0][1] + sx[1][1]) * kq;
       }
     }
 
-    // ---- online softmax for head row g over this thread's 4 tokens
-    const float kq = FP8 ? ksc * qscale : 1.f;
-    float s4[4] = {sc[0][0] * kq, sc[0][1] * kq, sc[1][0] * kq, sc[1][1] * kq};
+    // ---- online softmax for head row g over this thread's 4 NH tokens
+    float mx = -INFINITY;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int tok = (e >> 1) * 8 + 2 * tq + (e & 1);
-      if (tok >= n_here) s4[e] = -INFINITY;
-      else if (!scale_pos) s4[e] *= p.scale_log2;
+    for (int h = 0; h < NH; ++h) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tok = (e >> 1) * 8 + 2 * tq + (e & 1);
+        if (tok >= n_here[h]) s4[h][e] = -INFINITY;
+        else if (!scale_pos) s4[h][e] *= p.scale_log2;
+      }
+      mx = fmaxf(mx, fmaxf(fmaxf(s4[h][0], s4[h][1]), fmaxf(s4[h][2], s4[h][3])));
     }
-    float mx = fmaxf(fmaxf(s4[0], s4[1]), fmaxf(s4[2], s4[3]));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float m_new = fmaxf(m_run, mx * c2);
-    // nothing accumulated while m_run = -inf (also avoids -inf - -inf = NaN)
-    const float alpha = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_new);
-    const float base = (m_new == -INFINITY) ? 0.f : m_new;
-    float pr[4];
+    // lazy base: moves only when the max exceeds it by more than 8 (also true
+    // for the first finite max; alpha = 2^-inf = 0 then, nothing accumulated)
+    const float m_tile = mx * c2;
+    float alpha = 1.f;
+    if (m_tile > m_run + 8.f) {
+      alpha = ex2(m_run - m_tile);
+      m_run = m_tile;
+    }
+    const float base = (m_run == -INFINITY) ? 0.f : m_run;
+    // P^T rows (tokens) 2tq, 2tq+1 and 2tq+8, 2tq+9 of each chunk, column g
+    // (head): bf16 for a bf16 cache; for an E4M3 cache f16 of P * vs / vmax
+    // (<= 2^8), and the weights on the dequantised V are f16(P') * vmax / vs
+    uint32_t pb[NH][2];
+    float rs = 0.f, rr = 0.f;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) pr[e] = ex2(fmaf(s4[e], c2, -base));
-    // P^T rows (tokens) 2tq, 2tq+1 and 2tq+8, 2tq+9, column g (head): bf16 for a
-    // bf16 cache, f16 (P <= 1) for the f16 MMA of an E4M3 cache
-    const uint32_t pb0 = FP8 ? pack_f16x2(pr[0], pr[1]) : pack_bf16x2(pr[0], pr[1]);
-    const uint32_t pb1 = FP8 ? pack_f16x2(pr[2], pr[3]) : pack_bf16x2(pr[2], pr[3]);
-    float rs = (pr[0] + pr[1]) + (pr[2] + pr[3]);
-    float rr = FP8 ? (f16_to_f32(pb0) + f16_to_f32(pb0 >> 16)) +
-                         (f16_to_f32(pb1) + f16_to_f32(pb1 >> 16))
-                   : sum_f32x2(add_f32x2(bf16x2_to_f32x2(pb0), bf16x2_to_f32x2(pb1)));
+    for (int h = 0; h < NH; ++h) {
+      float pr[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) pr[e] = ex2(fmaf(s4[h][e], c2, -base));
+      rs += (pr[0] + pr[1]) + (pr[2] + pr[3]);
+      if (!FP8) {
+        pb[h][0] = pack_bf16x2(pr[0], pr[1]);
+        pb[h][1] = pack_bf16x2(pr[2], pr[3]);
+        rr += sum_f32x2(add_f32x2(bf16x2_to_f32x2(pb[h][0]), bf16x2_to_f32x2(pb[h][1])));
+      } else {
+        const float rv = vsc[h] * inv_vmax;
+        pb[h][0] = pack_f16x2(pr[0] * rv, pr[1] * rv);
+        pb[h][1] = pack_f16x2(pr[2] * rv, pr[3] * rv);
+        const float back = vsc[h] > 0.f ? vmax / vsc[h] : 0.f;  // no token of a bad page
+        rr += ((f16_to_f32(pb[h][0]) + f16_to_f32(pb[h][0] >> 16)) +
+               (f16_to_f32(pb[h][1]) + f16_to_f32(pb[h][1] >> 16))) * back;
+      }
+    }
     rs += __shfl_xor_sync(0xffffffffu, rs, 1);
     rr += __shfl_xor_sync(0xffffffffu, rr, 1);
     rs += __shfl_xor_sync(0xffffffffu, rs, 2);
     rr += __shfl_xor_sync(0xffffffffu, rr, 2);
     l_run = l_run * alpha + rs;
     lr_run = lr_run * alpha + rr;
-    m_run = m_new;
 
     // ---- O^T += V^T P^T; accumulator columns are heads 2tq and 2tq+1.  V^T
     // rows d = (D/8)*g + 2*mc (+1), columns = tokens 2tq, 2tq+1, 2tq+8, 2tq+9.
-    uint32_t vw[4][VW > 0 ? VW : 1];
+    uint32_t vw[NH][4][VW > 0 ? VW : 1];
 #pragma unroll
-    for (int ti = 0; ti < 4; ++ti) {
-      const int tok = 2 * tq + (ti & 1) + 8 * (ti >> 1);
-      const int byte0 = (D * C::E / 8) * g;
-      if constexpr (VW >= 4) {
+    for (int h = 0; h < NH; ++h) {
+      const uint32_t vt = st + h * C::CHUNK + C::TILE;
 #pragma unroll
-        for (int w = 0; w < VW / 4; ++w) {
-          const uint4 x = lds_u4(vt + dec_tile_off<D, FP8>(tok, byte0 + 16 * w));
-          vw[ti][4 * w + 0] = x.x;
-          vw[ti][4 * w + 1] = x.y;
-          vw[ti][4 * w + 2] = x.z;
-          vw[ti][4 * w + 3] = x.w;
+      for (int ti = 0; ti < 4; ++ti) {
+        const int tok = 2 * tq + (ti & 1) + 8 * (ti >> 1);
+        const int byte0 = (D * C::E / 8) * g;
+        if constexpr (VW >= 4) {
+#pragma unroll
+          for (int w = 0; w < VW / 4; ++w) {
+            const uint4 x = lds_u4(vt + dec_tile_off<D, FP8>(tok, byte0 + 16 * w));
+            vw[h][ti][4 * w + 0] = x.x;
+            vw[h][ti][4 * w + 1] = x.y;
+            vw[h][ti][4 * w + 2] = x.z;
+            vw[h][ti][4 * w + 3] = x.w;
+          }
+        } else {
+          const uint2 x = lds_u2(vt + dec_tile_off<D, FP8>(tok, byte0));
+          vw[h][ti][0] = x.x;
+          vw[h][ti][1] = x.y;
         }
-      } else {
-        const uint2 x = lds_u2(vt + dec_tile_off<D, FP8>(tok, byte0));
-        vw[ti][0] = x.x;
-        vw[ti][1] = x.y;
-      }
-      if (tok >= n_here) {  // masked tokens must not inject NaN
+        if (tok >= n_here[h]) {  // masked tokens must not inject NaN
 #pragma unroll
-        for (int w = 0; w < VW; ++w) vw[ti][w] = 0u;
+          for (int w = 0; w < VW; ++w) vw[h][ti][w] = 0u;
+        }
       }
     }
     __syncwarp();  // every lane has read the slot; it may be refilled
-    const float a_h0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
-    const float a_h1 = __shfl_sync(0xffffffffu, alpha, (2 * tq + 1) * 4);
+    if (__any_sync(0xffffffffu, alpha != 1.f)) {  // some head row moved its base
+      const float a_h0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
+      const float a_h1 = __shfl_sync(0xffffffffu, alpha, (2 * tq + 1) * 4);
 #pragma unroll
-    for (int mc = 0; mc < D / 16; ++mc) {
-      if (!FP8) {
+      for (int mc = 0; mc < D / 16; ++mc) {
         acc[mc][0] *= a_h0;
         acc[mc][1] *= a_h1;
         acc[mc][2] *= a_h0;
         acc[mc][3] *= a_h1;
-        mma_m16n8k16_bf16(acc[mc], prmt(vw[0][mc], vw[1][mc], 0x5410u),
-                          prmt(vw[0][mc], vw[1][mc], 0x7632u), prmt(vw[2][mc], vw[3][mc], 0x5410u),
-                          prmt(vw[2][mc], vw[3][mc], 0x7632u), pb0, pb1);
-      } else {
-        uint32_t vh[4];
+      }
+    }
 #pragma unroll
-        for (int ti = 0; ti < 4; ++ti) vh[ti] = e4m3x2_to_f16x2(vw[ti][mc >> 1] >> (16 * (mc & 1)));
-        float part[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_m16n8k16_f16(part, prmt(vh[0], vh[1], 0x5410u), prmt(vh[0], vh[1], 0x7632u),
-                         prmt(vh[2], vh[3], 0x5410u), prmt(vh[2], vh[3], 0x7632u), pb0, pb1);
-        acc[mc][0] = fmaf(vsc, part[0], acc[mc][0] * a_h0);
-        acc[mc][1] = fmaf(vsc, part[1], acc[mc][1] * a_h1);
-        acc[mc][2] = fmaf(vsc, part[2], acc[mc][2] * a_h0);
-        acc[mc][3] = fmaf(vsc, part[3], acc[mc][3] * a_h1);
+    for (int mc = 0; mc < D / 16; ++mc) {
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        if (!FP8) {
+          mma_m16n8k16_bf16(acc[mc], prmt(vw[h][0][mc], vw[h][1][mc], 0x5410u),
+                            prmt(vw[h][0][mc], vw[h][1][mc], 0x7632u),
+                            prmt(vw[h][2][mc], vw[h][3][mc], 0x5410u),
+                            prmt(vw[h][2][mc], vw[h][3][mc], 0x7632u), pb[h][0], pb[h][1]);
+        } else {
+          // pair the two tokens of each fragment register byte-wise, then widen:
+          // bytes (tok a, d0), (tok b, d0) -> f16x2 for row d0, likewise d1
+          const int w = mc >> 1;
+          const uint32_t sel_d0 = (mc & 1) ? 0x6262u : 0x4040u;  // d = 2 (mc & 1)
+          const uint32_t sel_d1 = (mc & 1) ? 0x7373u : 0x5151u;  // d = 2 (mc & 1) + 1
+          mma_m16n8k16_f16(acc[mc], e4m3x2_to_f16x2(prmt(vw[h][0][w], vw[h][1][w], sel_d0)),
+                           e4m3x2_to_f16x2(prmt(vw[h][0][w], vw[h][1][w], sel_d1)),
+                           e4m3x2_to_f16x2(prmt(vw[h][2][w], vw[h][3][w], sel_d0)),
+                           e4m3x2_to_f16x2(prmt(vw[h][2][w], vw[h][3][w], sel_d1)), pb[h][0],
+                           pb[h][1]);
+        }
       }
     }
   }
@@ -442,8 +522,8 @@ __global__ void __launch_bounds__(32) attn_decode_split_tma_kernel(
   const int h0 = 2 * tq, h1 = 2 * tq + 1;
   const float l_h0 = __shfl_sync(0xffffffffu, lr_run, h0 * 4);
   const float l_h1 = __shfl_sync(0xffffffffu, lr_run, h1 * 4);
-  const float inv0 = l_h0 > 0.f ? 1.f / l_h0 : 0.f;
-  const float inv1 = l_h1 > 0.f ? 1.f / l_h1 : 0.f;
+  const float inv0 = l_h0 > 0.f ? vmax / l_h0 : 0.f;  // vmax = 1 for a bf16 cache
+  const float inv1 = l_h1 > 0.f ? vmax / l_h1 : 0.f;
   const int dbase = (D / 8) * g;
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {

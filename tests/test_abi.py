@@ -105,6 +105,8 @@ def _dec(lib, q=FAKE, kc=FAKE, vc=FAKE, tbl=FAKE, lens=FAKE, ps=16, B_=2, Hq=8, 
     (dict(ws=None), B.ATTN_ERR_WORKSPACE),
     (dict(ws_bytes=16), B.ATTN_ERR_WORKSPACE),
     (dict(ws=FAKE + 8), B.ATTN_ERR_ALIGNMENT),
+    # 2^21 splits of 512 tokens x 2048 KV heads: more (split, KV head) CTAs than a grid row holds
+    (dict(Hq=4096, Hkv=2048, maxp=1 << 22, ps=256), B.ATTN_ERR_INVALID_ARG),
 ])
 def test_decode_validation(lib, kw, status):
     assert _dec(lib, **kw) == status
