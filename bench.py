@@ -5,15 +5,18 @@
                     [--workload NAME] [--decode-workload NAME] [--no-e2e] [--no-cpu-baseline]
 
 One step = one pass of the whole hot path over one batch of synthetic input:
-  * prefill: attn_fwd on the named prefill workload (default mha_causal_2k:
-    B=4, H=16, S=2048, d=128, causal), and
+  * prefill: attn_fwd on the named prefill workload (default gqa_causal_32k:
+    B=1, Hq=32, Hkv=8, S=32768, d=128, causal), and
   * decode: attn_decode_paged (split kernel + merge kernel) on paged_decode
     (B=64, Hq=32, Hkv=8, d=128, pages of 16, lengths U[512, 8192]).
 Each kernel is timed with CUDA events on the stream it is launched on; L2 is
 flushed (a 256 MiB write) before each timed kernel.  The headline `value` is
 prefill TFLOPS (FLOPs = 4*B*Hq*Sq*Sk*d, halved when causal) over all ranks;
-`decode` reports KV GB/s (K+V bytes of the attended tokens).  Under torchrun
-every rank runs the same per-GPU workload (weak scaling; the work units are
+`decode` reports KV GB/s (K+V bytes of the attended tokens).  Side legs time
+the other prefill workloads, ragged and paged prefill (bf16 and E4M3 caches),
+the FP8 prefill, the backward, the E4M3 decode, the host-buffer call
+(`e2e`) and the CPU oracle's sample, each on its own.  Under torchrun every
+rank runs the same per-GPU workload (weak scaling; the work units are
 independent, so there is no data-path collective) and times are the max over
 ranks.
 
