@@ -89,3 +89,41 @@ def test_repeated_calls_reuse_one_workspace():
     torch.cuda.synchronize()
     for (o, lse), (o_ref, lse_ref) in zip(outs, refs):
         assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+
+
+def test_concurrent_calls_from_two_host_threads():
+    """Two host threads, each with its own stream and workspace, calling at once:
+    the library's copy streams are shared, every result must still be its own."""
+    import threading
+    B, Hq, Hkv, S, d = 2, 8, 2, 384, 128
+    scale = 1.0 / math.sqrt(d)
+    cases = []
+    for seed in (11, 12):
+        q, k, v = W.prefill_inputs(B, Hq, Hkv, S, S, d, seed=seed)
+        cases.append((q.pin_memory(), k.pin_memory(), v.pin_memory()))
+    results = [None, None]
+    errors = []
+
+    def worker(t):
+        try:
+            stream = torch.cuda.Stream(device=DEV)
+            ws = torch.empty(1 << 24, dtype=torch.uint8, device=DEV)
+            outs = []
+            for _ in range(3):
+                outs.append(attn_fwd_host(*cases[t], True, scale, workspace=ws, device=DEV,
+                                          stream=stream))
+            stream.synchronize()
+            results[t] = outs
+        except Exception as e:  # surfaced below
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(t,)) for t in range(2)]
+    for th in threads:
+        th.start()
+    for th in threads:
+        th.join()
+    assert not errors, errors
+    for t in range(2):
+        o_ref, lse_ref = _device_reference(*cases[t], True, scale, None)
+        for o, lse in results[t]:
+            assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
