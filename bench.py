@@ -313,7 +313,7 @@ def config_dict(cfg, dcfg):
 # every row; an int = that many seeded rows (the 32k configuration: the 512
 # (head, row) pairs its parity test checks, timed and extrapolated).
 CPU_SAMPLE_ROWS = {"tiny_mha": None, "mha_causal_2k": None, "gqa_causal_8k": None,
-                   "gqa_causal_8k_padded": None, "gqa_causal_32k": 512}
+                   "gqa_causal_8k_padded": None, "gqa_causal_32k": 24576}
 CPU_SAMPLE_SEED = {"gqa_causal_32k": 41}
 
 
