@@ -32,11 +32,12 @@
 // power of two into f16's range; its fp32 scores are multiplied back and by
 // the page's K scale.  P^T V is an f16 MMA that accumulates straight into the
 // fp32 accumulator: the 16 tokens of a step always lie in one page, so the
-// page's V scale enters as a factor vs / vmax <= 1 on P before P is rounded
-// to f16 (vmax = the largest V scale of the split's pages), and the
-// accumulator, in units of vmax, is multiplied by vmax once at the end.  The
-// normaliser sums the weights as applied to the dequantised V: f16(P') * vmax
-// / vs per token.
+// page's V scale enters as a factor vs / vmax (|.| <= 1, the scale's sign) on
+// P before P is rounded to f16 (vmax = the largest V scale magnitude of the
+// split's pages), and the accumulator, in units of vmax, is multiplied by vmax
+// once at the end.  The normaliser sums the weights as applied to the
+// dequantised V, f16(P') * vmax / vs per token (f16(P) on a page whose scale
+// is zero).
 //
 // Rescaling is lazy, as in the prefill kernel: the exponent base of a head
 // row moves only when the row max exceeds it by more than 8 (log2 units), so
@@ -265,8 +266,8 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
   };
   int n_issued = 0;
   for (; n_issued < C::STAGES - 1 && n_issued < n_steps; ++n_issued) issue(n_issued);
-  // E4M3: the largest V scale of the split's pages (bad pages hold 0)
-  float vmax = FP8 ? my_vs : 1.f;
+  // E4M3: the largest V scale magnitude of the split's pages (bad pages hold 0)
+  float vmax = FP8 ? fabsf(my_vs) : 1.f;
   if (FP8) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
@@ -430,12 +431,19 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
         pb[h][1] = pack_bf16x2(pr[2], pr[3]);
         rr += sum_f32x2(add_f32x2(bf16x2_to_f32x2(pb[h][0]), bf16x2_to_f32x2(pb[h][1])));
       } else {
-        const float rv = vsc[h] * inv_vmax;
+        const float rv = vsc[h] * inv_vmax;  // |rv| <= 1, the sign of the scale
         pb[h][0] = pack_f16x2(pr[0] * rv, pr[1] * rv);
         pb[h][1] = pack_f16x2(pr[2] * rv, pr[3] * rv);
-        const float back = vsc[h] > 0.f ? vmax / vsc[h] : 0.f;  // no token of a bad page
-        rr += ((f16_to_f32(pb[h][0]) + f16_to_f32(pb[h][0] >> 16)) +
-               (f16_to_f32(pb[h][1]) + f16_to_f32(pb[h][1] >> 16))) * back;
+        if (vsc[h] != 0.f) {
+          const float back = vmax / vsc[h];
+          rr += ((f16_to_f32(pb[h][0]) + f16_to_f32(pb[h][0] >> 16)) +
+                 (f16_to_f32(pb[h][1]) + f16_to_f32(pb[h][1] >> 16))) * back;
+        } else {
+          // a zero scale: the page's values add nothing, but its weights still
+          // count in the normaliser (as f16, the rounding of the other pages)
+          const uint32_t w0 = pack_f16x2(pr[0], pr[1]), w1 = pack_f16x2(pr[2], pr[3]);
+          rr += (f16_to_f32(w0) + f16_to_f32(w0 >> 16)) + (f16_to_f32(w1) + f16_to_f32(w1 >> 16));
+        }
       }
     }
     rs += __shfl_xor_sync(0xffffffffu, rs, 1);

@@ -115,3 +115,27 @@ def test_fp8_slots_past_the_length_never_reach_the_result():
     c2 = W.PagedFp8Inputs(c.q, kc, vc, c.k_scale, c.v_scale, c.block_table, c.seq_lens, 16)
     o2, l2 = _run(c2, 0.088)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_fp8_scales_of_any_sign_and_zero():
+    """The schema allows any finite scale: negative K and V scales flip the
+    sign of a page's scores or values, and a zero V scale removes a page's
+    values but not its weights from the softmax.  GPU against the oracle on
+    the same scales, with pages of each kind inside one split and across
+    splits (lengths up to 1300 tokens: three 512-token splits)."""
+    c = W.fp8_paged_inputs(torch.tensor([1300, 97, 530], dtype=torch.int32), 8, 2, 128, 16,
+                           seed=43)
+    scale = 1 / math.sqrt(128)
+    g = torch.Generator().manual_seed(44)
+    ks, vs = c.k_scale.clone(), c.v_scale.clone()
+    flip_k = torch.rand(ks.shape, generator=g) < 0.3
+    flip_v = torch.rand(vs.shape, generator=g) < 0.3
+    zero_v = torch.rand(vs.shape, generator=g) < 0.15
+    ks[flip_k] = -ks[flip_k]
+    vs[flip_v] = -vs[flip_v]
+    vs[zero_v] = 0.0
+    c2 = W.PagedFp8Inputs(c.q, c.k_cache, c.v_cache, ks, vs, c.block_table, c.seq_lens,
+                          c.page_size)
+    o, lse = _run(c2, scale)
+    o_ref, lse_ref = _ref(c2, scale)
+    check(o, o_ref, lse, lse_ref, what="fp8 scales of any sign")
