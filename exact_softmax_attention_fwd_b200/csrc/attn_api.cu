@@ -421,11 +421,21 @@ int decode_paged_common(bool fp8, const void* q, const void* k_cache, const void
     st = fp8 ? launch_decode_split<64, true>(mk, mv, pf, grid_split, stream)
              : launch_decode_split<64, false>(mk, mv, pf, grid_split, stream);
   if (st != ATTN_OK) return st;
-  if (d == 128)
-    attn_decode_merge_kernel<128><<<grid_merge, 128, 0, stream>>>(prm);
-  else
-    attn_decode_merge_kernel<64><<<grid_merge, 128, 0, stream>>>(prm);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  // the merge kernel as a programmatic dependent of the split kernel: its
+  // launch overlaps the split grid's drain, its reads wait for the writes
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid_merge;
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = d == 128 ? cudaLaunchKernelEx(&cfg, attn_decode_merge_kernel<128>, prm)
+                                 : cudaLaunchKernelEx(&cfg, attn_decode_merge_kernel<64>, prm);
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 int check_paged_prefill_args(const void* q, const void* k_cache, const void* v_cache,

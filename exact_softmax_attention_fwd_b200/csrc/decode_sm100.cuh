@@ -15,11 +15,11 @@
 //   S (heads x 16 tokens)  = q (16 padded heads x d) . K^T
 //   O^T (d x heads)       += V^T (d x 16 tokens) . P^T (16 tokens x heads)
 // The contraction index of each MMA may be permuted freely as long as both
-// operands use the same permutation, and an output index may be relabelled
-// if the write-back uses the same labels.  Both are chosen so that every
-// thread reads 16-byte contiguous pieces of K and V rows: for K a thread owns
-// a contiguous quarter of a row, for V a contiguous eighth of four rows.
-// K and V reach the warp through a ring of shared-memory slots filled by
+// operands use the same permutation.  For K a thread owns a contiguous quarter
+// of a row (16-byte loads); V^T's fragments come from transposing fragment
+// loads (ldmatrix .trans) of 16-byte pieces of V rows, and for an E4M3 cache
+// the token order of the scores is permuted to match the byte order those
+// loads deliver.  K and V reach the warp through a ring of shared-memory slots filled by
 // tensor-memory-access copies (see attn_decode_split_tma_kernel), so that the
 // bytes in flight cost no registers.
 //
@@ -48,7 +48,9 @@
 // order: LSE = M + log2 sum_s 2^(lse_s - M), O = sum_s 2^(lse_s - LSE) o_s,
 // giving empty splits (lse = -inf) zero weight; no atomics, so the result is
 // the same on every run.  Partial log-sum-exps are kept in log2 units inside
-// the workspace; the final LSE is converted to the natural log.
+// the workspace; the final LSE is converted to the natural log.  It is launched
+// as a programmatic dependent of the split kernel, so that its launch overlaps
+// the split grid's drain; it waits for the split grid's writes before reading.
 #pragma once
 
 #include "sm100_primitives.cuh"
@@ -77,6 +79,16 @@ struct DecodeFp8Params {
   const float* v_scale;
 };
 
+// Programmatic dependent launch: the merge grid may be launched while the
+// split grid drains; it waits here for the split grid's writes.  Outside such
+// a launch both instructions do nothing.
+__device__ __forceinline__ void decode_wait_prior_grid() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void decode_allow_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ int decode_clamped_len(const DecodeParams& p, int b, bool report) {
   int len = p.seq_lens[b];
   const long long cap = (long long)p.max_pages * p.page_size;
@@ -92,6 +104,14 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
   uint32_t r;
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"((unsigned short)(two & 0xFFFFu)));
   return r;
+}
+
+// Four E4M3 bytes -> two f16x2 (exact): bytes 0-1 -> lo, bytes 2-3 -> hi.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t four, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(four));
 }
 
 __device__ __forceinline__ float f16_to_f32(uint32_t h16) {
@@ -125,8 +145,8 @@ __device__ __forceinline__ void mma_m16n8k16_f16(float (&c)[4], uint32_t a0, uin
 // warps reading the same pages run together.  The K and V rows of each step
 // arrive by tensor-memory-access copies (cp.async.bulk.tensor, no multicast)
 // into a STAGES-deep ring of shared memory, so the bytes in flight cost no
-// registers: lane 0 keeps the next STAGES - 1 steps' copies outstanding while
-// the warp computes.  The cache is read by the copies as the token-major
+// registers: all slots are filled up front, and lane 0 refills a slot with
+// step i + STAGES as soon as the warp has read step i out of it.  The cache is read by the copies as the token-major
 // tensor [num_pages * page_size, Hkv, D] (page p starts at token p *
 // page_size).  A step is NH chunks of 16 tokens (one for bf16 caches, two for
 // E4M3 caches, whose rows are half as long, so that both move about the same
@@ -134,22 +154,24 @@ __device__ __forceinline__ void mma_m16n8k16_f16(float (&c)[4], uint32_t a0, uin
 // 16), so it is one box of 16 rows x (up to) 128 bytes per 128-byte column
 // block, for K and for V.  The boxes land 128-byte swizzled (64-byte for
 // 64-byte rows), which keeps the fragment loads from shared memory free of
-// bank conflicts for K.
+// bank conflicts.
 //
 // Each lane reads one block-table entry (and, for E4M3 caches, one pair of
 // scales) up front: the split has at most 32 chunks, one per lane, and a
 // chunk's page is fetched from its lane by a shuffle.  Tokens past the length
-// and chunks on a page id outside the pool contribute exact zeros (their
-// fragments are zeroed after the shared-memory load, so stale or non-finite
-// slot contents never reach the MMAs); bad ids are flagged.
+// and chunks on a page id outside the pool contribute exact zeros: their
+// scores are set to -inf after the q K^T MMA (a K row only reaches its own
+// score column) and their V fragments are zeroed after the shared-memory load,
+// so stale or non-finite slot contents never reach the output; bad ids are
+// flagged.
 // ---------------------------------------------------------------------------
 template <int D, bool FP8>
 struct DecodeTmaCfg {
   static constexpr int NH = FP8 ? 2 : 1;           // 16-token chunks per step
   // ring depth: the bytes in flight per warp against the warps an SM holds
   // (shared memory per warp grows with the depth).  Measured on paged_decode:
-  // 3 slots of 8 KB for bf16 (2 slots: -2%); 2 slots of 8 KB for E4M3, which
-  // fits 13 warps per SM (3 slots: -4%, 4 slots: -15%)
+  // 3 slots of 8 KB for bf16 (2 slots: -2%); 2 slots of 8 KB for E4M3, 12
+  // warps per SM (3 slots: no gain, 4 slots: -15%)
   static constexpr int STAGES = FP8 ? 2 : 3;
   static constexpr int E = FP8 ? 1 : 2;            // bytes per element
   static constexpr int ROW = D * E;                // bytes per token row of one head
@@ -188,6 +210,24 @@ __device__ __forceinline__ uint2 lds_u2(uint32_t addr) {
   return r;
 }
 
+// Transposing fragment loads from shared memory (16-byte rows, one row
+// address per lane).  m8n8.x4.b16: lanes 8i..8i+7 address the rows of matrix
+// i; register i of lane t holds row t / 4, elements 2 (t % 4) and 2 (t % 4) + 1
+// of the transposed matrix i.  m16n16.x1.b8: lanes 0-15 address rows 0-15;
+// lane t receives rows 4 (t % 4) .. 4 (t % 4) + 3 of column t / 4 (register 0)
+// and of column t / 4 + 8 (register 1), one byte each, in row order.
+__device__ __forceinline__ void ldsm_x4_trans_b16(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_m16n16_trans_b8(uint32_t (&r)[2], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m16n16.x1.trans.shared.b8 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(addr));
+}
+
 template <int D, bool FP8>
 __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -195,8 +235,8 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
   using C = DecodeTmaCfg<D, FP8>;
   constexpr int NH = C::NH;
   constexpr int KW = D * C::E / 16;   // 32-bit words of a thread's K quarter row
-  constexpr int VW = D * C::E / 32;   // 32-bit words of a thread's V eighth row
   const DecodeParams& p = f.d;
+  decode_allow_dependents();  // the merge grid may start filling in as CTAs retire
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
@@ -211,6 +251,26 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
   const int t_end = min(t_begin + kSplitTokens, len);
   const int n_chunks = (t_end - t_begin + 15) / 16;
   const int n_steps = (n_chunks + NH - 1) / NH;
+  const int g = lane >> 2;   // MMA group id: head row of S / P, d-row block of V^T
+  const int tq = lane & 3;   // thread within the group
+  const int hq0 = kvh * p.group;
+
+  // q rows first: their loads need no page and overlap the block-table reads
+  uint32_t qraw[D / 8];
+  if (g < p.group) {
+    const uint16_t* src = p.q + ((size_t)b * p.Hq + hq0 + g) * D + (D / 4) * tq;
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) {
+      const uint4 x = *reinterpret_cast<const uint4*>(src + 8 * w);
+      qraw[4 * w + 0] = x.x;
+      qraw[4 * w + 1] = x.y;
+      qraw[4 * w + 2] = x.z;
+      qraw[4 * w + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int w = 0; w < D / 8; ++w) qraw[w] = 0u;
+  }
 
   // this lane's chunk: its page (or -1 when the id is outside the pool, or
   // past the split) and scales
@@ -265,7 +325,7 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
     }
   };
   int n_issued = 0;
-  for (; n_issued < C::STAGES - 1 && n_issued < n_steps; ++n_issued) issue(n_issued);
+  for (; n_issued < C::STAGES && n_issued < n_steps; ++n_issued) issue(n_issued);
   // E4M3: the largest V scale magnitude of the split's pages (bad pages hold 0)
   float vmax = FP8 ? fabsf(my_vs) : 1.f;
   if (FP8) {
@@ -274,31 +334,18 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
     if (!(vmax > 0.f)) vmax = 1.f;
   }
   const float inv_vmax = FP8 ? 1.f / vmax : 1.f;
-
-  const int g = lane >> 2;   // MMA group id: head row of S / P, d-row block of V^T
-  const int tq = lane & 3;   // thread within the group
-  const int hq0 = kvh * p.group;
+  // E4M3: this lane's chunk's factor on P (|.| <= 1) and the factor that takes
+  // the applied weights back to weights on the dequantised V (0 marks a zero
+  // scale, whose weights count as f16(P))
+  const float my_rv = my_vs * inv_vmax;
+  const float my_back = (FP8 && my_vs != 0.f) ? vmax / my_vs : 0.f;
 
   // q as the A operand (rows = heads, padded to 16; layout as the register
   // kernels).  E4M3 caches: f16 q scaled by 2^-qe into f16's range.
   uint32_t qa[D / 16][2];
   float qscale = 1.f;
   {
-    uint32_t raw[D / 8];
-    if (g < p.group) {
-      const uint16_t* src = p.q + ((size_t)b * p.Hq + hq0 + g) * D + (D / 4) * tq;
-#pragma unroll
-      for (int w = 0; w < D / 32; ++w) {
-        const uint4 x = *reinterpret_cast<const uint4*>(src + 8 * w);
-        raw[4 * w + 0] = x.x;
-        raw[4 * w + 1] = x.y;
-        raw[4 * w + 2] = x.z;
-        raw[4 * w + 3] = x.w;
-      }
-    } else {
-#pragma unroll
-      for (int w = 0; w < D / 8; ++w) raw[w] = 0u;
-    }
+    const uint32_t (&raw)[D / 8] = qraw;
     if (!FP8) {
 #pragma unroll
       for (int w = 0; w < D / 8; ++w) qa[w >> 1][w & 1] = raw[w];
@@ -321,6 +368,7 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
     }
   }
 
+  const float my_kq = my_ks * qscale;  // E4M3: K scale times the power of two on q
   float c2 = p.scale_log2;
   const bool scale_pos = c2 > 0.f;
   if (!scale_pos) c2 = 1.f;
@@ -334,17 +382,17 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
   int i = 0;
 #pragma unroll 1
   for (; i < n_steps; ++i) {
-    if (n_issued < n_steps) issue(n_issued++);  // step i + C::STAGES - 1
     const int slot = i % C::STAGES;
     int n_here[NH];
-    float ksc[NH], vsc[NH];
+    float kqc[NH], rvc[NH], backc[NH];
 #pragma unroll
     for (int h = 0; h < NH; ++h) {
       const int c = NH * i + h;
       const int pg = __shfl_sync(0xffffffffu, my_page, c);
       n_here[h] = pg >= 0 ? min(16, t_end - (t_begin + 16 * c)) : 0;  // <= 0 past the end
-      ksc[h] = FP8 ? __shfl_sync(0xffffffffu, my_ks, c) : 1.f;
-      vsc[h] = FP8 ? __shfl_sync(0xffffffffu, my_vs, c) : 1.f;
+      kqc[h] = FP8 ? __shfl_sync(0xffffffffu, my_kq, c) : 1.f;
+      rvc[h] = FP8 ? __shfl_sync(0xffffffffu, my_rv, c) : 1.f;
+      backc[h] = FP8 ? __shfl_sync(0xffffffffu, my_back, c) : 1.f;
     }
     const uint32_t st = sbase + slot * C::STAGE;
     const bool landed = mbar_wait(bars + 8u * slot, (uint32_t)(i / C::STAGES) & 1u, nullptr);
@@ -358,7 +406,10 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
       const uint32_t kt = st + h * C::CHUNK;
 #pragma unroll
       for (int nc = 0; nc < 2; ++nc) {
-        const int tok = nc * 8 + g;
+        // the token in score column g of this MMA: for an E4M3 cache column 2j +
+        // e of MMA nc is token 4j + 2nc + e, so that lane tq ends up with the
+        // scores of tokens 4tq .. 4tq + 3, the rows its V fragments hold
+        const int tok = FP8 ? 4 * (g >> 1) + 2 * nc + (g & 1) : nc * 8 + g;
         uint32_t kw[KW];
 #pragma unroll
         for (int w = 0; w < KW / 4; ++w) {
@@ -368,10 +419,6 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
           kw[4 * w + 2] = x.z;
           kw[4 * w + 3] = x.w;
         }
-        if (tok >= n_here[h]) {
-#pragma unroll
-          for (int w = 0; w < KW; ++w) kw[w] = 0u;
-        }
         float sx[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         if (!FP8) {
 #pragma unroll
@@ -380,13 +427,13 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
         } else {
 #pragma unroll
           for (int kc = 0; kc < D / 16; ++kc) {
-            const uint32_t w = kw[kc];
-            mma_m16n8k16_f16(sx[kc & 1], qa[kc][0], 0u, qa[kc][1], 0u, e4m3x2_to_f16x2(w),
-                             e4m3x2_to_f16x2(w >> 16));
+            uint32_t k0, k1;
+            e4m3x4_to_f16x2x2(kw[kc], k0, k1);
+            mma_m16n8k16_f16(sx[kc & 1], qa[kc][0], 0u, qa[kc][1], 0u, k0, k1);
           }
         }
         // this thread's scores of head row g: tokens 8nc + 2tq and 8nc + 2tq + 1
-        const float kq = FP8 ? ksc[h] * qscale : 1.f;
+        const float kq = kqc[h];
         s4[h][2 * nc + 0] = (sx[0][0] + sx[1][0]) * kq;
         s4[h][2 * nc + 1] = (sx[0][1] + sx[1][1]) * kq;
       }
@@ -396,11 +443,17 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
     float mx = -INFINITY;
 #pragma unroll
     for (int h = 0; h < NH; ++h) {
+      if (!scale_pos) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int tok = (e >> 1) * 8 + 2 * tq + (e & 1);
-        if (tok >= n_here[h]) s4[h][e] = -INFINITY;
-        else if (!scale_pos) s4[h][e] *= p.scale_log2;
+        for (int e = 0; e < 4; ++e) s4[h][e] *= p.scale_log2;
+      }
+      // tokens past the length or on a bad page: their K rows may hold anything
+      // (only their own score columns see them), masked here
+      if (n_here[h] < 16) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if ((FP8 ? 4 * tq + e : (e >> 1) * 8 + 2 * tq + (e & 1)) >= n_here[h])
+            s4[h][e] = -INFINITY;
       }
       mx = fmaxf(mx, fmaxf(fmaxf(s4[h][0], s4[h][1]), fmaxf(s4[h][2], s4[h][3])));
     }
@@ -431,13 +484,12 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
         pb[h][1] = pack_bf16x2(pr[2], pr[3]);
         rr += sum_f32x2(add_f32x2(bf16x2_to_f32x2(pb[h][0]), bf16x2_to_f32x2(pb[h][1])));
       } else {
-        const float rv = vsc[h] * inv_vmax;  // |rv| <= 1, the sign of the scale
+        const float rv = rvc[h];  // |rv| <= 1, the sign of the scale
         pb[h][0] = pack_f16x2(pr[0] * rv, pr[1] * rv);
         pb[h][1] = pack_f16x2(pr[2] * rv, pr[3] * rv);
-        if (vsc[h] != 0.f) {
-          const float back = vmax / vsc[h];
+        if (backc[h] != 0.f) {
           rr += ((f16_to_f32(pb[h][0]) + f16_to_f32(pb[h][0] >> 16)) +
-                 (f16_to_f32(pb[h][1]) + f16_to_f32(pb[h][1] >> 16))) * back;
+                 (f16_to_f32(pb[h][1]) + f16_to_f32(pb[h][1] >> 16))) * backc[h];
         } else {
           // a zero scale: the page's values add nothing, but its weights still
           // count in the normaliser (as f16, the rounding of the other pages)
@@ -446,44 +498,61 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
         }
       }
     }
-    rs += __shfl_xor_sync(0xffffffffu, rs, 1);
-    rr += __shfl_xor_sync(0xffffffffu, rr, 1);
-    rs += __shfl_xor_sync(0xffffffffu, rs, 2);
-    rr += __shfl_xor_sync(0xffffffffu, rr, 2);
     l_run = l_run * alpha + rs;
     lr_run = lr_run * alpha + rr;
 
-    // ---- O^T += V^T P^T; accumulator columns are heads 2tq and 2tq+1.  V^T
-    // rows d = (D/8)*g + 2*mc (+1), columns = tokens 2tq, 2tq+1, 2tq+8, 2tq+9.
-    uint32_t vw[NH][4][VW > 0 ? VW : 1];
+    // ---- O^T += V^T P^T; accumulator columns are heads 2tq and 2tq+1, rows
+    // d = 16 mc + g and 16 mc + g + 8.  The V^T fragments come from transposing
+    // loads: bf16, the contraction runs over tokens 2tq, 2tq+1 (| +8); E4M3,
+    // over tokens 4tq .. 4tq + 3 in the order of the scores above.
+    uint32_t vw[NH][D / 16][FP8 ? 2 : 4];
 #pragma unroll
     for (int h = 0; h < NH; ++h) {
       const uint32_t vt = st + h * C::CHUNK + C::TILE;
 #pragma unroll
-      for (int ti = 0; ti < 4; ++ti) {
-        const int tok = 2 * tq + (ti & 1) + 8 * (ti >> 1);
-        const int byte0 = (D * C::E / 8) * g;
-        if constexpr (VW >= 4) {
+      for (int mc = 0; mc < D / 16; ++mc) {
+        if constexpr (FP8) {
+          uint32_t r[2];
+          ldsm_m16n16_trans_b8(r, vt + dec_tile_off<D, FP8>(lane & 15, 16 * mc));
+          vw[h][mc][0] = r[0];
+          vw[h][mc][1] = r[1];
+        } else {
+          uint32_t r[4];
+          const int mi = lane >> 3;
+          ldsm_x4_trans_b16(r, vt + dec_tile_off<D, FP8>((lane & 7) + 8 * (mi >> 1),
+                                                         32 * mc + 16 * (mi & 1)));
+          vw[h][mc][0] = r[0];
+          vw[h][mc][1] = r[1];
+          vw[h][mc][2] = r[2];
+          vw[h][mc][3] = r[3];
+        }
+      }
+      if (n_here[h] < 16) {  // masked tokens must not inject NaN
+        if constexpr (FP8) {
+          const int keep = min(max(n_here[h] - 4 * tq, 0), 4);  // bytes = tokens 4tq + b
+          const uint32_t m = keep >= 4 ? 0xFFFFFFFFu : ((1u << (8 * keep)) - 1u);
 #pragma unroll
-          for (int w = 0; w < VW / 4; ++w) {
-            const uint4 x = lds_u4(vt + dec_tile_off<D, FP8>(tok, byte0 + 16 * w));
-            vw[h][ti][4 * w + 0] = x.x;
-            vw[h][ti][4 * w + 1] = x.y;
-            vw[h][ti][4 * w + 2] = x.z;
-            vw[h][ti][4 * w + 3] = x.w;
+          for (int mc = 0; mc < D / 16; ++mc) {
+            vw[h][mc][0] &= m;
+            vw[h][mc][1] &= m;
           }
         } else {
-          const uint2 x = lds_u2(vt + dec_tile_off<D, FP8>(tok, byte0));
-          vw[h][ti][0] = x.x;
-          vw[h][ti][1] = x.y;
-        }
-        if (tok >= n_here[h]) {  // masked tokens must not inject NaN
+          const int t0 = 2 * tq;
+          const uint32_t m_lo = (t0 < n_here[h] ? 0xFFFFu : 0u) | (t0 + 1 < n_here[h] ? 0xFFFF0000u : 0u);
+          const uint32_t m_hi =
+              (t0 + 8 < n_here[h] ? 0xFFFFu : 0u) | (t0 + 9 < n_here[h] ? 0xFFFF0000u : 0u);
 #pragma unroll
-          for (int w = 0; w < VW; ++w) vw[h][ti][w] = 0u;
+          for (int mc = 0; mc < D / 16; ++mc) {
+            vw[h][mc][0] &= m_lo;
+            vw[h][mc][1] &= m_lo;
+            vw[h][mc][2] &= m_hi;
+            vw[h][mc][3] &= m_hi;
+          }
         }
       }
     }
-    __syncwarp();  // every lane has read the slot; it may be refilled
+    __syncwarp();  // every lane has read the slot: refill it with step i + C::STAGES
+    if (n_issued < n_steps) issue(n_issued++);
     if (__any_sync(0xffffffffu, alpha != 1.f)) {  // some head row moved its base
       const float a_h0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
       const float a_h1 = __shfl_sync(0xffffffffu, alpha, (2 * tq + 1) * 4);
@@ -499,22 +568,14 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
     for (int mc = 0; mc < D / 16; ++mc) {
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
-        if (!FP8) {
-          mma_m16n8k16_bf16(acc[mc], prmt(vw[h][0][mc], vw[h][1][mc], 0x5410u),
-                            prmt(vw[h][0][mc], vw[h][1][mc], 0x7632u),
-                            prmt(vw[h][2][mc], vw[h][3][mc], 0x5410u),
-                            prmt(vw[h][2][mc], vw[h][3][mc], 0x7632u), pb[h][0], pb[h][1]);
+        if constexpr (!FP8) {
+          mma_m16n8k16_bf16(acc[mc], vw[h][mc][0], vw[h][mc][1], vw[h][mc][2], vw[h][mc][3],
+                            pb[h][0], pb[h][1]);
         } else {
-          // pair the two tokens of each fragment register byte-wise, then widen:
-          // bytes (tok a, d0), (tok b, d0) -> f16x2 for row d0, likewise d1
-          const int w = mc >> 1;
-          const uint32_t sel_d0 = (mc & 1) ? 0x6262u : 0x4040u;  // d = 2 (mc & 1)
-          const uint32_t sel_d1 = (mc & 1) ? 0x7373u : 0x5151u;  // d = 2 (mc & 1) + 1
-          mma_m16n8k16_f16(acc[mc], e4m3x2_to_f16x2(prmt(vw[h][0][w], vw[h][1][w], sel_d0)),
-                           e4m3x2_to_f16x2(prmt(vw[h][0][w], vw[h][1][w], sel_d1)),
-                           e4m3x2_to_f16x2(prmt(vw[h][2][w], vw[h][3][w], sel_d0)),
-                           e4m3x2_to_f16x2(prmt(vw[h][2][w], vw[h][3][w], sel_d1)), pb[h][0],
-                           pb[h][1]);
+          uint32_t a0, a1, a2, a3;
+          e4m3x4_to_f16x2x2(vw[h][mc][0], a0, a2);
+          e4m3x4_to_f16x2x2(vw[h][mc][1], a1, a3);
+          mma_m16n8k16_f16(acc[mc], a0, a1, a2, a3, pb[h][0], pb[h][1]);
         }
       }
     }
@@ -526,27 +587,27 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
       mbar_wait(bars + 8u * (j % C::STAGES), (uint32_t)(j / C::STAGES) & 1u, nullptr);
   __syncwarp();
 
-  // ---- this split's normalised partial output and its log2-sum-exp
+  // ---- this split's normalised partial output and its log2-sum-exp (the
+  // row sums were kept per lane: every lane of a head row shares its base)
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  lr_run += __shfl_xor_sync(0xffffffffu, lr_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  lr_run += __shfl_xor_sync(0xffffffffu, lr_run, 2);
   const int h0 = 2 * tq, h1 = 2 * tq + 1;
   const float l_h0 = __shfl_sync(0xffffffffu, lr_run, h0 * 4);
   const float l_h1 = __shfl_sync(0xffffffffu, lr_run, h1 * 4);
   const float inv0 = l_h0 > 0.f ? vmax / l_h0 : 0.f;  // vmax = 1 for a bf16 cache
   const float inv1 = l_h1 > 0.f ? vmax / l_h1 : 0.f;
-  const int dbase = (D / 8) * g;
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
     const int h = hh ? h1 : h0;
     if (h >= p.group) continue;
     const float inv = hh ? inv1 : inv0;
-    float* dst = p.o_part + (((size_t)b * p.Hq + hq0 + h) * p.n_split + split) * D + dbase;
+    float* dst = p.o_part + (((size_t)b * p.Hq + hq0 + h) * p.n_split + split) * D + g;
 #pragma unroll
-    for (int mc = 0; mc < D / 16; mc += 2) {
-      float4 w;
-      w.x = acc[mc][hh] * inv;          // d = dbase + 2mc
-      w.y = acc[mc][2 + hh] * inv;      // d = dbase + 2mc + 1
-      w.z = acc[mc + 1][hh] * inv;      // d = dbase + 2mc + 2
-      w.w = acc[mc + 1][2 + hh] * inv;  // d = dbase + 2mc + 3
-      *reinterpret_cast<float4*>(dst + 2 * mc) = w;
+    for (int mc = 0; mc < D / 16; ++mc) {
+      dst[16 * mc] = acc[mc][hh] * inv;
+      dst[16 * mc + 8] = acc[mc][2 + hh] * inv;
     }
   }
   if (tq == 0 && g < p.group) {
@@ -557,6 +618,8 @@ __global__ void __launch_bounds__(32, 8) attn_decode_split_tma_kernel(
 
 template <int D>
 __global__ void __launch_bounds__(128) attn_decode_merge_kernel(const DecodeParams p) {
+  constexpr int PER = D / 32;  // output columns per lane
+  constexpr int R = 16;        // partial rows whose loads are in flight together
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int pair = blockIdx.x * 4 + warp;  // b * Hq + hq
@@ -564,37 +627,68 @@ __global__ void __launch_bounds__(128) attn_decode_merge_kernel(const DecodePara
   const int b = pair / p.Hq;
   const int len = decode_clamped_len(p, b, false);
   const int ns = (len + kSplitTokens - 1) / kSplitTokens;
+  decode_wait_prior_grid();  // the split kernel's partials
   const float* lse_s = p.lse_part + (size_t)pair * p.n_split;
-  float mx = -INFINITY;
-  for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, lse_s[s]);
+  const float* op = p.o_part + (size_t)pair * p.n_split * D + lane * PER;
+  auto load_row = [&](float (&x)[PER], int s) {
+    if constexpr (PER == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(op + (size_t)s * D);
+      x[0] = v.x;
+      x[1 % PER] = v.y;
+      x[2 % PER] = v.z;
+      x[3 % PER] = v.w;
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(op + (size_t)s * D);
+      x[0] = v.x;
+      x[1 % PER] = v.y;
+    }
+  };
+  // the first R rows and the first 32 log-sum-exps in one round trip
+  float x0[R][PER];
+#pragma unroll
+  for (int u = 0; u < R; ++u)
+    if (u < ns) load_row(x0[u], u);
+  const float l0 = lane < ns ? lse_s[lane] : -INFINITY;
+  float mx = l0;
+  for (int s = lane + 32; s < ns; s += 32) mx = fmaxf(mx, lse_s[s]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  constexpr int PER = D / 32;  // output columns per lane
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   float wsum = 0.f;
   if (mx != -INFINITY) {
-    const float* op = p.o_part + (size_t)pair * p.n_split * D + lane * PER;
-    for (int s = 0; s < ns; ++s) {  // fixed order: deterministic
-      const float w = ex2(lse_s[s] - mx);
-      wsum += w;
-      if (PER == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(op + (size_t)s * D);
-        acc[0] += w * x.x;
-        acc[1 % PER] += w * x.y;
-        acc[2 % PER] += w * x.z;
-        acc[3 % PER] += w * x.w;
-      } else {
-        const float2 x = *reinterpret_cast<const float2*>(op + (size_t)s * D);
-        acc[0] += w * x.x;
-        acc[1 % PER] += w * x.y;
+    // rows in fixed order (split 0, 1, ...): deterministic
+    float w_l = ex2(l0 - mx);
+#pragma unroll
+    for (int u = 0; u < R; ++u) {
+      const float w = __shfl_sync(0xffffffffu, w_l, u);
+      if (u < ns) {
+        wsum += w;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] += w * x0[u][e];
+      }
+    }
+    for (int s0 = R; s0 < ns; s0 += R) {
+      if (s0 % 32 == 0) w_l = s0 + lane < ns ? ex2(lse_s[s0 + lane] - mx) : 0.f;
+      float x[R][PER];
+#pragma unroll
+      for (int u = 0; u < R; ++u)
+        if (s0 + u < ns) load_row(x[u], s0 + u);
+#pragma unroll
+      for (int u = 0; u < R; ++u) {
+        const float w = __shfl_sync(0xffffffffu, w_l, (s0 + u) & 31);
+        if (s0 + u < ns) {
+          wsum += w;
+#pragma unroll
+          for (int e = 0; e < PER; ++e) acc[e] += w * x[u][e];
+        }
       }
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   uint16_t* dst = p.o + (size_t)pair * D + lane * PER;
-  if (PER == 4) {
+  if constexpr (PER == 4) {
     uint2 w;
     w.x = pack_bf16x2(acc[0] * inv, acc[1 % PER] * inv);
     w.y = pack_bf16x2(acc[2 % PER] * inv, acc[3 % PER] * inv);
