@@ -348,6 +348,11 @@ size_t attn_decode_workspace_size(int B, int Hq, int max_pages_per_seq, int page
  * [0, max_pages_per_seq * page_size] is clamped and flags
  * ATTN_DEVERR_BAD_LENGTH.  The result is deterministic: the splits are merged
  * in a fixed order with no atomics.
+ * Launches: two kernels on `stream`, the split kernel and the merge kernel;
+ * the merge is launched with programmatic stream serialization, so that it
+ * may start while the split grid drains and waits (griddepcontrol.wait) for
+ * the split grid's writes before it reads them.  Both can be captured into a
+ * CUDA graph.
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA.
  */
 int attn_decode_paged(const void* q, const void* k_cache, const void* v_cache,
