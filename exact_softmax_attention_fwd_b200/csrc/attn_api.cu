@@ -225,7 +225,9 @@ int launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
   if (!set_smem_once(kern, C::SMEM_BYTES, smem_set)) return ATTN_ERR_CUDA;
   // persistent: one CTA per SM (or fewer when there are fewer work units)
   const long long units =
-      VARLEN ? max_units * prm.Hq : (long long)prm.n_qblocks * prm.Hq * prm.B;
+      VARLEN ? max_units * prm.Hq
+      : prm.head_pairs ? (long long)((prm.Sq + 127) / 128) * (prm.Hq / 2) * prm.B
+                       : (long long)prm.n_qblocks * prm.Hq * prm.B;
   const int sms = sm_count();
   if (sms <= 0) return ATTN_ERR_CUDA;
   dim3 grid((unsigned)(units < sms ? units : sms));
@@ -289,6 +291,9 @@ int prefill_dense(const void* q, const void* k, const void* v, void* o, float* l
   prm.group = Hq / Hkv;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.n_qblocks = (Sq + 255) / 256;
+  // windows and block masks: units of 128 rows x two query heads of one KV
+  // head (both tiles stream the same key tiles)
+  prm.head_pairs = (Hq / Hkv) % 2 == 0 && (window > 0 || block_mask != nullptr) ? 1 : 0;
   prm.window = window;
   prm.prefix = prefix;
   prm.block_mask = block_mask;

@@ -8,7 +8,13 @@
 //
 // Persistent organisation: one CTA per SM (384 threads) walks a list of work
 // units.  A unit is two 128-row query tiles of one (batch, query head): rows
-// [256*qb, 256*qb + 256).  Units are ranked heaviest first (largest causal
+// [256*qb, 256*qb + 256).  With a sliding window or a block mask (and an even
+// number of query heads per KV head) a unit is instead one 128-row query
+// tile of two query heads that share a KV head, so that both tiles stream the
+// same key tiles (measured: +8 to +25 % on windows, +9 to +19 % on sparse
+// block masks; on causal masks without them the staggered 256-row units
+// overlap one tile's epilogue with the other's last step and stay faster).
+// Units are ranked heaviest first (largest causal
 // q-block first) and dealt to the CTAs in a back-and-forth ("snake") order so
 // that every SM gets about the same number of KV tiles.  Inside a unit the
 // loop order is query tile outside, KV tiles inside, with the accumulator
@@ -69,6 +75,10 @@ struct PrefillParams {
   int group;            // Hq / Hkv
   float scale_log2;     // scale * log2(e)
   int n_qblocks;        // ceil(Sq / 256)
+  // fixed-length units of 128 query rows x two query heads of one KV head
+  // (Hq / Hkv even) instead of 256 rows x one head: both tiles then see the
+  // same keys and share every K/V tile
+  int head_pairs;
   // programmable masks (causal only; 0 = off): a row at key position p sees
   // keys (p - window, p] (sliding window), or keys below prefix as well (prefix-LM)
   int window, prefix;
@@ -179,6 +189,7 @@ __device__ __forceinline__ bool prefill_block_on(const PrefillParams& p, int b, 
 // One work unit: query rows [256*qb, 256*qb + 256) of head hq in sequence b.
 struct PrefillUnit {
   int qb, hq, b;
+  int hq_t[2];  // query head of each tile (hq, or hq and hq + 1 for head pairs)
   int sq;          // query rows of the sequence
   int klen;        // visible keys of the sequence
   int q_tok0;      // ragged batches: packed index of the sequence's first query
@@ -217,6 +228,15 @@ __device__ __forceinline__ bool prefill_unit(const PrefillParams& p, int k, Pref
       u.k_tok0 = __ldg(p.cu_k + u.b);
       u.klen = __ldg(p.cu_k + u.b + 1) - u.k_tok0;
     }
+  } else if (MASKS && p.head_pairs) {
+    const int n_hp = p.Hq >> 1;
+    const int n_qt = (p.Sq + 127) >> 7;
+    const long long HB = (long long)n_hp * p.B;
+    if (r >= (long long)n_qt * HB) return false;
+    u.qb = n_qt - 1 - (int)(r / HB);  // 128-row query tile
+    const int rem = (int)(r % HB);
+    u.hq = 2 * (rem % n_hp);
+    u.b = rem / n_hp;
   } else {
     const long long HB = (long long)p.Hq * p.B;
     if (r >= (long long)p.n_qblocks * HB) return false;
@@ -224,6 +244,8 @@ __device__ __forceinline__ bool prefill_unit(const PrefillParams& p, int k, Pref
     const int rem = (int)(r % HB);
     u.hq = rem % p.Hq;
     u.b = rem / p.Hq;
+  }
+  if (!VARLEN) {
     int klen = p.Sk;
     if (p.k_lens != nullptr) {
       klen = p.k_lens[u.b];
@@ -234,19 +256,21 @@ __device__ __forceinline__ bool prefill_unit(const PrefillParams& p, int k, Pref
     u.q_tok0 = 0;
     u.k_tok0 = 0;
   }
+  const bool pairs = MASKS && !VARLEN && p.head_pairs;
   u.kv_first = INT_MAX;
   u.kv_last = 0;
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    u.row0[i] = u.qb * 256 + i * 128;
+    u.hq_t[i] = pairs ? u.hq + i : u.hq;
+    u.row0[i] = pairs ? u.qb * 128 : u.qb * 256 + i * 128;
     prefill_kv_range(u.row0[i], u.sq, u.klen, CAUSAL, MASKS ? p.window : 0,
                      MASKS ? p.prefix : 0, u.kv_begin[i], u.kv_end[i]);
     if (MASKS && p.block_mask != nullptr) {
       // tighten the range to its first and last computed block, so that a
       // tile with no block left has an empty range (and no Q load)
       int lo = u.kv_begin[i], hi = u.kv_end[i];
-      while (lo < hi && !prefill_block_on(p, u.b, u.hq, u.row0[i], lo, hi, lo)) ++lo;
-      while (hi > lo && !prefill_block_on(p, u.b, u.hq, u.row0[i], lo, hi, hi - 1)) --hi;
+      while (lo < hi && !prefill_block_on(p, u.b, u.hq_t[i], u.row0[i], lo, hi, lo)) ++lo;
+      while (hi > lo && !prefill_block_on(p, u.b, u.hq_t[i], u.row0[i], lo, hi, hi - 1)) --hi;
       u.kv_begin[i] = lo < hi ? lo : 0;
       u.kv_end[i] = lo < hi ? hi : 0;
     }
@@ -340,7 +364,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int cb = 0; cb < C::NCB; ++cb)
           tma_load_3d(sbase + C::OFF_Q + i * C::TILE_BYTES + cb * C::CB_BYTES, &tm_q,
                       bar(C::B_QFULL + i), 64 * cb, VARLEN ? u.hq : u.row0[i],
-                      VARLEN ? u.q_tok0 + u.row0[i] : u.b * p.Hq + u.hq);
+                      VARLEN ? u.q_tok0 + u.row0[i] : u.b * p.Hq + u.hq_t[i]);
         ++n;
         return true;
       };
@@ -360,8 +384,8 @@ __global__ void __launch_bounds__(384, 1)
         for (int j = u.kv_first; j < u.kv_last; ++j) {
           // with a block mask, key tiles no query tile of the unit computes are not streamed
           if (MASKS && p.block_mask != nullptr &&
-              !prefill_block_on(p, u.b, u.hq, u.row0[0], u.kv_begin[0], u.kv_end[0], j) &&
-              !prefill_block_on(p, u.b, u.hq, u.row0[1], u.kv_begin[1], u.kv_end[1], j))
+              !prefill_block_on(p, u.b, u.hq_t[0], u.row0[0], u.kv_begin[0], u.kv_end[0], j) &&
+              !prefill_block_on(p, u.b, u.hq_t[1], u.row0[1], u.kv_begin[1], u.kv_end[1], j))
             continue;
           const int s = kv % C::STAGES;
           const uint32_t ph = (kv / C::STAGES) & 1u;
@@ -517,7 +541,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (MASKS && p.block_mask != nullptr) {
           auto on = [&](int i, int kb) {
-            return prefill_block_on(p, u.b, u.hq, u.row0[i], u.kv_begin[i], u.kv_end[i], kb);
+            return prefill_block_on(p, u.b, u.hq_t[i], u.row0[i], u.kv_begin[i], u.kv_end[i], kb);
           };
           auto next_pos = [&](int kb) {
             for (int x = kb + 1; x < je; ++x)
@@ -667,7 +691,8 @@ __global__ void __launch_bounds__(384, 1)
       const int kb = i ? u.kv_begin[1] : u.kv_begin[0];  // this tile's KV tiles [kb, ke)
       const int ke = i ? u.kv_end[1] : u.kv_end[0];
       const int row = row0 + r;
-      const int q_head_row = u.b * p.Hq + u.hq;
+      const int hq_i = i ? u.hq_t[1] : u.hq_t[0];
+      const int q_head_row = u.b * p.Hq + hq_i;
       if (!VARLEN && p.k_lens != nullptr && r == 0) {
         const int kl = p.k_lens[u.b];
         if (kl < 0 || kl > p.Sk) flag_device_error(kDevErrBadLength);
@@ -693,7 +718,7 @@ __global__ void __launch_bounds__(384, 1)
       float lr_run = 0.f;        // sum of bf16(P)
 
       for (int j = kb; j < ke; ++j) {
-        if (MASKS && p.block_mask != nullptr && !prefill_block_on(p, u.b, u.hq, row0, kb, ke, j))
+        if (MASKS && p.block_mask != nullptr && !prefill_block_on(p, u.b, hq_i, row0, kb, ke, j))
           continue;  // a block the mask switches off: no S, no P for it
         if (!(ok = mbar_wait_warp(bar(C::B_SFULL + i), s_waits & 1u, abort_flag))) break;
         ++s_waits;
