@@ -334,7 +334,19 @@ int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mdo, const CUtensorMap&
   auto dq = attn_bwd_dq_kernel<D, CAUSAL, VARLEN, MASKS>;
   static std::atomic<unsigned long long> q_smem_set{0};
   if (!set_smem_once(dq, C::Q_SMEM, q_smem_set)) return ATTN_ERR_CUDA;
-  dq<<<(unsigned)q_units, C::NUM_THREADS, C::Q_SMEM, stream>>>(mq, mdo, mk, mv, prm);
+  // dQ as a programmatic dependent of dK/dV (it reads only the inputs and the
+  // prep kernel's statistics, complete before dK/dV started)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)q_units);
+  cfg.blockDim = dim3(C::NUM_THREADS);
+  cfg.dynamicSmemBytes = C::Q_SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, dq, mq, mdo, mk, mv, prm) != cudaSuccess) return ATTN_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

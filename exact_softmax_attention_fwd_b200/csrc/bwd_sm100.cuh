@@ -288,6 +288,10 @@ __global__ void __launch_bounds__(384, 1)
                          const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const BwdParams p) {
   using C = BwdCfg<D>;
+  // the dQ grid does not read what this grid writes: it may be launched as
+  // soon as every CTA here has started, and fill the SMs this grid's tail
+  // leaves idle
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
@@ -829,6 +833,10 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after_sync();
   if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+  // launched as a programmatic dependent of the dK/dV grid: this grid does
+  // not complete before that one has, so work after the backward in the
+  // stream sees dK and dV as well
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace attn_b200

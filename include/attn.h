@@ -469,6 +469,9 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Sq);
  *   ignored and it must not be shared with a concurrent call.
  *   Deterministic: every output element is written by one CTA in a fixed
  *   order (no atomics), so repeated calls give identical bits.
+ *   Launches: three kernels on `stream` (row statistics, dK/dV, dQ); dQ is
+ *   launched as a programmatic dependent of dK/dV, whose outputs it does not
+ *   read, and does not complete before dK/dV has.
  * Errors: as attn_fwd_masked, plus INVALID_ARG for a NULL o, lse, d_o, dq or
  * workspace (dk, dv when Sk > 0), ALIGNMENT (o, d_o, dq, dk, dv, workspace
  * need 16 bytes, lse 4), WORKSPACE when workspace_bytes is too small.  Sk = 0

@@ -3,7 +3,8 @@
 The C ABI allocates nothing per call and never synchronises a stream in a
 launch, so its calls can be captured into a CUDA graph and replayed; the
 decode merge kernel is launched as a programmatic dependent of the split
-kernel, which a graph has to keep as such.  Each case runs a call eagerly,
+kernel, and the backward's dQ kernel as one of its dK/dV kernel, which a
+graph has to keep as such.  Each case runs a call eagerly,
 captures the same call (same buffers) into a graph, replays it and expects
 the eager bits; then it rewrites the inputs in place (new values, shorter
 lengths) and expects the replay to match an eager call on the new inputs.
@@ -13,7 +14,8 @@ import math
 import pytest
 import torch
 
-from exact_softmax_attention_fwd_b200 import (attn_decode_paged, attn_decode_paged_fp8,
+from exact_softmax_attention_fwd_b200 import (attn_bwd, attn_bwd_workspace_size,
+                                             attn_decode_paged, attn_decode_paged_fp8,
                                              attn_decode_workspace_size, attn_fwd_masked,
                                              attn_fwd_varlen, attn_fwd_varlen_workspace_size,
                                              attn_get_device_error)
@@ -145,3 +147,34 @@ def test_ragged_prefill_replay_matches_eager():
     torch.cuda.synchronize()
     _device_ok()
     assert torch.equal(o, o_ref) and _equal(lse, lse_ref)
+
+
+def test_backward_replay_matches_eager():
+    B, Hq, Hkv, S, d = 2, 8, 2, 700, 128
+    scale = 1.0 / math.sqrt(d)
+    q, k, v = (t.to(DEV) for t in W.prefill_inputs(B, Hq, Hkv, S, S, d, seed=31, value_scale=0.5))
+    d_o = W.grad_output(B, Hq, S, d, seed=32, value_scale=0.5).to(DEV)
+    o, lse = attn_fwd_masked(q, k, v, True, scale)
+    ws = torch.empty(attn_bwd_workspace_size(B, Hq, S), dtype=torch.uint8, device=DEV)
+    grads = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
+
+    def call(g=grads):
+        attn_bwd(q, k, v, o, lse, d_o, True, scale, dq=g[0], dk=g[1], dv=g[2], workspace=ws)
+
+    ref = [torch.empty_like(x) for x in grads]
+    call(ref)
+    graph = _capture(call)
+    for x in grads:
+        x.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    _device_ok()
+    for x, y in zip(grads, ref):
+        assert torch.equal(x, y)
+    d_o.mul_(-2.0)
+    graph.replay()
+    call(ref)
+    torch.cuda.synchronize()
+    _device_ok()
+    for x, y in zip(grads, ref):
+        assert torch.equal(x, y)
