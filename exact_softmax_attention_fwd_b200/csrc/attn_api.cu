@@ -314,7 +314,8 @@ int prefill_dense(const void* q, const void* k, const void* v, void* o, float* l
                 : launch_prefill<64, false>(mq, mk, mv, mo, prm, stream);
 }
 // Backward: the row-statistics pass, then dK/dV (one CTA per key tile and KV
-// head) and dQ (one CTA per query tile and query head), in stream order.
+// head), then dQ (one CTA per query tile and query head) as a programmatic
+// dependent of dK/dV.
 template <int D, bool CAUSAL, bool VARLEN = false, bool MASKS = false>
 int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mdo, const CUtensorMap& mk,
                const CUtensorMap& mv, const BwdParams& prm, cudaStream_t stream) {
