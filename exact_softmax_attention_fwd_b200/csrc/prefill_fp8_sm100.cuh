@@ -16,12 +16,17 @@
 //     codes is exact in fp32 up to accumulation order; the two block scales
 //     are one fp32 factor per (query tile, key tile), folded into the exponent
 //     multiplier of the softmax.
-//   * P V stays a bf16 MMA (kind::f16, P from tensor memory) so that P keeps
-//     bf16's precision: two warps widen each E4M3 V tile into a bf16 copy in
-//     shared memory (E4M3 values are exact in bf16) in the layout the MMA
-//     reads.  The V tile's scale is folded into the weights before they are
-//     rounded: P' = 2^(x + log2 v_scale), and the row sums are divided by
-//     v_scale again, so O = sum P' v_code / sum P' / v_scale.
+//   * P V is an f16 MMA (kind::f16, P from tensor memory), so that the weights
+//     keep 11 bits of precision: two warps widen each E4M3 V tile into an f16
+//     copy in shared memory (E4M3 values are exact in f16; one conversion per
+//     pair of codes) in the layout the MMA reads.  The V tile's scale enters
+//     the weights before they are rounded, relative to the largest V scale of
+//     the query tile's key range (vmax), which keeps them within f16's range:
+//     P' = 2^(x + log2(v_scale / vmax)) <= 2^8.  O accumulates in units of
+//     vmax and is normalised by the unrounded row sum of P (f16 rounds P' to
+//     2^-11 relative, below the forward's tolerance, and a V block whose scale
+//     is far below vmax -- whose weights underflow f16 -- still counts with its
+//     full weight): O = vmax * sum f16(P') v_code / sum P.
 //   * warp 0: TMA producer (E4M3 Q, K, V tiles; no multicast); warp 1: MMA
 //     issuer (elect.sync); warps 2-3: V widening; warps 4-11: two softmax
 //     warpgroups, one per query tile, thread = row = TMEM lane.
@@ -44,8 +49,8 @@ struct PrefillFp8Cfg {
   static constexpr int D = 128;
   static constexpr int STAGES = 2;
   static constexpr int T8 = 128 * 128;           // a 128-row E4M3 tile (Q, K or V)
-  static constexpr int VB = 128 * D * 2;         // a widened bf16 V tile
-  static constexpr int CB_BYTES = 128 * 128;     // one 64-column block of the bf16 tile
+  static constexpr int VB = 128 * D * 2;         // a widened f16 V tile
+  static constexpr int CB_BYTES = 128 * 128;     // one 64-column block of the f16 tile
   static constexpr int STG_BYTES = 32 * 128;     // per-warp epilogue staging
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * T8;
@@ -59,8 +64,8 @@ struct PrefillFp8Cfg {
   static constexpr int B_KEMPTY = B_KFULL + STAGES;
   static constexpr int B_VFULL = B_KEMPTY + STAGES;  // E4M3 V landed
   static constexpr int B_VEMPTY = B_VFULL + STAGES;  // E4M3 V widened (64 arrivals)
-  static constexpr int B_CFULL = B_VEMPTY + STAGES;  // bf16 V ready (64 arrivals)
-  static constexpr int B_CEMPTY = B_CFULL + STAGES;  // bf16 V read by its P V
+  static constexpr int B_CFULL = B_VEMPTY + STAGES;  // f16 V ready (64 arrivals)
+  static constexpr int B_CEMPTY = B_CFULL + STAGES;  // f16 V read by its P V
   static constexpr int B_SFULL = B_CEMPTY + STAGES;  // 2
   static constexpr int B_PFULL = B_SFULL + 2;        // 2
   static constexpr int B_OFULL = B_PFULL + 2;        // 2
@@ -95,15 +100,26 @@ __device__ __forceinline__ void umma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uin
       : "memory");
 }
 
-// Two E4M3 codes (bits 0-7, 8-15) -> bf16x2, exactly (via f16 and f32).
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two) {
-  uint32_t h;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((unsigned short)(two & 0xFFFFu)));
-  float lo, hi;
-  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
-      : "=f"(lo), "=f"(hi)
-      : "r"(h));
-  return pack_bf16x2(lo, hi);
+// Four E4M3 codes -> two f16x2 (exact: E4M3 values are f16 values), codes 0-1
+// -> lo, 2-3 -> hi.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2_v(uint32_t four, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(four));
+}
+
+// Two floats -> packed f16x2 (round to nearest even); `lo` lands in bits 0-15.
+__device__ __forceinline__ uint32_t pack_f16x2_p(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Instruction descriptor of a kind::f16 MMA on f16 A and B, f32 accumulate.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_major) {
+  return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 template <bool CAUSAL>
@@ -213,7 +229,7 @@ __global__ void __launch_bounds__(384, 1)
     } else if (warp == 1) {
       // ======================= tcgen05 MMA issuer =======================
       constexpr uint32_t idesc_qk = idesc_e4m3_f32(128, 128);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+      constexpr uint32_t idesc_pv = idesc_f16_f32(128, D, true);
       auto wait = [&](uint32_t b, uint32_t ph) -> bool {
         if (__all_sync(0xffffffffu, mbar_test(b, ph))) return true;
         const bool r = mbar_wait_slow(b, ph, abort_flag);
@@ -229,7 +245,7 @@ __global__ void __launch_bounds__(384, 1)
           umma_ss_f8(dt, qd + (uint64_t)((ks * 32) >> 4), kd + (uint64_t)((ks * 32) >> 4), idesc_qk,
                      ks > 0 ? 1u : 0u);
       };
-      // O_i (+)= P_i V over the widened bf16 V tile (as the bf16 kernel)
+      // O_i (+)= P_i V over the widened f16 V tile
       auto issue_pv = [&](int i, int stage, bool accumulate) {
         const uint64_t vd =
             smem_desc_sw128(opaque_u32(sbase + C::OFF_VB + stage * C::VB), C::CB_BYTES, 1024);
@@ -273,7 +289,7 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t idx = kv + (uint32_t)(j - jb);
           const int s = idx % C::STAGES;
           const int s1 = (idx + 1) % C::STAGES;
-          // the widened bf16 copy of V_j (not the E4M3 tile) feeds P V
+          // the widened f16 copy of V_j (not the E4M3 tile) feeds P V
           if (!(ok = wait(bar(C::B_CFULL + s), (idx / C::STAGES) & 1u))) break;
           bool k_next = false;
 #pragma unroll
@@ -318,7 +334,7 @@ __global__ void __launch_bounds__(384, 1)
     } else {
       // ======================= V widening (warps 2-3) =======================
       // Each K/V step's E4M3 V tile (128 keys x 128 bytes, 128-byte swizzled
-      // as TMA lands it) becomes a bf16 tile in the MN-major layout the P V
+      // as TMA lands it) becomes an f16 tile in the MN-major layout the P V
       // MMA reads: two 64-column blocks of 128 rows x 128 bytes, 128-byte
       // swizzled.  Thread t handles 16-code chunks t, t + 64, ... (8 chunks
       // per key row).
@@ -342,15 +358,11 @@ __global__ void __launch_bounds__(384, 1)
             asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
                          : "r"(src + row * 128 + (((cc ^ (row & 7)) & 7) << 4)));
-            uint4 lo, hi;  // codes 0-7 and 8-15 of the chunk as bf16
-            lo.x = e4m3x2_to_bf16x2(x.x);
-            lo.y = e4m3x2_to_bf16x2(x.x >> 16);
-            lo.z = e4m3x2_to_bf16x2(x.y);
-            lo.w = e4m3x2_to_bf16x2(x.y >> 16);
-            hi.x = e4m3x2_to_bf16x2(x.z);
-            hi.y = e4m3x2_to_bf16x2(x.z >> 16);
-            hi.z = e4m3x2_to_bf16x2(x.w);
-            hi.w = e4m3x2_to_bf16x2(x.w >> 16);
+            uint4 lo, hi;  // codes 0-7 and 8-15 of the chunk as f16
+            e4m3x4_to_f16x2x2_v(x.x, lo.x, lo.y);
+            e4m3x4_to_f16x2x2_v(x.y, lo.z, lo.w);
+            e4m3x4_to_f16x2x2_v(x.z, hi.x, hi.y);
+            e4m3x4_to_f16x2x2_v(x.w, hi.z, hi.w);
             // dims 16cc .. 16cc+15: block cc/4, 16-byte chunks 2(cc%4) and 2(cc%4)+1
             const int blk = cc >> 2, q0 = (cc & 3) * 2;
             uint8_t* rowp = dst + blk * C::CB_BYTES + row * 128;
@@ -399,9 +411,16 @@ __global__ void __launch_bounds__(384, 1)
       }
       // the query tile's block scale (scale_log2 carries the softmax scale)
       const float qsl = p.scale_log2 * __ldg(f.q_scale + (size_t)q_head_row * p.n_qt + row0 / 128);
+      // the largest V block scale of this tile's key range: P' = P v_scale / vmax
+      // <= 2^8 stays in f16's range, and O accumulates in units of vmax
+      float vmax = 1e-30f;
+      for (int jj = kb + lane; jj < ke; jj += 32)
+        vmax = fmaxf(vmax, __ldg(f.v_scale + (size_t)kv_head_row * p.n_kt + jj));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+      if (!(vmax < INFINITY)) vmax = 1e30f;
       float m_run = -INFINITY;
-      float l_run = 0.f;   // sum of P (f32): the LSE
-      float lr_run = 0.f;  // sum of bf16(P'), P' = P * v_scale, divided by v_scale per step
+      float l_run = 0.f;   // sum of P (f32): the LSE and the normaliser of O
 
       for (int j = kb; j < ke; ++j) {
         const float ksc = __ldg(f.k_scale + (size_t)kv_head_row * p.n_kt + j);
@@ -460,12 +479,12 @@ __global__ void __launch_bounds__(384, 1)
           m_run = m_tile;
         }
         const float base = (m_run == -INFINITY) ? 0.f : m_run;
-        // P' = 2^(s*c2 - base + log2 v_scale) = P * v_scale
-        const float nb = lg2(vsc) - base;
+        // P' = 2^(s*c2 - base + log2(v_scale / vmax)) = P * v_scale / vmax
+        const float vrel = fminf(vsc, vmax) / vmax;
+        const float nb = lg2(vrel) - base;
         const uint64_t c2x2 = f32x2(c2, c2);
         const uint64_t nbx2 = f32x2(nb, nb);
         uint64_t la = 0ull, lb = 0ull;
-        float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
@@ -476,18 +495,15 @@ __global__ void __launch_bounds__(384, 1)
             split_f32x2(fma_f32x2(f32x2(s[cc], s[cc + 1]), c2x2, nbx2), x0, x1);
             split_f32x2(fma_f32x2(f32x2(s[cc + 2], s[cc + 3]), c2x2, nbx2), x2, x3);
             const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
-            pk[e] = pack_bf16x2(p0, p1);
-            pk[e + 1] = pack_bf16x2(p2, p3);
+            pk[e] = pack_f16x2_p(p0, p1);
+            pk[e + 1] = pack_f16x2_p(p2, p3);
             la = add_f32x2(la, f32x2(p0, p1));
             lb = add_f32x2(lb, f32x2(p2, p3));
-            add_bf16x2_halves(pk[e], r0, r1);
-            add_bf16x2_halves(pk[e + 1], r2, r3);
           }
           tmem_st32(t_s + 32 * half, pk);
         }
-        const float inv_vs = 1.f / vsc;
+        const float inv_vs = 1.f / vrel;
         l_run = l_run * alpha + (sum_f32x2(la) + sum_f32x2(lb)) * inv_vs;
-        lr_run = lr_run * alpha + ((r0 + r1) + (r2 + r3)) * inv_vs;
         if (j > kb && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
           for (int c = 0; c < D; c += 32) {
@@ -511,7 +527,10 @@ __global__ void __launch_bounds__(384, 1)
         ++o_waits;
       }
       tc_fence_after_sync();
-      const float inv = (lr_run > 0.f) ? (1.f / lr_run) : 0.f;
+      // O in units of vmax, normalised by the unrounded weights: f16 rounds P'
+      // to 2^-11 relative, and a V block whose scale is far below vmax (a zero
+      // block) still counts with its full weight
+      const float o_mul = (l_run > 0.f) ? vmax / l_run : 0.f;
       const bool warp_has_rows = row0 + quarter * 32 < p.Sq;
 #pragma unroll 1
       for (int cb = 0; cb < D / 64; ++cb) {
@@ -533,10 +552,10 @@ __global__ void __launch_bounds__(384, 1)
           for (int q4 = 0; q4 < 4; ++q4) {
             const int chunk = 4 * half + q4;
             uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * inv, __uint_as_float(v[8 * q4 + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv, __uint_as_float(v[8 * q4 + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv, __uint_as_float(v[8 * q4 + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv, __uint_as_float(v[8 * q4 + 7]) * inv);
+            w.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * o_mul, __uint_as_float(v[8 * q4 + 1]) * o_mul);
+            w.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * o_mul, __uint_as_float(v[8 * q4 + 3]) * o_mul);
+            w.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * o_mul, __uint_as_float(v[8 * q4 + 5]) * o_mul);
+            w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * o_mul, __uint_as_float(v[8 * q4 + 7]) * o_mul);
             *reinterpret_cast<uint4*>(stg_ptr + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = w;
           }
         }

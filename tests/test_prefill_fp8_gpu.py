@@ -7,8 +7,9 @@ with scale = amax / 448 (``workloads.quantize_e4m3_blocks``); the CUDA path
 gets the codes and scales, the float64 oracle (``oracle/kv_fp8.py``,
 ``attn_fwd_fp8``) the same bytes, dequantised from the format's definition.
 The comparison uses the forward's bar (``tests/parity.py``): the kernel's
-score products of E4M3 codes are exact, V is widened exactly, and the
-weights are rounded to bf16 as in the bf16 kernel.
+score products of E4M3 codes are exact, V is widened exactly (to f16), and
+the weights, scaled by each V block's scale over the largest one, are rounded
+to f16 for the P.V product.
 """
 import math
 
@@ -88,3 +89,18 @@ def test_fp8_prefill_deterministic():
     a = _run(*x, True, 0.088)
     b = _run(*x, True, 0.088)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_fp8_prefill_v_block_scales_far_apart():
+    """V block scales twelve orders of magnitude apart, and one of zero: such a
+    block's weights underflow f16 in the P.V product, but they still count in
+    the normaliser (its values are ~0, its attention mass is not)."""
+    B, Hq, Hkv, S = 1, 4, 2, 600
+    q8, k8, v8, qs, ks, vs = W.fp8_prefill_inputs(B, Hq, Hkv, S, S, 128, seed=311)
+    vs = vs.clone()
+    vs[:, :, 1] = 1e-12
+    vs[:, 0, 3] = 0.0
+    for causal in (True, False):
+        o, lse = _run(q8, k8, v8, qs, ks, vs, causal, 0.088)
+        o_ref, lse_ref = oracle_fp8(q8, k8, v8, qs, ks, vs, causal, 0.088)
+        check(o, o_ref, lse, lse_ref, what=f"fp8 V scales far apart causal={causal}")
