@@ -221,8 +221,9 @@ int launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
   using C = PrefillCfg<D>;
   constexpr bool VARLEN = LAYOUT != kLayoutDense;
   auto kern = attn_prefill_sm100_kernel<D, CAUSAL, LAYOUT, MASKS>;
+  constexpr int smem = MASKS ? C::SMEM_BYTES_MASKS : C::SMEM_BYTES;
   static std::atomic<unsigned long long> smem_set{0};
-  if (!set_smem_once(kern, C::SMEM_BYTES, smem_set)) return ATTN_ERR_CUDA;
+  if (!set_smem_once(kern, smem, smem_set)) return ATTN_ERR_CUDA;
   // persistent: one CTA per SM (or fewer when there are fewer work units)
   const long long units =
       VARLEN ? max_units * prm.Hq
@@ -231,7 +232,7 @@ int launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
   const int sms = sm_count();
   if (sms <= 0) return ATTN_ERR_CUDA;
   dim3 grid((unsigned)(units < sms ? units : sms));
-  kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, prm);
+  kern<<<grid, C::NUM_THREADS, smem, stream>>>(mq, mk, mv, mo, prm);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -300,6 +301,10 @@ int prefill_dense(const void* q, const void* k, const void* v, void* o, float* l
   prm.mask_heads = mask_heads;
   prm.n_qt = (Sq + 127) / 128;
   prm.n_kt = (Sk + 127) / 128;
+  // a block mask shared by the heads: units ranked by their visible blocks
+  const long long sched_rows = (long long)B * (prm.head_pairs ? prm.n_qt : prm.n_qblocks);
+  if (block_mask != nullptr && mask_heads == 1 && sched_rows <= kPrefillSchedMax)
+    prm.sched_rows = (int)sched_rows;
   if (window > 0 || prefix > 0 || block_mask != nullptr) {  // window / prefix need causal
     if (d == 128)
       return causal ? launch_prefill<128, true, kLayoutDense, true>(mq, mk, mv, mo, prm, stream)

@@ -86,6 +86,10 @@ struct PrefillParams {
   // n_qt, n_kt] over 128 x 128 (query tile, key tile) blocks, 0 = skipped
   const uint8_t* block_mask;
   int mask_heads, n_qt, n_kt;
+  // block masks shared by the heads: the unit rows (sequence, query block) are
+  // ranked by their visible blocks in each CTA's prologue; the row count, or 0
+  // to keep the causal ranking (see prefill_unit)
+  int sched_rows;
   // ragged batches: packed token-major tensors, cumulative sequence lengths
   // and the unit list written by attn_varlen_schedule_kernel
   uint16_t* o;          // [total_q, Hq, d] bf16
@@ -99,6 +103,10 @@ struct PrefillParams {
   const int* unit_count;
   int total_q;
 };
+
+// Most unit rows (sequence, query block) a block-mask launch ranks in shared
+// memory; larger launches keep the causal ranking.
+constexpr int kPrefillSchedMax = 768;
 
 template <int D>
 struct PrefillCfg {
@@ -128,6 +136,9 @@ struct PrefillCfg {
   static constexpr int NUM_BARS = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem base, abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + runtime 1024-B alignment
+  // masked instantiations: + the ranked block-mask unit rows (uint16)
+  static constexpr int OFF_SCHED = OFF_MISC + 16;
+  static constexpr int SMEM_BYTES_MASKS = SMEM_BYTES + 2 * kPrefillSchedMax;
   static constexpr uint32_t TMEM_COLS = 512;
   // TMEM columns of S_i (P_i aliases its first 64) and of O_i
   __host__ __device__ static constexpr uint32_t tmem_s(int i) { return i ? 128u : 0u; }
@@ -141,7 +152,7 @@ struct PrefillCfg {
   static_assert(128 * ((REGS_PRODUCER + 16) + 2 * (REGS_SOFTMAX - 16)) <= NUM_THREADS * REGS_LAUNCH,
                 "the masked split must fit too");
   static_assert(D == 64 || D == 128, "head dim");
-  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static_assert(SMEM_BYTES_MASKS <= 232448, "shared memory");
 };
 
 // Tensor layouts of a prefill kernel instantiation: dense [B, H, S, d]; a
@@ -204,11 +215,15 @@ struct PrefillUnit {
 // The k-th unit of this CTA, or false when the CTA has no more work.  Ranks
 // are ordered heaviest first (q-blocks descending, heads inner) and dealt
 // back and forth across the CTAs: rank k*G + c for even k, k*G + G-1-c for odd.
-// For a ragged batch the (sequence, q-block) order comes from the unit list.
+// For a ragged batch the (sequence, q-block) order comes from the unit list;
+// for a block mask shared by the heads (p.sched_rows > 0) from `sched`, the
+// rows (b, query block) sorted by visible blocks in the prologue, heads inner
+// -- the random cost of such rows makes the causal ranking a poor proxy.
 // MASKS: the instantiation honours p.window / p.prefix; without it both are
 // the constant 0, so every range starts at tile 0 and the extra bounds fold away.
 template <bool CAUSAL, int LAYOUT, bool MASKS>
-__device__ __forceinline__ bool prefill_unit(const PrefillParams& p, int k, PrefillUnit& u) {
+__device__ __forceinline__ bool prefill_unit(const PrefillParams& p, int k, PrefillUnit& u,
+                                             const uint16_t* sched = nullptr) {
   constexpr bool VARLEN = LAYOUT != kLayoutDense;
   const long long G = gridDim.x;
   const long long c = blockIdx.x;
@@ -231,12 +246,26 @@ __device__ __forceinline__ bool prefill_unit(const PrefillParams& p, int k, Pref
   } else if (MASKS && p.head_pairs) {
     const int n_hp = p.Hq >> 1;
     const int n_qt = (p.Sq + 127) >> 7;
-    const long long HB = (long long)n_hp * p.B;
-    if (r >= (long long)n_qt * HB) return false;
-    u.qb = n_qt - 1 - (int)(r / HB);  // 128-row query tile
-    const int rem = (int)(r % HB);
-    u.hq = 2 * (rem % n_hp);
-    u.b = rem / n_hp;
+    if (p.sched_rows > 0) {
+      if (r >= (long long)p.sched_rows * n_hp) return false;
+      const int row = sched[r / n_hp];
+      u.qb = row % n_qt;  // 128-row query tile
+      u.b = row / n_qt;
+      u.hq = 2 * (int)(r % n_hp);
+    } else {
+      const long long HB = (long long)n_hp * p.B;
+      if (r >= (long long)n_qt * HB) return false;
+      u.qb = n_qt - 1 - (int)(r / HB);  // 128-row query tile
+      const int rem = (int)(r % HB);
+      u.hq = 2 * (rem % n_hp);
+      u.b = rem / n_hp;
+    }
+  } else if (MASKS && p.sched_rows > 0) {
+    if (r >= (long long)p.sched_rows * p.Hq) return false;
+    const int row = sched[r / p.Hq];
+    u.qb = row % p.n_qblocks;
+    u.b = row / p.n_qblocks;
+    u.hq = (int)(r % p.Hq);
   } else {
     const long long HB = (long long)p.Hq * p.B;
     if (r >= (long long)p.n_qblocks * HB) return false;
@@ -332,6 +361,40 @@ __global__ void __launch_bounds__(384, 1)
       ring[x] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
   }
+  uint16_t* sched = reinterpret_cast<uint16_t*>(sbase_ptr + C::OFF_SCHED);
+  if (MASKS && !VARLEN && p.sched_rows > 0) {
+    // Rank the unit rows of a shared block mask by their computed blocks
+    // (the MMA work of the row's query tiles), largest first and by index
+    // among equals, so that every CTA derives the same order.  The costs sit
+    // in the epilogue staging buffers, which are idle until the first unit ends.
+    int* cost = reinterpret_cast<int*>(sbase_ptr + C::OFF_STG);
+    const int n_q = p.head_pairs ? p.n_qt : p.n_qblocks;
+    for (int t = threadIdx.x; t < p.sched_rows; t += C::NUM_THREADS) {
+      const int b = t / n_q, qr = t % n_q;
+      int klen = p.Sk;
+      if (p.k_lens != nullptr) klen = min(max(__ldg(p.k_lens + b), 0), p.Sk);
+      int c = 0;
+      for (int i = 0; i < (p.head_pairs ? 1 : 2); ++i) {
+        const int row0 = p.head_pairs ? qr * 128 : qr * 256 + i * 128;
+        int lo, hi;
+        prefill_kv_range(row0, p.Sq, klen, CAUSAL, p.window, p.prefix, lo, hi);
+        const uint8_t* m = p.block_mask + ((size_t)b * p.n_qt + row0 / 128) * p.n_kt;
+#pragma unroll 16
+        for (int j = lo; j < hi; ++j) c += __ldg(m + j) != 0;
+      }
+      cost[t] = c;
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < p.sched_rows; t += C::NUM_THREADS) {
+      const int ct = cost[t];
+      int rank = 0;
+      for (int j = 0; j < p.sched_rows; ++j) {
+        const int cj = cost[j];
+        rank += (cj > ct) | ((cj == ct) & (j < t));
+      }
+      sched[rank] = (uint16_t)t;
+    }
+  }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
@@ -369,7 +432,7 @@ __global__ void __launch_bounds__(384, 1)
         return true;
       };
       PrefillUnit u;
-      for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT, MASKS>(p, k, u); ++k) {
+      for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT, MASKS>(p, k, u, sched); ++k) {
         const bool has0 = u.kv_end[0] > u.kv_begin[0], has1 = u.kv_end[1] > u.kv_begin[1];
         const int kvh = u.hq / p.group;
         const int kv_row = u.b * p.Hkv + kvh;
@@ -435,7 +498,7 @@ __global__ void __launch_bounds__(384, 1)
     uint32_t kv = 0;                  // K/V tiles issued so far (ring position)
     bool ok = true;
     PrefillUnit u;
-    for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT, MASKS>(p, k, u); ++k) {
+    for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT, MASKS>(p, k, u, sched); ++k) {
       const int kvh = u.hq / p.group;
       const int ppt = 128 / p.page_size;
       const int n_lp = (u.klen + p.page_size - 1) / p.page_size;  // <= max_pages
@@ -514,7 +577,7 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t p_waits0 = 0, p_waits1 = 0;  // P_FULL phases consumed per tile slot
       bool ok = true;
       PrefillUnit u;
-      for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT, MASKS>(p, k, u); ++k) {
+      for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT, MASKS>(p, k, u, sched); ++k) {
         const int jb = u.kv_first, je = u.kv_last;  // the unit's K/V stream
         if (je <= jb) continue;
         {
@@ -685,7 +748,7 @@ __global__ void __launch_bounds__(384, 1)
     bool stores_pending = false;
     bool ok = true;
     PrefillUnit u;
-    for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT, MASKS>(p, k, u); ++k) {
+    for (int k = 0; ok && prefill_unit<CAUSAL, LAYOUT, MASKS>(p, k, u, sched); ++k) {
       const int row0 = i ? u.row0[1] : u.row0[0];
       if (row0 >= u.sq) continue;  // this tile slot holds no rows in this unit
       const int kb = i ? u.kv_begin[1] : u.kv_begin[0];  // this tile's KV tiles [kb, ke)

@@ -124,6 +124,35 @@ def test_block_sparse_parity(case):
     check(o, o_ref, lse, lse_ref, what=f"block sparse {case}")
 
 
+SHARED_CASES = [
+    # (B, Hq, Hkv, S, causal, key padding)
+    (2, 8, 2, 4096, True, True),     # head-pair units, rows ranked by visible blocks
+    (3, 3, 3, 2000, True, False),    # 256-row units of one head, ranked
+    (2, 4, 4, 1500, False, True),    # non-causal, ranked
+    (13, 2, 1, 8192, True, False),   # 832 unit rows: more than a CTA ranks, causal order kept
+]
+
+
+@pytest.mark.parametrize("case", SHARED_CASES, ids=[str(c) for c in SHARED_CASES])
+def test_block_sparse_shared_mask_matches_per_head_copy(case):
+    # A mask shared by the heads has its unit rows ranked by their visible
+    # blocks in every CTA; the same mask repeated per head keeps the causal
+    # ranking.  Each unit is computed the same way whichever CTA takes it, so
+    # the two launches must agree bit for bit -- every unit exactly once.
+    B, Hq, Hkv, S, causal, padded = case
+    q, k, v = W.prefill_inputs(B, Hq, Hkv, S, S, 128, seed=229)
+    bm = _blocks(B, 1, S, S, 0.25, seed=233)
+    k_lens = None
+    if padded:
+        g = torch.Generator().manual_seed(239)
+        k_lens = torch.randint(S // 2, S + 1, (B,), generator=g, dtype=torch.int32)
+    scale = 1 / math.sqrt(128)
+    o1, lse1 = _run_bs(q, k, v, bm, causal, scale, k_lens)
+    o2, lse2 = _run_bs(q, k, v, bm.expand(B, Hq, -1, -1).contiguous(), causal, scale, k_lens)
+    assert torch.equal(o1, o2) and torch.equal(lse1, lse2)
+    assert bool(torch.isfinite(o1).all())
+
+
 def test_block_sparse_band_with_key_padding():
     B, Hq, Hkv, S, d = 2, 4, 2, 900, 128
     q, k, v = W.prefill_inputs(B, Hq, Hkv, S, S, d, seed=223)
