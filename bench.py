@@ -70,6 +70,8 @@ def parse_args():
     ap.add_argument("--no-paged-prefill", action="store_true")
     ap.add_argument("--no-paged-prefill-fp8", action="store_true")
     ap.add_argument("--paged-prefill-workload", default="paged_prefill_gqa")
+    ap.add_argument("--no-masks", action="store_true")
+    ap.add_argument("--masks-workload", default="gqa_causal_8k")
     return ap.parse_args()
 
 
@@ -599,6 +601,8 @@ def run_ours(args, world, rank, local):
             legs[name] = prefill_leg(args, W.CONFIGS[name], dev, world, peaks, cpu)
     if legs:
         line["prefill_legs"] = legs
+    if not args.no_masks:
+        line["masks"] = masks_leg(args, W.CONFIGS[args.masks_workload], dev, world, peaks)
     if not args.no_prefill_fp8:
         line["prefill_fp8"] = prefill_fp8_leg(args, W.CONFIGS[args.prefill_fp8_workload], dev,
                                               world, peaks)
@@ -621,6 +625,84 @@ def run_ours(args, world, rank, local):
         if dcfg is not None:
             line["decode"]["cpu_baseline"] = cpu_baseline_decode(dcfg, dinp)
     return line if rank == 0 else None
+
+
+# The programmable-mask legs: a sliding window and a block mask shared by the
+# heads, causal, on a fixed-length configuration's inputs.
+MASK_WINDOW = 1024
+MASK_DENSITY = 0.25
+
+
+def visible_pairs_window(S: int, window: int) -> int:
+    """(query row, key) pairs a causal sliding window of `window` keys leaves
+    for Sq = Sk = S: row i sees min(i + 1, window) keys."""
+    w = min(window, S)
+    return w * (w + 1) // 2 + (S - w) * w
+
+
+def visible_pairs_blocks(mask, S: int, causal: bool) -> int:
+    """Pairs a block mask uint8 [B, 1, n, n] (Sq = Sk = S, 128 x 128 blocks)
+    leaves per query head, summed over the batch: each kept block contributes
+    its (row, key) pairs, causal ones only below the diagonal."""
+    import numpy as np
+
+    n = -(-S // 128)
+    edge = np.minimum(np.arange(n) * 128 + 128, S) - np.arange(n) * 128  # rows (keys) per tile
+    full = np.outer(edge, edge)
+    if causal:
+        qt, kt = np.meshgrid(np.arange(n), np.arange(n), indexing="ij")
+        # a diagonal tile of m rows and keys holds m (m + 1) / 2 causal pairs
+        diag = np.diag(edge * (edge + 1) // 2)
+        full = np.where(kt < qt, full, 0) + diag
+    m = np.asarray(mask, dtype=np.int64)[:, 0]
+    return int((m * full[None]).sum())
+
+
+def masks_leg(args, cfg, dev, world, peaks):
+    """attn_fwd_window (window MASK_WINDOW) and attn_fwd_block_sparse (a mask of
+    density MASK_DENSITY shared by the heads, causal) on a configuration's
+    inputs, timed like the other legs; FLOPs counted over the visible (query,
+    key) pairs only, 4 d per pair and query head."""
+    import torch
+
+    from exact_softmax_attention_fwd_b200 import (attn_fwd_block_sparse, attn_fwd_window,
+                                                 attn_get_device_error)
+    from exact_softmax_attention_fwd_b200 import workloads as W
+
+    assert cfg.causal and not cfg.padded
+    q_h, k_h, v_h, _ = W.config_inputs(cfg)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((cfg.B, cfg.Hq, cfg.S), dtype=torch.float32, device=dev)
+    bm_h = W.block_mask(cfg.B, 1, cfg.S, cfg.S, MASK_DENSITY)
+    bm = bm_h.to(dev)
+    cases = {
+        f"window_{MASK_WINDOW}": (
+            lambda: attn_fwd_window(q, k, v, cfg.scale, window=MASK_WINDOW, out=o, lse=lse),
+            cfg.B * visible_pairs_window(cfg.S, MASK_WINDOW),
+            f"causal sliding window of {MASK_WINDOW} keys"),
+        f"blocks_{MASK_DENSITY}": (
+            lambda: attn_fwd_block_sparse(q, k, v, bm, True, cfg.scale, out=o, lse=lse),
+            visible_pairs_blocks(bm_h, cfg.S, True),
+            f"causal, 128 x 128 block mask shared by the heads, density {MASK_DENSITY} "
+            f"(seed {W.SEED_BLOCK_MASK})"),
+    }
+    legs = {}
+    for name, (one, pairs, what) in cases.items():
+        ms, clocks = timed_calls(args, dev, world, one)
+        st, fl = attn_get_device_error()
+        if st != 0:
+            raise RuntimeError(f"device error word set in the {name} leg: {fl:#x}")
+        flops = 4.0 * cfg.d * cfg.Hq * pairs
+        rl = tensor_roofline(flops, ms, peaks, "attn_prefill_sm100_kernel",
+                             f"{cfg.name}_{name}", world)
+        legs[name] = {"workload": f"{cfg.name}, {what}", "value": world * rl["achieved"],
+                      "unit": "TFLOPS", "flops_counted": "visible (query, key) pairs x 4 d x Hq",
+                      "visible_fraction": pairs / (cfg.B * cfg.S * (cfg.S + 1) / 2),
+                      "ms": rl["mean_ms"], "median_ms": rl["median_ms"], "calls": len(ms),
+                      "gpu_launches_per_call": 1, "clocks": clocks, "roofline": rl}
+    del q, k, v, o, lse, bm
+    return legs
 
 
 def prefill_fp8_leg(args, cfg, dev, world, peaks):

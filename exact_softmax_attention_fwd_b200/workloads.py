@@ -28,6 +28,7 @@ import torch
 SEED_PADDING = 1100
 SEED_DECODE_LENS = 2000
 SEED_DECODE_PERM = 2001
+SEED_BLOCK_MASK = 211
 
 
 @dataclass(frozen=True)
@@ -185,6 +186,15 @@ def prefill_inputs(B, Hq, Hkv, Sq, Sk, d, seed, value_scale=1.0):
 def grad_output(B, Hq, Sq, d, seed, value_scale=1.0):
     """dO [B,Hq,Sq,d] bf16 on the host: the gradient a backward pass receives."""
     return randn_bf16((B, Hq, Sq, d), seed * 16 + 3, value_scale)
+
+
+def block_mask(B: int, heads: int, Sq: int, Sk: int, density: float,
+               seed: int = SEED_BLOCK_MASK) -> torch.Tensor:
+    """uint8 [B, heads, ceil(Sq/128), ceil(Sk/128)] on the host: each 128 x 128
+    (query tile, key tile) block kept (1) with probability ``density``, drawn
+    as float32 U[0,1) from a seeded generator."""
+    g = torch.Generator().manual_seed(seed)
+    return (torch.rand(B, heads, -(-Sq // 128), -(-Sk // 128), generator=g) < density).to(torch.uint8)
 
 
 def key_padding(B: int, Sk: int, seed: int = SEED_PADDING, max_frac: float = 0.25) -> torch.Tensor:

@@ -5,7 +5,9 @@
   their own (or the shared primitives) must;
 * a stale hash makes ``ncu_traffic`` report nothing rather than an old figure;
 * the FP8 cache's algorithmic bytes: one byte per K and V element of the
-  attended tokens plus the K and V scale of every page they touch.
+  attended tokens plus the K and V scale of every page they touch;
+* the visible (query, key) pairs the mask legs count their FLOPs over, against
+  an element-by-element count of the same masks.
 """
 import json
 import os
@@ -79,3 +81,34 @@ def test_fp8_kv_bytes_formula():
     assert W.fp8_kv_bytes(lens, Hkv, d, ps) == 134 * Hkv * d * 2 + pages * Hkv * 4 * 2
     # half the bf16 cache's K/V bytes, plus the scales
     assert W.fp8_kv_bytes(lens, Hkv, d, ps) - pages * Hkv * 8 == W.decode_kv_bytes(lens, Hkv, d) // 2
+
+
+@pytest.mark.parametrize("S,window", [(1, 1), (300, 1), (300, 100), (300, 299), (300, 1000),
+                                      (1024, 1024), (1030, 128)])
+def test_window_visible_pairs(S, window):
+    i = torch.arange(S)[:, None]
+    j = torch.arange(S)[None, :]
+    brute = int(((j <= i) & (j > i - window)).sum())
+    assert bench.visible_pairs_window(S, window) == brute
+
+
+@pytest.mark.parametrize("S,causal,density", [(1, True, 1.0), (128, True, 1.0), (300, True, 0.5),
+                                               (300, False, 0.5), (513, True, 0.25),
+                                               (640, False, 0.0)])
+def test_block_mask_visible_pairs(S, causal, density):
+    m = W.block_mask(2, 1, S, S, density, seed=17)
+    i = torch.arange(S)[:, None]
+    j = torch.arange(S)[None, :]
+    vis = (j <= i) if causal else torch.ones(S, S, dtype=torch.bool)
+    brute = 0
+    for b in range(2):
+        keep = m[b, 0].repeat_interleave(128, 0).repeat_interleave(128, 1)[:S, :S] > 0
+        brute += int((vis & keep).sum())
+    assert bench.visible_pairs_blocks(m, S, causal) == brute
+
+
+def test_block_mask_generator_is_seeded_and_shaped():
+    a = W.block_mask(2, 3, 300, 700, 0.4, seed=5)
+    assert a.dtype == torch.uint8 and tuple(a.shape) == (2, 3, 3, 6)
+    assert torch.equal(a, W.block_mask(2, 3, 300, 700, 0.4, seed=5))
+    assert set(a.unique().tolist()) <= {0, 1}

@@ -124,6 +124,25 @@ def test_block_sparse_parity(case):
     check(o, o_ref, lse, lse_ref, what=f"block sparse {case}")
 
 
+@pytest.mark.parametrize("kind", ["window", "blocks"])
+def test_gqa_causal_8k_mask_legs_full(kind):
+    """Every element of the two mask workloads bench.py times: the 8k GQA inputs
+    (B=2, Hq=32, Hkv=8, S=8192) with a causal sliding window, and with a causal
+    block mask shared by the heads (seeded, the bench's density)."""
+    import bench
+
+    c = W.CONFIGS["gqa_causal_8k"]
+    q, k, v, _ = W.config_inputs(c)
+    if kind == "window":
+        o, lse = _run(q, k, v, c.scale, window=bench.MASK_WINDOW)
+        o_ref, lse_ref = oracle.attn_fwd(q, k, v, True, c.scale, window=bench.MASK_WINDOW)
+    else:
+        bm = W.block_mask(c.B, 1, c.S, c.S, bench.MASK_DENSITY)
+        o, lse = _run_bs(q, k, v, bm, True, c.scale)
+        o_ref, lse_ref = oracle.attn_fwd(q, k, v, True, c.scale, block_mask=bm)
+    check(o, o_ref, lse, lse_ref, what=f"{c.name} {kind}")
+
+
 SHARED_CASES = [
     # (B, Hq, Hkv, S, causal, key padding)
     (2, 8, 2, 4096, True, True),     # head-pair units, rows ranked by visible blocks
