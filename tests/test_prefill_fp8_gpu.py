@@ -66,6 +66,34 @@ def test_fp8_prefill_mha_causal_2k_full():
     check(o, o_ref, lse, lse_ref, what="fp8 mha_causal_2k")
 
 
+def test_fp8_prefill_gqa_causal_8k_two_kv_groups():
+    """The launch the bench times: the gqa_causal_8k inputs (B=2, Hq=32, Hkv=8,
+    S=8192, causal) quantised and run whole.  Checked: the first and the last
+    1024 query rows of two KV-head groups (batch 0 / KV head 0 and batch 1 /
+    KV head 7, four query heads each), every element, against the oracle run
+    on those rows alone -- the first rows see only the first 1024 keys, the
+    last rows all 8192 keys with the bottom-right causal rule, and both
+    slices start on a 128-row block, so their scales are the launch's own."""
+    c = W.CONFIGS["gqa_causal_8k"]
+    x = W.fp8_prefill_inputs(c.B, c.Hq, c.Hkv, c.S, c.S, c.d, c.seed, c.value_scale)
+    o, lse = _run(*x, True, c.scale)
+    q8, k8, v8, qs, ks, vs = x
+    g, S, R = c.Hq // c.Hkv, c.S, 1024
+    for b, kvh in ((0, 0), (c.B - 1, c.Hkv - 1)):
+        bb, hs, kv = slice(b, b + 1), slice(kvh * g, (kvh + 1) * g), slice(kvh, kvh + 1)
+        last, last_blk = slice(S - R, S), slice((S - R) // 128, S // 128)
+        o_ref, lse_ref = oracle_fp8(q8[bb, hs, last], k8[bb, kv], v8[bb, kv], qs[bb, hs, last_blk],
+                                    ks[bb, kv], vs[bb, kv], True, c.scale)
+        check(o[bb, hs, last], o_ref, lse[bb, hs, last], lse_ref,
+              what=f"fp8 gqa_causal_8k batch {b} KV head {kvh}, last {R} rows")
+        first, first_blk = slice(0, R), slice(0, R // 128)
+        o_ref, lse_ref = oracle_fp8(q8[bb, hs, first], k8[bb, kv, first], v8[bb, kv, first],
+                                    qs[bb, hs, first_blk], ks[bb, kv, first_blk],
+                                    vs[bb, kv, first_blk], True, c.scale)
+        check(o[bb, hs, first], o_ref, lse[bb, hs, first], lse_ref,
+              what=f"fp8 gqa_causal_8k batch {b} KV head {kvh}, first {R} rows")
+
+
 def test_fp8_prefill_key_padding_and_empty_rows():
     x = W.fp8_prefill_inputs(3, 4, 2, 256, 256, 128, seed=303)
     k_lens = torch.tensor([0, 77, 256], dtype=torch.int32)
