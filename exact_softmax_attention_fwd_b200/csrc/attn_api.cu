@@ -332,20 +332,23 @@ int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mdo, const CUtensorMap&
   if (prep_blocks > INT_MAX || kv_units > INT_MAX || q_units > INT_MAX) return ATTN_ERR_INVALID_ARG;
   attn_bwd_prep_kernel<D, VARLEN><<<(unsigned)prep_blocks, 256, 0, stream>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  // the masked instantiations keep a list of the blocks they walk in shared memory
+  constexpr int kv_smem = MASKS ? C::KV_SMEM_MASKS : C::KV_SMEM;
+  constexpr int q_smem = MASKS ? C::Q_SMEM_MASKS : C::Q_SMEM;
   auto kv = attn_bwd_dkdv_kernel<D, CAUSAL, VARLEN, MASKS>;
   static std::atomic<unsigned long long> kv_smem_set{0};
-  if (!set_smem_once(kv, C::KV_SMEM, kv_smem_set)) return ATTN_ERR_CUDA;
-  kv<<<(unsigned)kv_units, C::NUM_THREADS, C::KV_SMEM, stream>>>(mq, mdo, mk, mv, prm);
+  if (!set_smem_once(kv, kv_smem, kv_smem_set)) return ATTN_ERR_CUDA;
+  kv<<<(unsigned)kv_units, C::NUM_THREADS, kv_smem, stream>>>(mq, mdo, mk, mv, prm);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   auto dq = attn_bwd_dq_kernel<D, CAUSAL, VARLEN, MASKS>;
   static std::atomic<unsigned long long> q_smem_set{0};
-  if (!set_smem_once(dq, C::Q_SMEM, q_smem_set)) return ATTN_ERR_CUDA;
+  if (!set_smem_once(dq, q_smem, q_smem_set)) return ATTN_ERR_CUDA;
   // dQ as a programmatic dependent of dK/dV (it reads only the inputs and the
   // prep kernel's statistics, complete before dK/dV started)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)q_units);
   cfg.blockDim = dim3(C::NUM_THREADS);
-  cfg.dynamicSmemBytes = C::Q_SMEM;
+  cfg.dynamicSmemBytes = q_smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -88,6 +88,29 @@ __device__ __forceinline__ bool bwd_block_on(const BwdParams& p, int b, int hq, 
   return __ldg(p.block_mask + (((size_t)b * p.mask_heads + h) * p.n_qt + qt) * p.n_kt + kt) != 0;
 }
 
+// Block-sparse backward: the candidate iterations [0, n) whose block is on,
+// listed in ascending order by all threads of the CTA (flags first, then one
+// warp compacts them with ballots), so that every role walks the same list.
+// The caller's next __syncthreads publishes list[0, *count).
+template <typename On>
+__device__ __forceinline__ void bwd_list_blocks(int n, On on, uint16_t* list, uint8_t* flag,
+                                                int* count) {
+  for (int c = threadIdx.x; c < n; c += blockDim.x) flag[c] = on(c) ? 1 : 0;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int cnt = 0;
+    for (int base = 0; base < n; base += 32) {
+      const int c = base + lane;
+      const bool keep = c < n && flag[c] != 0;
+      const unsigned m = __ballot_sync(0xffffffffu, keep);
+      if (keep) list[cnt + __popc(m & ((1u << lane) - 1u))] = (uint16_t)c;
+      cnt += __popc(m);
+    }
+    if (lane == 0) *count = cnt;
+  }
+}
+
 // One sequence of a backward call: query rows [q0, q0 + lq) and keys
 // [k0, k0 + lk) of the packed tensors (fixed-length batches: q0 = k0 = 0,
 // lq = Sq, lk = the clamped key length).  False when a ragged sequence's
@@ -150,6 +173,11 @@ struct BwdCfg {
   static constexpr int KB_NUM = KB_ACC + 1;
   static constexpr int KV_OFF_MISC = KV_OFF_BAR + KB_NUM * 8;
   static constexpr int KV_SMEM = KV_OFF_MISC + 16 + 1024;
+  // block masks: the iterations a CTA keeps, listed as uint16 ids, then one
+  // flag byte per candidate (masked instantiations only)
+  static constexpr int LIST_MAX = 4096;
+  static constexpr int KV_OFF_LIST = KV_OFF_MISC + 16;
+  static constexpr int KV_SMEM_MASKS = KV_SMEM + 3 * LIST_MAX;
   // ---- dQ kernel: Q, dO resident; K, V in a ring
   static constexpr int Q_OFF_Q = 0;
   static constexpr int Q_OFF_DO = TILE_BYTES;
@@ -166,6 +194,8 @@ struct BwdCfg {
   static constexpr int QB_NUM = QB_ACC + 1;
   static constexpr int Q_OFF_MISC = Q_OFF_BAR + QB_NUM * 8;
   static constexpr int Q_SMEM = Q_OFF_MISC + 16 + 1024;
+  static constexpr int Q_OFF_LIST = Q_OFF_MISC + 16;
+  static constexpr int Q_SMEM_MASKS = Q_SMEM + 3 * LIST_MAX;
   // ---- tensor memory (512 columns)
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t KV_TM_S = 0;        // S^T
@@ -180,7 +210,7 @@ struct BwdCfg {
   static constexpr uint32_t REGS_SOFTMAX = 192;
   static_assert(128 * (REGS_PRODUCER + 2 * REGS_SOFTMAX) <= NUM_THREADS * 168,
                 "register reallocation must fit the launch allocation");
-  static_assert(KV_SMEM <= 232448 && Q_SMEM <= 232448, "shared memory");
+  static_assert(KV_SMEM_MASKS <= 232448 && Q_SMEM_MASKS <= 232448, "shared memory");
   static_assert(D == 64 || D == 128, "head dim");
 };
 
@@ -328,7 +358,16 @@ __global__ void __launch_bounds__(384, 1)
     }
   }
   const int nq = (!seq_ok || key0 >= klen || qt_hi <= qt_lo) ? 0 : qt_hi - qt_lo;
-  const int N = p.group * nq;  // (query head, query tile) iterations
+  const int N = p.group * nq;  // (query head, query tile) candidates
+  // with a block mask, only the candidates whose block is on are walked
+  const bool listed = MASKS && p.block_mask != nullptr && N > 0 && N <= C::LIST_MAX;
+  const uint16_t* list = reinterpret_cast<const uint16_t*>(sbase_ptr + C::KV_OFF_LIST);
+  int* list_count = reinterpret_cast<int*>(sbase_ptr + C::KV_OFF_MISC + 8);
+  if (listed)
+    bwd_list_blocks(
+        N, [&](int c) { return bwd_block_on(p, b, kvh * p.group + c / nq, qt_lo + c % nq, kb); },
+        reinterpret_cast<uint16_t*>(sbase_ptr + C::KV_OFF_LIST),
+        sbase_ptr + C::KV_OFF_LIST + 2 * C::LIST_MAX, list_count);
   // dK/dV rows this CTA writes: a ragged sequence's own keys only (rows past
   // them belong to the next sequence); fixed-length batches write every key
   // row of the tile (padded keys get zeros)
@@ -357,6 +396,8 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  const int NI = listed ? *list_count : N;  // iterations walked
+  auto cand = [&](int n) { return listed ? (int)list[n] : n; };
   const uint32_t sK = sbase + C::KV_OFF_K, sV = sbase + C::KV_OFF_V;
   auto sQ = [&](int s) { return sbase + C::KV_OFF_Q + (uint32_t)s * C::TILE_BYTES; };
   auto sDO = [&](int s) { return sbase + C::KV_OFF_DO + (uint32_t)s * C::TILE_BYTES; };
@@ -364,7 +405,7 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp < 4) {
     warpgroup_reg_dealloc<C::REGS_PRODUCER>();
-    if (warp == 0 && lane == 0 && N > 0) {
+    if (warp == 0 && lane == 0 && NI > 0) {
       // ======================= TMA producer =======================
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_do);
@@ -380,13 +421,14 @@ __global__ void __launch_bounds__(384, 1)
       }
       int issued = 0;
       bool ok = true;
-      for (int n = 0; n < N; ++n) {
+      for (int n = 0; n < NI; ++n) {
         const int s = n % C::STAGES;
         if (n >= C::STAGES &&
             !(ok = mbar_wait(bar(C::KB_QE + s), ((n / C::STAGES) - 1) & 1u, abort_flag)))
           break;
-        const int hq = kvh * p.group + n / nq;
-        const int qt = qt_lo + n % nq;
+        const int c = cand(n);
+        const int hq = kvh * p.group + c / nq;
+        const int qt = qt_lo + c % nq;
         const int bh_q = b * p.Hq + hq;
         mbar_arrive_expect_tx(bar(C::KB_QF + s), 2 * C::TILE_BYTES + C::STAT_BYTES);
         const int qy = VARLEN ? hq : qt * 128, qz = VARLEN ? sq.q0 + qt * 128 : bh_q;
@@ -403,7 +445,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_wait(bar(C::KB_KV), 0, nullptr);
       for (int n = (issued > C::STAGES ? issued - C::STAGES : 0); n < issued; ++n)
         mbar_wait(bar(C::KB_QF + n % C::STAGES), (n / C::STAGES) & 1u, nullptr);
-    } else if (warp == 1 && lane == 0 && N > 0) {
+    } else if (warp == 1 && lane == 0 && NI > 0) {
       // ======================= tcgen05 MMA issuer =======================
       const uint32_t tS = tmem + C::KV_TM_S, tDP = tmem + C::KV_TM_DP;
       const uint32_t tDV = tmem + C::KV_TM_DV, tDK = tmem + C::KV_TM_DK;
@@ -415,9 +457,9 @@ __global__ void __launch_bounds__(384, 1)
         bwd_mma_ss<D>(tDP, sV, sDO(0));
         umma_commit(bar(C::KB_DPF));
       }
-      for (int n = 0; ok && n < N; ++n) {
+      for (int n = 0; ok && n < NI; ++n) {
         const int s = n % C::STAGES, s1 = (n + 1) % C::STAGES;
-        if (n + 1 < N) {
+        if (n + 1 < NI) {
           // S^T of the next query tile, as soon as this tile's S^T has been read
           if (!(ok = mbar_wait(bar(C::KB_SE), n & 1u, abort_flag))) break;
           if (!(ok = mbar_wait(bar(C::KB_QF + s1), ((n + 1) / C::STAGES) & 1u, abort_flag))) break;
@@ -430,7 +472,7 @@ __global__ void __launch_bounds__(384, 1)
         bwd_mma_ts<D>(tDV, tDP + 32, sDO(s), n > 0);  // dV += P^T dO
         bwd_mma_ts<D>(tDK, tDP, sQ(s), n > 0);        // dK += dS^T Q
         umma_commit(bar(C::KB_QE + s));  // Q and dO of stage s read for the last time
-        if (n + 1 < N) {
+        if (n + 1 < NI) {
           // dP^T of the next tile overwrites P^T and dS^T only after the two MMAs
           // above read them (MMAs of one thread run in issue order)
           bwd_mma_ss<D>(tDP, sV, sDO(s1));
@@ -456,9 +498,10 @@ __global__ void __launch_bounds__(384, 1)
     const float c2 = p.scale_log2;
     const uint64_t c2x2 = f32x2(c2, c2);
     bool ok = true;
-    for (int n = 0; ok && n < N; ++n) {
+    for (int n = 0; ok && n < NI; ++n) {
       const int s = n % C::STAGES;
-      const int qt = qt_lo + n % nq;
+      const int cn = cand(n);
+      const int qt = qt_lo + cn % nq;
       // columns c >= cmin are visible to this key (c relative to this warpgroup's run)
       long long cm = (j >= klen) ? 64 : (CAUSAL ? (long long)j - koff - qt * 128 - c0 : 0);
       long long cx = 64;  // columns [cmin, cmax) are visible to this key
@@ -468,7 +511,7 @@ __global__ void __launch_bounds__(384, 1)
           cm = 0;
           cx = 64;
         }
-        if (!bwd_block_on(p, b, kvh * p.group + n / nq, qt, kb)) cm = 64;
+        if (!bwd_block_on(p, b, kvh * p.group + cn / nq, qt, kb)) cm = 64;
       }
       const int cmin = (int)(cm < 0 ? 0 : (cm > 64 ? 64 : cm));
       const int cmax = MASKS ? (int)(cx < 0 ? 0 : (cx > 64 ? 64 : cx)) : 64;
@@ -552,7 +595,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_arrive(bar(C::KB_QE + s));  // this thread is done with stage s's statistics
     }
     // ---- epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (times scale)
-    bool have = N > 0;
+    bool have = NI > 0;
     if (have && ok) {
       ok = mbar_wait_warp(bar(C::KB_ACC), 0, abort_flag);
       tc_fence_after_sync();
@@ -629,6 +672,15 @@ __global__ void __launch_bounds__(384, 1)
   // key tiles [kt_lo, kt_lo + N); none for a tile past the sequence's rows
   const int kt_end = max_key < 0 ? 0 : (int)(max_key / 128) + 1;
   const int N = (row0 >= n_rows || kt_end <= kt_lo) ? 0 : kt_end - kt_lo;
+  // with a block mask, only the key tiles whose block is on are walked
+  const bool listed = MASKS && p.block_mask != nullptr && N > 0 && N <= C::LIST_MAX;
+  const uint16_t* list = reinterpret_cast<const uint16_t*>(sbase_ptr + C::Q_OFF_LIST);
+  int* list_count = reinterpret_cast<int*>(sbase_ptr + C::Q_OFF_MISC + 8);
+  if (listed)
+    bwd_list_blocks(
+        N, [&](int c) { return bwd_block_on(p, b, hq, qt, kt_lo + c); },
+        reinterpret_cast<uint16_t*>(sbase_ptr + C::Q_OFF_LIST),
+        sbase_ptr + C::Q_OFF_LIST + 2 * C::LIST_MAX, list_count);
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::QB_QF), 1);
@@ -653,13 +705,15 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  const int NI = listed ? *list_count : N;  // key tiles walked
+  auto cand = [&](int n) { return listed ? (int)list[n] : n; };
   const uint32_t sQ = sbase + C::Q_OFF_Q, sDO = sbase + C::Q_OFF_DO;
   auto sK = [&](int s) { return sbase + C::Q_OFF_K + (uint32_t)s * C::TILE_BYTES; };
   auto sV = [&](int s) { return sbase + C::Q_OFF_V + (uint32_t)s * C::TILE_BYTES; };
 
   if (warp < 4) {
     warpgroup_reg_dealloc<C::REGS_PRODUCER>();
-    if (warp == 0 && lane == 0 && N > 0) {
+    if (warp == 0 && lane == 0 && NI > 0) {
       // ======================= TMA producer =======================
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_do);
@@ -673,13 +727,13 @@ __global__ void __launch_bounds__(384, 1)
       }
       int issued = 0;
       bool ok = true;
-      for (int n = 0; n < N; ++n) {
+      for (int n = 0; n < NI; ++n) {
         const int s = n % C::STAGES;
         if (n >= C::STAGES &&
             !(ok = mbar_wait(bar(C::QB_KVE + s), ((n / C::STAGES) - 1) & 1u, abort_flag)))
           break;
         mbar_arrive_expect_tx(bar(C::QB_KVF + s), 2 * C::TILE_BYTES);
-        const int kt = kt_lo + n;
+        const int kt = kt_lo + cand(n);
         const int ky = VARLEN ? kvh : kt * 128, kz = VARLEN ? sq.k0 + kt * 128 : bh_kv;
         for (int cb = 0; cb < C::NCB; ++cb) {
           tma_load_3d(sK(s) + cb * C::CB_BYTES, &tm_k, bar(C::QB_KVF + s), 64 * cb, ky, kz);
@@ -690,7 +744,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_wait(bar(C::QB_QF), 0, nullptr);
       for (int n = (issued > C::STAGES ? issued - C::STAGES : 0); n < issued; ++n)
         mbar_wait(bar(C::QB_KVF + n % C::STAGES), (n / C::STAGES) & 1u, nullptr);
-    } else if (warp == 1 && lane == 0 && N > 0) {
+    } else if (warp == 1 && lane == 0 && NI > 0) {
       // ======================= tcgen05 MMA issuer =======================
       const uint32_t tDP = tmem + C::Q_TM_DP, tDQ = tmem + C::Q_TM_DQ;
       auto tS = [&](int n) { return tmem + ((n & 1) ? C::Q_TM_S1 : C::Q_TM_S0); };
@@ -702,9 +756,9 @@ __global__ void __launch_bounds__(384, 1)
         bwd_mma_ss<D>(tDP, sDO, sV(0));
         umma_commit(bar(C::QB_DPF));
       }
-      for (int n = 0; ok && n < N; ++n) {
+      for (int n = 0; ok && n < NI; ++n) {
         const int s = n % C::STAGES, s1 = (n + 1) % C::STAGES;
-        if (n + 1 < N) {
+        if (n + 1 < NI) {
           if (!(ok = mbar_wait(bar(C::QB_KVF + s1), ((n + 1) / C::STAGES) & 1u, abort_flag))) break;
           tc_fence_after_sync();
           bwd_mma_ss<D>(tS(n + 1), sQ, sK(s1));
@@ -714,7 +768,7 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after_sync();
         bwd_mma_ts<D>(tDQ, tDP, sK(s), n > 0);  // dQ += dS K
         umma_commit(bar(C::QB_KVE + s));
-        if (n + 1 < N) {
+        if (n + 1 < NI) {
           // dP of the next key tile: overwrites dS only after the MMA above read it
           bwd_mma_ss<D>(tDP, sDO, sV(s1));
           umma_commit(bar(C::QB_DPF));
@@ -745,10 +799,11 @@ __global__ void __launch_bounds__(384, 1)
       kend = min(kend, max((long long)row + koff, MASKS ? (long long)p.prefix - 1 : -1LL) + 1);
     if (MASKS && p.window > 0) klo = max(0LL, (long long)row + koff - p.window + 1);
     bool ok = true;
-    for (int n = 0; ok && n < N; ++n) {
-      const long long t0 = (long long)(kt_lo + n) * 128 + c0;  // this run's first key
+    for (int n = 0; ok && n < NI; ++n) {
+      const int kt = kt_lo + cand(n);
+      const long long t0 = (long long)kt * 128 + c0;  // this run's first key
       long long cm = kend - t0;  // visible iff cmin <= c < cmax
-      if (MASKS && !bwd_block_on(p, b, hq, qt, kt_lo + n)) cm = 0;
+      if (MASKS && !bwd_block_on(p, b, hq, qt, kt)) cm = 0;
       const long long cn = MASKS ? klo - t0 : 0;
       const int cmin = (int)(cn < 0 ? 0 : (cn > 64 ? 64 : cn));
       const int cmax = (int)(cm < 0 ? 0 : (cm > 64 ? 64 : cm));
@@ -803,7 +858,7 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
     // ---- epilogue: each warpgroup writes half of the dQ row (times scale)
-    const bool have = N > 0;
+    const bool have = NI > 0;
     if (have && ok) {
       ok = mbar_wait_warp(bar(C::QB_ACC), 0, abort_flag);
       tc_fence_after_sync();

@@ -503,7 +503,9 @@ int attn_bwd_window(const void* q, const void* k, const void* v, const void* o, 
  * Source: as attn_bwd_window; "可编程 mask" (block-level sparsity).
  *   block_mask, mask_heads exactly as given to attn_fwd_block_sparse: uint8
  *   [B, mask_heads, ceil(Sq/128), ceil(Sk/128)] device array, mask_heads 1 or
- *   Hq; 0 hides the 128 x 128 block.  Other arguments as attn_bwd.
+ *   Hq; 0 hides the 128 x 128 block, which is then neither loaded nor
+ *   computed (for units of up to 4096 candidate blocks; larger ones stream
+ *   it and weight it zero).  Other arguments as attn_bwd.
  * Errors: as attn_bwd, plus INVALID_ARG for a NULL block_mask or another
  * mask_heads.
  */
