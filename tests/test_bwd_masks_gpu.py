@@ -92,6 +92,7 @@ def test_bwd_block_sparse(case):
     g = torch.Generator().manual_seed(423 + Sq)
     mask = (torch.rand(B, Hq if per_head else 1, nq, nk, generator=g) < 0.5).to(torch.uint8)
     mask[:, :, 0, :] = 0  # a query tile with no block at all: zero dQ, no gradient from it
+    mask[:, :, :, 1] = 0  # a key tile no query tile keeps: its dK / dV units walk nothing
     scale = 1 / math.sqrt(d)
     qd, kd, vd, dod, md = (x.to(DEV) for x in (q, k, v, do, mask))
     o, lse = attn_fwd_block_sparse(qd, kd, vd, md, causal, scale)
@@ -102,6 +103,8 @@ def test_bwd_block_sparse(case):
     ref = oracle_bwd(q, k, v, do, causal, scale, block_mask=mask.numpy())
     _check(got, ref, f"blocks {case}")
     assert not got[0][:, :, :128].float().abs().sum()  # rows of the empty query tile
+    assert not got[1][:, :, 128:256].float().abs().sum()  # rows of the empty key tile
+    assert not got[2][:, :, 128:256].float().abs().sum()
 
 
 def test_bwd_all_ones_block_mask_equals_plain_backward():
