@@ -72,6 +72,8 @@ def parse_args():
     ap.add_argument("--paged-prefill-workload", default="paged_prefill_gqa")
     ap.add_argument("--no-masks", action="store_true")
     ap.add_argument("--masks-workload", default="gqa_causal_8k")
+    ap.add_argument("--mask-legs", default="window,blocks",
+                    help="which mask legs to time: window, blocks or both")
     return ap.parse_args()
 
 
@@ -687,8 +689,11 @@ def masks_leg(args, cfg, dev, world, peaks):
             f"causal, 128 x 128 block mask shared by the heads, density {MASK_DENSITY} "
             f"(seed {W.SEED_BLOCK_MASK})"),
     }
+    wanted = {x.strip() for x in args.mask_legs.split(",") if x.strip()}
     legs = {}
     for name, (one, pairs, what) in cases.items():
+        if name.split("_")[0] not in wanted:
+            continue
         ms, clocks = timed_calls(args, dev, world, one)
         st, fl = attn_get_device_error()
         if st != 0:
